@@ -1,0 +1,179 @@
+"""CPU oracle for NABLA block-sparse attention -- test infrastructure only.
+
+This package wraps ``oracle.c`` (plain scalar C, OpenMP over independent
+rows) with ctypes.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it.
+The product path (``block_sparse_attention_flatten_b200``) never imports it
+and shares no code with it.
+
+Every function restates one step of the method as described on the page
+"Resumo Tecnico: NABLA - Atencao de Bloco Adaptativa de Vizinhanca para
+Geracao de Video Eficiente" (section "Metodologia: NABLA"); the C source
+names the item each one follows.
+
+Parity unpinned: the STA window geometry beyond "a static local window"
+(centred, truncated at the border, temporal tile = one frame) is a reading
+of the pages, checked only against its own closed-form count.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+BLOCK = 64  # N = P * P tokens per block (P = 8)
+BAND = 1e-5  # |c - (1 - thr)| below this marks a band block
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (no fused multiply-add)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
+               "-o", _LIB_PATH + ".tmp", _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB_PATH + ".tmp", _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        i, i64, f, d = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double
+        lib.oracle_flatten.argtypes = [P, P, i, i, i, i, i, i64]
+        lib.oracle_unflatten.argtypes = [P, P, i, i, i, i, i, i64]
+        lib.oracle_pool.argtypes = [P, P, i, i, i, i]
+        lib.oracle_mask.argtypes = [P, P, i, i, i, i, f, f, i, i, i, i, i, d, P, P, P, P]
+        lib.oracle_attention.argtypes = [P, P, P, P, P, i, i, i, i, d, P, i, P, P]
+        lib.oracle_block_probs_row.argtypes = [P, P, i, i, f, i, P]
+        lib.oracle_cdf_keep.argtypes = [P, i, f, P, P]
+        lib.oracle_cdf_keep.restype = i
+        lib.oracle_sta.argtypes = [i, i, i, i, i, i, i]
+        lib.oracle_sta.restype = i
+        lib.oracle_num_threads.restype = i
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def _bits(x: np.ndarray) -> np.ndarray:
+    """bf16 data as raw uint16 bits (accepts a uint16 array or a torch bf16 tensor)."""
+    if hasattr(x, "view") and not isinstance(x, np.ndarray):  # torch tensor
+        import torch
+        x = x.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return np.ascontiguousarray(x, dtype=np.uint16)
+
+
+def flatten(x, T: int, H: int, W: int, P: int = 8) -> np.ndarray:
+    """Fractal flattening of a grid-order [B, S, row] bf16 array (uint16 bits)."""
+    x = _bits(x)
+    B = x.shape[0]
+    row = int(np.prod(x.shape[2:]))
+    out = np.empty_like(x)
+    _load().oracle_flatten(_ptr(x), _ptr(out), B, T, H, W, P, row)
+    return out
+
+
+def unflatten(x, T: int, H: int, W: int, P: int = 8) -> np.ndarray:
+    """Inverse of :func:`flatten`."""
+    x = _bits(x)
+    B = x.shape[0]
+    row = int(np.prod(x.shape[2:]))
+    out = np.empty_like(x)
+    _load().oracle_unflatten(_ptr(x), _ptr(out), B, T, H, W, P, row)
+    return out
+
+
+def pool(xf) -> np.ndarray:
+    """Block means of a flattened [B, S, Hh, D] bf16 array -> fp32 [B, Hh, Nb, D]."""
+    xf = _bits(xf)
+    B, S, Hh, D = xf.shape
+    out = np.empty((B, Hh, S // BLOCK, D), dtype=np.float32)
+    _load().oracle_pool(_ptr(xf), _ptr(out), B, S, Hh, D)
+    return out
+
+
+def block_probs_row(qbar_bh: np.ndarray, kbar_bh: np.ndarray, i: int, scale: float) -> np.ndarray:
+    """Reduced-attention probabilities of query block i for one (b, head)."""
+    qbar_bh = np.ascontiguousarray(qbar_bh, dtype=np.float32)
+    kbar_bh = np.ascontiguousarray(kbar_bh, dtype=np.float32)
+    Nb, D = kbar_bh.shape
+    p = np.empty(Nb, dtype=np.float32)
+    _load().oracle_block_probs_row(_ptr(qbar_bh), _ptr(kbar_bh), Nb, D, scale, i, _ptr(p))
+    return p
+
+
+def cdf_keep(p: np.ndarray, thr: float):
+    """CDF keep flags and per-block cumulative mass for one probability row."""
+    p = np.ascontiguousarray(p, dtype=np.float32)
+    keep = np.empty(p.shape[0], dtype=np.uint8)
+    cum = np.empty(p.shape[0], dtype=np.float64)
+    argmax = _load().oracle_cdf_keep(_ptr(p), p.shape[0], thr, _ptr(keep), _ptr(cum))
+    return keep.astype(bool), cum, argmax
+
+
+def sta(i: int, j: int, nbh: int, nbw: int, window=(3, 3, 3)) -> bool:
+    return bool(_load().oracle_sta(i, j, nbh, nbw, *window))
+
+
+def build_mask(qbar: np.ndarray, kbar: np.ndarray, thr: float, scale: float, nbh: int, nbw: int,
+               sta_window=(0, 0, 0), band: float = BAND, want_status: bool = True,
+               want_probs: bool = False):
+    """Masks for every row.  Returns (kv_count, kv_idx, status, probs).
+
+    kv_count int32 [B,Hh,Nb]; kv_idx int32 [B,Hh,Nb,Nb] (ascending, padded
+    with -1 past the count); status uint8 [B,Hh,Nb,Nb] (bit0 kept, bit1 band)
+    or None; probs fp32 [B,Hh,Nb,Nb] or None.
+    """
+    qbar = np.ascontiguousarray(qbar, dtype=np.float32)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float32)
+    B, Hh, Nb, D = qbar.shape
+    kv_count = np.zeros((B, Hh, Nb), dtype=np.int32)
+    kv_idx = np.full((B, Hh, Nb, Nb), -1, dtype=np.int32)
+    status = np.zeros((B, Hh, Nb, Nb), dtype=np.uint8) if want_status else None
+    probs = np.zeros((B, Hh, Nb, Nb), dtype=np.float32) if want_probs else None
+    _load().oracle_mask(_ptr(qbar), _ptr(kbar), B, Hh, Nb, D, scale, thr, nbh, nbw,
+                        int(sta_window[0]), int(sta_window[1]), int(sta_window[2]), band,
+                        _ptr(kv_count), _ptr(kv_idx),
+                        _ptr(status) if status is not None else None,
+                        _ptr(probs) if probs is not None else None)
+    return kv_count, kv_idx, status, probs
+
+
+def attention(qf, kf, vf, kv_count: np.ndarray, kv_idx: np.ndarray, scale: float, qblocks=None):
+    """Masked attention (fp64) for the listed query blocks (all heads).
+
+    Returns (out fp64 [B, nq*64, Hh, D], lse fp64 [B, Hh, nq*64]).
+    """
+    qf, kf, vf = _bits(qf), _bits(kf), _bits(vf)
+    B, S, Hh, D = qf.shape
+    Nb = S // BLOCK
+    if qblocks is None:
+        qblocks = np.arange(Nb, dtype=np.int32)
+    qblocks = np.ascontiguousarray(qblocks, dtype=np.int32)
+    nq = qblocks.shape[0]
+    kv_count = np.ascontiguousarray(kv_count, dtype=np.int32)
+    kv_idx = np.ascontiguousarray(kv_idx, dtype=np.int32)
+    assert kv_idx.shape == (B, Hh, Nb, Nb)
+    out = np.zeros((B, nq * BLOCK, Hh, D), dtype=np.float64)
+    lse = np.zeros((B, Hh, nq * BLOCK), dtype=np.float64)
+    _load().oracle_attention(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(kv_count), _ptr(kv_idx), B, S, Hh, D,
+                             scale, _ptr(qblocks), nq, _ptr(out), _ptr(lse))
+    return out, lse

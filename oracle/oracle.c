@@ -1,0 +1,350 @@
+/*
+ * CPU oracle for NABLA block-sparse attention -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, scalar C that restates what the method computes so the CUDA
+ * path can be checked against it.  Only the test suite, the smoke check and
+ * the benchmark's CPU-baseline leg may load this library; the product path
+ * never calls it and shares no code with it.
+ *
+ * Source of every step: the page "Resumo Tecnico: NABLA - Atencao de Bloco
+ * Adaptativa de Vizinhanca para Geracao de Video Eficiente" (gist.science,
+ * paper 2507.13546), section "Metodologia: NABLA":
+ *   item 1  "Reordenacao de Tokens (Fractal Flattening)"       -> oracle_flatten
+ *   item 2  "Downsampling"                                     -> oracle_pool
+ *           "Atencao Reduzida"                                 -> block_probs
+ *           "Limiarizacao CDF"                                 -> cdf_keep_row
+ *           "Expansao"                                         -> kv lists
+ *   item 3  "Integracao Hibrida com STA", M = M_nabla OR M_STA -> sta_keep
+ * and the attention on the kept N x N blocks (same section, "Expansao"),
+ * with dropped blocks absent from both numerator and normaliser (the
+ * AB-Attention news page, section "Onde os esquemas esparsos anteriores
+ * falham", second bullet) -> oracle_attention.
+ *
+ * Precision: the mask is fp32 (pooled vectors, scores, exponentials,
+ * probabilities) with fp64 accumulation of the softmax normaliser and of the
+ * CDF; attention accumulates in fp64.  Build with -ffp-contract=off so every
+ * a*b+c below is two roundings, as written.
+ *
+ * Parity pins (each in tests/): see the functions' comments.  Functions with
+ * no external pin say "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_BLOCK 64 /* N = P*P tokens per block, P = 8 */
+
+static inline float bf16_bits_to_f32(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Fractal flattening (NABLA summary, Metodologia item 1).                   */
+/* Grid order s = (t*H + h)*W + w.  Flattened order: frame-major, then the   */
+/* P x P patch (bh, bw) row-major, then the token inside the patch           */
+/* row-major:  f = t*H*W + (bh*nbw + bw)*P*P + (h%P)*P + (w%P).              */
+/* Pinned by: an independent reshape/transpose formulation, bijectivity,     */
+/* unflatten(flatten(x)) == x, and the T=1,H=W=P identity case.              */
+/* ------------------------------------------------------------------------ */
+static int64_t flat_index(int t, int h, int w, int H, int W, int P) {
+  int nbw = W / P;
+  int bh = h / P, bw = w / P;
+  return (int64_t)t * H * W + (int64_t)(bh * nbw + bw) * P * P + (h % P) * P + (w % P);
+}
+
+void oracle_flatten(const uint16_t* in, uint16_t* out, int B, int T, int H, int W, int P,
+                    int64_t row_elems) {
+  int64_t S = (int64_t)T * H * W;
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < T; ++t)
+      for (int h = 0; h < H; ++h)
+        for (int w = 0; w < W; ++w) {
+          int64_t src = ((int64_t)t * H + h) * W + w;
+          int64_t dst = flat_index(t, h, w, H, W, P);
+          memcpy(out + (b * S + dst) * row_elems, in + (b * S + src) * row_elems,
+                 (size_t)row_elems * 2);
+        }
+}
+
+void oracle_unflatten(const uint16_t* in, uint16_t* out, int B, int T, int H, int W, int P,
+                      int64_t row_elems) {
+  int64_t S = (int64_t)T * H * W;
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < T; ++t)
+      for (int h = 0; h < H; ++h)
+        for (int w = 0; w < W; ++w) {
+          int64_t grid = ((int64_t)t * H + h) * W + w;
+          int64_t flat = flat_index(t, h, w, H, W, P);
+          memcpy(out + (b * S + grid) * row_elems, in + (b * S + flat) * row_elems,
+                 (size_t)row_elems * 2);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block average pooling (NABLA summary, Metodologia item 2, "Downsampling"):*/
+/* xbar[b,hd,i,:] = (sum_{r=0..63} x[b, 64 i + r, hd, :]) / 64, summed in    */
+/* fp32 with r ascending; dividing by 64 is exact.                           */
+/* x is flattened BSHD bf16 [B][S][Hh][D]; xbar is fp32 [B][Hh][Nb][D].      */
+/* Pinned by bilinearity: qbar_i . kbar_j equals the mean of the 64 x 64     */
+/* token-logit tile (checked in fp64).                                       */
+/* ------------------------------------------------------------------------ */
+void oracle_pool(const uint16_t* x, float* xbar, int B, int S, int Hh, int D) {
+  int Nb = S / ORACLE_BLOCK;
+  for (int b = 0; b < B; ++b)
+    for (int hd = 0; hd < Hh; ++hd)
+      for (int i = 0; i < Nb; ++i)
+        for (int d = 0; d < D; ++d) {
+          float acc = 0.0f;
+          for (int r = 0; r < ORACLE_BLOCK; ++r) {
+            int64_t tok = (int64_t)i * ORACLE_BLOCK + r;
+            acc = acc + bf16_bits_to_f32(x[(((int64_t)b * S + tok) * Hh + hd) * D + d]);
+          }
+          xbar[(((int64_t)b * Hh + hd) * Nb + i) * D + d] = acc * (1.0f / 64.0f);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Reduced attention (NABLA summary, "Atencao Reduzida"): one row i of the   */
+/* block-level softmax.  s_ij = fp32(exact dot(qbar_i, kbar_j)) * scale in    */
+/* fp32; m = max_j s_ij; e_j = expf(s_ij - m); Z = sum_j e_j in fp64;         */
+/* p_j = fp32(e_j / Z).                                                      */
+/* Pinned by: scores against the fp64 mean of token logits; sum p = 1 within */
+/* Nb * 2^-24; the all-equal-scores case giving exactly 1/Nb.                */
+/* ------------------------------------------------------------------------ */
+static void block_probs(const float* qbar_i, const float* kbar, int Nb, int D, float scale,
+                        float* p) {
+  float m = -INFINITY;
+  for (int j = 0; j < Nb; ++j) {
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d) dot += (double)qbar_i[d] * (double)kbar[(int64_t)j * D + d];
+    float s = (float)dot * scale;
+    p[j] = s;
+    if (s > m) m = s;
+  }
+  double Z = 0.0;
+  for (int j = 0; j < Nb; ++j) {
+    float e = expf(p[j] - m);
+    p[j] = e;
+    Z += (double)e;
+  }
+  for (int j = 0; j < Nb; ++j) p[j] = (float)((double)p[j] / Z);
+}
+
+typedef struct {
+  float p;
+  int j;
+} pj_t;
+
+/* Ascending by probability, ties by ascending block index. */
+static int cmp_pj(const void* a, const void* b) {
+  const pj_t* x = (const pj_t*)a;
+  const pj_t* y = (const pj_t*)b;
+  if (x->p < y->p) return -1;
+  if (x->p > y->p) return 1;
+  return (x->j > y->j) - (x->j < y->j);
+}
+
+/* ------------------------------------------------------------------------ */
+/* CDF thresholding (NABLA summary, "Limiarizacao CDF"): sort the row's       */
+/* probabilities ascending, take the running sum c_k (fp64) and keep the      */
+/* block at position k iff c_k > 1 - thr.  thr >= 1 keeps every block; the    */
+/* arg-max (last position) is always kept.  cum[j] receives c at block j's    */
+/* position (used to mark blocks whose decision is within the 1e-5 band).    */
+/* Pinned by: an exact-rational top-p (nucleus) restatement on random rows,  */
+/* kept mass >= thr and minimality, and the uniform Nb=16 case.              */
+/* ------------------------------------------------------------------------ */
+static int cdf_keep_row(const float* p, int Nb, float thr, uint8_t* keep, double* cum,
+                        pj_t* scratch) {
+  for (int j = 0; j < Nb; ++j) {
+    scratch[j].p = p[j];
+    scratch[j].j = j;
+  }
+  qsort(scratch, (size_t)Nb, sizeof(pj_t), cmp_pj);
+  double tau = 1.0 - (double)thr;
+  double c = 0.0;
+  for (int k = 0; k < Nb; ++k) {
+    c += (double)scratch[k].p;
+    int j = scratch[k].j;
+    cum[j] = c;
+    keep[j] = (uint8_t)((thr >= 1.0f) || (c > tau) || (k == Nb - 1));
+  }
+  return scratch[Nb - 1].j; /* the arg-max block */
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sliding Tile Attention window in block space (NABLA summary, Metodologia  */
+/* item 3): blocks i=(ti,hi,wi) and j=(tj,hj,wj) interact iff each           */
+/* coordinate differs by at most floor(window/2); the window is centred and  */
+/* truncated at the grid border.  A window size of 0 disables STA.           */
+/* Pinned by the closed-form per-row count prod_axis(min(x+r,n-1) -          */
+/* max(x-r,0) + 1) and its totals per configuration.                         */
+/* ------------------------------------------------------------------------ */
+static int sta_keep(int i, int j, int nbh, int nbw, int st, int sh, int sw) {
+  if (st <= 0 || sh <= 0 || sw <= 0) return 0;
+  int per_t = nbh * nbw;
+  int ti = i / per_t, hi = (i % per_t) / nbw, wi = i % nbw;
+  int tj = j / per_t, hj = (j % per_t) / nbw, wj = j % nbw;
+  return abs(ti - tj) <= st / 2 && abs(hi - hj) <= sh / 2 && abs(wi - wj) <= sw / 2;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Full mask construction for every (b, head, query block) row, producing    */
+/* the block-CSR lists consumed by the attention ("Expansao"):               */
+/*   kv_count[b,hd,i]   number of kept key blocks                            */
+/*   kv_idx[b,hd,i,:]   kept key-block indices ascending (row stride Nb)      */
+/* status (optional, [B,Hh,Nb,Nb] uint8): bit0 = kept, bit1 = band block     */
+/* (decided by the CDF alone and |c - (1-thr)| < band).                       */
+/* probs (optional, [B,Hh,Nb,Nb] fp32): the row probabilities p.             */
+/* qbar/kbar: fp32 [B][Hh][Nb][D].  Rows are independent; OpenMP splits them */
+/* without changing any element's arithmetic.                                */
+/* ------------------------------------------------------------------------ */
+void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, int D, float scale,
+                 float thr, int nbh, int nbw, int sta_t, int sta_h, int sta_w, double band,
+                 int32_t* kv_count, int32_t* kv_idx, uint8_t* status, float* probs) {
+  int64_t rows = (int64_t)B * Hh * Nb;
+#pragma omp parallel
+  {
+    float* p = (float*)malloc(sizeof(float) * (size_t)Nb);
+    uint8_t* keep = (uint8_t*)malloc((size_t)Nb);
+    double* cum = (double*)malloc(sizeof(double) * (size_t)Nb);
+    pj_t* scratch = (pj_t*)malloc(sizeof(pj_t) * (size_t)Nb);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t row = 0; row < rows; ++row) {
+      int64_t bh = row / Nb;
+      int i = (int)(row % Nb);
+      const float* qi = qbar + (bh * Nb + i) * D;
+      const float* kb = kbar + bh * Nb * D;
+      block_probs(qi, kb, Nb, D, scale, p);
+      int argmax = cdf_keep_row(p, Nb, thr, keep, cum, scratch);
+      double tau = 1.0 - (double)thr;
+      int32_t n = 0;
+      for (int j = 0; j < Nb; ++j) {
+        int cdf_kept = keep[j];
+        int sta = sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w);
+        int kept = cdf_kept || sta;
+        if (kept) kv_idx[row * Nb + n++] = j;
+        if (status) {
+          /* A block is "band" only when the CDF comparison alone decides it. */
+          int forced = sta || thr >= 1.0f;
+          int in_band = !forced && j != argmax && fabs(cum[j] - tau) < band;
+          status[row * Nb + j] = (uint8_t)(kept | (in_band << 1));
+        }
+        if (probs) probs[row * Nb + j] = p[j];
+      }
+      kv_count[row] = n;
+    }
+    free(p);
+    free(keep);
+    free(cum);
+    free(scratch);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention restricted to the kept 64 x 64 tiles ("Expansao"), for the      */
+/* query blocks listed in qblocks (all heads).  For query token a of block i */
+/* and every token c of the kept blocks of row (b,hd,i):                     */
+/*   l = (sum_d q_a,d k_c,d) * scale (fp64),  w = exp(l - max_c l),          */
+/*   O_a = sum_c w v_c / sum_c w,   LSE_a = max + log(sum_c w).              */
+/* Dropped tiles enter neither numerator nor normaliser.  A row with no kept */
+/* block gives O = 0 and LSE = -inf.                                         */
+/* out: fp64 [B][nq*64][Hh][D]; lse: fp64 [B][Hh][nq*64] (may be NULL).      */
+/* Pinned by: thr=1 equals dense softmax attention computed independently in */
+/* grid order; V constant -> O constant; Q = 0 -> O = mean of kept V;        */
+/* a row keeping only its own block equals tile-local attention.             */
+/* ------------------------------------------------------------------------ */
+void oracle_attention(const uint16_t* qf, const uint16_t* kf, const uint16_t* vf,
+                      const int32_t* kv_count, const int32_t* kv_idx, int B, int S, int Hh, int D,
+                      double scale, const int32_t* qblocks, int nq, double* out, double* lse) {
+  int Nb = S / ORACLE_BLOCK;
+  int64_t units = (int64_t)B * Hh * nq * ORACLE_BLOCK;
+#pragma omp parallel
+  {
+    double* logit = (double*)malloc(sizeof(double) * (size_t)S);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t u = 0; u < units; ++u) {
+      int r = (int)(u % ORACLE_BLOCK);
+      int64_t t1 = u / ORACLE_BLOCK;
+      int qn = (int)(t1 % nq);
+      int64_t t2 = t1 / nq;
+      int hd = (int)(t2 % Hh);
+      int b = (int)(t2 / Hh);
+      int i = qblocks[qn];
+      int64_t a = (int64_t)i * ORACLE_BLOCK + r;
+      int64_t row = ((int64_t)b * Hh + hd) * Nb + i;
+      int cnt = kv_count[row];
+      const int32_t* lst = kv_idx + row * Nb;
+      const uint16_t* q = qf + (((int64_t)b * S + a) * Hh + hd) * D;
+      int64_t out_row = (int64_t)qn * ORACLE_BLOCK + r;
+      double* o = out + (((int64_t)b * nq * ORACLE_BLOCK + out_row) * Hh + hd) * D;
+      double mx = -INFINITY;
+      int64_t n = 0;
+      for (int e = 0; e < cnt; ++e) {
+        int j = lst[e];
+        for (int c = 0; c < ORACLE_BLOCK; ++c) {
+          int64_t tok = (int64_t)j * ORACLE_BLOCK + c;
+          const uint16_t* k = kf + (((int64_t)b * S + tok) * Hh + hd) * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d) dot += (double)bf16_bits_to_f32(q[d]) * (double)bf16_bits_to_f32(k[d]);
+          double l = dot * scale;
+          logit[n++] = l;
+          if (l > mx) mx = l;
+        }
+      }
+      for (int d = 0; d < D; ++d) acc[d] = 0.0;
+      double den = 0.0;
+      n = 0;
+      for (int e = 0; e < cnt; ++e) {
+        int j = lst[e];
+        for (int c = 0; c < ORACLE_BLOCK; ++c) {
+          int64_t tok = (int64_t)j * ORACLE_BLOCK + c;
+          const uint16_t* v = vf + (((int64_t)b * S + tok) * Hh + hd) * D;
+          double w = exp(logit[n++] - mx);
+          den += w;
+          for (int d = 0; d < D; ++d) acc[d] += w * (double)bf16_bits_to_f32(v[d]);
+        }
+      }
+      for (int d = 0; d < D; ++d) o[d] = cnt > 0 ? acc[d] / den : 0.0;
+      if (lse) lse[((int64_t)b * Hh + hd) * nq * ORACLE_BLOCK + out_row] = cnt > 0 ? mx + log(den) : -INFINITY;
+    }
+    free(logit);
+    free(acc);
+  }
+}
+
+/* Probability row for one (b, head, i): exposed so tests can pin the softmax
+ * and CDF steps on their own. */
+void oracle_block_probs_row(const float* qbar, const float* kbar, int Nb, int D, float scale,
+                            int i, float* p_out) {
+  block_probs(qbar + (int64_t)i * D, kbar, Nb, D, scale, p_out);
+}
+
+/* CDF keep decision for one probability row (see cdf_keep_row). */
+int oracle_cdf_keep(const float* p, int Nb, float thr, uint8_t* keep, double* cum) {
+  pj_t* scratch = (pj_t*)malloc(sizeof(pj_t) * (size_t)Nb);
+  int argmax = cdf_keep_row(p, Nb, thr, keep, cum, scratch);
+  free(scratch);
+  return argmax;
+}
+
+/* STA predicate for one block pair (see sta_keep). */
+int oracle_sta(int i, int j, int nbh, int nbw, int sta_t, int sta_h, int sta_w) {
+  return sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w);
+}
