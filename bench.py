@@ -1,0 +1,401 @@
+"""Benchmark: one NABLA attention layer per step on B200, through the C ABI.
+
+A step is the whole hot path on one batch of synthetic input already
+resident in HBM: fractal flattening of Q, K and V, the adaptive block mask
+(pooling + reduced attention + CDF + compaction), block-sparse attention on
+the kept tiles, and unflattening of the output.  L2 is flushed (a 256 MB
+write) between timed steps, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan13b]
+    python bench.py --impl reference ...   # the CPU oracle, same metric
+
+Prints one JSON line (rank 0).  `value` is kept-tile attention TFLOP/s over
+the whole step (4*64*64*D FLOP per kept 64x64 tile); the per-stage figures
+(ms per layer = mask + attention, mask-build GB/s, attention TFLOP/s) are
+extra keys.  With --gpus N > 1 each rank runs an independent replica of the
+layer (the method runs on one GPU; there is no exchange between ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_flatten_b200 import inputs  # noqa: E402
+
+METRIC = "sparse-attn TFLOP/s on kept tiles & ms/layer; mask-build GB/s (1×B200)"
+CONFIGS = {
+    "tiny": inputs.TINY,
+    "wan13b": inputs.WAN13B,
+    "hunyuan": inputs.HUNYUAN,
+    "long": inputs.LONG,
+}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def config_dict(w: inputs.Workload):
+    return {
+        "workload": w.name,
+        "B": w.B,
+        "heads": w.Hh,
+        "head_dim": w.D,
+        "grid_THW": [w.T, w.H, w.W],
+        "tokens": w.S,
+        "blocks": w.Nb,
+        "thr": w.thr,
+        "sta": list(w.sta) if any(w.sta) else None,
+        "locality_amplitude": w.alpha,
+        "seed": w.seed,
+        "l2": "flushed between timed steps (256 MB write)",
+    }
+
+
+def kept_flops(w, total_kept):
+    return 4.0 * 64 * 64 * w.D * total_kept
+
+
+def mask_bytes(w, total_kept):
+    return 2.0 * w.B * w.S * w.Hh * w.D * 2 + 4.0 * w.B * w.Hh * w.Nb + 4.0 * total_kept
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[4:8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    from block_sparse_attention_flatten_b200 import nabla
+    from block_sparse_attention_flatten_b200 import build as nbuild
+
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = CONFIGS[args.config]
+    q, k, v = inputs.make_qkv(w)
+    stream = torch.cuda.current_stream()
+
+    # device-resident inputs and outputs (allocated once; the library allocates nothing)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    qf, kf, vf = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    of, og = torch.empty_like(qd), torch.empty_like(qd)
+    kv_count = torch.empty((w.B, w.Hh, w.Nb), dtype=torch.int32, device=dev)
+    kv_idx = torch.empty((w.B, w.Hh, w.Nb, w.Nb), dtype=torch.int32, device=dev)
+    prm = nabla.params(w.thr, w.sta)
+    ws = torch.empty(nabla.mask_workspace_bytes(w.B, w.Hh, w.D, w.T, w.H, w.W, prm), dtype=torch.uint8, device=dev)
+    lse = torch.empty((w.B, w.Hh, w.S), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        nabla.flatten(qd, w.T, w.H, w.W, out=qf)
+        nabla.flatten(kd, w.T, w.H, w.W, out=kf)
+        nabla.flatten(vd, w.T, w.H, w.W, out=vf)
+        if ev is not None:
+            ev[1].record(stream)
+        nabla.build_mask(qf, kf, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+        nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=of, lse=lse)
+        if ev is not None:
+            ev[3].record(stream)
+        nabla.unflatten(of, w.T, w.H, w.W, out=og)
+        if ev is not None:
+            ev[4].record(stream)
+
+    launches_per_step = 3 + 2 + 1 + 1
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = nabla.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {nabla.strerror(status)}")
+    total_kept = float(kv_count.double().sum().item())
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 or True else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for s in range(args.steps):
+        flush.zero_()
+        step(events[s])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    status = nabla.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {nabla.strerror(status)}")
+
+    def stage(a, b):
+        return [events[s][a].elapsed_time(events[s][b]) for s in range(args.steps)]
+
+    step_ms = stage(0, 4)
+    flat_ms, mask_ms, attn_ms, unflat_ms = stage(0, 1), stage(1, 2), stage(2, 3), stage(3, 4)
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms_max = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, result out
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        oh = torch.empty(og.shape, dtype=og.dtype, pin_memory=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_ms = []
+        for s in range(args.e2e_steps + 1):
+            flush.zero_()
+            e0.record(stream)
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(og, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if s > 0:
+                e2e_ms.append(e0.elapsed_time(e1))
+        te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        bi = 3 * qd.numel() * qd.element_size()
+        bo = og.numel() * og.element_size()
+        e2e = {"value": world * kept_flops(w, total_kept) * len(e2e_ms) / (float(te.item()) * 1e-3) / 1e12,
+               "unit": "TFLOP/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+               "ms_per_step": float(te.item()) / len(e2e_ms)}
+
+    peak_tf, peak_gbs, peak_kind = load_peaks()
+    attn_avg = statistics.mean(attn_ms)
+    mask_avg = statistics.mean(mask_ms)
+    achieved = kept_flops(w, total_kept) / (attn_avg * 1e-3) / 1e12
+    traffic = load_traffic(args.config)
+    result = {
+        "metric": METRIC,
+        "value": world * kept_flops(w, total_kept) * args.steps / (total_ms_max * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": config_dict(w),
+        "ms_per_layer": mask_avg + attn_avg,
+        "stages_ms": {"flatten_qkv": statistics.mean(flat_ms), "build_mask": mask_avg, "sparse_attn": attn_avg,
+                      "unflatten_o": statistics.mean(unflat_ms)},
+        "attn_tflops_kept": achieved,
+        "mask_build_gbs": mask_bytes(w, total_kept) / (mask_avg * 1e-3) / 1e9,
+        "flatten_gbs": 3 * 2.0 * qd.numel() * 2 / (statistics.mean(flat_ms) * 1e-3) / 1e9,
+        "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
+                     "traffic": traffic},
+        "mask_roofline": {"bound": "hbm", "achieved": mask_bytes(w, total_kept) / (mask_avg * 1e-3) / 1e9,
+                          "peak": peak_gbs, "unit": "GB/s",
+                          "frac": mask_bytes(w, total_kept) / (mask_avg * 1e-3) / 1e9 / peak_gbs},
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    return result, (q, k, v, w, total_kept)
+
+
+def load_traffic(config):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    matches the current kernel; else None."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{config}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh)
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample(w, q, k, v, n_blocks, total_kept=None):
+    """Time the CPU oracle on a bounded sample of the layer: flattening,
+    pooling and the full mask, plus attention on n_blocks seeded query blocks
+    (all heads).  Returns the dict for `cpu_baseline`."""
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    qf = oracle.flatten(q, w.T, w.H, w.W).reshape(q.shape)
+    kf = oracle.flatten(k, w.T, w.H, w.W).reshape(k.shape)
+    vf = oracle.flatten(v, w.T, w.H, w.W).reshape(v.shape)
+    t1 = time.perf_counter()
+    qbar, kbar = oracle.pool(qf), oracle.pool(kf)
+    cnt, idx, _, _ = oracle.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, sta_window=w.sta,
+                                       want_status=False)
+    t2 = time.perf_counter()
+    qblocks = inputs.sample_query_blocks(w.Nb, n_blocks, seed=1234)
+    oracle.attention(qf, kf, vf, cnt, idx, w.scale, qblocks=qblocks)
+    t3 = time.perf_counter()
+    all_kept = float(cnt.astype(np.float64).sum())
+    sample_kept = float(cnt[:, :, qblocks].astype(np.float64).sum())
+    attn_full_s = (t3 - t2) * all_kept / max(sample_kept, 1.0)
+    step_s = (t1 - t0) + (t2 - t1) + attn_full_s
+    return {
+        "value": kept_flops(w, all_kept) / step_s / 1e12,
+        "unit": "TFLOP/s",
+        "cores": oracle.num_threads(),
+        "kind": "oracle",
+        "sample": (f"flatten+pool+full mask ({t2 - t0:.2f} s) and attention on {len(qblocks)} seeded query blocks x "
+                   f"{w.Hh} heads ({t3 - t2:.2f} s), attention extrapolated to all {w.Nb} blocks by kept-tile count"),
+        "ms_per_step_extrapolated": step_s * 1e3,
+    }
+
+
+def run_reference(args):
+    w = CONFIGS[args.config]
+    q, k, v = inputs.make_qkv(w)
+    times, vals = [], []
+    last = None
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        last = oracle_sample(w, q, k, v, args.ref_blocks)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            vals.append(last["value"])
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": statistics.mean(times) * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="wan13b", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-blocks", type=int, default=8, help="query blocks in the CPU-baseline sample")
+    ap.add_argument("--ref-blocks", type=int, default=4, help="query blocks per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        result, (q, k, v, w, total_kept) = run_gpu(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                result["cpu_baseline"] = oracle_sample(w, q, k, v, args.cpu_blocks)
+            else:
+                result["cpu_baseline"] = None
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,15 @@
+"""NABLA adaptive block-sparse attention for one NVIDIA B200 (sm_100a).
+
+The compute path is libnabla.so (hand-written CUDA, C ABI in
+include/nabla.h); this package is its thin Python binding.  PyTorch only
+provides device memory and streams.
+
+    from block_sparse_attention_flatten_b200 import nabla
+    qf = nabla.flatten(q, T, H, W)                       # per tensor, once per sequence
+    kv_count, kv_idx, _ = nabla.build_mask(qf, kf, T, H, W, thr=0.9, sta=(3, 3, 3))
+    of, lse = nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx)
+    o = nabla.unflatten(of, T, H, W)
+"""
+from . import _lib as nabla  # noqa: F401
+
+__all__ = ["nabla"]

@@ -1,0 +1,209 @@
+"""ctypes binding of libnabla.so: argument marshalling only.
+
+Every function here checks that its tensors are CUDA tensors of the right
+dtype and layout, allocates missing outputs with torch (the library itself
+allocates no device memory), and passes raw device pointers, sizes and the
+current CUDA stream to the C entry point of the same name (include/nabla.h).
+There is no CPU fallback: a missing library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnabla.so")
+BLOCK = 64
+
+NABLA_OK = 0
+NABLA_ERR_INVALID = 1
+NABLA_ERR_ALIGN = 2
+NABLA_ERR_CUDA = 3
+NABLA_ERR_DEVICE_TIMEOUT = 4
+NABLA_ERR_DEVICE_BOUNDS = 5
+NABLA_ERR_UNSUPPORTED = 6
+
+EXPORTS = (
+    "nabla_flatten",
+    "nabla_unflatten",
+    "nabla_mask_workspace_bytes",
+    "nabla_build_mask",
+    "nabla_sparse_attn_fwd",
+    "nabla_get_status",
+    "nabla_validate_mask",
+    "nabla_strerror",
+)
+
+
+class NablaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+class NablaParams(ctypes.Structure):
+    _fields_ = [
+        ("P", ctypes.c_int),
+        ("thr", ctypes.c_float),
+        ("sta_t", ctypes.c_int),
+        ("sta_h", ctypes.c_int),
+        ("sta_w", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("flags", ctypes.c_uint),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load libnabla.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libnabla.so is missing at {LIB_PATH}; build it with "
+                               "`python -m block_sparse_attention_flatten_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        pp = ctypes.POINTER(NablaParams)
+        L.nabla_flatten.argtypes = [vp, vp, i, i, i, i, i, i, vp]
+        L.nabla_unflatten.argtypes = [vp, vp, i, i, i, i, i, i, vp]
+        L.nabla_mask_workspace_bytes.argtypes = [i, i, i, i, i, i, pp]
+        L.nabla_mask_workspace_bytes.restype = sz
+        L.nabla_build_mask.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
+        L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
+        L.nabla_get_status.argtypes = [vp]
+        L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
+        L.nabla_strerror.argtypes = [i]
+        L.nabla_strerror.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            if name not in ("nabla_mask_workspace_bytes", "nabla_strerror"):
+                getattr(L, name).restype = i
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().nabla_strerror(int(code)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != NABLA_OK:
+        raise NablaError(rc, where)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def params(thr: float, sta=(0, 0, 0), scale: float = 0.0, P: int = 8) -> NablaParams:
+    return NablaParams(P, float(thr), int(sta[0]), int(sta[1]), int(sta[2]), float(scale), 0)
+
+
+def _permute(fn, x: torch.Tensor, T: int, H: int, W: int, out, stream, P: int):
+    if out is None:
+        out = torch.empty_like(x)
+    B = x.shape[0]
+    row = x[0, 0].numel() if x.dim() > 2 else 1
+    _check(fn(_dev(x, torch.bfloat16, "x"), _dev(out, torch.bfloat16, "out"), B, T, H, W, P, row, _stream(stream)),
+           "nabla_flatten" if fn is lib().nabla_flatten else "nabla_unflatten")
+    return out
+
+
+def flatten(x: torch.Tensor, T: int, H: int, W: int, out=None, stream=None, P: int = 8) -> torch.Tensor:
+    """Fractal flattening of a grid-order [B, S, ...] bf16 CUDA tensor."""
+    return _permute(lib().nabla_flatten, x, T, H, W, out, stream, P)
+
+
+def unflatten(x: torch.Tensor, T: int, H: int, W: int, out=None, stream=None, P: int = 8) -> torch.Tensor:
+    """Inverse of :func:`flatten`."""
+    return _permute(lib().nabla_unflatten, x, T, H, W, out, stream, P)
+
+
+def mask_workspace_bytes(B: int, Hh: int, D: int, T: int, H: int, W: int, prm: NablaParams) -> int:
+    return int(lib().nabla_mask_workspace_bytes(B, Hh, D, T, H, W, ctypes.byref(prm)))
+
+
+def build_mask(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),
+               scale: float = 0.0, kv_count=None, kv_idx=None, workspace=None, stream=None, P: int = 8):
+    """Adaptive block mask from flattened Q, K [B, S, Hh, D] (bf16, CUDA).
+
+    Returns (kv_count int32 [B,Hh,Nb], kv_idx int32 [B,Hh,Nb,Nb], workspace
+    uint8 holding the pooled qbar then kbar, fp32 [B,Hh,Nb,D] each).
+    """
+    B, S, Hh, D = qf.shape
+    Nb = S // BLOCK
+    prm = params(thr, sta, scale, P)
+    dev = qf.device
+    if kv_count is None:
+        kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)
+    if workspace is None:
+        nbytes = mask_workspace_bytes(B, Hh, D, T, H, W, prm)
+        if nbytes == 0:
+            raise NablaError(NABLA_ERR_INVALID, "nabla_mask_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(lib().nabla_build_mask(_dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"), B, Hh, D, T, H, W,
+                                  ctypes.byref(prm), _dev(kv_count, torch.int32, "kv_count"),
+                                  _dev(kv_idx, torch.int32, "kv_idx"), _dev(workspace, torch.uint8, "workspace"),
+                                  _stream(stream)), "nabla_build_mask")
+    return kv_count, kv_idx, workspace
+
+
+def pooled_from_workspace(workspace: torch.Tensor, B: int, Hh: int, Nb: int, D: int):
+    """Views of qbar and kbar inside a mask workspace."""
+    f = workspace.view(torch.float32)
+    n = B * Hh * Nb * D
+    return f[:n].view(B, Hh, Nb, D), f[n:2 * n].view(B, Hh, Nb, D)
+
+
+def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_count: torch.Tensor,
+                    kv_idx: torch.Tensor, scale: float = 0.0, out=None, lse=None, want_lse: bool = True,
+                    stream=None):
+    """Block-sparse attention on the kept tiles; returns (out, lse or None)."""
+    B, S, Hh, D = qf.shape
+    if out is None:
+        out = torch.empty_like(qf)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hh, S), dtype=torch.float32, device=qf.device)
+    lse_p = _dev(lse, torch.float32, "lse") if lse is not None else None
+    _check(lib().nabla_sparse_attn_fwd(_dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"),
+                                       _dev(vf, torch.bfloat16, "vf"), _dev(kv_count, torch.int32, "kv_count"),
+                                       _dev(kv_idx, torch.int32, "kv_idx"), B, S, Hh, D, float(scale),
+                                       _dev(out, torch.bfloat16, "out"), lse_p, _stream(stream)),
+           "nabla_sparse_attn_fwd")
+    return out, lse
+
+
+def get_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word."""
+    return int(lib().nabla_get_status(_stream(stream)))
+
+
+def validate_mask(kv_count: torch.Tensor, kv_idx: torch.Tensor, stream=None) -> int:
+    """Number of malformed block-list rows (synchronises)."""
+    B, Hh, Nb = kv_count.shape
+    bad = torch.zeros(1, dtype=torch.int32, device=kv_count.device)
+    _check(lib().nabla_validate_mask(_dev(kv_count, torch.int32, "kv_count"), _dev(kv_idx, torch.int32, "kv_idx"),
+                                     B, Hh, Nb, _dev(bad, torch.int32, "bad_rows"), _stream(stream)),
+           "nabla_validate_mask")
+    return int(bad.item())
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

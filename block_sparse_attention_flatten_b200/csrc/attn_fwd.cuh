@@ -1,0 +1,394 @@
+// Block-sparse flash-attention forward on the kept 64 x 64 tiles (NABLA
+// technical summary, "Metodologia: NABLA", item 2 "Expansao": only the
+// listed N x N blocks are computed; a dropped block is in neither the
+// numerator nor the softmax normaliser).
+//
+// One CTA owns a query tile of 128 rows = two consecutive 64-token query
+// blocks (2p, 2p+1) of one (batch, head), so every tcgen05.mma runs at the
+// full M = 128.  It walks the ascending union of the two blocks' key-block
+// lists; a key block listed by only one of them is masked for the other
+// half's rows (their probabilities are set to zero and their running max and
+// sum are left alone).
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread t owns query row t = TMEM lane t.  Reads the
+//              64 scores of its row from TMEM, keeps an online max/sum,
+//              rescales its O row in TMEM when the max grew by more than
+//              2^8, writes bf16 probabilities to a 128-byte-swizzled shared
+//              tile, and finally normalises O and stores it with the LSE.
+//   warp 4     TMA producer: Q once, then K_j and V_j of each listed block j
+//              (contiguous 64-token boxes of the flattened layout) into a
+//              ring of kStages stages.
+//   warp 5     MMA issuer (one thread): S = Q K_j^T into one of two TMEM
+//              score buffers (M=128, N=64, K=D), and O += P V_j (M=128, N=D,
+//              K=64) with V read MN-major straight from its TMA tile.
+// Every wait is bounded (see mbar_wait); a timeout raises the CTA's abort
+// flag, records NABLA_ERR_DEVICE_TIMEOUT and all roles drain and exit, with
+// the tensor memory freed.
+#pragma once
+
+#include "common.cuh"
+
+namespace nabla {
+
+constexpr int kAttnThreads = 192;
+constexpr int kStages = 3;
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kChunks = D / 64;          // 64-element (128-byte) column chunks
+  static constexpr int kQBytes = 128 * 128 * kChunks;
+  static constexpr int kKVBytes = 64 * 128 * kChunks;
+  static constexpr int kPBytes = 128 * 128;
+  // offsets from a 1024-byte-aligned base
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kQBytes;
+  static constexpr int kV = kK + kStages * kKVBytes;
+  static constexpr int kP = kV + kStages * kKVBytes;
+  static constexpr int kBars = kP + 2 * kPBytes;
+  // q, k/v full + empty, s full/free, p full, pv done, mma drain
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 * 4 + 1;
+  static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, abort flag, list length
+  static constexpr int kList = kMisc + 16;
+  static size_t bytes(int Nb) {
+    const int words = (Nb + 31) / 32;
+    return 1024 + kList + static_cast<size_t>(Nb) * 4 + 2 * static_cast<size_t>(words) * 4;
+  }
+};
+
+struct AttnArgs {
+  const int32_t* kv_count;  // [B][Hh][Nb]
+  const int32_t* kv_idx;    // [B][Hh][Nb][Nb]
+  __nv_bfloat16* out;       // [B][S][Hh][D]
+  float* lse;               // [B][Hh][S] or null
+  int S, Hh, Nb;
+  float scale_log2;         // scale * log2(e)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using L = AttnSmem<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + kStages;
+  uint64_t* kv_empty = v_full + kStages;
+  uint64_t* s_full = kv_empty + kStages;  // [2]
+  uint64_t* s_free = s_full + 2;          // [2]
+  uint64_t* p_full = s_free + 2;          // [2]
+  uint64_t* pv_done = p_full + 2;         // [2]
+  uint64_t* mma_drain = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
+  int* list_len = reinterpret_cast<int*>(sm + L::kMisc + 8);
+  uint32_t* list = reinterpret_cast<uint32_t*>(sm + L::kList);
+  const int Nb = a.Nb;
+  const int words = (Nb + 31) >> 5;
+  uint32_t* bm0 = list + Nb;
+  uint32_t* bm1 = bm0 + words;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pair = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
+  const int blk0 = 2 * pair, blk1 = 2 * pair + 1;
+  const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
+
+  // ---- set-up: barriers, tensor memory, merged block list
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(k_full + s, 1);
+      mbar_init(v_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(s_free + s, 128);
+      mbar_init(p_full + s, 128);
+      mbar_init(pv_done + s, 1);
+    }
+    mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+  }
+  for (int w = tid; w < 2 * words; w += kAttnThreads) bm0[w] = 0u;
+  __syncthreads();
+  for (int half = 0; half < 2; ++half) {
+    const int blk = half == 0 ? blk0 : blk1;
+    if (blk >= Nb) continue;
+    int cnt = a.kv_count[bh * Nb + blk];
+    if (cnt < 0 || cnt > Nb) {
+      if (tid == 0) report(NABLA_ERR_DEVICE_BOUNDS);
+      cnt = cnt < 0 ? 0 : Nb;
+    }
+    const int32_t* src = a.kv_idx + (bh * Nb + blk) * static_cast<int64_t>(Nb);
+    uint32_t* bm = half == 0 ? bm0 : bm1;
+    for (int e = tid; e < cnt; e += kAttnThreads) {
+      const int j = src[e];
+      if (j < 0 || j >= Nb) {
+        report(NABLA_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      atomicOr(bm + (j >> 5), 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t x0 = w < words ? bm0[w] : 0u, x1 = w < words ? bm1[w] : 0u;
+      uint32_t u = x0 | x1;
+      const int n = __popc(u);
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int pos = base + incl - n;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        const uint32_t m = 1u << bit;
+        list[pos++] = static_cast<uint32_t>(w * 32 + bit) | ((x0 & m) ? (1u << 24) : 0u) | ((x1 & m) ? (1u << 25) : 0u);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) *list_len = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int L_n = *list_len;
+  const uint32_t tS0 = tmem, tS1 = tmem + 64, tO = tmem + 128;
+
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+  const uint32_t sQ = smem_u32(sm + L::kQ), sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV),
+                 sP = smem_u32(sm + L::kP);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && L_n > 0) {
+      mbar_arrive_expect_tx(q_full, L::kQBytes);
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_4d(sm + L::kQ + c * 128 * 128, &tmQ, q_full, c * 64, hd, pair * 128, b);
+      int issued = 0;
+      for (int n = 0; n < L_n; ++n) {
+        const int s = n % kStages;
+        if (n >= kStages && !mbar_wait(kv_empty + s, ((n / kStages) - 1) & 1, abort_flag)) break;
+        const int j = static_cast<int>(list[n] & 0xFFFFFFu);
+        mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(sm + L::kK + s * L::kKVBytes + c * 64 * 128, &tmK, k_full + s, c * 64, hd, j * 64, b);
+        mbar_arrive_expect_tx(v_full + s, L::kKVBytes);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(sm + L::kV + s * L::kKVBytes + c * 64 * 128, &tmV, v_full + s, c * 64, hd, j * 64, b);
+        issued = n + 1;
+      }
+      // Drain: wait for the last issued loads of every stage so no copy is in
+      // flight when the CTA exits, also on the abort path (time-bounded).
+      mbar_wait_drain(q_full, 0);
+      for (int n = (issued > kStages ? issued - kStages : 0); n < issued; ++n) {
+        const int s = n % kStages;
+        mbar_wait_drain(k_full + s, (n / kStages) & 1);
+        mbar_wait_drain(v_full + s, (n / kStages) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------- MMA issue
+    if (lane == 0 && L_n > 0) {
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      tc_fence_after();
+      auto issue_pv = [&](int m) -> bool {
+        const int s = m % kStages;
+        if (!mbar_wait(p_full + (m & 1), (m >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(v_full + s, (m / kStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t pa = sP + (m & 1) * L::kPBytes;
+        const uint32_t vb = sV + s * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, 64 * 128, 1024);
+          umma_bf16_ss(tO, ad, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(pv_done + (m & 1));
+        umma_commit(kv_empty + s);
+        return true;
+      };
+      for (int n = 0; ok && n < L_n; ++n) {
+        const int s = n % kStages;
+        if (!mbar_wait(k_full + s, (n / kStages) & 1, abort_flag)) { ok = false; break; }
+        if (n >= 2 && !mbar_wait(s_free + (n & 1), ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kb = sK + s * L::kKVBytes;
+        const uint32_t tS = (n & 1) ? tS1 : tS0;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t ad = smem_desc_sw128(sQ + c * 128 * 128 + off, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(kb + c * 64 * 128 + off, 16, 1024);
+          umma_bf16_ss(tS, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + (n & 1));
+        if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(L_n - 1);
+      // Every MMA this thread issued must finish before the tensor memory is
+      // freed, also on the abort path (time-bounded).
+      umma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0);
+    }
+  } else {
+    // --------------------------------------------------------------- softmax
+    const int r = tid;  // query row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t flag = 1u << (24 + (r >> 6));
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    unsigned char* prow_base = sm + L::kP + r * 128;
+    for (int n = 0; n < L_n; ++n) {
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + (n & 1), (n >> 1) & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[4][16];
+      const uint32_t tS = ((n & 1) ? tS1 : tS0) + lane_off;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld16(tS + c * 16, sv[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence16(sv[c]);
+      tc_fence_before();
+      mbar_arrive(s_free + (n & 1));
+
+      const bool inc = (list[n] & flag) != 0u;
+      float factor = 1.f;
+      bool need = false;
+      if (inc) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) mx = fmaxf(mx, __uint_as_float(sv[c][e]));
+        mx *= a.scale_log2;
+        if (mx > m_run + 8.f) {  // also true while m_run is -inf
+          factor = ex2_approx(m_run - mx);  // 0 when m_run = -inf
+          need = (n > 0) && (l_run > 0.f);  // an all-zero O row needs no rescale
+          m_run = mx;
+        }
+      }
+      float rowsum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float p0 = 0.f, p1 = 0.f;
+          if (inc) {
+            p0 = ex2_approx(fmaf(__uint_as_float(sv[c][e]), a.scale_log2, -m_run));
+            p1 = ex2_approx(fmaf(__uint_as_float(sv[c][e + 1]), a.scale_log2, -m_run));
+          }
+          rowsum += p0 + p1;
+          pk[c * 8 + e / 2] = pack_bf16x2(p0, p1);
+        }
+      l_run = l_run * factor + rowsum;
+
+      // P buffer (n & 1) is free once PV(n-2) has completed.
+      if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(pv_done + (n & 1), ((n - 2) >> 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        __syncwarp();
+        // O must not be rescaled while PV(n-1) still accumulates into it.
+        if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = need ? factor : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t ov[16];
+          tmem_ld16(tO + lane_off + c * 16, ov);
+          tmem_ld_wait();
+          reg_fence16(ov);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          tmem_st16(tO + lane_off + c * 16, ov);
+        }
+        tmem_st_wait();
+      }
+      unsigned char* prow = prow_base + (n & 1) * L::kPBytes;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full + (n & 1));
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    const int64_t row_g = static_cast<int64_t>(pair) * 128 + r;
+    const bool row_valid = row_g < a.S;
+    if (ok && L_n > 0) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((L_n - 1) & 1), ((L_n - 1) >> 1) & 1, abort_flag));
+    tc_fence_after();
+    __syncwarp();
+    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+    __nv_bfloat16* orow = a.out + ((static_cast<int64_t>(b) * a.S + row_g) * a.Hh + hd) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t ov[16];
+      if (ok && L_n > 0) {
+        tmem_ld16(tO + lane_off + c * 16, ov);
+        tmem_ld_wait();
+        reg_fence16(ov);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ov[e] = 0u;
+      }
+      uint4 w0, w1;
+      w0.x = pack_bf16x2(__uint_as_float(ov[0]) * inv_l, __uint_as_float(ov[1]) * inv_l);
+      w0.y = pack_bf16x2(__uint_as_float(ov[2]) * inv_l, __uint_as_float(ov[3]) * inv_l);
+      w0.z = pack_bf16x2(__uint_as_float(ov[4]) * inv_l, __uint_as_float(ov[5]) * inv_l);
+      w0.w = pack_bf16x2(__uint_as_float(ov[6]) * inv_l, __uint_as_float(ov[7]) * inv_l);
+      w1.x = pack_bf16x2(__uint_as_float(ov[8]) * inv_l, __uint_as_float(ov[9]) * inv_l);
+      w1.y = pack_bf16x2(__uint_as_float(ov[10]) * inv_l, __uint_as_float(ov[11]) * inv_l);
+      w1.z = pack_bf16x2(__uint_as_float(ov[12]) * inv_l, __uint_as_float(ov[13]) * inv_l);
+      w1.w = pack_bf16x2(__uint_as_float(ov[14]) * inv_l, __uint_as_float(ov[15]) * inv_l);
+      if (row_valid) {
+        reinterpret_cast<uint4*>(orow + c * 16)[0] = w0;
+        reinterpret_cast<uint4*>(orow + c * 16)[1] = w1;
+      }
+    }
+    if (row_valid && a.lse != nullptr)
+      a.lse[bh * a.S + row_g] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace nabla

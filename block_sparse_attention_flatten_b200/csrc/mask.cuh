@@ -1,0 +1,285 @@
+// Adaptive block mask (NABLA technical summary, "Metodologia: NABLA", item 2
+// "Construcao de Mascara Adaptativa" and item 3 "Integracao Hibrida com STA").
+//
+// pool_kernel       Downsampling: per 64-token block the fp32 mean of the
+//                   flattened queries and keys (Q and K read once from HBM).
+// mask_rows_kernel  Reduced attention, CDF threshold, STA union and block-CSR
+//                   compaction, R query-block rows per CTA:
+//   1. scores s_ij = (qbar_i . kbar_j) * scale (fp32 FMA chain over d) into
+//      shared memory, one row of Nb scores per query block;
+//   2. softmax per row (one warp per row): max, e = expf(s - max), fp64 sum,
+//      p = fp32(e / Z);
+//   3. the CDF rule "keep where the ascending cumulative mass exceeds 1 - thr"
+//      without a full sort: a mass-weighted radix select over the fp32 bit
+//      patterns of p (4 passes of 8 bits, 256-bin histograms in shared memory)
+//      finds the boundary element (p*, j*) of the ascending (p, j) order;
+//      masses are integers p * 2^56 so every partial sum is exact and
+//      independent of summation order;
+//   4. keep = (p, j) >= (p*, j*)  OR arg-max  OR STA window, compacted with
+//      warp ballots into ascending kv_idx and kv_count.
+#pragma once
+
+#include "common.cuh"
+
+namespace nabla {
+
+// ------------------------------------------------------------------ pooling
+// grid (Nb, B, 2): z = 0 pools Q into qbar, z = 1 pools K into kbar.
+// Thread c handles elements 8c..8c+7 of a token row (Hh*D elements), summing
+// the block's 64 rows in ascending order in fp32.
+__global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                   const __nv_bfloat16* __restrict__ k, float* __restrict__ qbar,
+                                                   float* __restrict__ kbar, int S, int Hh, int D) {
+  const int i = blockIdx.x, b = blockIdx.y;
+  const int Nb = S >> 6;
+  const __nv_bfloat16* x = blockIdx.z == 0 ? q : k;
+  float* out = blockIdx.z == 0 ? qbar : kbar;
+  const int row = Hh * D;
+  const int chunks = row >> 3;
+  const uint4* base = reinterpret_cast<const uint4*>(x + (static_cast<int64_t>(b) * S + static_cast<int64_t>(i) * 64) * row);
+  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 64; r0 += 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(base + static_cast<int64_t>(r0 + u) * chunks + c);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 f = __bfloat1622float2(h2[e]);
+          acc[2 * e] = __fadd_rn(acc[2 * e], f.x);
+          acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], f.y);
+        }
+      }
+    }
+    const int col = c * 8;
+    const int h = col / D, d = col - h * D;
+    float4* o = reinterpret_cast<float4*>(out + ((static_cast<int64_t>(b) * Hh + h) * Nb + i) * D + d);
+    o[0] = make_float4(acc[0] * (1.f / 64.f), acc[1] * (1.f / 64.f), acc[2] * (1.f / 64.f), acc[3] * (1.f / 64.f));
+    o[1] = make_float4(acc[4] * (1.f / 64.f), acc[5] * (1.f / 64.f), acc[6] * (1.f / 64.f), acc[7] * (1.f / 64.f));
+  }
+}
+
+// -------------------------------------------------------------- mask rows
+struct MaskArgs {
+  const float* qbar;  // [B][Hh][Nb][D]
+  const float* kbar;
+  int32_t* kv_count;  // [B][Hh][Nb]
+  int32_t* kv_idx;    // [B][Hh][Nb][Nb]
+  int Hh, Nb, D;
+  int nbh, nbw;       // blocks per frame row / column
+  int sta_rt, sta_rh, sta_rw;  // STA half-widths; sta_on = 0 disables
+  int sta_on;
+  int keep_all;       // thr >= 1
+  float scale;
+  unsigned long long tau_fixed;  // floor((1 - thr) * 2^56)
+};
+
+constexpr int kMaskThreads = 256;
+constexpr int kMaskWarps = kMaskThreads / 32;
+
+__device__ __forceinline__ unsigned long long mass_fixed(float p) {
+  return __double2ull_rz(static_cast<double>(p) * 72057594037927936.0);  // p * 2^56, exact scaling
+}
+
+template <int R>
+__global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int D = a.D, Nb = a.Nb;
+  float* qs = reinterpret_cast<float*>(smem_raw);                       // [R][D]
+  float* rows = qs + R * D;                                             // [R][Nb]
+  unsigned long long* hist_all = reinterpret_cast<unsigned long long*>(rows + static_cast<size_t>(R) * Nb);
+  // hist_all is 8-byte aligned because R*D and R*Nb are even.
+
+  const int i0 = blockIdx.x * R;
+  const int hd = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
+  const float* qb = a.qbar + (bh * Nb + i0) * D;
+  const float* kb = a.kbar + bh * Nb * D;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  for (int e = tid; e < R * D; e += kMaskThreads) {
+    const int r = e / D;
+    qs[e] = (i0 + r < Nb) ? qb[e] : 0.f;
+  }
+  __syncthreads();
+
+  // 1. scores
+  for (int j = tid; j < Nb; j += kMaskThreads) {
+    float acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    const float4* kp = reinterpret_cast<const float4*>(kb + static_cast<int64_t>(j) * D);
+    for (int d4 = 0; d4 < (D >> 2); ++d4) {
+      const float4 kv = __ldg(kp + d4);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float4 qv = reinterpret_cast<const float4*>(qs + r * D)[d4];
+        float t = acc[r];
+        t = fmaf(qv.x, kv.x, t);
+        t = fmaf(qv.y, kv.y, t);
+        t = fmaf(qv.z, kv.z, t);
+        t = fmaf(qv.w, kv.w, t);
+        acc[r] = t;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) rows[static_cast<size_t>(r) * Nb + j] = acc[r] * a.scale;
+  }
+  __syncthreads();
+
+  unsigned long long* hist = hist_all + warp * 256;
+  for (int r = warp; r < R; r += kMaskWarps) {
+    const int i = i0 + r;
+    if (i >= Nb) break;
+    float* row = rows + static_cast<size_t>(r) * Nb;
+
+    // 2. softmax
+    float m = -INFINITY;
+    for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    double z = 0.0;
+    for (int j = lane; j < Nb; j += 32) {
+      const float e = expf(row[j] - m);
+      row[j] = e;
+      z += static_cast<double>(e);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    unsigned long long best = 0;  // (bits(p) << 32) | j, max = arg-max with ties to the larger j
+    unsigned long long total = 0;
+    for (int j = lane; j < Nb; j += 32) {
+      const float p = static_cast<float>(static_cast<double>(row[j]) / z);
+      row[j] = p;
+      const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(p)) << 32) | static_cast<unsigned>(j);
+      best = key > best ? key : best;
+      total += mass_fixed(p);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
+      best = ob > best ? ob : best;
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+    }
+    const int argmax = static_cast<int>(best & 0xffffffffu);
+
+    // 3. CDF boundary by mass-weighted radix select
+    unsigned long long kstar = ~0ull;  // keep (p,j) with key >= kstar
+    if (!a.keep_all && total > a.tau_fixed) {
+      uint32_t prefix = 0, pmask = 0;
+      unsigned long long below = 0;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0ull;
+        __syncwarp();
+        for (int j = lane; j < Nb; j += 32) {
+          const float p = row[j];
+          const uint32_t u = __float_as_uint(p);
+          if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], mass_fixed(p));
+        }
+        __syncwarp();
+        unsigned long long loc[8], lsum = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          loc[t] = hist[lane * 8 + t];
+          lsum += loc[t];
+        }
+        unsigned long long incl = lsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        unsigned long long cum = below + (incl - lsum);
+        int found = -1;
+        unsigned long long before = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (found < 0 && cum + loc[t] > a.tau_fixed) {
+            found = lane * 8 + t;
+            before = cum;
+          }
+          cum += loc[t];
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
+        const int win = __ffs(ball) - 1;  // ball != 0: the range's cumulative mass exceeds tau
+        const int bin = __shfl_sync(0xffffffffu, found, win);
+        below = __shfl_sync(0xffffffffu, before, win);
+        prefix |= static_cast<uint32_t>(bin) << shift;
+        pmask |= 255u << shift;
+        __syncwarp();
+      }
+      // Ties at p*: the boundary is the m-th smallest index among them.
+      const unsigned long long wstar = mass_fixed(__uint_as_float(prefix));
+      const unsigned long long need = (a.tau_fixed - below) / wstar + 1ull;
+      unsigned long long seen = 0;
+      int jstar = Nb;
+      for (int base = 0; base < Nb; base += 32) {
+        const int j = base + lane;
+        const bool hit = j < Nb && __float_as_uint(row[j]) == prefix;
+        const unsigned bal = __ballot_sync(0xffffffffu, hit);
+        const unsigned c = __popc(bal);
+        if (seen + c >= need) {
+          unsigned bb = bal;
+          for (unsigned long long s = seen + 1; s < need; ++s) bb &= bb - 1;  // drop lower hits
+          jstar = base + __ffs(bb) - 1;
+          break;
+        }
+        seen += c;
+      }
+      kstar = (static_cast<unsigned long long>(prefix) << 32) | static_cast<unsigned>(jstar);
+    }
+
+    // 4. union with the STA window and compaction
+    const int per_t = a.nbh * a.nbw;
+    const int ti = i / per_t, hi = (i % per_t) / a.nbw, wi = i % a.nbw;
+    int32_t* out = a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb);
+    int count = 0;
+    for (int base = 0; base < Nb; base += 32) {
+      const int j = base + lane;
+      bool keep = false;
+      if (j < Nb) {
+        const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(row[j])) << 32) | static_cast<unsigned>(j);
+        keep = a.keep_all || key >= kstar || j == argmax;
+        if (!keep && a.sta_on) {
+          const int tj = j / per_t, hj = (j % per_t) / a.nbw, wj = j % a.nbw;
+          keep = abs(ti - tj) <= a.sta_rt && abs(hi - hj) <= a.sta_rh && abs(wi - wj) <= a.sta_rw;
+        }
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[count + __popc(bal & ((1u << lane) - 1u))] = j;
+      count += __popc(bal);
+    }
+    if (lane == 0) a.kv_count[bh * Nb + i] = count;
+  }
+}
+
+// --------------------------------------------------------- mask validation
+__global__ void validate_mask_kernel(const int32_t* __restrict__ kv_count, const int32_t* __restrict__ kv_idx,
+                                     int64_t rows, int Nb, int32_t* bad_rows) {
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  const int c = kv_count[r];
+  bool bad = c < 1 || c > Nb;
+  if (!bad) {
+    const int32_t* l = kv_idx + r * Nb;
+    int prev = -1;
+    for (int e = 0; e < c; ++e) {
+      const int j = l[e];
+      if (j <= prev || j >= Nb) {
+        bad = true;
+        break;
+      }
+      prev = j;
+    }
+  }
+  if (bad) atomicAdd(bad_rows, 1);
+}
+
+}  // namespace nabla

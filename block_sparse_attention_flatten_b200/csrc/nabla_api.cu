@@ -1,0 +1,316 @@
+// C ABI of libnabla.so (declared in include/nabla.h): argument checks, TMA
+// descriptor set-up and kernel launches.  Everything here is host code; the
+// kernels live in the .cuh files included below (one translation unit, so
+// the device status word is a single symbol).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_fwd.cuh"
+#include "common.cuh"
+#include "flatten.cuh"
+#include "mask.cuh"
+#include "nabla.h"
+
+namespace nabla {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  bool ready = false;
+  bool sm100 = false;
+  int sms = 0;
+  int max_smem_optin = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+// Per-device facts, looked up once.
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NABLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return NABLA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return NABLA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NABLA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    d.sm100 = (major == 10 && minor == 0);
+    d.ready = true;
+  }
+  *out = d;
+  return NABLA_OK;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NABLA_OK : NABLA_ERR_CUDA;
+}
+
+// ----------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// View of a BSHD bf16 tensor as 4-D (D, Hh, S, B), box (64, 1, rows, 1),
+// 128-byte swizzle: one box is `rows` tokens x 64 head-dim elements.
+bool make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int Hh, int D, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hh), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hh) * D * 2,
+                                 static_cast<cuuint64_t>(S) * Hh * D * 2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int check_grid(int B, int T, int H, int W, int P) {
+  if (B <= 0 || T <= 0 || H <= 0 || W <= 0) return NABLA_ERR_INVALID;
+  if (P != 8 || H % P != 0 || W % P != 0) return NABLA_ERR_INVALID;
+  const int64_t S = static_cast<int64_t>(T) * H * W;
+  if (S > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
+  return NABLA_OK;
+}
+
+template <bool kInverse>
+int permute(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems, cudaStream_t stream) {
+  int rc = check_grid(B, T, H, W, P);
+  if (rc != NABLA_OK) return rc;
+  if (row_elems <= 0 || row_elems % 8 != 0) return NABLA_ERR_INVALID;
+  if (in == nullptr || out == nullptr || in == out) return NABLA_ERR_INVALID;
+  if (!aligned16(in) || !aligned16(out)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != NABLA_OK) return rc;
+  const int64_t S = static_cast<int64_t>(T) * H * W;
+  const int64_t rows = S * B;
+  const int chunks = row_elems / 8;
+  const int64_t blocks_needed = (rows + 7) / 8;
+  const int grid = static_cast<int>(blocks_needed < int64_t{di.sms} * 16 ? blocks_needed : int64_t{di.sms} * 16);
+  permute_rows_kernel<kInverse><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out),
+                                                           rows, S, GridShape{T, H, W, P}, chunks);
+  return launch_status();
+}
+
+size_t mask_smem_bytes(int R, int D, int Nb) {
+  return static_cast<size_t>(R) * D * 4 + static_cast<size_t>(R) * Nb * 4 + kMaskWarps * 256 * 8;
+}
+
+template <int R>
+int launch_mask(const MaskArgs& a, int B, const DeviceInfo& di, cudaStream_t stream) {
+  const size_t smem = mask_smem_bytes(R, a.D, a.Nb);
+  if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
+  if (cudaFuncSetAttribute(mask_rows_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return NABLA_ERR_CUDA;
+  dim3 grid((a.Nb + R - 1) / R, a.Hh, B);
+  mask_rows_kernel<R><<<grid, kMaskThreads, smem, stream>>>(a);
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace nabla
+
+using namespace nabla;
+
+extern "C" {
+
+int nabla_flatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
+                  nabla_stream_t stream) {
+  return permute<false>(in, out, B, T, H, W, P, row_elems, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int nabla_unflatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
+                    nabla_stream_t stream) {
+  return permute<true>(in, out, B, T, H, W, P, row_elems, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W, const nabla_params* params) {
+  const int P = params ? params->P : 8;
+  if (check_grid(B, T, H, W, P) != NABLA_OK || Hh <= 0 || (D != 64 && D != 128)) return 0;
+  const size_t Nb = static_cast<size_t>(T) * H * W / 64;
+  return 2 * static_cast<size_t>(B) * Hh * Nb * D * sizeof(float);
+}
+
+int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
+                     const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, void* workspace,
+                     nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (params == nullptr) return NABLA_ERR_INVALID;
+  const nabla_params& p = *params;
+  int rc = check_grid(B, T, H, W, p.P);
+  if (rc != NABLA_OK) return rc;
+  if (Hh <= 0 || (D != 64 && D != 128) || p.flags != 0u) return NABLA_ERR_INVALID;
+  if (!(p.thr >= 0.f && p.thr <= 1.f)) return NABLA_ERR_INVALID;
+  if (!(p.scale >= 0.f) || std::isinf(p.scale)) return NABLA_ERR_INVALID;
+  const bool sta_on = p.sta_t != 0 || p.sta_h != 0 || p.sta_w != 0;
+  if (sta_on && (p.sta_t <= 0 || p.sta_h <= 0 || p.sta_w <= 0 || p.sta_t % 2 == 0 || p.sta_h % 2 == 0 ||
+                 p.sta_w % 2 == 0))
+    return NABLA_ERR_INVALID;
+  if (qf == nullptr || kf == nullptr || kv_count == nullptr || kv_idx == nullptr || workspace == nullptr)
+    return NABLA_ERR_INVALID;
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(workspace) || !aligned16(kv_count) || !aligned16(kv_idx))
+    return NABLA_ERR_ALIGN;
+  if (static_cast<int64_t>(Hh) * D > 3072 * 4) return NABLA_ERR_INVALID;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != NABLA_OK) return rc;
+  const int S = T * H * W;
+  const int Nb = S / 64;
+  float* qbar = static_cast<float*>(workspace);
+  float* kbar = qbar + static_cast<size_t>(B) * Hh * Nb * D;
+
+  const int pool_threads = (Hh * D / 8) < 384 ? (Hh * D / 8) : 384;
+  pool_kernel<<<dim3(Nb, B, 2), pool_threads, 0, stream>>>(static_cast<const __nv_bfloat16*>(qf),
+                                                            static_cast<const __nv_bfloat16*>(kf), qbar, kbar, S, Hh, D);
+  if ((rc = launch_status()) != NABLA_OK) return rc;
+
+  MaskArgs a;
+  a.qbar = qbar;
+  a.kbar = kbar;
+  a.kv_count = kv_count;
+  a.kv_idx = kv_idx;
+  a.Hh = Hh;
+  a.Nb = Nb;
+  a.D = D;
+  a.nbh = H / p.P;
+  a.nbw = W / p.P;
+  a.sta_on = sta_on ? 1 : 0;
+  a.sta_rt = p.sta_t / 2;
+  a.sta_rh = p.sta_h / 2;
+  a.sta_rw = p.sta_w / 2;
+  a.keep_all = p.thr >= 1.f ? 1 : 0;
+  a.scale = p.scale > 0.f ? p.scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  // (1 - thr) is exact in double; scaling by 2^56 is exact; floor keeps the
+  // comparison "cumulative mass > 1 - thr" exact for integer masses.
+  a.tau_fixed = static_cast<unsigned long long>(std::floor((1.0 - static_cast<double>(p.thr)) * 72057594037927936.0));
+
+  // Rows per CTA: as many as fit ~128 KB of score rows, at most 32.
+  const size_t per_row = static_cast<size_t>(Nb) * 4;
+  const size_t fit = (128u * 1024u) / per_row;
+  if (fit >= 32) return launch_mask<32>(a, B, di, stream);
+  if (fit >= 16) return launch_mask<16>(a, B, di, stream);
+  if (fit >= 8) return launch_mask<8>(a, B, di, stream);
+  if (fit >= 4) return launch_mask<4>(a, B, di, stream);
+  if (mask_smem_bytes(2, D, Nb) <= static_cast<size_t>(di.max_smem_optin)) return launch_mask<2>(a, B, di, stream);
+  return NABLA_ERR_INVALID;
+}
+
+int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+                          const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
+                          nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
+  if (static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
+  if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
+  if (qf == nullptr || kf == nullptr || vf == nullptr || kv_count == nullptr || kv_idx == nullptr || out == nullptr)
+    return NABLA_ERR_INVALID;
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(vf) || !aligned16(out) || !aligned16(kv_idx) ||
+      !aligned16(kv_count))
+    return NABLA_ERR_ALIGN;
+  if (lse != nullptr && !aligned16(lse)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc != NABLA_OK) return rc;
+  if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
+  const int Nb = S / 64;
+  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+
+  CUtensorMap tq, tk, tv;
+  if (!make_bshd_map(&tq, qf, B, S, Hh, D, 128) || !make_bshd_map(&tk, kf, B, S, Hh, D, 64) ||
+      !make_bshd_map(&tv, vf, B, S, Hh, D, 64))
+    return NABLA_ERR_CUDA;
+  AttnArgs a;
+  a.kv_count = kv_count;
+  a.kv_idx = kv_idx;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.S = S;
+  a.Hh = Hh;
+  a.Nb = Nb;
+  a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
+  const dim3 grid((Nb + 1) / 2, Hh, B);
+  if (D == 128) {
+    const size_t smem = AttnSmem<128>::bytes(Nb);
+    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
+    if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    attn_fwd_kernel<128><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    const size_t smem = AttnSmem<64>::bytes(Nb);
+    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
+    if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    attn_fwd_kernel<64><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
+  }
+  return launch_status();
+}
+
+int nabla_get_status(nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return NABLA_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return NABLA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return NABLA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return NABLA_ERR_CUDA;
+  return v;
+}
+
+int nabla_validate_mask(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb, int32_t* bad_rows,
+                        nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B <= 0 || Hh <= 0 || Nb <= 0 || kv_count == nullptr || kv_idx == nullptr || bad_rows == nullptr)
+    return NABLA_ERR_INVALID;
+  if (cudaMemsetAsync(bad_rows, 0, sizeof(int32_t), stream) != cudaSuccess) return NABLA_ERR_CUDA;
+  const int64_t rows = static_cast<int64_t>(B) * Hh * Nb;
+  validate_mask_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(kv_count, kv_idx, rows, Nb,
+                                                                                       bad_rows);
+  return launch_status();
+}
+
+const char* nabla_strerror(int code) {
+  switch (code) {
+    case NABLA_OK: return "ok";
+    case NABLA_ERR_INVALID: return "invalid argument (shape or parameter)";
+    case NABLA_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    case NABLA_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
+    case NABLA_ERR_DEVICE_TIMEOUT: return "device wait exceeded its time limit";
+    case NABLA_ERR_DEVICE_BOUNDS: return "block index or count out of range";
+    case NABLA_ERR_UNSUPPORTED: return "device is not an sm_100 GPU";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+/*
+ * nabla.h -- C ABI of libnabla.so: NABLA adaptive block-sparse attention on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * The method (page "Resumo Tecnico: NABLA - Atencao de Bloco Adaptativa de
+ * Vizinhanca para Geracao de Video Eficiente", gist.science paper 2507.13546,
+ * section "Metodologia: NABLA") has three stages, each an entry point here:
+ *   1. fractal flattening of the T x H x W token grid   -> nabla_flatten
+ *   2. adaptive block mask (pool, reduced attention, CDF
+ *      threshold, optional STA union)                   -> nabla_build_mask
+ *   3. attention on the kept 64 x 64 tiles               -> nabla_sparse_attn_fwd
+ *
+ * Conventions shared by every call
+ *   - Tensors are bf16 in BSHD layout [B][S][Hh][D] (D contiguous), S = T*H*W
+ *     tokens, Hh heads, head dimension D in {64, 128}.  A block is P*P = 64
+ *     consecutive tokens of the flattened order (P = 8); Nb = S / 64.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, who
+ *     allocates it (the library allocates no device memory) and keeps it alive
+ *     until the stream has executed the call.  Inputs and outputs never alias.
+ *   - Calls are asynchronous on the given stream (0 = legacy default stream)
+ *     and never synchronise, except nabla_get_status.
+ *   - Return value: NABLA_OK, or an error code; on error nothing is launched.
+ *     Device-side faults of the data (an out-of-range block index, a wait that
+ *     ran out of time) are recorded in a per-device status word that
+ *     nabla_get_status reads and clears.
+ */
+#ifndef NABLA_H_
+#define NABLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nabla_stream_t; /* same object as cudaStream_t */
+
+enum {
+  NABLA_OK = 0,
+  NABLA_ERR_INVALID = 1,        /* bad shape or parameter */
+  NABLA_ERR_ALIGN = 2,          /* pointer not 16-byte aligned */
+  NABLA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+  NABLA_ERR_DEVICE_TIMEOUT = 4, /* (device status) a bounded wait expired */
+  NABLA_ERR_DEVICE_BOUNDS = 5,  /* (device status) a block index or count was out of range */
+  NABLA_ERR_UNSUPPORTED = 6     /* no sm_100 device */
+};
+
+/* Mask parameters.
+ *   P      patch side; must be 8 (64-token blocks).
+ *   thr    CDF threshold in [0, 1]: per row, blocks sorted by probability
+ *          ascending are kept where the cumulative mass exceeds 1 - thr
+ *          ("Limiarizacao CDF").  thr = 1 keeps every block; the row's
+ *          arg-max block is always kept.
+ *   sta_t, sta_h, sta_w
+ *          Sliding-Tile window in blocks (frames, patch rows, patch columns),
+ *          odd sizes; all three 0 disables the STA union ("Integracao Hibrida
+ *          com STA", M = M_nabla OR M_STA).  The window is centred on the query
+ *          block and truncated at the grid border.
+ *   scale  score scale; 0 selects 1/sqrt(D).
+ *   flags  reserved, must be 0. */
+typedef struct {
+  int P;
+  float thr;
+  int sta_t, sta_h, sta_w;
+  float scale;
+  unsigned flags;
+} nabla_params;
+
+/* Fractal flattening ("Metodologia: NABLA", item 1, "Reordenacao de Tokens"):
+ * out[b, f(t,h,w), :] = in[b, (t*H + h)*W + w, :] with
+ *   f = t*H*W + ((h/P)*(W/P) + w/P)*P*P + (h%P)*P + (w%P),
+ * so each P x P spatial patch of a frame becomes P*P contiguous rows and the
+ * frames stay in order.
+ *   in, out     device bf16 [B][T*H*W][row_elems]; row_elems*2 bytes per row
+ *               (e.g. Hh*D), a multiple of 16 bytes; both 16-byte aligned.
+ * Errors: NABLA_ERR_INVALID unless P == 8, H % P == 0, W % P == 0, all sizes
+ * positive and row_elems % 8 == 0; NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
+int nabla_flatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
+                  nabla_stream_t stream);
+
+/* Inverse of nabla_flatten (same arguments and rules): takes flattened rows
+ * back to grid order. */
+int nabla_unflatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
+                    nabla_stream_t stream);
+
+/* Bytes of device workspace nabla_build_mask needs: the pooled queries and
+ * keys, fp32 [B][Hh][Nb][D] each (queries first).  Returns 0 for invalid
+ * sizes. */
+size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W,
+                                  const nabla_params* params);
+
+/* Adaptive block mask ("Metodologia: NABLA", item 2, and item 3):
+ *   1. pooling: qbar[b,hd,i,:] = mean of the 64 flattened query rows of block
+ *      i (fp32 accumulation, rows in ascending order), same for keys
+ *      ("Downsampling");
+ *   2. reduced attention: s_ij = (qbar_i . kbar_j) * scale in fp32,
+ *      p_i = softmax_j(s_i) ("Atencao Reduzida");
+ *   3. CDF threshold as described for nabla_params.thr ("Limiarizacao CDF");
+ *   4. optional STA union, then compaction into block lists ("Expansao").
+ *   qf, kf      device bf16 [B][S][Hh][D], flattened order.
+ *   kv_count    device int32 [B][Hh][Nb]: kept key blocks per query block.
+ *   kv_idx      device int32 [B][Hh][Nb][Nb]: row (b,hd,i) holds its kept key
+ *               blocks ascending in entries [0, kv_count); later entries are
+ *               not written.
+ *   workspace   device buffer of nabla_mask_workspace_bytes() bytes, 16-byte
+ *               aligned; on return it holds qbar then kbar.
+ * Errors: NABLA_ERR_INVALID (shape, D not 64/128, thr outside [0,1], even or
+ * negative STA sizes, flags != 0); NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
+int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
+                     const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
+                     void* workspace, nabla_stream_t stream);
+
+/* Block-sparse attention forward on the kept tiles ("Expansao": only the
+ * listed N x N blocks are computed; a dropped block is in neither the
+ * numerator nor the softmax normaliser).  For query block i of (b, hd):
+ *   O_i = softmax over the tokens of kv_idx[b,hd,i,0..kv_count) of
+ *         (Q_i K^T * scale), applied to V;   LSE = log of the normaliser.
+ *   qf, kf, vf  device bf16 [B][S][Hh][D], flattened order, 16-byte aligned;
+ *               S a multiple of 64.
+ *   kv_count, kv_idx   block lists as written by nabla_build_mask (entries
+ *               must be ascending and < Nb; a bad entry is skipped and
+ *               recorded as NABLA_ERR_DEVICE_BOUNDS).
+ *   scale       0 selects 1/sqrt(D).
+ *   out         device bf16 [B][S][Hh][D], flattened order.
+ *   lse         device fp32 [B][Hh][S] (natural log) or NULL.
+ * A query block with kv_count == 0 gets O = 0 and LSE = -inf.
+ * Errors: NABLA_ERR_INVALID (D not 64/128, S % 64 != 0, sizes); NABLA_ERR_ALIGN;
+ * NABLA_ERR_CUDA; NABLA_ERR_UNSUPPORTED when the device is not sm_100. */
+int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+                          const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out,
+                          float* lse, nabla_stream_t stream);
+
+/* Synchronises the stream, then returns and clears the current device's
+ * status word (NABLA_OK, NABLA_ERR_DEVICE_TIMEOUT or NABLA_ERR_DEVICE_BOUNDS),
+ * or NABLA_ERR_CUDA if the synchronisation itself failed. */
+int nabla_get_status(nabla_stream_t stream);
+
+/* Debug check of block lists on the device: every row must have
+ * 1 <= count <= Nb and strictly ascending entries in [0, Nb).  Writes the
+ * number of bad rows to *bad_rows (device int32, zeroed by the call).
+ * Asynchronous like the others. */
+int nabla_validate_mask(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb,
+                        int32_t* bad_rows, nabla_stream_t stream);
+
+/* Static description of an error code. */
+const char* nabla_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NABLA_H_ */

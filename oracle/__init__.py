@@ -160,6 +160,9 @@ def build_mask(qbar: np.ndarray, kbar: np.ndarray, thr: float, scale: float, nbh
 def attention(qf, kf, vf, kv_count: np.ndarray, kv_idx: np.ndarray, scale: float, qblocks=None):
     """Masked attention (fp64) for the listed query blocks (all heads).
 
+    kv_count/kv_idx are the full lists [B,Hh,Nb] / [B,Hh,Nb,Nb] or, when
+    qblocks is given, may already be restricted to those blocks
+    ([B,Hh,nq] / [B,Hh,nq,Nb]).
     Returns (out fp64 [B, nq*64, Hh, D], lse fp64 [B, Hh, nq*64]).
     """
     qf, kf, vf = _bits(qf), _bits(kf), _bits(vf)
@@ -169,9 +172,14 @@ def attention(qf, kf, vf, kv_count: np.ndarray, kv_idx: np.ndarray, scale: float
         qblocks = np.arange(Nb, dtype=np.int32)
     qblocks = np.ascontiguousarray(qblocks, dtype=np.int32)
     nq = qblocks.shape[0]
+    kv_count = np.asarray(kv_count)
+    kv_idx = np.asarray(kv_idx)
+    if kv_count.shape[-1] != nq:
+        kv_count = kv_count[:, :, qblocks]
+        kv_idx = kv_idx[:, :, qblocks]
     kv_count = np.ascontiguousarray(kv_count, dtype=np.int32)
     kv_idx = np.ascontiguousarray(kv_idx, dtype=np.int32)
-    assert kv_idx.shape == (B, Hh, Nb, Nb)
+    assert kv_count.shape == (B, Hh, nq) and kv_idx.shape == (B, Hh, nq, Nb)
     out = np.zeros((B, nq * BLOCK, Hh, D), dtype=np.float64)
     lse = np.zeros((B, Hh, nq * BLOCK), dtype=np.float64)
     _load().oracle_attention(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(kv_count), _ptr(kv_idx), B, S, Hh, D,

@@ -264,6 +264,8 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
 /*   O_a = sum_c w v_c / sum_c w,   LSE_a = max + log(sum_c w).              */
 /* Dropped tiles enter neither numerator nor normaliser.  A row with no kept */
 /* block gives O = 0 and LSE = -inf.                                         */
+/* kv_count: int32 [B][Hh][nq] and kv_idx: int32 [B][Hh][nq][Nb] hold the    */
+/* lists of the listed query blocks only, in qblocks order.                  */
 /* out: fp64 [B][nq*64][Hh][D]; lse: fp64 [B][Hh][nq*64] (may be NULL).      */
 /* Pinned by: thr=1 equals dense softmax attention computed independently in */
 /* grid order; V constant -> O constant; Q = 0 -> O = mean of kept V;        */
@@ -288,7 +290,7 @@ void oracle_attention(const uint16_t* qf, const uint16_t* kf, const uint16_t* vf
       int b = (int)(t2 / Hh);
       int i = qblocks[qn];
       int64_t a = (int64_t)i * ORACLE_BLOCK + r;
-      int64_t row = ((int64_t)b * Hh + hd) * Nb + i;
+      int64_t row = ((int64_t)b * Hh + hd) * nq + qn;
       int cnt = kv_count[row];
       const int32_t* lst = kv_idx + row * Nb;
       const uint16_t* q = qf + (((int64_t)b * S + a) * Hh + hd) * D;

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load on a machine without a GPU, export every function
+include/nabla.h declares, and reject bad arguments before touching the
+device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_flatten_b200 import build as nbuild
+from block_sparse_attention_flatten_b200 import nabla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nbuild.build()
+    return nabla.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "nabla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nabla_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for name in nabla.EXPORTS:
+        assert name in fns
+    assert set(fns) == set(nabla.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_strerror_covers_codes(lib):
+    for code in range(0, 7):
+        assert nabla.strerror(code) != "unknown error"
+    assert nabla.strerror(99) == "unknown error"
+
+
+def test_params_struct_layout_matches_header():
+    assert ctypes.sizeof(nabla.NablaParams) == 28
+    assert nabla.NablaParams.thr.offset == 4 and nabla.NablaParams.flags.offset == 24
+
+
+def test_workspace_bytes(lib):
+    prm = nabla.params(0.9)
+    assert nabla.mask_workspace_bytes(1, 12, 128, 16, 48, 80, prm) == 2 * 12 * 960 * 128 * 4
+    assert nabla.mask_workspace_bytes(1, 2, 96, 4, 16, 16, prm) == 0  # D not supported
+    assert nabla.mask_workspace_bytes(1, 2, 64, 4, 12, 16, prm) == 0  # H not a multiple of 8
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    L = lib
+    s = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x1000)
+    # P must be 8; H, W multiples of P; rows a multiple of 16 bytes
+    assert L.nabla_flatten(fake, ctypes.c_void_p(0x2000), 1, 4, 16, 16, 7, 128, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_flatten(fake, ctypes.c_void_p(0x2000), 1, 4, 12, 16, 8, 128, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_flatten(fake, ctypes.c_void_p(0x2000), 1, 4, 16, 16, 8, 12, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_flatten(fake, fake, 1, 4, 16, 16, 8, 128, s) == nabla.NABLA_ERR_INVALID  # aliasing
+    assert L.nabla_flatten(ctypes.c_void_p(0x1001), ctypes.c_void_p(0x2000), 1, 4, 16, 16, 8, 128,
+                           s) == nabla.NABLA_ERR_ALIGN
+    prm = nabla.params(1.5)
+    assert L.nabla_build_mask(fake, fake, 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake, fake, fake,
+                              s) == nabla.NABLA_ERR_INVALID
+    prm = nabla.params(0.9, sta=(2, 3, 3))
+    assert L.nabla_build_mask(fake, fake, 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake, fake, fake,
+                              s) == nabla.NABLA_ERR_INVALID
+    prm = nabla.params(0.9)
+    assert L.nabla_build_mask(fake, fake, 1, 2, 80, 4, 16, 16, ctypes.byref(prm), fake, fake, fake,
+                              s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask(ctypes.c_void_p(0x1008), fake, 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake, fake,
+                              fake, s) == nabla.NABLA_ERR_ALIGN
+    assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 100, 2, 64, ctypes.c_float(0.0), fake, None,
+                                   s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 128, 2, 48, ctypes.c_float(0.0), fake, None,
+                                   s) == nabla.NABLA_ERR_INVALID
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 64, 8, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        nabla.flatten(x, 1, 8, 8)
