@@ -10,18 +10,22 @@
 // half's rows (their probabilities are set to zero and their running max and
 // sum are left alone).
 //
-// Warp roles (192 threads):
+// Warp roles (192 threads, two CTAs per SM):
 //   warps 0-3  softmax: thread t owns query row t = TMEM lane t.  Reads the
 //              64 scores of its row from TMEM, keeps an online max/sum,
 //              rescales its O row in TMEM when the max grew by more than
-//              2^8, writes bf16 probabilities to a 128-byte-swizzled shared
-//              tile, and finally normalises O and stores it with the LSE.
+//              2^8, writes the bf16 probabilities back into the first 32
+//              columns of the same TMEM score buffer, and finally normalises
+//              O and stores it with the LSE.
 //   warp 4     TMA producer: Q once, then K_j and V_j of each listed block j
 //              (contiguous 64-token boxes of the flattened layout) into a
 //              ring of kStages stages.
 //   warp 5     MMA issuer (one thread): S = Q K_j^T into one of two TMEM
-//              score buffers (M=128, N=64, K=D), and O += P V_j (M=128, N=D,
-//              K=64) with V read MN-major straight from its TMA tile.
+//              score buffers (M=128, N=64, K=D), and O += P V_j with P read
+//              from tensor memory and V MN-major straight from its TMA tile
+//              (M=128, N=D, K=64).
+// Tensor memory per CTA: S0 | S1 (64 columns each, P aliases their first 32)
+// | O (D columns) = 256 columns, so two CTAs share an SM's 512 columns.
 // Every wait is bounded (see mbar_wait); a timeout raises the CTA's abort
 // flag, records NABLA_ERR_DEVICE_TIMEOUT and all roles drain and exit, with
 // the tensor memory freed.
@@ -32,27 +36,27 @@
 namespace nabla {
 
 constexpr int kAttnThreads = 192;
-constexpr int kStages = 3;
+constexpr int kMaxListBlocks = 16383;  // list entries hold a 14-bit block index
 
 template <int D>
 struct AttnSmem {
   static constexpr int kChunks = D / 64;          // 64-element (128-byte) column chunks
+  static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr int kQBytes = 128 * 128 * kChunks;
   static constexpr int kKVBytes = 64 * 128 * kChunks;
-  static constexpr int kPBytes = 128 * 128;
   // offsets from a 1024-byte-aligned base
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQBytes;
   static constexpr int kV = kK + kStages * kKVBytes;
-  static constexpr int kP = kV + kStages * kKVBytes;
-  static constexpr int kBars = kP + 2 * kPBytes;
-  // q, k/v full + empty, s full/free, p full, pv done, mma drain
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 * 4 + 1;
+  static constexpr int kBars = kV + kStages * kKVBytes;
+  // q, k/v full + empty, s full, p full, pv done, mma drain
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 * 3 + 1;
   static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, abort flag, list length
   static constexpr int kList = kMisc + 16;
+  __host__ __device__ static size_t list_bytes(int Nb) { return (static_cast<size_t>(Nb) * 2 + 15) & ~size_t(15); }
   static size_t bytes(int Nb) {
     const int words = (Nb + 31) / 32;
-    return 1024 + kList + static_cast<size_t>(Nb) * 4 + 2 * static_cast<size_t>(words) * 4;
+    return 1024 + kList + list_bytes(Nb) + 2 * static_cast<size_t>(words) * 4;
   }
 };
 
@@ -66,10 +70,11 @@ struct AttnArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using L = AttnSmem<D>;
+  constexpr int kStages = L::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
@@ -78,17 +83,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* v_full = k_full + kStages;
   uint64_t* kv_empty = v_full + kStages;
   uint64_t* s_full = kv_empty + kStages;  // [2]
-  uint64_t* s_free = s_full + 2;          // [2]
-  uint64_t* p_full = s_free + 2;          // [2]
+  uint64_t* p_full = s_full + 2;          // [2]
   uint64_t* pv_done = p_full + 2;         // [2]
   uint64_t* mma_drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
   int* list_len = reinterpret_cast<int*>(sm + L::kMisc + 8);
-  uint32_t* list = reinterpret_cast<uint32_t*>(sm + L::kList);
+  uint16_t* list = reinterpret_cast<uint16_t*>(sm + L::kList);
   const int Nb = a.Nb;
   const int words = (Nb + 31) >> 5;
-  uint32_t* bm0 = list + Nb;
+  uint32_t* bm0 = reinterpret_cast<uint32_t*>(sm + L::kList + L::list_bytes(Nb));
   uint32_t* bm1 = bm0 + words;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -106,7 +110,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(s_free + s, 128);
       mbar_init(p_full + s, 128);
       mbar_init(pv_done + s, 1);
     }
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int bit = __ffs(u) - 1;
         u &= u - 1;
         const uint32_t m = 1u << bit;
-        list[pos++] = static_cast<uint32_t>(w * 32 + bit) | ((x0 & m) ? (1u << 24) : 0u) | ((x1 & m) ? (1u << 25) : 0u);
+        list[pos++] = static_cast<uint16_t>((w * 32 + bit) | ((x0 & m) ? 0x4000u : 0u) | ((x1 & m) ? 0x8000u : 0u));
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
@@ -178,8 +181,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, false, false);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
-  const uint32_t sQ = smem_u32(sm + L::kQ), sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV),
-                 sP = smem_u32(sm + L::kP);
+  const uint32_t sQ = smem_u32(sm + L::kQ), sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV);
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int n = 0; n < L_n; ++n) {
         const int s = n % kStages;
         if (n >= kStages && !mbar_wait(kv_empty + s, ((n / kStages) - 1) & 1, abort_flag)) break;
-        const int j = static_cast<int>(list[n] & 0xFFFFFFu);
+        const int j = static_cast<int>(list[n] & 0x3FFFu);
         mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_4d(sm + L::kK + s * L::kKVBytes + c * 64 * 128, &tmK, k_full + s, c * 64, hd, j * 64, b);
@@ -219,13 +221,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(p_full + (m & 1), (m >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait(v_full + s, (m / kStages) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = sP + (m & 1) * L::kPBytes;
+        const uint32_t pa = (m & 1) ? tS1 : tS0;
         const uint32_t vb = sV + s * L::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, 64 * 128, 1024);
-          umma_bf16_ss(tO, ad, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tO, pa + kk * 8, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(pv_done + (m & 1));
         umma_commit(kv_empty + s);
@@ -234,7 +235,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int n = 0; ok && n < L_n; ++n) {
         const int s = n % kStages;
         if (!mbar_wait(k_full + s, (n / kStages) & 1, abort_flag)) { ok = false; break; }
-        if (n >= 2 && !mbar_wait(s_free + (n & 1), ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+        // S buffer (n & 1) still holds P(n-2) until PV(n-2) has read it.
+        if (n >= 2 && !mbar_wait(pv_done + (n & 1), ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kb = sK + s * L::kKVBytes;
         const uint32_t tS = (n & 1) ? tS1 : tS0;
@@ -258,10 +260,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // --------------------------------------------------------------- softmax
     const int r = tid;  // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t flag = 1u << (24 + (r >> 6));
+    const uint32_t flag = 0x4000u << (r >> 6);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    unsigned char* prow_base = sm + L::kP + r * 128;
     for (int n = 0; n < L_n; ++n) {
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + (n & 1), (n >> 1) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
@@ -272,10 +273,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence16(sv[c]);
-      tc_fence_before();
-      mbar_arrive(s_free + (n & 1));
 
-      const bool inc = (list[n] & flag) != 0u;
+      const bool inc = (static_cast<uint32_t>(list[n]) & flag) != 0u;
       float factor = 1.f;
       bool need = false;
       if (inc) {
@@ -292,7 +291,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       float rowsum = 0.f;
-      uint32_t pk[32];
+      uint32_t pk[2][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -303,17 +302,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             p1 = ex2_approx(fmaf(__uint_as_float(sv[c][e + 1]), a.scale_log2, -m_run));
           }
           rowsum += p0 + p1;
-          pk[c * 8 + e / 2] = pack_bf16x2(p0, p1);
+          const int k = c * 8 + e / 2;
+          pk[k >> 4][k & 15] = pack_bf16x2(p0, p1);
         }
       l_run = l_run * factor + rowsum;
 
-      // P buffer (n & 1) is free once PV(n-2) has completed.
-      if (n >= 2 && !__all_sync(0xffffffffu, mbar_wait(pv_done + (n & 1), ((n - 2) >> 1) & 1, abort_flag))) {
-        ok = false;
-        break;
-      }
+      __syncwarp();
       if (__any_sync(0xffffffffu, need)) {
-        __syncwarp();
         // O must not be rescaled while PV(n-1) still accumulates into it.
         if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag))) {
           ok = false;
@@ -331,15 +326,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
           tmem_st16(tO + lane_off + c * 16, ov);
         }
-        tmem_st_wait();
       }
-      unsigned char* prow = prow_base + (n & 1) * L::kPBytes;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
+      // P(n): bf16 pairs into the first 32 columns of the score buffer.
+      tmem_st16(tS, pk[0]);
+      tmem_st16(tS + 16, pk[1]);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full + (n & 1));
     }

@@ -7,15 +7,15 @@
 //                   compaction, R query-block rows per CTA:
 //   1. scores s_ij = (qbar_i . kbar_j) * scale (fp32 FMA chain over d) into
 //      shared memory, one row of Nb scores per query block;
-//   2. softmax per row (one warp per row): max, e = expf(s - max), fp64 sum,
-//      p = fp32(e / Z);
+//   2. softmax numerators per row (one warp per row): max, e = expf(s - max);
+//      p = e / sum(e) is never formed: the order of e is the order of p, and
+//      the masses are integers e * 2^40, so every partial sum is exact and
+//      independent of summation order;
 //   3. the CDF rule "keep where the ascending cumulative mass exceeds 1 - thr"
 //      without a full sort: a mass-weighted radix select over the fp32 bit
-//      patterns of p (4 passes of 8 bits, 256-bin histograms in shared memory)
-//      finds the boundary element (p*, j*) of the ascending (p, j) order;
-//      masses are integers p * 2^56 so every partial sum is exact and
-//      independent of summation order;
-//   4. keep = (p, j) >= (p*, j*)  OR arg-max  OR STA window, compacted with
+//      patterns of e (4 passes of 8 bits, 256-bin histograms in shared memory)
+//      finds the boundary element (e*, j*) of the ascending (e, j) order;
+//   4. keep = (e, j) >= (e*, j*)  OR arg-max  OR STA window, compacted with
 //      warp ballots into ascending kv_idx and kv_count.
 #pragma once
 
@@ -77,14 +77,18 @@ struct MaskArgs {
   int sta_on;
   int keep_all;       // thr >= 1
   float scale;
-  unsigned long long tau_fixed;  // floor((1 - thr) * 2^56)
+  double tau;         // 1 - thr (exact in double)
 };
 
-constexpr int kMaskThreads = 256;
+constexpr int kMaskThreads = 512;
 constexpr int kMaskWarps = kMaskThreads / 32;
 
-__device__ __forceinline__ unsigned long long mass_fixed(float p) {
-  return __double2ull_rz(static_cast<double>(p) * 72057594037927936.0);  // p * 2^56, exact scaling
+// Integer mass of an unnormalised probability e in (0, 1]: e * 2^40,
+// truncated (exact for e >= 2^-16; smaller masses lose < 2^-40 each).  The
+// row's CDF rule "cumulative p > 1 - thr" becomes, with p = e / sum(e),
+// "cumulative mass > floor((1 - thr) * total mass)" in exact integers.
+__device__ __forceinline__ unsigned long long mass_fixed(float e) {
+  return __float2ull_rz(e * 1099511627776.0f);
 }
 
 template <int R>
@@ -109,12 +113,13 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs 
   }
   __syncthreads();
 
-  // 1. scores
+  // 1. scores: one fused multiply-add chain per (row, block) over d ascending
   for (int j = tid; j < Nb; j += kMaskThreads) {
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
     const float4* kp = reinterpret_cast<const float4*>(kb + static_cast<int64_t>(j) * D);
+#pragma unroll 2
     for (int d4 = 0; d4 < (D >> 2); ++d4) {
       const float4 kv = __ldg(kp + d4);
 #pragma unroll
@@ -139,27 +144,26 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs 
     if (i >= Nb) break;
     float* row = rows + static_cast<size_t>(r) * Nb;
 
-    // 2. softmax
+    // 2. softmax numerators e = exp(s - max) (<= 1), integer masses, the
+    //    arg-max and the first radix digit's histogram, in one pass
     float m = -INFINITY;
     for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    double z = 0.0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0ull;
+    __syncwarp();
+    unsigned long long best = 0;  // (bits(e) << 32) | j; max = arg-max, ties to the larger j
+    unsigned long long total = 0;
     for (int j = lane; j < Nb; j += 32) {
       const float e = expf(row[j] - m);
       row[j] = e;
-      z += static_cast<double>(e);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    unsigned long long best = 0;  // (bits(p) << 32) | j, max = arg-max with ties to the larger j
-    unsigned long long total = 0;
-    for (int j = lane; j < Nb; j += 32) {
-      const float p = static_cast<float>(static_cast<double>(row[j]) / z);
-      row[j] = p;
-      const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(p)) << 32) | static_cast<unsigned>(j);
+      const uint32_t u = __float_as_uint(e);
+      const unsigned long long w = mass_fixed(e);
+      const unsigned long long key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
       best = key > best ? key : best;
-      total += mass_fixed(p);
+      total += w;
+      atomicAdd(&hist[u >> 24], w);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -167,23 +171,29 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs 
       best = ob > best ? ob : best;
       total += __shfl_xor_sync(0xffffffffu, total, o);
     }
+    __syncwarp();
     const int argmax = static_cast<int>(best & 0xffffffffu);
+    const unsigned long long tau_m =
+        static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
 
-    // 3. CDF boundary by mass-weighted radix select
-    unsigned long long kstar = ~0ull;  // keep (p,j) with key >= kstar
-    if (!a.keep_all && total > a.tau_fixed) {
+    // 3. CDF boundary by mass-weighted radix select over the bits of e
+    //    (order of e = order of p); keep (e, j) >= (e*, j*)
+    unsigned long long kstar = ~0ull;
+    if (!a.keep_all && total > tau_m) {
       uint32_t prefix = 0, pmask = 0;
       unsigned long long below = 0;
       for (int shift = 24; shift >= 0; shift -= 8) {
+        if (shift < 24) {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0ull;
-        __syncwarp();
-        for (int j = lane; j < Nb; j += 32) {
-          const float p = row[j];
-          const uint32_t u = __float_as_uint(p);
-          if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], mass_fixed(p));
+          for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0ull;
+          __syncwarp();
+          for (int j = lane; j < Nb; j += 32) {
+            const float e = row[j];
+            const uint32_t u = __float_as_uint(e);
+            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], mass_fixed(e));
+          }
+          __syncwarp();
         }
-        __syncwarp();
         unsigned long long loc[8], lsum = 0;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
@@ -201,23 +211,23 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs 
         unsigned long long before = 0;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          if (found < 0 && cum + loc[t] > a.tau_fixed) {
+          if (found < 0 && cum + loc[t] > tau_m) {
             found = lane * 8 + t;
             before = cum;
           }
           cum += loc[t];
         }
         const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
-        const int win = __ffs(ball) - 1;  // ball != 0: the range's cumulative mass exceeds tau
+        const int win = __ffs(ball) - 1;  // ball != 0: the range's cumulative mass exceeds tau_m
         const int bin = __shfl_sync(0xffffffffu, found, win);
         below = __shfl_sync(0xffffffffu, before, win);
         prefix |= static_cast<uint32_t>(bin) << shift;
         pmask |= 255u << shift;
         __syncwarp();
       }
-      // Ties at p*: the boundary is the m-th smallest index among them.
+      // Equal values at e*: the boundary is the m-th smallest index among them.
       const unsigned long long wstar = mass_fixed(__uint_as_float(prefix));
-      const unsigned long long need = (a.tau_fixed - below) / wstar + 1ull;
+      const unsigned long long need = (tau_m - below) / wstar + 1ull;
       unsigned long long seen = 0;
       int jstar = Nb;
       for (int base = 0; base < Nb; base += 32) {

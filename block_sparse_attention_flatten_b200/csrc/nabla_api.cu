@@ -208,15 +208,13 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
   a.sta_rw = p.sta_w / 2;
   a.keep_all = p.thr >= 1.f ? 1 : 0;
   a.scale = p.scale > 0.f ? p.scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  // (1 - thr) is exact in double; scaling by 2^56 is exact; floor keeps the
-  // comparison "cumulative mass > 1 - thr" exact for integer masses.
-  a.tau_fixed = static_cast<unsigned long long>(std::floor((1.0 - static_cast<double>(p.thr)) * 72057594037927936.0));
+  a.tau = 1.0 - static_cast<double>(p.thr);  // exact in double
 
-  // Rows per CTA: as many as fit ~128 KB of score rows, at most 32.
+  // Rows per CTA: 16 while the score rows fit ~64 KB (two CTAs per SM), else
+  // as many as fit ~128 KB.
   const size_t per_row = static_cast<size_t>(Nb) * 4;
+  if (16 * per_row <= 64u * 1024u) return launch_mask<16>(a, B, di, stream);
   const size_t fit = (128u * 1024u) / per_row;
-  if (fit >= 32) return launch_mask<32>(a, B, di, stream);
-  if (fit >= 16) return launch_mask<16>(a, B, di, stream);
   if (fit >= 8) return launch_mask<8>(a, B, di, stream);
   if (fit >= 4) return launch_mask<4>(a, B, di, stream);
   if (mask_smem_bytes(2, D, Nb) <= static_cast<size_t>(di.max_smem_optin)) return launch_mask<2>(a, B, di, stream);
@@ -241,6 +239,7 @@ int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const 
   if (rc != NABLA_OK) return rc;
   if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
   const int Nb = S / 64;
+  if (Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
   const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
 
   CUtensorMap tq, tk, tv;

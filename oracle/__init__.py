@@ -55,7 +55,7 @@ def _load():
         lib.oracle_mask.argtypes = [P, P, i, i, i, i, f, f, i, i, i, i, i, d, P, P, P, P]
         lib.oracle_attention.argtypes = [P, P, P, P, P, i, i, i, i, d, P, i, P, P]
         lib.oracle_block_probs_row.argtypes = [P, P, i, i, f, i, P]
-        lib.oracle_cdf_keep.argtypes = [P, i, f, P, P]
+        lib.oracle_cdf_keep.argtypes = [P, i, f, P, P, P, d]
         lib.oracle_cdf_keep.restype = i
         lib.oracle_sta.argtypes = [i, i, i, i, i, i, i]
         lib.oracle_sta.restype = i
@@ -120,13 +120,15 @@ def block_probs_row(qbar_bh: np.ndarray, kbar_bh: np.ndarray, i: int, scale: flo
     return p
 
 
-def cdf_keep(p: np.ndarray, thr: float):
-    """CDF keep flags and per-block cumulative mass for one probability row."""
+def cdf_keep(p: np.ndarray, thr: float, band: float = BAND):
+    """CDF keep flags, per-block cumulative mass, band flags and the arg-max
+    for one probability row."""
     p = np.ascontiguousarray(p, dtype=np.float32)
     keep = np.empty(p.shape[0], dtype=np.uint8)
     cum = np.empty(p.shape[0], dtype=np.float64)
-    argmax = _load().oracle_cdf_keep(_ptr(p), p.shape[0], thr, _ptr(keep), _ptr(cum))
-    return keep.astype(bool), cum, argmax
+    bandf = np.empty(p.shape[0], dtype=np.uint8)
+    argmax = _load().oracle_cdf_keep(_ptr(p), p.shape[0], thr, _ptr(keep), _ptr(cum), _ptr(bandf), band)
+    return keep.astype(bool), cum, bandf.astype(bool), argmax
 
 
 def sta(i: int, j: int, nbh: int, nbw: int, window=(3, 3, 3)) -> bool:

@@ -121,9 +121,13 @@ void oracle_pool(const uint16_t* x, float* xbar, int B, int S, int Hh, int D) {
 
 /* ------------------------------------------------------------------------ */
 /* Reduced attention (NABLA summary, "Atencao Reduzida"): one row i of the   */
-/* block-level softmax.  s_ij = fp32(exact dot(qbar_i, kbar_j)) * scale in    */
-/* fp32; m = max_j s_ij; e_j = expf(s_ij - m); Z = sum_j e_j in fp64;         */
-/* p_j = fp32(e_j / Z).                                                      */
+/* block-level softmax, in fp32 as the method's mask stage is:               */
+/*   s_ij = fl32(sum_d qbar_id * kbar_jd) * scale, the sum a chain of fused  */
+/*          multiply-adds in ascending d (fmaf), then one fp32 multiply;     */
+/*   m    = max_j s_ij;                                                      */
+/*   e_j  = exp(s_ij - m) correctly rounded to fp32 (s - m in fp32, exp in   */
+/*          fp64, then rounded);                                             */
+/*   Z    = sum_j e_j in fp64;  p_j = fl32(e_j / Z).                          */
 /* Pinned by: scores against the fp64 mean of token logits; sum p = 1 within */
 /* Nb * 2^-24; the all-equal-scores case giving exactly 1/Nb.                */
 /* ------------------------------------------------------------------------ */
@@ -131,15 +135,15 @@ static void block_probs(const float* qbar_i, const float* kbar, int Nb, int D, f
                         float* p) {
   float m = -INFINITY;
   for (int j = 0; j < Nb; ++j) {
-    double dot = 0.0;
-    for (int d = 0; d < D; ++d) dot += (double)qbar_i[d] * (double)kbar[(int64_t)j * D + d];
-    float s = (float)dot * scale;
+    float dot = 0.0f;
+    for (int d = 0; d < D; ++d) dot = fmaf(qbar_i[d], kbar[(int64_t)j * D + d], dot);
+    float s = dot * scale;
     p[j] = s;
     if (s > m) m = s;
   }
   double Z = 0.0;
   for (int j = 0; j < Nb; ++j) {
-    float e = expf(p[j] - m);
+    float e = (float)exp((double)(p[j] - m));
     p[j] = e;
     Z += (double)e;
   }
@@ -160,17 +164,27 @@ static int cmp_pj(const void* a, const void* b) {
   return (x->j > y->j) - (x->j < y->j);
 }
 
+/* Probabilities within this relative distance of each other are treated as  */
+/* tied by rounding when marking band blocks (about 8-16 fp32 ulps).         */
+#define ORACLE_TIE_REL (1.0 / 1048576.0) /* 2^-20 */
+
 /* ------------------------------------------------------------------------ */
 /* CDF thresholding (NABLA summary, "Limiarizacao CDF"): sort the row's       */
 /* probabilities ascending, take the running sum c_k (fp64) and keep the      */
 /* block at position k iff c_k > 1 - thr.  thr >= 1 keeps every block; the    */
 /* arg-max (last position) is always kept.  cum[j] receives c at block j's    */
-/* position (used to mark blocks whose decision is within the 1e-5 band).    */
+/* position.  band[j] (if not NULL) marks blocks whose decision rounding can  */
+/* change: |c - (1-thr)| < band_width, or a run of rounding-tied             */
+/* probabilities (consecutive in the order, each within ORACLE_TIE_REL of the */
+/* next) whose positions straddle 1 - thr, since the order inside such a run */
+/* is set by rounding, not by the method; the same holds for the run that    */
+/* holds the arg-max when it has more than one member (which block is the   */
+/* forced arg-max is then set by rounding).                                  */
 /* Pinned by: an exact-rational top-p (nucleus) restatement on random rows,  */
 /* kept mass >= thr and minimality, and the uniform Nb=16 case.              */
 /* ------------------------------------------------------------------------ */
 static int cdf_keep_row(const float* p, int Nb, float thr, uint8_t* keep, double* cum,
-                        pj_t* scratch) {
+                        uint8_t* band, double band_width, pj_t* scratch) {
   for (int j = 0; j < Nb; ++j) {
     scratch[j].p = p[j];
     scratch[j].j = j;
@@ -183,6 +197,24 @@ static int cdf_keep_row(const float* p, int Nb, float thr, uint8_t* keep, double
     int j = scratch[k].j;
     cum[j] = c;
     keep[j] = (uint8_t)((thr >= 1.0f) || (c > tau) || (k == Nb - 1));
+  }
+  if (band) {
+    int a = 0;
+    while (a < Nb) {
+      int b = a;
+      while (b + 1 < Nb && (double)scratch[b + 1].p <= (double)scratch[b].p * (1.0 + ORACLE_TIE_REL)) ++b;
+      double ca = cum[scratch[a].j], cb = cum[scratch[b].j];
+      int flag;
+      if (b == Nb - 1) {
+        flag = b > a; /* the run holding the forced arg-max */
+      } else {
+        int near = 0;
+        for (int k = a; k <= b; ++k) near |= fabs(cum[scratch[k].j] - tau) < band_width;
+        flag = (ca <= tau && cb > tau) || near;
+      }
+      for (int k = a; k <= b; ++k) band[scratch[k].j] = (uint8_t)flag;
+      a = b + 1;
+    }
   }
   return scratch[Nb - 1].j; /* the arg-max block */
 }
@@ -209,7 +241,7 @@ static int sta_keep(int i, int j, int nbh, int nbw, int st, int sh, int sw) {
 /*   kv_count[b,hd,i]   number of kept key blocks                            */
 /*   kv_idx[b,hd,i,:]   kept key-block indices ascending (row stride Nb)      */
 /* status (optional, [B,Hh,Nb,Nb] uint8): bit0 = kept, bit1 = band block     */
-/* (decided by the CDF alone and |c - (1-thr)| < band).                       */
+/* (decided by the CDF alone and within the band, see cdf_keep_row).         */
 /* probs (optional, [B,Hh,Nb,Nb] fp32): the row probabilities p.             */
 /* qbar/kbar: fp32 [B][Hh][Nb][D].  Rows are independent; OpenMP splits them */
 /* without changing any element's arithmetic.                                */
@@ -222,6 +254,7 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
   {
     float* p = (float*)malloc(sizeof(float) * (size_t)Nb);
     uint8_t* keep = (uint8_t*)malloc((size_t)Nb);
+    uint8_t* bandf = (uint8_t*)malloc((size_t)Nb);
     double* cum = (double*)malloc(sizeof(double) * (size_t)Nb);
     pj_t* scratch = (pj_t*)malloc(sizeof(pj_t) * (size_t)Nb);
 #pragma omp for schedule(dynamic, 4)
@@ -231,8 +264,7 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
       const float* qi = qbar + (bh * Nb + i) * D;
       const float* kb = kbar + bh * Nb * D;
       block_probs(qi, kb, Nb, D, scale, p);
-      int argmax = cdf_keep_row(p, Nb, thr, keep, cum, scratch);
-      double tau = 1.0 - (double)thr;
+      int argmax = cdf_keep_row(p, Nb, thr, keep, cum, status ? bandf : NULL, band, scratch);
       int32_t n = 0;
       for (int j = 0; j < Nb; ++j) {
         int cdf_kept = keep[j];
@@ -242,7 +274,8 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
         if (status) {
           /* A block is "band" only when the CDF comparison alone decides it. */
           int forced = sta || thr >= 1.0f;
-          int in_band = !forced && j != argmax && fabs(cum[j] - tau) < band;
+          /* the arg-max is forced unless rounding-tied (then bandf marks it) */
+          int in_band = !forced && bandf[j];
           status[row * Nb + j] = (uint8_t)(kept | (in_band << 1));
         }
         if (probs) probs[row * Nb + j] = p[j];
@@ -251,6 +284,7 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
     }
     free(p);
     free(keep);
+    free(bandf);
     free(cum);
     free(scratch);
   }
@@ -339,9 +373,10 @@ void oracle_block_probs_row(const float* qbar, const float* kbar, int Nb, int D,
 }
 
 /* CDF keep decision for one probability row (see cdf_keep_row). */
-int oracle_cdf_keep(const float* p, int Nb, float thr, uint8_t* keep, double* cum) {
+int oracle_cdf_keep(const float* p, int Nb, float thr, uint8_t* keep, double* cum, uint8_t* band,
+                    double band_width) {
   pj_t* scratch = (pj_t*)malloc(sizeof(pj_t) * (size_t)Nb);
-  int argmax = cdf_keep_row(p, Nb, thr, keep, cum, scratch);
+  int argmax = cdf_keep_row(p, Nb, thr, keep, cum, band, band_width, scratch);
   free(scratch);
   return argmax;
 }

@@ -197,7 +197,7 @@ def test_cdf_rule_equals_exact_top_p(oracle_lib, thr):
     for hd in range(w.Hh):
         for i in range(w.Nb):
             p = oracle_lib.block_probs_row(qbar[0, hd], kbar[0, hd], i, w.scale)
-            keep, cum, argmax = oracle_lib.cdf_keep(p, thr)
+            keep, cum, band, argmax = oracle_lib.cdf_keep(p, thr)
             assert set(np.nonzero(keep)[0].tolist()) == exact_top_p(p, thr)
             assert keep[int(np.argmax(p))]
 
@@ -390,3 +390,36 @@ def test_generator_is_deterministic_and_shaped():
         assert torch.equal(x, y)
     idx = inputs.sample_query_blocks(960)
     assert len(idx) == 64 and len(set(idx.tolist())) == 64 and np.all(np.diff(idx) > 0)
+
+
+def test_band_marks_rounding_ties_straddling_the_threshold(oracle_lib):
+    """Band blocks: within 1e-5 of 1 - thr, or a run of probabilities equal to
+    within fp32 rounding whose positions straddle 1 - thr (their order, and so
+    which of them is kept, is set by rounding)."""
+    one_ulp_up = np.nextafter(np.float32(0.06), np.float32(1.0))
+    # ascending: 0.06 (c=0.06 <= 0.1), 0.06+ulp (c=0.12 > 0.1): a tied pair across the threshold
+    p = np.array([0.8, 0.06, one_ulp_up, 0.2], dtype=np.float32)
+    keep, cum, band, argmax = oracle_lib.cdf_keep(p, 0.9)
+    assert keep.tolist() == [True, False, True, True]
+    assert band.tolist() == [False, True, True, False]
+    # same masses but clearly ordered: nothing is band
+    p2 = np.array([0.8, 0.06, 0.062, 0.2], dtype=np.float32)
+    keep2, _, band2, _ = oracle_lib.cdf_keep(p2, 0.9)
+    assert keep2.tolist() == [True, False, True, True] and not band2.any()
+    # a block whose cumulative mass sits 5e-6 above the threshold
+    tau = 1.0 - float(np.float32(0.9))
+    p3 = np.array([0.7, np.float32(tau + 5e-6), 0.3], dtype=np.float32)
+    keep3, cum3, band3, _ = oracle_lib.cdf_keep(p3, 0.9)
+    assert keep3.tolist() == [True, True, True]
+    assert band3.tolist() == [False, True, False]
+
+
+def test_band_marks_a_rounding_tied_arg_max(oracle_lib):
+    top = np.float32(0.4)
+    p = np.array([0.2, top, np.nextafter(top, np.float32(1.0)), 0.0001], dtype=np.float32)
+    keep, cum, band, argmax = oracle_lib.cdf_keep(p, 0.0)  # thr 0: only the arg-max is kept
+    assert argmax == 2 and keep.tolist() == [False, False, True, False]
+    assert band.tolist() == [False, True, True, False]
+    p2 = np.array([0.2, 0.39, 0.41, 0.0001], dtype=np.float32)  # clear arg-max: nothing band
+    _, _, band2, _ = oracle_lib.cdf_keep(p2, 0.0)
+    assert not band2.any()
