@@ -278,13 +278,21 @@ def run_gpu(args, rank, world, local_rank):
 
 
 def load_traffic(config):
-    """DRAM bytes per attention launch from the committed ncu summary, if it
-    matches the current kernel; else None."""
+    """DRAM bytes (read + write) per attention launch from the committed ncu
+    capture of this workload, or None when there is none or the kernel source
+    changed since it was taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", f"attn_fwd_{config}.json")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
         d = json.load(fh)
+    h = hashlib.sha256()
+    for name in ("attn_fwd.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_flatten_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != d.get("source_sha256"):
+        return None
     return d.get("dram_bytes_per_launch")
 
 
