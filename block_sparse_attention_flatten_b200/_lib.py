@@ -25,12 +25,15 @@ NABLA_ERR_CUDA = 3
 NABLA_ERR_DEVICE_TIMEOUT = 4
 NABLA_ERR_DEVICE_BOUNDS = 5
 NABLA_ERR_UNSUPPORTED = 6
+NABLA_ERR_TOO_LARGE = 7
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTS = (
     "nabla_flatten",
     "nabla_unflatten",
     "nabla_mask_workspace_bytes",
     "nabla_build_mask",
+    "nabla_build_mask_noalloc",
     "nabla_sparse_attn_fwd",
     "nabla_get_status",
     "nabla_validate_mask",
@@ -74,6 +77,7 @@ def lib():
         L.nabla_mask_workspace_bytes.argtypes = [i, i, i, i, i, i, pp]
         L.nabla_mask_workspace_bytes.restype = sz
         L.nabla_build_mask.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
+        L.nabla_build_mask_noalloc.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
         L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
@@ -163,6 +167,27 @@ def build_mask(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: 
                                   _dev(kv_idx, torch.int32, "kv_idx"), _dev(workspace, torch.uint8, "workspace"),
                                   _stream(stream)), "nabla_build_mask")
     return kv_count, kv_idx, workspace
+
+
+def build_mask_noalloc(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),
+                       scale: float = 0.0, kv_count=None, kv_idx=None, stream=None, P: int = 8):
+    """The mask of :func:`build_mask` through nabla_build_mask_noalloc: the
+    library keeps the pooled vectors in its own static device buffer (16 MiB)
+    and allocates nothing; calls sharing that buffer must not overlap on the
+    GPU.  Returns (kv_count, kv_idx)."""
+    B, S, Hh, D = qf.shape
+    Nb = S // BLOCK
+    prm = params(thr, sta, scale, P)
+    dev = qf.device
+    if kv_count is None:
+        kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)
+    _check(lib().nabla_build_mask_noalloc(_dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"), B, Hh, D,
+                                          T, H, W, ctypes.byref(prm), _dev(kv_count, torch.int32, "kv_count"),
+                                          _dev(kv_idx, torch.int32, "kv_idx"), _stream(stream)),
+           "nabla_build_mask_noalloc")
+    return kv_count, kv_idx
 
 
 def pooled_from_workspace(workspace: torch.Tensor, B: int, Hh: int, Nb: int, D: int):

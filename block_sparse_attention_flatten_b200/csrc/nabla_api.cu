@@ -136,6 +136,13 @@ int launch_mask(const MaskArgs& a, int B, const DeviceInfo& di, cudaStream_t str
   return launch_status();
 }
 
+// Scratch of nabla_build_mask_noalloc: the pooled queries then keys.  In host
+// code this name is only a stand-in for the device symbol; its device address
+// comes from cudaGetSymbolAddress, once per device.
+__device__ __align__(256) unsigned char g_noalloc_scratch[NABLA_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
 }  // namespace
 }  // namespace nabla
 
@@ -274,6 +281,27 @@ int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const 
   return launch_status();
 }
 
+int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
+                             const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
+                             nabla_stream_t stream) {
+  const size_t need = nabla_mask_workspace_bytes(B, Hh, D, T, H, W, params);
+  if (params == nullptr || need == 0) return NABLA_ERR_INVALID;
+  if (need > NABLA_NOALLOC_SCRATCH_BYTES) return NABLA_ERR_TOO_LARGE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NABLA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NABLA_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return nabla_build_mask(qf, kf, B, Hh, D, T, H, W, params, kv_count, kv_idx, scratch, stream);
+}
+
 int nabla_get_status(nabla_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (cudaStreamSynchronize(stream) != cudaSuccess) return NABLA_ERR_CUDA;
@@ -308,6 +336,7 @@ const char* nabla_strerror(int code) {
     case NABLA_ERR_DEVICE_TIMEOUT: return "device wait exceeded its time limit";
     case NABLA_ERR_DEVICE_BOUNDS: return "block index or count out of range";
     case NABLA_ERR_UNSUPPORTED: return "device is not an sm_100 GPU";
+    case NABLA_ERR_TOO_LARGE: return "mask workspace exceeds the static scratch of nabla_build_mask_noalloc (16 MiB)";
     default: return "unknown error";
   }
 }

@@ -43,7 +43,8 @@ enum {
   NABLA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
   NABLA_ERR_DEVICE_TIMEOUT = 4, /* (device status) a bounded wait expired */
   NABLA_ERR_DEVICE_BOUNDS = 5,  /* (device status) a block index or count was out of range */
-  NABLA_ERR_UNSUPPORTED = 6     /* no sm_100 device */
+  NABLA_ERR_UNSUPPORTED = 6,    /* no sm_100 device */
+  NABLA_ERR_TOO_LARGE = 7       /* problem exceeds NABLA_NOALLOC_SCRATCH_BYTES */
 };
 
 /* Mask parameters.
@@ -130,6 +131,30 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out,
                           float* lse, nabla_stream_t stream);
+
+/* Same mask as nabla_build_mask, for callers that cannot allocate device
+ * memory.  This entry point has no counterpart in the paper; it exists for
+ * code that hands the library only its input and output buffers: a plug-in
+ * host or serving runtime that owns all device memory and exposes no
+ * allocator, or a latency-critical path where cudaMalloc's implicit
+ * device-wide synchronisation is not acceptable.
+ *   The pooled queries and keys (the workspace of nabla_build_mask) live in
+ *   a static device buffer of NABLA_NOALLOC_SCRATCH_BYTES inside the library;
+ *   every GPU that loads the library holds that buffer until the process
+ *   exits.  The call allocates nothing and frees nothing.
+ *   Arguments, layouts and results are those of nabla_build_mask without the
+ *   workspace argument.  A problem whose workspace
+ *   (nabla_mask_workspace_bytes) exceeds NABLA_NOALLOC_SCRATCH_BYTES is
+ *   rejected with NABLA_ERR_TOO_LARGE before anything is launched.
+ *   The first call on a device looks up the buffer's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one buffer and each call overwrites it completely:
+ *   calls that overlap on the GPU (other streams, other host threads) race
+ *   on it, so the caller must order them. */
+#define NABLA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
+                             const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
+                             nabla_stream_t stream);
 
 /* Synchronises the stream, then returns and clears the current device's
  * status word (NABLA_OK, NABLA_ERR_DEVICE_TIMEOUT or NABLA_ERR_DEVICE_BOUNDS),
