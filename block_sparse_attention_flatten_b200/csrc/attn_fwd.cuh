@@ -49,8 +49,8 @@ struct AttnSmem {
   static constexpr int kK = kQ + kQBytes;
   static constexpr int kV = kK + kStages * kKVBytes;
   static constexpr int kBars = kV + kStages * kKVBytes;
-  // q, k/v full + empty, s full, p full, pv done, mma drain
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 * 3 + 1;
+  // q, k full + empty, v full + empty, s full, p full, pv done, mma drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 * 3 + 1;
   static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, abort flag, list length
   static constexpr int kList = kMisc + 16;
   __host__ __device__ static size_t list_bytes(int Nb) { return (static_cast<size_t>(Nb) * 2 + 15) & ~size_t(15); }
@@ -81,8 +81,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kStages;
-  uint64_t* kv_empty = v_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;  // [2]
+  uint64_t* k_empty = v_full + kStages;
+  uint64_t* v_empty = k_empty + kStages;
+  uint64_t* s_full = v_empty + kStages;   // [2]
   uint64_t* p_full = s_full + 2;          // [2]
   uint64_t* pv_done = p_full + 2;         // [2]
   uint64_t* mma_drain = pv_done + 2;
@@ -106,7 +107,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(v_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
@@ -116,12 +118,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // Q does not depend on the block lists: start its load right away.
+    tma_prefetch_desc(&tmQ);
+    mbar_arrive_expect_tx(q_full, L::kQBytes);
+    for (int c = 0; c < L::kChunks; ++c)
+      tma_load_4d(sm + L::kQ + c * 128 * 128, &tmQ, q_full, c * 64, hd, pair * 128, b);
   }
   if (warp == 4) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
@@ -185,32 +191,48 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
+    // One thread streams K and V through two rings.  A K stage frees as soon
+    // as its QK^T MMA is done, a V stage after its PV MMA; the MMA order is
+    // QK(n), PV(n-1), so K runs one block ahead of V: step n loads K(n) (its
+    // stage freed by QK(n-2)) and then V(n-1) (freed by PV(n-3)).  Blocking
+    // waits of a second producer lane in this warp would stall this one.
     if (lane == 0 && L_n > 0) {
-      mbar_arrive_expect_tx(q_full, L::kQBytes);
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_4d(sm + L::kQ + c * 128 * 128, &tmQ, q_full, c * 64, hd, pair * 128, b);
-      int issued = 0;
-      for (int n = 0; n < L_n; ++n) {
-        const int s = n % kStages;
-        if (n >= kStages && !mbar_wait(kv_empty + s, ((n / kStages) - 1) & 1, abort_flag)) break;
-        const int j = static_cast<int>(list[n] & 0x3FFFu);
-        mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sm + L::kK + s * L::kKVBytes + c * 64 * 128, &tmK, k_full + s, c * 64, hd, j * 64, b);
-        mbar_arrive_expect_tx(v_full + s, L::kKVBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sm + L::kV + s * L::kKVBytes + c * 64 * 128, &tmV, v_full + s, c * 64, hd, j * 64, b);
-        issued = n + 1;
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (int n = 0; ok && n <= L_n; ++n) {
+        if (n < L_n) {
+          const int s = n % kStages;
+          if (n >= kStages && !mbar_wait(k_empty + s, ((n / kStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int j = static_cast<int>(list[n] & 0x3FFFu);
+          mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sm + L::kK + s * L::kKVBytes + c * 64 * 128, &tmK, k_full + s, c * 64, hd, j * 64, b);
+          k_issued = n + 1;
+        }
+        if (n >= 1) {
+          const int m = n - 1, s = m % kStages;
+          if (m >= kStages && !mbar_wait(v_empty + s, ((m / kStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int j = static_cast<int>(list[m] & 0x3FFFu);
+          mbar_arrive_expect_tx(v_full + s, L::kKVBytes);
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(sm + L::kV + s * L::kKVBytes + c * 64 * 128, &tmV, v_full + s, c * 64, hd, j * 64, b);
+          v_issued = m + 1;
+        }
       }
       // Drain: wait for the last issued loads of every stage so no copy is in
       // flight when the CTA exits, also on the abort path (time-bounded).
-      mbar_wait_drain(q_full, 0);
-      for (int n = (issued > kStages ? issued - kStages : 0); n < issued; ++n) {
-        const int s = n % kStages;
-        mbar_wait_drain(k_full + s, (n / kStages) & 1);
-        mbar_wait_drain(v_full + s, (n / kStages) & 1);
-      }
+      for (int n = (k_issued > kStages ? k_issued - kStages : 0); n < k_issued; ++n)
+        mbar_wait_drain(k_full + n % kStages, (n / kStages) & 1);
+      for (int n = (v_issued > kStages ? v_issued - kStages : 0); n < v_issued; ++n)
+        mbar_wait_drain(v_full + n % kStages, (n / kStages) & 1);
     }
+    if (lane == 0) mbar_wait_drain(q_full, 0);
   } else if (warp == 5) {
     // ------------------------------------------------------------- MMA issue
     if (lane == 0 && L_n > 0) {
@@ -229,7 +251,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           umma_bf16_ts(tO, pa + kk * 8, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(pv_done + (m & 1));
-        umma_commit(kv_empty + s);
+        umma_commit(v_empty + s);
         return true;
       };
       for (int n = 0; ok && n < L_n; ++n) {
@@ -248,6 +270,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           umma_bf16_ss(tS, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full + (n & 1));
+        umma_commit(k_empty + s);
         if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
       }
       if (ok) issue_pv(L_n - 1);
@@ -278,11 +301,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       float factor = 1.f;
       bool need = false;
       if (inc) {
-        float mx = -INFINITY;
+        float mc[4];  // four independent max chains
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c) {
+          mc[c] = __uint_as_float(sv[c][0]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) mx = fmaxf(mx, __uint_as_float(sv[c][e]));
+          for (int e = 1; e < 16; ++e) mc[c] = fmaxf(mc[c], __uint_as_float(sv[c][e]));
+        }
+        float mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
         mx *= a.scale_log2;
         if (mx > m_run + 8.f) {  // also true while m_run is -inf
           factor = ex2_approx(m_run - mx);  // 0 when m_run = -inf
@@ -290,7 +316,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           m_run = mx;
         }
       }
-      float rowsum = 0.f;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
       uint32_t pk[2][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -301,11 +327,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             p0 = ex2_approx(fmaf(__uint_as_float(sv[c][e]), a.scale_log2, -m_run));
             p1 = ex2_approx(fmaf(__uint_as_float(sv[c][e + 1]), a.scale_log2, -m_run));
           }
-          rowsum += p0 + p1;
+          rs[c] += p0 + p1;
           const int k = c * 8 + e / 2;
           pk[k >> 4][k & 15] = pack_bf16x2(p0, p1);
         }
-      l_run = l_run * factor + rowsum;
+      l_run = l_run * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
 
       __syncwarp();
       if (__any_sync(0xffffffffu, need)) {
@@ -344,16 +370,24 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
     __nv_bfloat16* orow = a.out + ((static_cast<int64_t>(b) * a.S + row_g) * a.Hh + hd) * D;
 #pragma unroll 1
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t ov[16];
+    for (int c0 = 0; c0 < D / 16; c0 += 4) {
+      uint32_t ob[4][16];
       if (ok && L_n > 0) {
-        tmem_ld16(tO + lane_off + c * 16, ov);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tmem_ld16(tO + lane_off + (c0 + u) * 16, ob[u]);
         tmem_ld_wait();
-        reg_fence16(ov);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) reg_fence16(ob[u]);
       } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) ov[e] = 0u;
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ob[u][e] = 0u;
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u;
+      const uint32_t (&ov)[16] = ob[u];
       uint4 w0, w1;
       w0.x = pack_bf16x2(__uint_as_float(ov[0]) * inv_l, __uint_as_float(ov[1]) * inv_l);
       w0.y = pack_bf16x2(__uint_as_float(ov[2]) * inv_l, __uint_as_float(ov[3]) * inv_l);
@@ -366,6 +400,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       if (row_valid) {
         reinterpret_cast<uint4*>(orow + c * 16)[0] = w0;
         reinterpret_cast<uint4*>(orow + c * 16)[1] = w1;
+      }
       }
     }
     if (row_valid && a.lse != nullptr)
