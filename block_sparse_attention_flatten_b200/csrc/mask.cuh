@@ -12,9 +12,10 @@
 //      the masses are integers e * 2^40, so every partial sum is exact and
 //      independent of summation order;
 //   3. the CDF rule "keep where the ascending cumulative mass exceeds 1 - thr"
-//      without a full sort: a mass-weighted radix select over the fp32 bit
-//      patterns of e (4 passes of 8 bits, 256-bin histograms in shared memory)
-//      finds the boundary element (e*, j*) of the ascending (e, j) order;
+//      without a full sort: a binary search over the fp32 bit patterns of e
+//      with warp-summed exact masses finds the boundary element (e*, j*) of
+//      the ascending (e, j) order (shared-memory histograms with atomics
+//      serialise on the few bins most masses fall into);
 //   4. keep = (e, j) >= (e*, j*)  OR arg-max  OR STA window, compacted with
 //      warp ballots into ascending kv_idx and kv_count.
 #pragma once
@@ -83,22 +84,24 @@ struct MaskArgs {
 constexpr int kMaskThreads = 512;
 constexpr int kMaskWarps = kMaskThreads / 32;
 
-// Integer mass of an unnormalised probability e in (0, 1]: e * 2^40,
-// truncated (exact for e >= 2^-16; smaller masses lose < 2^-40 each).  The
-// row's CDF rule "cumulative p > 1 - thr" becomes, with p = e / sum(e),
-// "cumulative mass > floor((1 - thr) * total mass)" in exact integers.
-__device__ __forceinline__ unsigned long long mass_fixed(float e) {
-  return __float2ull_rz(e * 1099511627776.0f);
+// Integer mass of an unnormalised probability e in [0, 1], from its bit
+// pattern u: floor(e * 2^40) (exact for e >= 2^-16; smaller masses lose
+// < 2^-40 each).  The row's CDF rule "cumulative p > 1 - thr" becomes, with
+// p = e / sum(e), "cumulative mass > floor((1 - thr) * total mass)" in exact
+// integers, independent of summation order.
+__device__ __forceinline__ unsigned long long mass_bits(uint32_t u) {
+  const int sh = static_cast<int>(u >> 23) - 110;  // biased exponent - (150 - 40)
+  const unsigned long long m24 = (u & 0x7FFFFFu) | 0x800000u;
+  return sh >= 0 ? (m24 << sh) : (sh > -24 ? (m24 >> -sh) : 0ull);
 }
 
 template <int R>
-__global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs a) {
+__global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int D = a.D, Nb = a.Nb;
   float* qs = reinterpret_cast<float*>(smem_raw);                       // [R][D]
   float* rows = qs + R * D;                                             // [R][Nb]
-  unsigned long long* hist_all = reinterpret_cast<unsigned long long*>(rows + static_cast<size_t>(R) * Nb);
-  // hist_all is 8-byte aligned because R*D and R*Nb are even.
+  int* cand_all = reinterpret_cast<int*>(rows + static_cast<size_t>(R) * Nb);  // [warps][32]
 
   const int i0 = blockIdx.x * R;
   const int hd = blockIdx.y, b = blockIdx.z;
@@ -138,32 +141,27 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs 
   }
   __syncthreads();
 
-  unsigned long long* hist = hist_all + warp * 256;
+  int* cand = cand_all + warp * 32;
   for (int r = warp; r < R; r += kMaskWarps) {
     const int i = i0 + r;
     if (i >= Nb) break;
     float* row = rows + static_cast<size_t>(r) * Nb;
 
-    // 2. softmax numerators e = exp(s - max) (<= 1), integer masses, the
-    //    arg-max and the first radix digit's histogram, in one pass
+    // 2. softmax numerators e = exp(s - max) (<= 1), their total integer
+    //    mass and the arg-max, in one pass
     float m = -INFINITY;
     for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-#pragma unroll
-    for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0ull;
-    __syncwarp();
     unsigned long long best = 0;  // (bits(e) << 32) | j; max = arg-max, ties to the larger j
     unsigned long long total = 0;
     for (int j = lane; j < Nb; j += 32) {
       const float e = expf(row[j] - m);
       row[j] = e;
       const uint32_t u = __float_as_uint(e);
-      const unsigned long long w = mass_fixed(e);
       const unsigned long long key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
       best = key > best ? key : best;
-      total += w;
-      atomicAdd(&hist[u >> 24], w);
+      total += mass_bits(u);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -171,79 +169,112 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_kernel(const MaskArgs 
       best = ob > best ? ob : best;
       total += __shfl_xor_sync(0xffffffffu, total, o);
     }
-    __syncwarp();
     const int argmax = static_cast<int>(best & 0xffffffffu);
     const unsigned long long tau_m =
         static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
 
-    // 3. CDF boundary by mass-weighted radix select over the bits of e
-    //    (order of e = order of p); keep (e, j) >= (e*, j*)
+    // 3. CDF boundary: the element (e*, j*) of the ascending (e, j) order at
+    //    which the cumulative mass first exceeds tau_m; keep (e, j) >= it.
+    //    bits(e*) is the largest bit pattern x with mass(bits(e) < x) <= tau_m
+    //    (positive floats order like their bit patterns), found MSB first by
+    //    a binary search of exact warp-summed masses (no atomics).  After the
+    //    top 11 bits, if at most 32 blocks share them they are sorted by a
+    //    warp bitonic sort and the boundary read off their prefix sums.
     unsigned long long kstar = ~0ull;
     if (!a.keep_all && total > tau_m) {
-      uint32_t prefix = 0, pmask = 0;
-      unsigned long long below = 0;
-      for (int shift = 24; shift >= 0; shift -= 8) {
-        if (shift < 24) {
+      uint32_t prefix = 0;
+      unsigned long long below = 0;  // mass(bits(e) < prefix)
+      auto mass_below = [&](uint32_t x) -> unsigned long long {
+        unsigned long long sum = 0;
+        for (int j = lane; j < Nb; j += 32) {
+          const uint32_t u = __float_as_uint(row[j]);
+          if (u < x) sum += mass_bits(u);
+        }
 #pragma unroll
-          for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0ull;
-          __syncwarp();
-          for (int j = lane; j < Nb; j += 32) {
-            const float e = row[j];
-            const uint32_t u = __float_as_uint(e);
-            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], mass_fixed(e));
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        return sum;
+      };
+      for (int bit = 30; bit >= 20; --bit) {
+        const uint32_t c = prefix | (1u << bit);
+        const unsigned long long sm_ = mass_below(c);
+        if (sm_ <= tau_m) {
+          prefix = c;
+          below = sm_;
+        }
+      }
+      // e* lies in [prefix, prefix + 2^20): gather those blocks (ascending j).
+      int ncand = 0;
+      for (int base = 0; base < Nb && ncand <= 32; base += 32) {
+        const int j = base + lane;
+        const bool hit = j < Nb && (__float_as_uint(row[j]) >> 20) == (prefix >> 20);
+        const unsigned bal = __ballot_sync(0xffffffffu, hit);
+        const int pos = ncand + __popc(bal & ((1u << lane) - 1u));
+        if (hit && pos < 32) cand[pos] = j;
+        ncand += __popc(bal);
+      }
+      __syncwarp();
+      if (ncand <= 32) {
+        unsigned long long key = ~0ull, w = 0ull;
+        if (lane < ncand) {
+          const int j = cand[lane];
+          const uint32_t u = __float_as_uint(row[j]);
+          key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
+          w = mass_bits(u);
+        }
+        // bitonic sort of (key, w) ascending by key across the warp
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const unsigned long long okey = __shfl_xor_sync(0xffffffffu, key, stride);
+            const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
+            const bool up = (lane & size) == 0;
+            const bool lower = (lane & stride) == 0;
+            if (lower == up ? (okey < key) : (okey > key)) {
+              key = okey;
+              w = ow;
+            }
           }
-          __syncwarp();
         }
-        unsigned long long loc[8], lsum = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          loc[t] = hist[lane * 8 + t];
-          lsum += loc[t];
-        }
-        unsigned long long incl = lsum;
+        unsigned long long cw = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
+          const unsigned long long v = __shfl_up_sync(0xffffffffu, cw, o);
+          if (lane >= o) cw += v;
         }
-        unsigned long long cum = below + (incl - lsum);
-        int found = -1;
-        unsigned long long before = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (found < 0 && cum + loc[t] > tau_m) {
-            found = lane * 8 + t;
-            before = cum;
+        // below + (mass of the whole group) > tau_m, so some lane qualifies
+        const unsigned hitb = __ballot_sync(0xffffffffu, lane < ncand && below + cw > tau_m);
+        kstar = __shfl_sync(0xffffffffu, key, __ffs(hitb) - 1);
+      } else {
+        for (int bit = 19; bit >= 0; --bit) {
+          const uint32_t c = prefix | (1u << bit);
+          const unsigned long long sm_ = mass_below(c);
+          if (sm_ <= tau_m) {
+            prefix = c;
+            below = sm_;
           }
-          cum += loc[t];
         }
-        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
-        const int win = __ffs(ball) - 1;  // ball != 0: the range's cumulative mass exceeds tau_m
-        const int bin = __shfl_sync(0xffffffffu, found, win);
-        below = __shfl_sync(0xffffffffu, before, win);
-        prefix |= static_cast<uint32_t>(bin) << shift;
-        pmask |= 255u << shift;
-        __syncwarp();
-      }
-      // Equal values at e*: the boundary is the m-th smallest index among them.
-      const unsigned long long wstar = mass_fixed(__uint_as_float(prefix));
-      const unsigned long long need = (tau_m - below) / wstar + 1ull;
-      unsigned long long seen = 0;
-      int jstar = Nb;
-      for (int base = 0; base < Nb; base += 32) {
-        const int j = base + lane;
-        const bool hit = j < Nb && __float_as_uint(row[j]) == prefix;
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        const unsigned c = __popc(bal);
-        if (seen + c >= need) {
-          unsigned bb = bal;
-          for (unsigned long long s = seen + 1; s < need; ++s) bb &= bb - 1;  // drop lower hits
-          jstar = base + __ffs(bb) - 1;
-          break;
+        // Equal values at e*: the boundary is the m-th smallest index among them.
+        const unsigned long long wstar = mass_bits(prefix);
+        const unsigned long long need = (tau_m - below) / wstar + 1ull;
+        unsigned long long seen = 0;
+        int jstar = Nb;
+        for (int base = 0; base < Nb; base += 32) {
+          const int j = base + lane;
+          const bool hit = j < Nb && __float_as_uint(row[j]) == prefix;
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
+          const unsigned c = __popc(bal);
+          if (seen + c >= need) {
+            unsigned bb = bal;
+            for (unsigned long long t = seen + 1; t < need; ++t) bb &= bb - 1;  // drop lower hits
+            jstar = base + __ffs(bb) - 1;
+            break;
+          }
+          seen += c;
         }
-        seen += c;
+        kstar = (static_cast<unsigned long long>(prefix) << 32) | static_cast<unsigned>(jstar);
       }
-      kstar = (static_cast<unsigned long long>(prefix) << 32) | static_cast<unsigned>(jstar);
+      __syncwarp();
     }
 
     // 4. union with the STA window and compaction

@@ -121,7 +121,7 @@ int permute(const void* in, void* out, int B, int T, int H, int W, int P, int ro
 }
 
 size_t mask_smem_bytes(int R, int D, int Nb) {
-  return static_cast<size_t>(R) * D * 4 + static_cast<size_t>(R) * Nb * 4 + kMaskWarps * 256 * 8;
+  return static_cast<size_t>(R) * D * 4 + static_cast<size_t>(R) * Nb * 4 + kMaskWarps * 32 * 4;
 }
 
 template <int R>
