@@ -40,6 +40,7 @@ CONFIGS = {
     "hunyuan": inputs.HUNYUAN,
     "long": inputs.LONG,
 }
+CONFIGS.update({f"sweep-a{w.alpha}-t{w.thr}": w for w in inputs.sweep_points()})
 L2_FLUSH_BYTES = 256 << 20
 
 

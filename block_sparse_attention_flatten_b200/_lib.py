@@ -37,6 +37,7 @@ EXPORTS = (
     "nabla_sparse_attn_fwd",
     "nabla_get_status",
     "nabla_validate_mask",
+    "nabla_selftest_wait_timeout",
     "nabla_strerror",
 )
 
@@ -81,6 +82,7 @@ def lib():
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
         L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
+        L.nabla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
         L.nabla_strerror.argtypes = [i]
         L.nabla_strerror.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -228,6 +230,13 @@ def validate_mask(kv_count: torch.Tensor, kv_idx: torch.Tensor, stream=None) -> 
                                      B, Hh, Nb, _dev(bad, torch.int32, "bad_rows"), _stream(stream)),
            "nabla_validate_mask")
     return int(bad.item())
+
+
+def selftest_wait_timeout(limit_cycles: int = 2_000_000, stream=None) -> int:
+    """Run the bounded-wait self-test and return the status it leaves
+    (synchronises; NABLA_ERR_DEVICE_TIMEOUT when the wait gave up)."""
+    _check(lib().nabla_selftest_wait_timeout(int(limit_cycles), _stream(stream)), "nabla_selftest_wait_timeout")
+    return get_status(stream)
 
 
 def default_scale(D: int) -> float:

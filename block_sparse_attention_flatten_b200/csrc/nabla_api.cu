@@ -136,6 +136,21 @@ int launch_mask(const MaskArgs& a, int B, const DeviceInfo& di, cudaStream_t str
   return launch_status();
 }
 
+// Failure-detection self-test: every thread of one CTA waits on an mbarrier
+// nothing arrives on, with the kernels' bounded wait and a short limit.
+__global__ void wait_timeout_selftest_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait_limit(&bar, 0, &abort_flag, limit);
+  __syncthreads();
+}
+
 // Scratch of nabla_build_mask_noalloc: the pooled queries then keys.  In host
 // code this name is only a stand-in for the device symbol; its device address
 // comes from cudaGetSymbolAddress, once per device.
@@ -300,6 +315,12 @@ int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int 
     scratch = g_noalloc_ptr[dev];
   }
   return nabla_build_mask(qf, kf, B, Hh, D, T, H, W, params, kv_count, kv_idx, scratch, stream);
+}
+
+int nabla_selftest_wait_timeout(long long limit_cycles, nabla_stream_t stream_) {
+  if (limit_cycles < 1000 || limit_cycles > kWaitLimitCycles) return NABLA_ERR_INVALID;
+  wait_timeout_selftest_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream_)>>>(limit_cycles);
+  return launch_status();
 }
 
 int nabla_get_status(nabla_stream_t stream_) {

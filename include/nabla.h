@@ -168,6 +168,15 @@ int nabla_get_status(nabla_stream_t stream);
 int nabla_validate_mask(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb,
                         int32_t* bad_rows, nabla_stream_t stream);
 
+/* Failure-detection self-test (no counterpart in the paper): launches one CTA
+ * whose threads wait on an mbarrier that nothing arrives on, using the same
+ * bounded wait as the kernels with a limit of limit_cycles SM cycles
+ * (1000 .. 4e9).  The wait gives up, records NABLA_ERR_DEVICE_TIMEOUT in the
+ * status word and the kernel returns normally, so the context stays usable;
+ * read the code with nabla_get_status.  NABLA_ERR_INVALID for a limit out of
+ * range. */
+int nabla_selftest_wait_timeout(long long limit_cycles, nabla_stream_t stream);
+
 /* Static description of an error code. */
 const char* nabla_strerror(int code);
 

@@ -86,6 +86,11 @@ def test_invalid_arguments_rejected_before_launch(lib):
                                    s) == nabla.NABLA_ERR_INVALID
 
 
+def test_selftest_rejects_out_of_range_limits(lib):
+    assert lib.nabla_selftest_wait_timeout(10, None) == nabla.NABLA_ERR_INVALID
+    assert lib.nabla_selftest_wait_timeout(10 ** 12, None) == nabla.NABLA_ERR_INVALID
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     x = torch.zeros(1, 64, 8, dtype=torch.bfloat16)

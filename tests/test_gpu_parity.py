@@ -201,3 +201,15 @@ def test_stream_argument_is_honoured():
     case = Case(w, q, k, v)
     out2, _ = case.attention()
     assert torch.equal(out, out2) and torch.equal(cnt, case.kv_count)
+
+
+def test_bounded_wait_times_out_without_faulting():
+    """A wait on a barrier nothing completes gives up after its limit, records
+    NABLA_ERR_DEVICE_TIMEOUT, and leaves the context usable."""
+    assert nabla.get_status() == 0
+    assert nabla.selftest_wait_timeout(2_000_000) == nabla.NABLA_ERR_DEVICE_TIMEOUT
+    assert nabla.get_status() == 0  # read-and-clear
+    w = inputs.Workload("after timeout", 1, 2, 64, 1, 8, 16, 0.0, 0.9, seed=51)
+    case = Case(w)
+    out, lse = case.attention()
+    assert torch.isfinite(out.float()).all()
