@@ -166,7 +166,7 @@ def run_gpu(args, rank, world, local_rank):
         nabla.build_mask(qf, kf, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx, workspace=ws)
         if ev is not None:
             ev[2].record(stream)
-        nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=of, lse=lse)
+        nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=of, lse=lse, grid=(w.T, w.H, w.W))
         if ev is not None:
             ev[3].record(stream)
         nabla.unflatten(of, w.T, w.H, w.W, out=og)

@@ -7,7 +7,7 @@ provides device memory and streams.
     from block_sparse_attention_flatten_b200 import nabla
     qf = nabla.flatten(q, T, H, W)                       # per tensor, once per sequence
     kv_count, kv_idx, _ = nabla.build_mask(qf, kf, T, H, W, thr=0.9, sta=(3, 3, 3))
-    of, lse = nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx)
+    of, lse = nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, grid=(T, H, W))
     o = nabla.unflatten(of, T, H, W)
 """
 from . import _lib as nabla  # noqa: F401

@@ -35,6 +35,7 @@ EXPORTS = (
     "nabla_build_mask",
     "nabla_build_mask_noalloc",
     "nabla_sparse_attn_fwd",
+    "nabla_sparse_attn_fwd_grid",
     "nabla_get_status",
     "nabla_validate_mask",
     "nabla_selftest_wait_timeout",
@@ -80,6 +81,7 @@ def lib():
         L.nabla_build_mask.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
         L.nabla_build_mask_noalloc.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
+        L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
         L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
         L.nabla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
@@ -193,27 +195,43 @@ def build_mask_noalloc(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: in
 
 
 def pooled_from_workspace(workspace: torch.Tensor, B: int, Hh: int, Nb: int, D: int):
-    """Views of qbar and kbar inside a mask workspace."""
+    """qbar [B,Hh,Nb,D] and kbar [B,Hh,Nb,D] from a mask workspace (kbar is
+    stored transposed, [B,Hh,D,Nbp] with Nbp = Nb rounded up to 4; the
+    returned kbar is a strided view of its first Nb columns)."""
     f = workspace.view(torch.float32)
     n = B * Hh * Nb * D
-    return f[:n].view(B, Hh, Nb, D), f[n:2 * n].view(B, Hh, Nb, D)
+    nbp = (Nb + 3) // 4 * 4
+    kt = f[n:n + B * Hh * D * nbp].view(B, Hh, D, nbp)
+    return f[:n].view(B, Hh, Nb, D), kt[..., :Nb].transpose(2, 3)
 
 
 def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_count: torch.Tensor,
                     kv_idx: torch.Tensor, scale: float = 0.0, out=None, lse=None, want_lse: bool = True,
-                    stream=None):
-    """Block-sparse attention on the kept tiles; returns (out, lse or None)."""
+                    stream=None, grid=None):
+    """Block-sparse attention on the kept tiles; returns (out, lse or None).
+
+    grid = (T, H, W) of the flattened tokens calls nabla_sparse_attn_fwd_grid,
+    which pairs query blocks by their lists' overlap; None calls
+    nabla_sparse_attn_fwd (pairs 2p, 2p+1)."""
     B, S, Hh, D = qf.shape
     if out is None:
         out = torch.empty_like(qf)
     if lse is None and want_lse:
         lse = torch.empty((B, Hh, S), dtype=torch.float32, device=qf.device)
     lse_p = _dev(lse, torch.float32, "lse") if lse is not None else None
-    _check(lib().nabla_sparse_attn_fwd(_dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"),
-                                       _dev(vf, torch.bfloat16, "vf"), _dev(kv_count, torch.int32, "kv_count"),
-                                       _dev(kv_idx, torch.int32, "kv_idx"), B, S, Hh, D, float(scale),
-                                       _dev(out, torch.bfloat16, "out"), lse_p, _stream(stream)),
-           "nabla_sparse_attn_fwd")
+    ptrs = (_dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"), _dev(vf, torch.bfloat16, "vf"),
+            _dev(kv_count, torch.int32, "kv_count"), _dev(kv_idx, torch.int32, "kv_idx"))
+    o_p = _dev(out, torch.bfloat16, "out")
+    if grid is None:
+        _check(lib().nabla_sparse_attn_fwd(*ptrs, B, S, Hh, D, float(scale), o_p, lse_p, _stream(stream)),
+               "nabla_sparse_attn_fwd")
+    else:
+        T, H, W = (int(x) for x in grid)
+        if T * H * W != S:
+            raise ValueError(f"grid {grid} does not hold {S} tokens")
+        _check(lib().nabla_sparse_attn_fwd_grid(*ptrs, B, Hh, D, T, H, W, float(scale), o_p, lse_p,
+                                                _stream(stream)),
+               "nabla_sparse_attn_fwd_grid")
     return out, lse
 
 

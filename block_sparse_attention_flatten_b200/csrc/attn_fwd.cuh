@@ -3,12 +3,20 @@
 // listed N x N blocks are computed; a dropped block is in neither the
 // numerator nor the softmax normaliser).
 //
-// One CTA owns a query tile of 128 rows = two consecutive 64-token query
-// blocks (2p, 2p+1) of one (batch, head), so every tcgen05.mma runs at the
-// full M = 128.  It walks the ascending union of the two blocks' key-block
-// lists; a key block listed by only one of them is masked for the other
-// half's rows (their probabilities are set to zero and their running max and
-// sum are left alone).
+// One CTA owns a query tile of 128 rows = two 64-token query blocks of one
+// (batch, head), so every tcgen05.mma runs at the full M = 128.  It walks the
+// ascending union of the two blocks' key-block lists; a key block listed by
+// only one of them is masked for the other half's rows (their probabilities
+// are set to zero and their running max and sum are left alone).  Which two
+// blocks share a CTA decides how many masked half-tiles it runs:
+//   - without the token grid, blocks 2p and 2p+1 of the flattened order
+//     (horizontally adjacent patches of one frame);
+//   - with the grid, each 2 x 2 group {(t, w), (t, w+1), (t+1, w), (t+1, w+1)}
+//     of patch positions (same patch row, two frames) is split into two CTAs
+//     either along w or along t, whichever pairing has the smaller total
+//     union of lists.  Both CTAs of a group take the same decision from the
+//     same four lists; one block of each CTA is the same under both pairings,
+//     so its half of Q is loaded before the lists are read.
 //
 // Warp roles (192 threads, two CTAs per SM):
 //   warps 0-3  softmax: thread t owns query row t = TMEM lane t.  Reads the
@@ -51,12 +59,14 @@ struct AttnSmem {
   static constexpr int kBars = kV + kStages * kKVBytes;
   // q, k full + empty, v full + empty, s full, p full, pv done, mma drain
   static constexpr int kNumBars = 1 + 4 * kStages + 2 * 3 + 1;
-  static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, abort flag, list length
-  static constexpr int kList = kMisc + 16;
+  // tmem base, abort flag, list length, the two query blocks
+  static constexpr int kMisc = kBars + 8 * kNumBars;
+  static constexpr int kList = kMisc + 32;
   __host__ __device__ static size_t list_bytes(int Nb) { return (static_cast<size_t>(Nb) * 2 + 15) & ~size_t(15); }
+  // followed by four key-block bitmaps of (Nb + 31) / 32 words
   static size_t bytes(int Nb) {
     const int words = (Nb + 31) / 32;
-    return 1024 + kList + list_bytes(Nb) + 2 * static_cast<size_t>(words) * 4;
+    return 1024 + kList + list_bytes(Nb) + 4 * static_cast<size_t>(words) * 4;
   }
 };
 
@@ -66,6 +76,8 @@ struct AttnArgs {
   __nv_bfloat16* out;       // [B][S][Hh][D]
   float* lse;               // [B][Hh][S] or null
   int S, Hh, Nb;
+  int grp_F;                // query blocks per frame for 2 x 2 (w, t) grouping, 0 = pairs 2p, 2p+1
+  int grp_nbw;              // blocks per patch row (W / 8) when grp_F > 0
   float scale_log2;         // scale * log2(e)
 };
 
@@ -90,16 +102,37 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
   int* list_len = reinterpret_cast<int*>(sm + L::kMisc + 8);
+  int* half_blk = reinterpret_cast<int*>(sm + L::kMisc + 12);  // [2]; -1 = no block
   uint16_t* list = reinterpret_cast<uint16_t*>(sm + L::kList);
   const int Nb = a.Nb;
   const int words = (Nb + 31) >> 5;
-  uint32_t* bm0 = reinterpret_cast<uint32_t*>(sm + L::kList + L::list_bytes(Nb));
-  uint32_t* bm1 = bm0 + words;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(sm + L::kList + L::list_bytes(Nb));  // [4][words]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int pair = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
-  const int blk0 = 2 * pair, blk1 = 2 * pair + 1;
+  const int p = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
+
+  // Candidate query blocks.  Group mode: cand = {(t,w), (t,w+1), (t+1,w),
+  // (t+1,w+1)}; CTA slot 0 owns cand[0] in half 0 and slot 1 owns cand[3] in
+  // half 1; the other half is cand[1] or cand[2] (see the decision below).
+  // Pair mode: cand = {2p, 2p+1} in halves 0 and 1.
+  const bool grouped = a.grp_F > 0;
+  const int slot = p & 1;
+  int cand[4];
+  if (grouped) {
+    const int g = p >> 1, ngw = a.grp_nbw >> 1, nbh = a.grp_F / a.grp_nbw;
+    const int bw2 = g % ngw, rest = g / ngw;
+    const int a0 = 2 * (rest / nbh) * a.grp_F + (rest % nbh) * a.grp_nbw + 2 * bw2;
+    cand[0] = a0;
+    cand[1] = a0 + 1;
+    cand[2] = a0 + a.grp_F;
+    cand[3] = a0 + a.grp_F + 1;
+  } else {
+    cand[0] = 2 * p;
+    cand[1] = 2 * p + 1 < Nb ? 2 * p + 1 : -1;
+    cand[2] = cand[3] = -1;
+  }
+  const int nlists = grouped ? 4 : 2;
 
   // ---- set-up: barriers, tensor memory, merged block list
   if (tid == 0) {
@@ -118,11 +151,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // Q does not depend on the block lists: start its load right away.
+    // The half of Q whose block is already known loads right away; in pair
+    // mode both halves do (a missing second block loads the first one again:
+    // its rows are never listed and never stored).
     tma_prefetch_desc(&tmQ);
     mbar_arrive_expect_tx(q_full, L::kQBytes);
-    for (int c = 0; c < L::kChunks; ++c)
-      tma_load_4d(sm + L::kQ + c * 128 * 128, &tmQ, q_full, c * 64, hd, pair * 128, b);
+    if (grouped) {
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_4d(sm + L::kQ + c * 128 * 128 + slot * 64 * 128, &tmQ, q_full, c * 64, hd,
+                    cand[slot ? 3 : 0] * 64, b);
+    } else {
+      const int q1 = cand[1] >= 0 ? cand[1] : cand[0];
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_4d(sm + L::kQ + c * 128 * 128, &tmQ, q_full, c * 64, hd, cand[0] * 64, b);
+        tma_load_4d(sm + L::kQ + c * 128 * 128 + 64 * 128, &tmQ, q_full, c * 64, hd, q1 * 64, b);
+      }
+    }
   }
   if (warp == 4) {
     tmem_alloc(tmem_slot, 256);
@@ -132,29 +176,71 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tma_prefetch_desc(&tmV);
     }
   }
-  for (int w = tid; w < 2 * words; w += kAttnThreads) bm0[w] = 0u;
+  // The counts and the first kAttnThreads entries of every list are loaded
+  // together (entries past a row's count are read and ignored; a row has Nb
+  // entries), so the list set-up waits for one memory latency, not two.
+  int cnt[4], first[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const bool have = h < nlists && cand[h] >= 0;
+    const int64_t row = bh * Nb + (have ? cand[h] : 0);
+    cnt[h] = have ? __ldg(a.kv_count + row) : 0;
+    first[h] = (have && tid < Nb) ? __ldg(a.kv_idx + row * Nb + tid) : 0;
+  }
+  for (int w = tid; w < 4 * words; w += kAttnThreads) bm[w] = 0u;
   __syncthreads();
-  for (int half = 0; half < 2; ++half) {
-    const int blk = half == 0 ? blk0 : blk1;
-    if (blk >= Nb) continue;
-    int cnt = a.kv_count[bh * Nb + blk];
-    if (cnt < 0 || cnt > Nb) {
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    int c = cnt[h];
+    if (c < 0 || c > Nb) {
       if (tid == 0) report(NABLA_ERR_DEVICE_BOUNDS);
-      cnt = cnt < 0 ? 0 : Nb;
+      c = c < 0 ? 0 : Nb;
     }
-    const int32_t* src = a.kv_idx + (bh * Nb + blk) * static_cast<int64_t>(Nb);
-    uint32_t* bm = half == 0 ? bm0 : bm1;
-    for (int e = tid; e < cnt; e += kAttnThreads) {
-      const int j = src[e];
+    uint32_t* bmh = bm + h * words;
+    const int32_t* src = a.kv_idx + (bh * Nb + (cand[h] >= 0 ? cand[h] : 0)) * static_cast<int64_t>(Nb);
+    for (int e = tid; e < c; e += kAttnThreads) {
+      const int j = e == tid ? first[h] : src[e];
       if (j < 0 || j >= Nb) {
         report(NABLA_ERR_DEVICE_BOUNDS);
         continue;
       }
-      atomicOr(bm + (j >> 5), 1u << (j & 31));
+      atomicOr(bmh + (j >> 5), 1u << (j & 31));
     }
   }
   __syncthreads();
   if (warp == 0) {
+    int x_half0 = 0, x_half1 = 1;  // which candidate (bitmap) each half holds
+    if (grouped) {
+      // Split along t when the two unions along t hold fewer blocks in total
+      // than the two along w.
+      int cw = 0, ct = 0;
+      for (int w = lane; w < words; w += 32) {
+        const uint32_t b0 = bm[w], b1 = bm[words + w], b2 = bm[2 * words + w], b3 = bm[3 * words + w];
+        cw += __popc(b0 | b1) + __popc(b2 | b3);
+        ct += __popc(b0 | b2) + __popc(b1 | b3);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        cw += __shfl_xor_sync(0xffffffffu, cw, o);
+        ct += __shfl_xor_sync(0xffffffffu, ct, o);
+      }
+      const bool along_t = ct < cw;
+      x_half0 = slot == 0 ? 0 : (along_t ? 1 : 2);
+      x_half1 = slot == 0 ? (along_t ? 2 : 1) : 3;
+      if (lane == 0) {
+        // the other half of Q; q_full already expects its bytes
+        const int other = slot ? x_half0 : x_half1;
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_4d(sm + L::kQ + c * 128 * 128 + (slot ? 0 : 64 * 128), &tmQ, q_full, c * 64, hd,
+                      cand[other] * 64, b);
+      }
+    }
+    if (lane == 0) {
+      half_blk[0] = cand[x_half0];
+      half_blk[1] = cand[x_half1];
+    }
+    const uint32_t* bm0 = bm + x_half0 * words;
+    const uint32_t* bm1 = bm + x_half1 * words;
     int base = 0;
     for (int w0 = 0; w0 < words; w0 += 32) {
       const int w = w0 + lane;
@@ -362,8 +448,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
 
     // ---------------------------------------------------------------- epilogue
-    const int64_t row_g = static_cast<int64_t>(pair) * 128 + r;
-    const bool row_valid = row_g < a.S;
+    const int qblk = half_blk[r >> 6];
+    const bool row_valid = qblk >= 0;
+    const int64_t row_g = static_cast<int64_t>(row_valid ? qblk : 0) * 64 + (r & 63);
     if (ok && L_n > 0) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((L_n - 1) & 1), ((L_n - 1) >> 1) & 1, abort_flag));
     tc_fence_after();
     __syncwarp();

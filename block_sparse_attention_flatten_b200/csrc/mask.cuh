@@ -12,10 +12,11 @@
 //      the masses are integers e * 2^40, so every partial sum is exact and
 //      independent of summation order;
 //   3. the CDF rule "keep where the ascending cumulative mass exceeds 1 - thr"
-//      without a full sort: a binary search over the fp32 bit patterns of e
-//      with warp-summed exact masses finds the boundary element (e*, j*) of
-//      the ascending (e, j) order (shared-memory histograms with atomics
-//      serialise on the few bins most masses fall into);
+//      without a full sort: a search over the fp32 bit patterns of e, two
+//      bits per pass, with warp-summed exact masses finds the boundary
+//      element (e*, j*) of the ascending (e, j) order (shared-memory
+//      histograms with atomics serialise on the few bins most masses fall
+//      into);
 //   4. keep = (e, j) >= (e*, j*)  OR arg-max  OR STA window, compacted with
 //      warp ballots into ascending kv_idx and kv_count.
 #pragma once
@@ -25,7 +26,9 @@
 namespace nabla {
 
 // ------------------------------------------------------------------ pooling
-// grid (Nb, B, 2): z = 0 pools Q into qbar, z = 1 pools K into kbar.
+// grid (Nb, B, 2): z = 0 pools Q into qbar [B][Hh][Nb][D], z = 1 pools K
+// into kbar^T [B][Hh][D][Nbp] (Nbp = Nb rounded up to a multiple of 4; the
+// padding columns are never written).
 // Thread c handles elements 8c..8c+7 of a token row (Hh*D elements), summing
 // the block's 64 rows in ascending order in fp32.
 __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restrict__ q,
@@ -60,9 +63,18 @@ __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restri
     }
     const int col = c * 8;
     const int h = col / D, d = col - h * D;
-    float4* o = reinterpret_cast<float4*>(out + ((static_cast<int64_t>(b) * Hh + h) * Nb + i) * D + d);
-    o[0] = make_float4(acc[0] * (1.f / 64.f), acc[1] * (1.f / 64.f), acc[2] * (1.f / 64.f), acc[3] * (1.f / 64.f));
-    o[1] = make_float4(acc[4] * (1.f / 64.f), acc[5] * (1.f / 64.f), acc[6] * (1.f / 64.f), acc[7] * (1.f / 64.f));
+    if (blockIdx.z == 0) {
+      float4* o = reinterpret_cast<float4*>(out + ((static_cast<int64_t>(b) * Hh + h) * Nb + i) * D + d);
+      o[0] = make_float4(acc[0] * (1.f / 64.f), acc[1] * (1.f / 64.f), acc[2] * (1.f / 64.f), acc[3] * (1.f / 64.f));
+      o[1] = make_float4(acc[4] * (1.f / 64.f), acc[5] * (1.f / 64.f), acc[6] * (1.f / 64.f), acc[7] * (1.f / 64.f));
+    } else {
+      // keys transposed: kbar^T [B][Hh][D][Nbp], so the score phase reads
+      // them coalesced along the key blocks
+      const int Nbp = (Nb + 3) & ~3;
+      float* o = out + ((static_cast<int64_t>(b) * Hh + h) * D + d) * Nbp + i;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[static_cast<int64_t>(e) * Nbp] = acc[e] * (1.f / 64.f);
+    }
   }
 }
 
@@ -81,8 +93,20 @@ struct MaskArgs {
   double tau;         // 1 - thr (exact in double)
 };
 
-constexpr int kMaskThreads = 512;
+constexpr int kMaskThreads = 256;
 constexpr int kMaskWarps = kMaskThreads / 32;
+constexpr int kMaskCols = 2;  // adjacent key blocks per thread in the score phase
+
+// Column count of the transposed pooled keys kbar^T [D][Nbp]: Nb rounded up
+// to a multiple of 4 so every thread's pair of columns is an aligned 8-byte
+// load.
+__host__ __device__ inline int kbar_cols(int Nb) { return (Nb + 3) & ~3; }
+
+// d = a * b + d on two fp32 lanes at once; each lane is one fmaf (round to
+// nearest even), so a lane's chain of these equals the scalar fmaf chain.
+__device__ __forceinline__ void ffma2(unsigned long long& d, unsigned long long a, unsigned long long b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
 
 // Integer mass of an unnormalised probability e in [0, 1], from its bit
 // pattern u: floor(e * 2^40) (exact for e >= 2^-16; smaller masses lose
@@ -95,49 +119,74 @@ __device__ __forceinline__ unsigned long long mass_bits(uint32_t u) {
   return sh >= 0 ? (m24 << sh) : (sh > -24 ? (m24 >> -sh) : 0ull);
 }
 
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// R query-block rows per CTA, 256 threads.  Shared memory: q pairs [D][R]
+// (each fp32 qbar value twice, the second operand of a two-lane FMA), score
+// rows [R][Nb], per-warp candidate slots.
 template <int R>
 __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int D = a.D, Nb = a.Nb;
-  float* qs = reinterpret_cast<float*>(smem_raw);                       // [R][D]
-  float* rows = qs + R * D;                                             // [R][Nb]
-  int* cand_all = reinterpret_cast<int*>(rows + static_cast<size_t>(R) * Nb);  // [warps][32]
+  const int D = a.D, Nb = a.Nb, Nbp = kbar_cols(Nb);
+  unsigned long long* qd = reinterpret_cast<unsigned long long*>(smem_raw);          // [D][R]
+  float* rows = reinterpret_cast<float*>(qd + static_cast<size_t>(R) * D);          // [R][Nb]
+  int* cand_all = reinterpret_cast<int*>(rows + static_cast<size_t>(R) * Nb);      // [warps][32]
 
   const int i0 = blockIdx.x * R;
   const int hd = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
   const float* qb = a.qbar + (bh * Nb + i0) * D;
-  const float* kb = a.kbar + bh * Nb * D;
+  const float* kt = a.kbar + bh * static_cast<int64_t>(D) * Nbp;  // kbar^T [D][Nbp]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   for (int e = tid; e < R * D; e += kMaskThreads) {
-    const int r = e / D;
-    qs[e] = (i0 + r < Nb) ? qb[e] : 0.f;
+    const int r = e / D, d = e - r * D;
+    const uint32_t u = __float_as_uint((i0 + r < Nb) ? qb[e] : 0.f);
+    qd[d * R + r] = (static_cast<unsigned long long>(u) << 32) | u;
   }
   __syncthreads();
 
-  // 1. scores: one fused multiply-add chain per (row, block) over d ascending
-  for (int j = tid; j < Nb; j += kMaskThreads) {
-    float acc[R];
+  // 1. scores: thread owns key blocks j, j+1 and all R rows; per (row, block)
+  //    one fused multiply-add chain over d ascending (the oracle's order),
+  //    two blocks per instruction.  kbar^T rows are read coalesced, eight d
+  //    ahead of use.
+  for (int j = tid * kMaskCols; j < Nb; j += kMaskThreads * kMaskCols) {
+    unsigned long long acc[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    const float4* kp = reinterpret_cast<const float4*>(kb + static_cast<int64_t>(j) * D);
-#pragma unroll 2
-    for (int d4 = 0; d4 < (D >> 2); ++d4) {
-      const float4 kv = __ldg(kp + d4);
+    for (int r = 0; r < R; ++r) acc[r] = 0ull;
+    const unsigned long long* kp = reinterpret_cast<const unsigned long long*>(kt + j);
+    const int kstride = Nbp / 2;  // in column pairs
+    unsigned long long kv[8];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float4 qv = reinterpret_cast<const float4*>(qs + r * D)[d4];
-        float t = acc[r];
-        t = fmaf(qv.x, kv.x, t);
-        t = fmaf(qv.y, kv.y, t);
-        t = fmaf(qv.z, kv.z, t);
-        t = fmaf(qv.w, kv.w, t);
-        acc[r] = t;
+    for (int u = 0; u < 8; ++u) kv[u] = __ldg(kp + static_cast<int64_t>(u) * kstride);
+    for (int d0 = 0; d0 < D; d0 += 8) {
+      unsigned long long kn[8];
+      const bool more = d0 + 8 < D;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) kn[u] = more ? __ldg(kp + static_cast<int64_t>(d0 + 8 + u) * kstride) : 0ull;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const ulonglong2* qrow = reinterpret_cast<const ulonglong2*>(qd + (d0 + u) * R);
+#pragma unroll
+        for (int r2 = 0; r2 < R / 2; ++r2) {
+          const ulonglong2 qq = qrow[r2];
+          ffma2(acc[2 * r2], kv[u], qq.x);
+          ffma2(acc[2 * r2 + 1], kv[u], qq.y);
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) kv[u] = kn[u];
     }
 #pragma unroll
-    for (int r = 0; r < R; ++r) rows[static_cast<size_t>(r) * Nb + j] = acc[r] * a.scale;
+    for (int r = 0; r < R; ++r) {
+      float* row = rows + static_cast<size_t>(r) * Nb;
+      row[j] = __uint_as_float(static_cast<uint32_t>(acc[r])) * a.scale;
+      if (j + 1 < Nb) row[j + 1] = __uint_as_float(static_cast<uint32_t>(acc[r] >> 32)) * a.scale;
+    }
   }
   __syncthreads();
 
@@ -167,8 +216,8 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     for (int o = 16; o > 0; o >>= 1) {
       const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
       best = ob > best ? ob : best;
-      total += __shfl_xor_sync(0xffffffffu, total, o);
     }
+    total = warp_sum_u64(total);
     const int argmax = static_cast<int>(best & 0xffffffffu);
     const unsigned long long tau_m =
         static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
@@ -176,32 +225,55 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     // 3. CDF boundary: the element (e*, j*) of the ascending (e, j) order at
     //    which the cumulative mass first exceeds tau_m; keep (e, j) >= it.
     //    bits(e*) is the largest bit pattern x with mass(bits(e) < x) <= tau_m
-    //    (positive floats order like their bit patterns), found MSB first by
-    //    a binary search of exact warp-summed masses (no atomics).  After the
-    //    top 11 bits, if at most 32 blocks share them they are sorted by a
-    //    warp bitonic sort and the boundary read off their prefix sums.
+    //    (positive floats order like their bit patterns), found MSB first,
+    //    two bits per pass: each pass sums the exact masses below three
+    //    probes at once (warp sums, no atomics).  After the top 11 bits, if
+    //    at most 32 blocks share them they are sorted by a warp bitonic sort
+    //    and the boundary read off their prefix sums.
     unsigned long long kstar = ~0ull;
     if (!a.keep_all && total > tau_m) {
       uint32_t prefix = 0;
       unsigned long long below = 0;  // mass(bits(e) < prefix)
-      auto mass_below = [&](uint32_t x) -> unsigned long long {
-        unsigned long long sum = 0;
+      // Extends prefix by the bits [lo, hi] (one or two bits).
+      auto refine = [&](int hi, int lo) {
+        if (hi == lo) {
+          const uint32_t c = prefix | (1u << hi);
+          unsigned long long s = 0;
+          for (int j = lane; j < Nb; j += 32) {
+            const uint32_t u = __float_as_uint(row[j]);
+            if (u < c) s += mass_bits(u);
+          }
+          s = warp_sum_u64(s);
+          if (s <= tau_m) {
+            prefix = c;
+            below = s;
+          }
+          return;
+        }
+        const uint32_t c1 = prefix | (1u << lo), c2 = prefix | (2u << lo), c3 = prefix | (3u << lo);
+        unsigned long long s1 = 0, s2 = 0, s3 = 0;
         for (int j = lane; j < Nb; j += 32) {
           const uint32_t u = __float_as_uint(row[j]);
-          if (u < x) sum += mass_bits(u);
+          const unsigned long long w = mass_bits(u);
+          if (u < c1) s1 += w;
+          if (u < c2) s2 += w;
+          if (u < c3) s3 += w;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        return sum;
+        s1 = warp_sum_u64(s1);
+        s2 = warp_sum_u64(s2);
+        s3 = warp_sum_u64(s3);
+        if (s3 <= tau_m) {
+          prefix = c3;
+          below = s3;
+        } else if (s2 <= tau_m) {
+          prefix = c2;
+          below = s2;
+        } else if (s1 <= tau_m) {
+          prefix = c1;
+          below = s1;
+        }
       };
-      for (int bit = 30; bit >= 20; --bit) {
-        const uint32_t c = prefix | (1u << bit);
-        const unsigned long long sm_ = mass_below(c);
-        if (sm_ <= tau_m) {
-          prefix = c;
-          below = sm_;
-        }
-      }
+      for (int hi = 30; hi >= 20; hi -= 2) refine(hi, hi > 20 ? hi - 1 : hi);
       // e* lies in [prefix, prefix + 2^20): gather those blocks (ascending j).
       int ncand = 0;
       for (int base = 0; base < Nb && ncand <= 32; base += 32) {
@@ -246,14 +318,7 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
         const unsigned hitb = __ballot_sync(0xffffffffu, lane < ncand && below + cw > tau_m);
         kstar = __shfl_sync(0xffffffffu, key, __ffs(hitb) - 1);
       } else {
-        for (int bit = 19; bit >= 0; --bit) {
-          const uint32_t c = prefix | (1u << bit);
-          const unsigned long long sm_ = mass_below(c);
-          if (sm_ <= tau_m) {
-            prefix = c;
-            below = sm_;
-          }
-        }
+        for (int hi = 19; hi >= 0; hi -= 2) refine(hi, hi - 1);
         // Equal values at e*: the boundary is the m-th smallest index among them.
         const unsigned long long wstar = mass_bits(prefix);
         const unsigned long long need = (tau_m - below) / wstar + 1ull;

@@ -121,7 +121,7 @@ int permute(const void* in, void* out, int B, int T, int H, int W, int P, int ro
 }
 
 size_t mask_smem_bytes(int R, int D, int Nb) {
-  return static_cast<size_t>(R) * D * 4 + static_cast<size_t>(R) * Nb * 4 + kMaskWarps * 32 * 4;
+  return static_cast<size_t>(R) * D * 8 + static_cast<size_t>(R) * Nb * 4 + kMaskWarps * 32 * 4;
 }
 
 template <int R>
@@ -158,6 +158,62 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[NABLA_NOALLOC_SCRATCH_
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
+// Shared body of the two attention entry points; grp_F > 0 selects the 2 x 2
+// (w, t) grouping of query blocks (grp_F blocks per frame, grp_nbw per row).
+int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+                       const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
+                       int grp_F, int grp_nbw, cudaStream_t stream) {
+  if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
+  if (static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
+  if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
+  if (qf == nullptr || kf == nullptr || vf == nullptr || kv_count == nullptr || kv_idx == nullptr || out == nullptr)
+    return NABLA_ERR_INVALID;
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(vf) || !aligned16(out) || !aligned16(kv_idx) ||
+      !aligned16(kv_count))
+    return NABLA_ERR_ALIGN;
+  if (lse != nullptr && !aligned16(lse)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc != NABLA_OK) return rc;
+  if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
+  const int Nb = S / 64;
+  if (Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
+  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+
+  CUtensorMap tq, tk, tv;
+  if (!make_bshd_map(&tq, qf, B, S, Hh, D, 64) || !make_bshd_map(&tk, kf, B, S, Hh, D, 64) ||
+      !make_bshd_map(&tv, vf, B, S, Hh, D, 64))
+    return NABLA_ERR_CUDA;
+  AttnArgs a;
+  a.kv_count = kv_count;
+  a.kv_idx = kv_idx;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.S = S;
+  a.Hh = Hh;
+  a.Nb = Nb;
+  a.grp_F = grp_F;
+  a.grp_nbw = grp_nbw;
+  a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
+  const dim3 grid((Nb + 1) / 2, Hh, B);
+  if (D == 128) {
+    const size_t smem = AttnSmem<128>::bytes(Nb);
+    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
+    if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    attn_fwd_kernel<128><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    const size_t smem = AttnSmem<64>::bytes(Nb);
+    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
+    if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    attn_fwd_kernel<64><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
+  }
+  return launch_status();
+}
+
 }  // namespace
 }  // namespace nabla
 
@@ -179,7 +235,8 @@ size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W, con
   const int P = params ? params->P : 8;
   if (check_grid(B, T, H, W, P) != NABLA_OK || Hh <= 0 || (D != 64 && D != 128)) return 0;
   const size_t Nb = static_cast<size_t>(T) * H * W / 64;
-  return 2 * static_cast<size_t>(B) * Hh * Nb * D * sizeof(float);
+  const size_t Nbp = static_cast<size_t>(kbar_cols(static_cast<int>(Nb)));
+  return static_cast<size_t>(B) * Hh * (Nb + Nbp) * D * sizeof(float);
 }
 
 int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
@@ -245,55 +302,21 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
 
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
-                          nabla_stream_t stream_) {
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
-  if (static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
-  if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
-  if (qf == nullptr || kf == nullptr || vf == nullptr || kv_count == nullptr || kv_idx == nullptr || out == nullptr)
-    return NABLA_ERR_INVALID;
-  if (!aligned16(qf) || !aligned16(kf) || !aligned16(vf) || !aligned16(out) || !aligned16(kv_idx) ||
-      !aligned16(kv_count))
-    return NABLA_ERR_ALIGN;
-  if (lse != nullptr && !aligned16(lse)) return NABLA_ERR_ALIGN;
-  DeviceInfo di;
-  int rc = device_info(&di);
-  if (rc != NABLA_OK) return rc;
-  if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
-  const int Nb = S / 64;
-  if (Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
-  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+                          nabla_stream_t stream) {
+  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, S, Hh, D, scale, out, lse, 0, 0,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
 
-  CUtensorMap tq, tk, tv;
-  if (!make_bshd_map(&tq, qf, B, S, Hh, D, 128) || !make_bshd_map(&tk, kf, B, S, Hh, D, 64) ||
-      !make_bshd_map(&tv, vf, B, S, Hh, D, 64))
-    return NABLA_ERR_CUDA;
-  AttnArgs a;
-  a.kv_count = kv_count;
-  a.kv_idx = kv_idx;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.lse = lse;
-  a.S = S;
-  a.Hh = Hh;
-  a.Nb = Nb;
-  a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
-  const dim3 grid((Nb + 1) / 2, Hh, B);
-  if (D == 128) {
-    const size_t smem = AttnSmem<128>::bytes(Nb);
-    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return NABLA_ERR_CUDA;
-    attn_fwd_kernel<128><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
-  } else {
-    const size_t smem = AttnSmem<64>::bytes(Nb);
-    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return NABLA_ERR_CUDA;
-    attn_fwd_kernel<64><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
-  }
-  return launch_status();
+int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+                               const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
+                               void* out, float* lse, nabla_stream_t stream) {
+  if (T <= 0 || H <= 0 || W <= 0 || H % 8 != 0 || W % 8 != 0) return NABLA_ERR_INVALID;
+  const int64_t S = static_cast<int64_t>(T) * H * W;
+  if (S > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
+  const int nbw = W / 8, F = (H / 8) * nbw;
+  const bool groups = T % 2 == 0 && nbw % 2 == 0;
+  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
+                            groups ? F : 0, groups ? nbw : 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,

@@ -85,9 +85,10 @@ int nabla_flatten(const void* in, void* out, int B, int T, int H, int W, int P, 
 int nabla_unflatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
                     nabla_stream_t stream);
 
-/* Bytes of device workspace nabla_build_mask needs: the pooled queries and
- * keys, fp32 [B][Hh][Nb][D] each (queries first).  Returns 0 for invalid
- * sizes. */
+/* Bytes of device workspace nabla_build_mask needs: the pooled queries,
+ * fp32 [B][Hh][Nb][D], then the pooled keys transposed, fp32
+ * [B][Hh][D][Nbp] with Nbp = Nb rounded up to a multiple of 4 (columns
+ * >= Nb are padding).  Returns 0 for invalid sizes. */
 size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W,
                                   const nabla_params* params);
 
@@ -105,7 +106,8 @@ size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W,
  *               blocks ascending in entries [0, kv_count); later entries are
  *               not written.
  *   workspace   device buffer of nabla_mask_workspace_bytes() bytes, 16-byte
- *               aligned; on return it holds qbar then kbar.
+ *               aligned; on return it holds qbar then kbar^T (layouts as
+ *               for nabla_mask_workspace_bytes).
  * Errors: NABLA_ERR_INVALID (shape, D not 64/128, thr outside [0,1], even or
  * negative STA sizes, flags != 0); NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
 int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
@@ -131,6 +133,20 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out,
                           float* lse, nabla_stream_t stream);
+
+/* nabla_sparse_attn_fwd for a flattened T x H x W token grid (S = T*H*W,
+ * P = 8): same arguments, layouts, results and errors, plus NABLA_ERR_INVALID
+ * unless H and W are multiples of 8.  Knowing the grid lets the kernel choose
+ * which two query blocks share one 128-row tile: when T and W/8 are even,
+ * each 2 x 2 group of patch positions {(t, w), (t, w+1), (t+1, w), (t+1, w+1)}
+ * (same patch row) is split along w or along t, whichever leaves fewer key
+ * blocks listed by only one of the two (those run as half-masked tiles).
+ * The pairing changes the work done, never which keys a query attends to:
+ * every query block still attends exactly to its own kv_idx list.  With T or
+ * W/8 odd it behaves as nabla_sparse_attn_fwd. */
+int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+                               const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
+                               void* out, float* lse, nabla_stream_t stream);
 
 /* Same mask as nabla_build_mask, for callers that cannot allocate device
  * memory.  This entry point has no counterpart in the paper; it exists for

@@ -41,8 +41,12 @@ class Case:
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
 
-    def attention(self):
-        out, lse = nabla.sparse_attn_fwd(self.qf, self.kf, self.vf, self.kv_count, self.kv_idx)
+    def attention(self, grid: bool = True):
+        """grid=True calls the grid-aware entry point (the one bench.py times),
+        grid=False the plain one."""
+        w = self.w
+        out, lse = nabla.sparse_attn_fwd(self.qf, self.kf, self.vf, self.kv_count, self.kv_idx,
+                                         grid=(w.T, w.H, w.W) if grid else None)
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
         return out, lse

@@ -58,10 +58,12 @@ def test_small_layers_end_to_end(w):
     # masks: bit-exact outside the band
     bad, in_band, nband = compare_masks(case, status)
     assert bad == 0, f"{bad} mask mismatches outside the band ({in_band} inside, {nband} band blocks)"
-    # attention on every query block, against the oracle on the GPU's lists
-    out, lse = case.attention()
-    mx, mean, lse_err = check_attention(case, out, lse, np.arange(w.Nb), (qf_h, kf_h, vf_h))
-    assert mx <= MAX_ABS and mean <= MEAN_ABS and lse_err <= LSE_ABS, (mx, mean, lse_err)
+    # attention on every query block, against the oracle on the GPU's lists,
+    # through both entry points (pairs 2p, 2p+1 and the grid-aware pairing)
+    for grid in (False, True):
+        out, lse = case.attention(grid=grid)
+        mx, mean, lse_err = check_attention(case, out, lse, np.arange(w.Nb), (qf_h, kf_h, vf_h))
+        assert mx <= MAX_ABS and mean <= MEAN_ABS and lse_err <= LSE_ABS, (grid, mx, mean, lse_err)
     # unflatten brings the output back to grid order bit-exactly
     o_grid = nabla.unflatten(out, w.T, w.H, w.W)
     ref = oracle.unflatten(out.cpu(), w.T, w.H, w.W).reshape(out.shape)
@@ -142,6 +144,88 @@ def test_hand_built_lists_pairs_disagree(D, Nb_t, logit_scale):
     err = np.abs(out.double().cpu().numpy() - ref)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     assert np.abs(lse.double().cpu().numpy() - ref_lse).max() <= LSE_ABS * max(1.0, logit_scale)
+
+
+def grouped_lists(T, nbh, nbw, Hh, rng):
+    """Block lists on a T x nbh x nbw block grid whose 2 x 2 (w, t) groups
+    push the grid-aware pairing both ways: in 'w' groups the two horizontal
+    neighbours share their list and the frames differ, in 't' groups the two
+    frames share it and the neighbours differ; 'e' groups hold empty rows and
+    'r' groups random lists."""
+    Nb = T * nbh * nbw
+    F = nbh * nbw
+    cnt = np.zeros((1, Hh, Nb), dtype=np.int32)
+    idx = np.full((1, Hh, Nb, Nb), -1, dtype=np.int32)
+    kinds = []
+
+    def put(h, i, sel):
+        sel = np.unique(sel)
+        cnt[0, h, i] = sel.size
+        idx[0, h, i, :sel.size] = sel
+
+    for h in range(Hh):
+        for t in range(0, T, 2):
+            for bh in range(nbh):
+                for bw in range(0, nbw, 2):
+                    a = t * F + bh * nbw + bw
+                    g = [a, a + 1, a + F, a + F + 1]
+                    kind = "wter"[rng.integers(4)]
+                    kinds.append(kind)
+                    lists = [rng.choice(Nb, size=rng.integers(1, Nb // 3), replace=False) for _ in range(4)]
+                    if kind == "w":
+                        lists[1], lists[3] = lists[0], lists[2]
+                    elif kind == "t":
+                        lists[2], lists[3] = lists[0], lists[1]
+                    elif kind == "e":
+                        lists[rng.integers(4)] = np.array([], dtype=np.int64)
+                    for i, sel in zip(g, lists):
+                        put(h, i, sel)
+    return cnt, idx, kinds
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_grid_pairing_takes_both_decisions(D):
+    """The grid-aware entry point splits some groups along w and others along
+    t (and handles groups with an empty row); every query block must still
+    attend exactly to its own list."""
+    rng = np.random.default_rng(500 + D)
+    T, H, W, Hh, B = 4, 16, 32, 3, 1  # block grid 4 x 2 x 4, Nb = 32
+    S = T * H * W
+    nbh, nbw = H // 8, W // 8
+    g = torch.Generator().manual_seed(600 + D)
+    q, k, v = (torch.randn(B, S, Hh, D, generator=g).to(torch.bfloat16) for _ in range(3))
+    cnt, idx, kinds = grouped_lists(T, nbh, nbw, Hh, rng)
+    assert {"w", "t"} <= set(kinds)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    cnt_d = torch.from_numpy(cnt).cuda()
+    idx_d = torch.from_numpy(idx).cuda()
+    ref, ref_lse = oracle.attention(q, k, v, cnt, idx, 1.0 / math.sqrt(D))
+    for grid in (None, (T, H, W)):
+        out, lse = nabla.sparse_attn_fwd(qd, kd, vd, cnt_d, idx_d, grid=grid)
+        torch.cuda.synchronize()
+        assert nabla.get_status() == 0
+        err = np.abs(out.double().cpu().numpy() - ref)
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (grid, err.max(), err.mean())
+        got_lse = lse.double().cpu().numpy()
+        finite = np.isfinite(ref_lse)
+        assert np.array_equal(finite, np.isfinite(got_lse))
+        assert np.abs(got_lse[finite] - ref_lse[finite]).max() <= LSE_ABS
+        # empty rows: exactly zero output
+        empty = np.nonzero(cnt[0] == 0)
+        o = out.float().cpu()
+        for h, i in zip(*empty):
+            assert torch.all(o[0, i * 64:(i + 1) * 64, h] == 0)
+
+
+def test_grid_entry_point_rejects_bad_grids():
+    x = torch.zeros(1, 1024, 1, 64, dtype=torch.bfloat16, device="cuda")
+    cnt = torch.ones(1, 1, 16, dtype=torch.int32, device="cuda")
+    idx = torch.zeros(1, 1, 16, 16, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        nabla.sparse_attn_fwd(x, x, x, cnt, idx, grid=(4, 16, 8))  # 512 tokens, not 1024
+    with pytest.raises(nabla.NablaError):
+        nabla.sparse_attn_fwd(x, x, x, cnt, idx, grid=(4, 4, 64))  # H not a multiple of 8
+    assert nabla.get_status() == 0
 
 
 def test_empty_rows_give_zero_output_and_neg_inf_lse():
