@@ -18,7 +18,7 @@
 //     same four lists; one block of each CTA is the same under both pairings,
 //     so its half of Q is loaded before the lists are read.
 //
-// Warp roles (192 threads, two CTAs per SM):
+// Warp roles (224 threads, two CTAs per SM):
 //   warps 0-3  softmax: thread t owns query row t = TMEM lane t.  Reads the
 //              64 scores of its row from TMEM, keeps an online max/sum,
 //              rescales its O row in TMEM when the max grew by more than
@@ -28,10 +28,11 @@
 //   warp 4     TMA producer: Q once, then K_j and V_j of each listed block j
 //              (contiguous 64-token boxes of the flattened layout) into a
 //              ring of kStages stages.
-//   warp 5     MMA issuer (one thread): S = Q K_j^T into one of two TMEM
-//              score buffers (M=128, N=64, K=D), and O += P V_j with P read
-//              from tensor memory and V MN-major straight from its TMA tile
-//              (M=128, N=D, K=64).
+//   warp 5     QK^T issuer (one thread): S = Q K_j^T into one of two TMEM
+//              score buffers (M=128, N=64, K=D).
+//   warp 6     PV issuer (one thread): O += P V_j with P read from tensor
+//              memory and V MN-major straight from its TMA tile (M=128, N=D,
+//              K=64).
 // Tensor memory per CTA: S0 | S1 (64 columns each, P aliases their first 32)
 // | O (D columns) = 256 columns, so two CTAs share an SM's 512 columns.
 // Every wait is bounded (see mbar_wait); a timeout raises the CTA's abort
@@ -43,7 +44,7 @@
 
 namespace nabla {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 224;
 constexpr int kMaxListBlocks = 16383;  // list entries hold a 14-bit block index
 
 template <int D>
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(p_full + s, 128);
       mbar_init(pv_done + s, 1);
     }
-    mbar_init(mma_drain, 1);
+    mbar_init(mma_drain, 2);  // one commit from each MMA-issuing thread
     *abort_flag = 0;
     fence_mbar_init();
     // The half of Q whose block is already known loads right away; in pair
@@ -320,26 +321,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     if (lane == 0) mbar_wait_drain(q_full, 0);
   } else if (warp == 5) {
-    // ------------------------------------------------------------- MMA issue
+    // ---------------------------------------------------------- QK^T issue
     if (lane == 0 && L_n > 0) {
       bool ok = mbar_wait(q_full, 0, abort_flag);
       tc_fence_after();
-      auto issue_pv = [&](int m) -> bool {
-        const int s = m % kStages;
-        if (!mbar_wait(p_full + (m & 1), (m >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(v_full + s, (m / kStages) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t pa = (m & 1) ? tS1 : tS0;
-        const uint32_t vb = sV + s * L::kKVBytes;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, 64 * 128, 1024);
-          umma_bf16_ts(tO, pa + kk * 8, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(pv_done + (m & 1));
-        umma_commit(v_empty + s);
-        return true;
-      };
       for (int n = 0; ok && n < L_n; ++n) {
         const int s = n % kStages;
         if (!mbar_wait(k_full + s, (n / kStages) & 1, abort_flag)) { ok = false; break; }
@@ -357,16 +342,38 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         }
         umma_commit(s_full + (n & 1));
         umma_commit(k_empty + s);
-        if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
       }
-      if (ok) issue_pv(L_n - 1);
       // Every MMA this thread issued must finish before the tensor memory is
       // freed, also on the abort path (time-bounded).
       umma_commit(mma_drain);
       mbar_wait_drain(mma_drain, 0);
     }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------- PV issue
+    // A thread of its own, so a PV is issued as soon as its P is written
+    // instead of queueing behind the issue of the next QK^T.
+    if (lane == 0 && L_n > 0) {
+      bool ok = true;
+      for (int m = 0; ok && m < L_n; ++m) {
+        const int s = m % kStages;
+        if (!mbar_wait(p_full + (m & 1), (m >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(v_full + s, (m / kStages) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t pa = (m & 1) ? tS1 : tS0;
+        const uint32_t vb = sV + s * L::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = smem_desc_sw128(vb + kk * 16 * 128, 64 * 128, 1024);
+          umma_bf16_ts(tO, pa + kk * 8, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(pv_done + (m & 1));
+        umma_commit(v_empty + s);
+      }
+      umma_commit(mma_drain);
+      mbar_wait_drain(mma_drain, 0);
+    }
   } else {
-    // --------------------------------------------------------------- softmax
+    // --------------------------------------------------------------- softmax (warps 0-3)
     const int r = tid;  // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t flag = 0x4000u << (r >> 6);

@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     unsigned long long best = 0;  // (bits(e) << 32) | j; max = arg-max, ties to the larger j
     unsigned long long total = 0;
+    int n_tiny = 0;  // blocks with e < 2^-63
     for (int j = lane; j < Nb; j += 32) {
       const float e = expf(row[j] - m);
       row[j] = e;
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
       const unsigned long long key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
       best = key > best ? key : best;
       total += mass_bits(u);
+      n_tiny += u < 0x20000000u;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -218,6 +220,8 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
       best = ob > best ? ob : best;
     }
     total = warp_sum_u64(total);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_tiny += __shfl_xor_sync(0xffffffffu, n_tiny, o);
     const int argmax = static_cast<int>(best & 0xffffffffu);
     const unsigned long long tau_m =
         static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
@@ -225,67 +229,82 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     // 3. CDF boundary: the element (e*, j*) of the ascending (e, j) order at
     //    which the cumulative mass first exceeds tau_m; keep (e, j) >= it.
     //    bits(e*) is the largest bit pattern x with mass(bits(e) < x) <= tau_m
-    //    (positive floats order like their bit patterns), found MSB first,
-    //    two bits per pass: each pass sums the exact masses below three
-    //    probes at once (warp sums, no atomics).  After the top 11 bits, if
-    //    at most 32 blocks share them they are sorted by a warp bitonic sort
-    //    and the boundary read off their prefix sums.
+    //    (positive floats order like their bit patterns).  It is narrowed
+    //    inside a range [prefix, prefix + 2^span), two bits per pass: a pass
+    //    sums, per quarter of the range, the exact masses and counts of the
+    //    blocks in it (warp sums, no atomics; blocks outside the range cost a
+    //    compare).  As soon as at most 32 blocks remain in the range they are
+    //    sorted by a warp bitonic sort and the boundary is read off their
+    //    prefix sums.  Every block with positive mass has e >= 2^-40, so e*
+    //    does too and the search starts at [2^-63, 2): bits(e*) has bit 29
+    //    set and bit 30 clear, and nothing below 2^-63 carries mass.
     unsigned long long kstar = ~0ull;
     if (!a.keep_all && total > tau_m) {
-      uint32_t prefix = 0;
+      uint32_t prefix = 0x20000000u;
+      int span = 29;
       unsigned long long below = 0;  // mass(bits(e) < prefix)
-      // Extends prefix by the bits [lo, hi] (one or two bits).
-      auto refine = [&](int hi, int lo) {
-        if (hi == lo) {
-          const uint32_t c = prefix | (1u << hi);
-          unsigned long long s = 0;
-          for (int j = lane; j < Nb; j += 32) {
-            const uint32_t u = __float_as_uint(row[j]);
-            if (u < c) s += mass_bits(u);
-          }
-          s = warp_sum_u64(s);
-          if (s <= tau_m) {
-            prefix = c;
-            below = s;
-          }
-          return;
-        }
-        const uint32_t c1 = prefix | (1u << lo), c2 = prefix | (2u << lo), c3 = prefix | (3u << lo);
-        unsigned long long s1 = 0, s2 = 0, s3 = 0;
+      int n_lo = n_tiny, n_hi = Nb;  // blocks below prefix, below prefix + 2^span
+      while (span > 0 && n_hi - n_lo > 32) {
+        const int lo = span > 2 ? span - 2 : 0;
+        const uint32_t range = 1u << span;
+        unsigned long long m0 = 0, m1 = 0, m2 = 0;
+        int c0 = 0, c1 = 0, c2 = 0;
         for (int j = lane; j < Nb; j += 32) {
           const uint32_t u = __float_as_uint(row[j]);
-          const unsigned long long w = mass_bits(u);
-          if (u < c1) s1 += w;
-          if (u < c2) s2 += w;
-          if (u < c3) s3 += w;
+          const uint32_t d = u - prefix;
+          if (d < range) {
+            const uint32_t q = d >> lo;
+            const unsigned long long w = mass_bits(u);
+            m0 += q == 0 ? w : 0ull;
+            m1 += q == 1 ? w : 0ull;
+            m2 += q == 2 ? w : 0ull;
+            c0 += q == 0;
+            c1 += q == 1;
+            c2 += q == 2;
+          }
         }
-        s1 = warp_sum_u64(s1);
-        s2 = warp_sum_u64(s2);
-        s3 = warp_sum_u64(s3);
+        m0 = warp_sum_u64(m0);
+        m1 = warp_sum_u64(m1);
+        m2 = warp_sum_u64(m2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+          c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+          c2 += __shfl_xor_sync(0xffffffffu, c2, o);
+        }
+        const unsigned long long s1 = below + m0, s2 = s1 + m1, s3 = s2 + m2;
         if (s3 <= tau_m) {
-          prefix = c3;
+          prefix += 3u << lo;
           below = s3;
+          n_lo += c0 + c1 + c2;
         } else if (s2 <= tau_m) {
-          prefix = c2;
+          prefix += 2u << lo;
           below = s2;
+          n_lo += c0 + c1;
+          n_hi = n_lo + c2;
         } else if (s1 <= tau_m) {
-          prefix = c1;
+          prefix += 1u << lo;
           below = s1;
+          n_lo += c0;
+          n_hi = n_lo + c1;
+        } else {
+          n_hi = n_lo + c0;
         }
-      };
-      for (int hi = 30; hi >= 20; hi -= 2) refine(hi, hi > 20 ? hi - 1 : hi);
-      // e* lies in [prefix, prefix + 2^20): gather those blocks (ascending j).
-      int ncand = 0;
-      for (int base = 0; base < Nb && ncand <= 32; base += 32) {
-        const int j = base + lane;
-        const bool hit = j < Nb && (__float_as_uint(row[j]) >> 20) == (prefix >> 20);
-        const unsigned bal = __ballot_sync(0xffffffffu, hit);
-        const int pos = ncand + __popc(bal & ((1u << lane) - 1u));
-        if (hit && pos < 32) cand[pos] = j;
-        ncand += __popc(bal);
+        span = lo;
       }
-      __syncwarp();
-      if (ncand <= 32) {
+      const uint32_t range = 1u << span;
+      if (n_hi - n_lo <= 32) {
+        // gather the blocks of the range (ascending j), then sort them
+        int ncand = 0;
+        for (int base = 0; base < Nb && ncand < n_hi - n_lo; base += 32) {
+          const int j = base + lane;
+          const bool hit = j < Nb && __float_as_uint(row[j]) - prefix < range;
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
+          const int pos = ncand + __popc(bal & ((1u << lane) - 1u));
+          if (hit && pos < 32) cand[pos] = j;
+          ncand += __popc(bal);
+        }
+        __syncwarp();
         unsigned long long key = ~0ull, w = 0ull;
         if (lane < ncand) {
           const int j = cand[lane];
@@ -314,12 +333,12 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
           const unsigned long long v = __shfl_up_sync(0xffffffffu, cw, o);
           if (lane >= o) cw += v;
         }
-        // below + (mass of the whole group) > tau_m, so some lane qualifies
+        // below + (mass of the whole range) > tau_m, so some lane qualifies
         const unsigned hitb = __ballot_sync(0xffffffffu, lane < ncand && below + cw > tau_m);
         kstar = __shfl_sync(0xffffffffu, key, __ffs(hitb) - 1);
       } else {
-        for (int hi = 19; hi >= 0; hi -= 2) refine(hi, hi - 1);
-        // Equal values at e*: the boundary is the m-th smallest index among them.
+        // More than 32 blocks share the value e* = prefix: the boundary is
+        // the need-th smallest index among them.
         const unsigned long long wstar = mass_bits(prefix);
         const unsigned long long need = (tau_m - below) / wstar + 1ull;
         unsigned long long seen = 0;
@@ -342,9 +361,23 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
       __syncwarp();
     }
 
-    // 4. union with the STA window and compaction
-    const int per_t = a.nbh * a.nbw;
-    const int ti = i / per_t, hi = (i % per_t) / a.nbw, wi = i % a.nbw;
+    // 4. union with the STA window: the window's blocks get e = +inf, which
+    //    orders above every kept key; then compaction of keep = (e, j) >=
+    //    (e*, j*) or arg-max, ascending j
+    if (a.sta_on) {
+      const int per_t = a.nbh * a.nbw;
+      const int nbt = Nb / per_t;
+      const int ti = i / per_t, hi = (i - ti * per_t) / a.nbw, wi = i - ti * per_t - hi * a.nbw;
+      const int wh = 2 * a.sta_rh + 1, ww = 2 * a.sta_rw + 1, plane = wh * ww;
+      const int nwin = (2 * a.sta_rt + 1) * plane;
+      for (int e = lane; e < nwin; e += 32) {
+        const int et = e / plane, ehw = e - et * plane, eh = ehw / ww;
+        const int tj = ti + et - a.sta_rt, hj = hi + eh - a.sta_rh, wj = wi + (ehw - eh * ww) - a.sta_rw;
+        if (tj >= 0 && tj < nbt && hj >= 0 && hj < a.nbh && wj >= 0 && wj < a.nbw)
+          row[tj * per_t + hj * a.nbw + wj] = __uint_as_float(0x7F800000u);
+      }
+      __syncwarp();
+    }
     int32_t* out = a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb);
     int count = 0;
     for (int base = 0; base < Nb; base += 32) {
@@ -353,10 +386,6 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
       if (j < Nb) {
         const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(row[j])) << 32) | static_cast<unsigned>(j);
         keep = a.keep_all || key >= kstar || j == argmax;
-        if (!keep && a.sta_on) {
-          const int tj = j / per_t, hj = (j % per_t) / a.nbw, wj = j % a.nbw;
-          keep = abs(ti - tj) <= a.sta_rt && abs(hi - hj) <= a.sta_rh && abs(wi - wj) <= a.sta_rw;
-        }
       }
       const unsigned bal = __ballot_sync(0xffffffffu, keep);
       if (keep) out[count + __popc(bal & ((1u << lane) - 1u))] = j;
