@@ -95,10 +95,10 @@ struct MaskArgs {
 
 constexpr int kMaskThreads = 256;
 constexpr int kMaskWarps = kMaskThreads / 32;
-constexpr int kMaskCols = 2;  // adjacent key blocks per thread in the score phase
+constexpr int kMaskCols = 4;  // adjacent key blocks per thread in the score phase
 
 // Column count of the transposed pooled keys kbar^T [D][Nbp]: Nb rounded up
-// to a multiple of 4 so every thread's pair of columns is an aligned 8-byte
+// to a multiple of 4 so every thread's four columns are an aligned 16-byte
 // load.
 __host__ __device__ inline int kbar_cols(int Nb) { return (Nb + 3) & ~3; }
 
@@ -150,42 +150,50 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
   }
   __syncthreads();
 
-  // 1. scores: thread owns key blocks j, j+1 and all R rows; per (row, block)
+  // 1. scores: thread owns key blocks j..j+3 and all R rows; per (row, block)
   //    one fused multiply-add chain over d ascending (the oracle's order),
-  //    two blocks per instruction.  kbar^T rows are read coalesced, eight d
-  //    ahead of use.
+  //    two blocks per instruction.  kbar^T rows are read coalesced (16 bytes
+  //    a thread), two or four d ahead of use; each q pair loaded from shared memory
+  //    feeds four two-lane FMAs.
   for (int j = tid * kMaskCols; j < Nb; j += kMaskThreads * kMaskCols) {
-    unsigned long long acc[R];
+    unsigned long long acc[R][2];
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0ull;
-    const unsigned long long* kp = reinterpret_cast<const unsigned long long*>(kt + j);
-    const int kstride = Nbp / 2;  // in column pairs
-    unsigned long long kv[8];
+    for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = 0ull;
+    const ulonglong2* kp = reinterpret_cast<const ulonglong2*>(kt + j);
+    const int kstride = Nbp / 4;  // in groups of four columns
+    constexpr int PF = R >= 16 ? 2 : 4;  // d rows loaded ahead (registers allowing)
+    ulonglong2 kv[PF];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) kv[u] = __ldg(kp + static_cast<int64_t>(u) * kstride);
-    for (int d0 = 0; d0 < D; d0 += 8) {
-      unsigned long long kn[8];
-      const bool more = d0 + 8 < D;
+    for (int u = 0; u < PF; ++u) kv[u] = __ldg(kp + static_cast<int64_t>(u) * kstride);
+    for (int d0 = 0; d0 < D; d0 += PF) {
+      ulonglong2 kn[PF];
+      const bool more = d0 + PF < D;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) kn[u] = more ? __ldg(kp + static_cast<int64_t>(d0 + 8 + u) * kstride) : 0ull;
+      for (int u = 0; u < PF; ++u)
+        kn[u] = more ? __ldg(kp + static_cast<int64_t>(d0 + PF + u) * kstride) : make_ulonglong2(0ull, 0ull);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < PF; ++u) {
         const ulonglong2* qrow = reinterpret_cast<const ulonglong2*>(qd + (d0 + u) * R);
 #pragma unroll
         for (int r2 = 0; r2 < R / 2; ++r2) {
           const ulonglong2 qq = qrow[r2];
-          ffma2(acc[2 * r2], kv[u], qq.x);
-          ffma2(acc[2 * r2 + 1], kv[u], qq.y);
+          ffma2(acc[2 * r2][0], kv[u].x, qq.x);
+          ffma2(acc[2 * r2][1], kv[u].y, qq.x);
+          ffma2(acc[2 * r2 + 1][0], kv[u].x, qq.y);
+          ffma2(acc[2 * r2 + 1][1], kv[u].y, qq.y);
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) kv[u] = kn[u];
+      for (int u = 0; u < PF; ++u) kv[u] = kn[u];
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float* row = rows + static_cast<size_t>(r) * Nb;
-      row[j] = __uint_as_float(static_cast<uint32_t>(acc[r])) * a.scale;
-      if (j + 1 < Nb) row[j + 1] = __uint_as_float(static_cast<uint32_t>(acc[r] >> 32)) * a.scale;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const unsigned long long v = acc[r][c >> 1];
+        if (j + c < Nb) row[j + c] = __uint_as_float(static_cast<uint32_t>(c & 1 ? v >> 32 : v)) * a.scale;
+      }
     }
   }
   __syncthreads();
