@@ -74,8 +74,20 @@ def kept_flops(w, total_kept):
     return 4.0 * 64 * 64 * w.D * total_kept
 
 
-def mask_bytes(w, total_kept):
-    return 2.0 * w.B * w.S * w.Hh * w.D * 2 + 4.0 * w.B * w.Hh * w.Nb + 4.0 * total_kept
+def flatten_pool_bytes(w):
+    """Compulsory bytes of the flatten stage: Q, K, V read and written once,
+    plus the pooled Q and K (fp32)."""
+    return 6.0 * w.B * w.S * w.Hh * w.D * 2 + 2.0 * 4 * w.B * w.Hh * w.Nb * w.D
+
+
+def score_flops(w):
+    """fp32 FLOPs of the mask's block scores (2 per multiply-add)."""
+    return 2.0 * w.B * w.Hh * w.Nb * w.Nb * w.D
+
+
+# fp32 FMA peak of one B200: 148 SMs x 128 lanes x 2 FLOP per clock at the
+# 1965 MHz maximum SM clock
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -158,12 +170,12 @@ def run_gpu(args, rank, world, local_rank):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        nabla.flatten(qd, w.T, w.H, w.W, out=qf)
-        nabla.flatten(kd, w.T, w.H, w.W, out=kf)
+        # Q and K: flattening fused with the mask's pooling; V: flattening
+        nabla.flatten_pool_qk(qd, kd, w.T, w.H, w.W, qf=qf, kf=kf, workspace=ws, thr=w.thr, sta=w.sta)
         nabla.flatten(vd, w.T, w.H, w.W, out=vf)
         if ev is not None:
             ev[1].record(stream)
-        nabla.build_mask(qf, kf, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx, workspace=ws)
+        nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx)
         if ev is not None:
             ev[2].record(stream)
         nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=of, lse=lse, grid=(w.T, w.H, w.W))
@@ -173,7 +185,7 @@ def run_gpu(args, rank, world, local_rank):
         if ev is not None:
             ev[4].record(stream)
 
-    launches_per_step = 3 + 2 + 1 + 1
+    launches_per_step = 2 + 1 + 1 + 1  # flatten+pool, flatten V, mask rows, attention, unflatten
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -258,19 +270,18 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic",
         "config": config_dict(w),
-        "ms_per_layer": mask_avg + attn_avg,
-        "stages_ms": {"flatten_qkv": statistics.mean(flat_ms), "build_mask": mask_avg, "sparse_attn": attn_avg,
+        "stages_ms": {"flatten_pool_qkv": statistics.mean(flat_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg,
                       "unflatten_o": statistics.mean(unflat_ms)},
         "attn_tflops_kept": achieved,
-        "mask_build_gbs": mask_bytes(w, total_kept) / (mask_avg * 1e-3) / 1e9,
-        "flatten_gbs": 3 * 2.0 * qd.numel() * 2 / (statistics.mean(flat_ms) * 1e-3) / 1e9,
+        "flatten_pool_gbs": flatten_pool_bytes(w) / (statistics.mean(flat_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": traffic},
-        "mask_roofline": {"bound": "hbm", "achieved": mask_bytes(w, total_kept) / (mask_avg * 1e-3) / 1e9,
-                          "peak": peak_gbs, "unit": "GB/s",
-                          "frac": mask_bytes(w, total_kept) / (mask_avg * 1e-3) / 1e9 / peak_gbs},
+        "mask_roofline": {"bound": "alu", "kernel": "mask_rows_kernel", "achieved": score_flops(w) / (mask_avg * 1e-3) / 1e12,
+                          "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                          "frac": score_flops(w) / (mask_avg * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
+                          "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"},
         "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,

@@ -34,6 +34,8 @@ EXPORTS = (
     "nabla_mask_workspace_bytes",
     "nabla_build_mask",
     "nabla_build_mask_noalloc",
+    "nabla_flatten_pool_qk",
+    "nabla_build_mask_pooled",
     "nabla_sparse_attn_fwd",
     "nabla_sparse_attn_fwd_grid",
     "nabla_get_status",
@@ -80,6 +82,8 @@ def lib():
         L.nabla_mask_workspace_bytes.restype = sz
         L.nabla_build_mask.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
         L.nabla_build_mask_noalloc.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp]
+        L.nabla_flatten_pool_qk.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, pp, vp, vp]
+        L.nabla_build_mask_pooled.argtypes = [vp, i, i, i, i, i, i, pp, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
@@ -151,7 +155,8 @@ def build_mask(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: 
     """Adaptive block mask from flattened Q, K [B, S, Hh, D] (bf16, CUDA).
 
     Returns (kv_count int32 [B,Hh,Nb], kv_idx int32 [B,Hh,Nb,Nb], workspace
-    uint8 holding the pooled qbar then kbar, fp32 [B,Hh,Nb,D] each).
+    uint8 holding the pooled qbar [B,Hh,Nb,D] then kbar^T [B,Hh,D,Nbp], fp32;
+    see :func:`pooled_from_workspace`).
     """
     B, S, Hh, D = qf.shape
     Nb = S // BLOCK
@@ -171,6 +176,47 @@ def build_mask(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: 
                                   _dev(kv_idx, torch.int32, "kv_idx"), _dev(workspace, torch.uint8, "workspace"),
                                   _stream(stream)), "nabla_build_mask")
     return kv_count, kv_idx, workspace
+
+
+def flatten_pool_qk(q: torch.Tensor, k: torch.Tensor, T: int, H: int, W: int, qf=None, kf=None, workspace=None,
+                    thr: float = 0.0, sta=(0, 0, 0), stream=None, P: int = 8):
+    """Flatten Q and K (grid order [B, T*H*W, Hh, D], bf16, CUDA) and pool
+    them into a mask workspace in one pass (nabla_flatten_pool_qk).
+    Returns (qf, kf, workspace); finish the mask with :func:`build_mask_pooled`."""
+    B, S, Hh, D = q.shape
+    prm = params(thr, sta, 0.0, P)
+    if qf is None:
+        qf = torch.empty_like(q)
+    if kf is None:
+        kf = torch.empty_like(k)
+    if workspace is None:
+        nbytes = mask_workspace_bytes(B, Hh, D, T, H, W, prm)
+        if nbytes == 0:
+            raise NablaError(NABLA_ERR_INVALID, "nabla_mask_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(lib().nabla_flatten_pool_qk(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                       _dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"), B, Hh, D, T, H,
+                                       W, ctypes.byref(prm), _dev(workspace, torch.uint8, "workspace"),
+                                       _stream(stream)), "nabla_flatten_pool_qk")
+    return qf, kf, workspace
+
+
+def build_mask_pooled(workspace: torch.Tensor, B: int, Hh: int, D: int, T: int, H: int, W: int, thr: float,
+                      sta=(0, 0, 0), scale: float = 0.0, kv_count=None, kv_idx=None, stream=None, P: int = 8):
+    """The mask from a workspace that already holds the pooled Q and K
+    (nabla_build_mask_pooled).  Returns (kv_count, kv_idx)."""
+    Nb = T * H * W // BLOCK
+    prm = params(thr, sta, scale, P)
+    dev = workspace.device
+    if kv_count is None:
+        kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)
+    _check(lib().nabla_build_mask_pooled(_dev(workspace, torch.uint8, "workspace"), B, Hh, D, T, H, W,
+                                         ctypes.byref(prm), _dev(kv_count, torch.int32, "kv_count"),
+                                         _dev(kv_idx, torch.int32, "kv_idx"), _stream(stream)),
+           "nabla_build_mask_pooled")
+    return kv_count, kv_idx
 
 
 def build_mask_noalloc(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),

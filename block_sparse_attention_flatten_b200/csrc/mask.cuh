@@ -2,7 +2,8 @@
 // "Construcao de Mascara Adaptativa" and item 3 "Integracao Hibrida com STA").
 //
 // pool_kernel       Downsampling: per 64-token block the fp32 mean of the
-//                   flattened queries and keys (Q and K read once from HBM).
+//                   flattened queries and keys (Q and K read once from HBM),
+//                   optionally fused with their fractal flattening.
 // mask_rows_kernel  Reduced attention, CDF threshold, STA union and block-CSR
 //                   compaction, R query-block rows per CTA:
 //   1. scores s_ij = (qbar_i . kbar_j) * scale (fp32 FMA chain over d) into
@@ -30,26 +31,51 @@ namespace nabla {
 // into kbar^T [B][Hh][D][Nbp] (Nbp = Nb rounded up to a multiple of 4; the
 // padding columns are never written).
 // Thread c handles elements 8c..8c+7 of a token row (Hh*D elements), summing
-// the block's 64 rows in ascending order in fp32.
+// the block's 64 rows in ascending flattened order in fp32.
+// kFlatten = false: q, k are already flattened.  kFlatten = true: q, k are in
+// grid order; the kernel also writes the block's 64 rows, permuted, to
+// qf_out / kf_out (fractal flattening fused with the pooling, so Q and K are
+// read once).  Flattened rows 8u..8u+7 of a block are one run of 8
+// consecutive grid rows (patch row u).
+template <bool kFlatten>
 __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restrict__ q,
-                                                   const __nv_bfloat16* __restrict__ k, float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, int S, int Hh, int D) {
+                                                   const __nv_bfloat16* __restrict__ k, __nv_bfloat16* qf_out,
+                                                   __nv_bfloat16* kf_out, float* __restrict__ qbar,
+                                                   float* __restrict__ kbar, int S, int Hh, int D, int H, int W) {
   const int i = blockIdx.x, b = blockIdx.y;
   const int Nb = S >> 6;
   const __nv_bfloat16* x = blockIdx.z == 0 ? q : k;
   float* out = blockIdx.z == 0 ? qbar : kbar;
   const int row = Hh * D;
   const int chunks = row >> 3;
-  const uint4* base = reinterpret_cast<const uint4*>(x + (static_cast<int64_t>(b) * S + static_cast<int64_t>(i) * 64) * row);
+  const int64_t batch_rows = static_cast<int64_t>(b) * S;
+  // first grid row of the block's patch (kFlatten) or first flattened row
+  int64_t src0 = batch_rows + static_cast<int64_t>(i) * 64;
+  if (kFlatten) {
+    const int nbw = W >> 3, per_t = (H >> 3) * nbw;
+    const int t = i / per_t, rem = i - t * per_t, bh = rem / nbw, bw = rem - bh * nbw;
+    src0 = batch_rows + (static_cast<int64_t>(t) * H + bh * 8) * W + bw * 8;
+  }
+  const uint4* base = reinterpret_cast<const uint4*>(x) + src0 * chunks;
+  uint4* dst = kFlatten ? reinterpret_cast<uint4*>(blockIdx.z == 0 ? qf_out : kf_out) +
+                              (batch_rows + static_cast<int64_t>(i) * 64) * chunks
+                        : nullptr;
   for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll 1
     for (int r0 = 0; r0 < 64; r0 += 8) {
+      // rows r0..r0+7: flattened order; in grid order one run of 8 along w
+      const int64_t src_row = kFlatten ? static_cast<int64_t>(r0 >> 3) * W : r0;
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldg(base + static_cast<int64_t>(r0 + u) * chunks + c);
+      for (int u = 0; u < 8; ++u)
+        v[u] = kFlatten ? __ldcs(base + (src_row + u) * chunks + c) : __ldg(base + (src_row + u) * chunks + c);
+      if (kFlatten) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dst[static_cast<int64_t>(r0 + u) * chunks + c] = v[u];
+      }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);

@@ -136,6 +136,78 @@ int launch_mask(const MaskArgs& a, int B, const DeviceInfo& di, cudaStream_t str
   return launch_status();
 }
 
+// Validated mask configuration shared by the mask entry points.
+struct MaskPlan {
+  MaskArgs a;
+  DeviceInfo di;
+  int S, H, W;
+};
+
+int mask_plan(int B, int Hh, int D, int T, int H, int W, const nabla_params* params, void* workspace,
+              int32_t* kv_count, int32_t* kv_idx, MaskPlan* mp) {
+  if (params == nullptr) return NABLA_ERR_INVALID;
+  const nabla_params& p = *params;
+  int rc = check_grid(B, T, H, W, p.P);
+  if (rc != NABLA_OK) return rc;
+  if (Hh <= 0 || (D != 64 && D != 128) || p.flags != 0u) return NABLA_ERR_INVALID;
+  if (!(p.thr >= 0.f && p.thr <= 1.f)) return NABLA_ERR_INVALID;
+  if (!(p.scale >= 0.f) || std::isinf(p.scale)) return NABLA_ERR_INVALID;
+  const bool sta_on = p.sta_t != 0 || p.sta_h != 0 || p.sta_w != 0;
+  if (sta_on && (p.sta_t <= 0 || p.sta_h <= 0 || p.sta_w <= 0 || p.sta_t % 2 == 0 || p.sta_h % 2 == 0 ||
+                 p.sta_w % 2 == 0))
+    return NABLA_ERR_INVALID;
+  if (workspace == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(workspace)) return NABLA_ERR_ALIGN;
+  if (static_cast<int64_t>(Hh) * D > 3072 * 4) return NABLA_ERR_INVALID;
+  const int S = T * H * W;
+  const int Nb = S / 64;
+  MaskArgs& a = mp->a;
+  a.qbar = static_cast<float*>(workspace);
+  a.kbar = const_cast<float*>(a.qbar) + static_cast<size_t>(B) * Hh * Nb * D;
+  a.kv_count = kv_count;
+  a.kv_idx = kv_idx;
+  a.Hh = Hh;
+  a.Nb = Nb;
+  a.D = D;
+  a.nbh = H / p.P;
+  a.nbw = W / p.P;
+  a.sta_on = sta_on ? 1 : 0;
+  a.sta_rt = p.sta_t / 2;
+  a.sta_rh = p.sta_h / 2;
+  a.sta_rw = p.sta_w / 2;
+  a.keep_all = p.thr >= 1.f ? 1 : 0;
+  a.scale = p.scale > 0.f ? p.scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  a.tau = 1.0 - static_cast<double>(p.thr);  // exact in double
+  mp->S = S;
+  mp->H = H;
+  mp->W = W;
+  return NABLA_OK;
+}
+
+template <bool kFlatten>
+int launch_pool(const MaskPlan& mp, int B, const void* q, const void* k, void* qf, void* kf, cudaStream_t stream) {
+  const int row = mp.a.Hh * mp.a.D;
+  const int pool_threads = (row / 8) < 384 ? (row / 8) : 384;
+  pool_kernel<kFlatten><<<dim3(mp.a.Nb, B, 2), pool_threads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(qf),
+      static_cast<__nv_bfloat16*>(kf), const_cast<float*>(mp.a.qbar), const_cast<float*>(mp.a.kbar), mp.S, mp.a.Hh,
+      mp.a.D, mp.H, mp.W);
+  return launch_status();
+}
+
+int launch_mask_rows(const MaskPlan& mp, int B, cudaStream_t stream) {
+  // Rows per CTA: 16 while the score rows fit ~64 KB (two CTAs per SM), else
+  // as many as fit ~128 KB.
+  const int Nb = mp.a.Nb, D = mp.a.D;
+  const size_t per_row = static_cast<size_t>(Nb) * 4;
+  if (16 * per_row <= 64u * 1024u) return launch_mask<16>(mp.a, B, mp.di, stream);
+  const size_t fit = (128u * 1024u) / per_row;
+  if (fit >= 8) return launch_mask<8>(mp.a, B, mp.di, stream);
+  if (fit >= 4) return launch_mask<4>(mp.a, B, mp.di, stream);
+  if (mask_smem_bytes(2, D, Nb) <= static_cast<size_t>(mp.di.max_smem_optin)) return launch_mask<2>(mp.a, B, mp.di, stream);
+  return NABLA_ERR_INVALID;
+}
+
 // Failure-detection self-test: every thread of one CTA waits on an mbarrier
 // nothing arrives on, with the kernels' bounded wait and a short limit.
 __global__ void wait_timeout_selftest_kernel(long long limit) {
@@ -243,61 +315,39 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
                      const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, void* workspace,
                      nabla_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (params == nullptr) return NABLA_ERR_INVALID;
-  const nabla_params& p = *params;
-  int rc = check_grid(B, T, H, W, p.P);
+  MaskPlan mp;
+  int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, kv_count, kv_idx, &mp);
   if (rc != NABLA_OK) return rc;
-  if (Hh <= 0 || (D != 64 && D != 128) || p.flags != 0u) return NABLA_ERR_INVALID;
-  if (!(p.thr >= 0.f && p.thr <= 1.f)) return NABLA_ERR_INVALID;
-  if (!(p.scale >= 0.f) || std::isinf(p.scale)) return NABLA_ERR_INVALID;
-  const bool sta_on = p.sta_t != 0 || p.sta_h != 0 || p.sta_w != 0;
-  if (sta_on && (p.sta_t <= 0 || p.sta_h <= 0 || p.sta_w <= 0 || p.sta_t % 2 == 0 || p.sta_h % 2 == 0 ||
-                 p.sta_w % 2 == 0))
-    return NABLA_ERR_INVALID;
-  if (qf == nullptr || kf == nullptr || kv_count == nullptr || kv_idx == nullptr || workspace == nullptr)
-    return NABLA_ERR_INVALID;
-  if (!aligned16(qf) || !aligned16(kf) || !aligned16(workspace) || !aligned16(kv_count) || !aligned16(kv_idx))
-    return NABLA_ERR_ALIGN;
-  if (static_cast<int64_t>(Hh) * D > 3072 * 4) return NABLA_ERR_INVALID;
-  DeviceInfo di;
-  if ((rc = device_info(&di)) != NABLA_OK) return rc;
-  const int S = T * H * W;
-  const int Nb = S / 64;
-  float* qbar = static_cast<float*>(workspace);
-  float* kbar = qbar + static_cast<size_t>(B) * Hh * Nb * D;
+  if (qf == nullptr || kf == nullptr || kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
+  if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
+  if ((rc = launch_pool<false>(mp, B, qf, kf, nullptr, nullptr, stream)) != NABLA_OK) return rc;
+  return launch_mask_rows(mp, B, stream);
+}
 
-  const int pool_threads = (Hh * D / 8) < 384 ? (Hh * D / 8) : 384;
-  pool_kernel<<<dim3(Nb, B, 2), pool_threads, 0, stream>>>(static_cast<const __nv_bfloat16*>(qf),
-                                                            static_cast<const __nv_bfloat16*>(kf), qbar, kbar, S, Hh, D);
-  if ((rc = launch_status()) != NABLA_OK) return rc;
+int nabla_flatten_pool_qk(const void* q, const void* k, void* qf, void* kf, int B, int Hh, int D, int T, int H,
+                          int W, const nabla_params* params, void* workspace, nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  MaskPlan mp;
+  int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, nullptr, nullptr, &mp);
+  if (rc != NABLA_OK) return rc;
+  if (q == nullptr || k == nullptr || qf == nullptr || kf == nullptr) return NABLA_ERR_INVALID;
+  if (q == qf || q == kf || k == qf || k == kf || qf == kf) return NABLA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qf) || !aligned16(kf)) return NABLA_ERR_ALIGN;
+  if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
+  return launch_pool<true>(mp, B, q, k, qf, kf, stream);
+}
 
-  MaskArgs a;
-  a.qbar = qbar;
-  a.kbar = kbar;
-  a.kv_count = kv_count;
-  a.kv_idx = kv_idx;
-  a.Hh = Hh;
-  a.Nb = Nb;
-  a.D = D;
-  a.nbh = H / p.P;
-  a.nbw = W / p.P;
-  a.sta_on = sta_on ? 1 : 0;
-  a.sta_rt = p.sta_t / 2;
-  a.sta_rh = p.sta_h / 2;
-  a.sta_rw = p.sta_w / 2;
-  a.keep_all = p.thr >= 1.f ? 1 : 0;
-  a.scale = p.scale > 0.f ? p.scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  a.tau = 1.0 - static_cast<double>(p.thr);  // exact in double
-
-  // Rows per CTA: 16 while the score rows fit ~64 KB (two CTAs per SM), else
-  // as many as fit ~128 KB.
-  const size_t per_row = static_cast<size_t>(Nb) * 4;
-  if (16 * per_row <= 64u * 1024u) return launch_mask<16>(a, B, di, stream);
-  const size_t fit = (128u * 1024u) / per_row;
-  if (fit >= 8) return launch_mask<8>(a, B, di, stream);
-  if (fit >= 4) return launch_mask<4>(a, B, di, stream);
-  if (mask_smem_bytes(2, D, Nb) <= static_cast<size_t>(di.max_smem_optin)) return launch_mask<2>(a, B, di, stream);
-  return NABLA_ERR_INVALID;
+int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, int H, int W,
+                            const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  MaskPlan mp;
+  int rc = mask_plan(B, Hh, D, T, H, W, params, const_cast<void*>(workspace), kv_count, kv_idx, &mp);
+  if (rc != NABLA_OK) return rc;
+  if (kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
+  if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
+  return launch_mask_rows(mp, B, stream);
 }
 
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,

@@ -114,6 +114,27 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
                      const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
                      void* workspace, nabla_stream_t stream);
 
+/* Fractal flattening of Q and K fused with the pooling stage of
+ * nabla_build_mask: one pass reads q and k (grid order), writes qf and kf
+ * (flattened, exactly as nabla_flatten with row_elems = Hh*D) and the pooled
+ * queries and transposed keys into `workspace` (layout of
+ * nabla_mask_workspace_bytes, identical bits to the pooling inside
+ * nabla_build_mask).  Saves the second read of the flattened Q and K.
+ *   q, k        device bf16 [B][T*H*W][Hh][D], grid order.
+ *   qf, kf      device bf16 [B][T*H*W][Hh][D] outputs, flattened order.
+ *   workspace   as for nabla_build_mask.
+ * The four tensors must not alias.  Errors: as nabla_build_mask (params are
+ * validated the same way although only P is used here). */
+int nabla_flatten_pool_qk(const void* q, const void* k, void* qf, void* kf, int B, int Hh, int D, int T, int H,
+                          int W, const nabla_params* params, void* workspace, nabla_stream_t stream);
+
+/* Stages 2-4 of nabla_build_mask (reduced attention, CDF threshold, STA
+ * union, compaction) on a workspace that already holds the pooled queries
+ * and keys (written by nabla_flatten_pool_qk or nabla_build_mask).  Same
+ * arguments, results and errors as nabla_build_mask without qf and kf. */
+int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, int H, int W,
+                            const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream);
+
 /* Block-sparse attention forward on the kept tiles ("Expansao": only the
  * listed N x N blocks are computed; a dropped block is in neither the
  * numerator nor the softmax normaliser).  For query block i of (b, hd):

@@ -80,6 +80,18 @@ def test_invalid_arguments_rejected_before_launch(lib):
                               s) == nabla.NABLA_ERR_INVALID
     assert L.nabla_build_mask(ctypes.c_void_p(0x1008), fake, 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake, fake,
                               fake, s) == nabla.NABLA_ERR_ALIGN
+    prm = nabla.params(0.9)
+    a1, a2, a3 = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), ctypes.c_void_p(0x3000)
+    assert L.nabla_flatten_pool_qk(a1, a2, a1, a3, 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake,
+                                   s) == nabla.NABLA_ERR_INVALID  # q aliases qf
+    assert L.nabla_flatten_pool_qk(a1, a2, a3, ctypes.c_void_p(0x4008), 1, 2, 64, 4, 16, 16, ctypes.byref(prm),
+                                   fake, s) == nabla.NABLA_ERR_ALIGN
+    assert L.nabla_flatten_pool_qk(a1, a2, a3, ctypes.c_void_p(0x4000), 1, 2, 96, 4, 16, 16, ctypes.byref(prm),
+                                   fake, s) == nabla.NABLA_ERR_INVALID  # D
+    assert L.nabla_build_mask_pooled(fake, 1, 2, 64, 4, 16, 16, ctypes.byref(prm), None, fake,
+                                     s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_pooled(ctypes.c_void_p(0x1004), 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake, fake,
+                                     s) == nabla.NABLA_ERR_ALIGN
     assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 100, 2, 64, ctypes.c_float(0.0), fake, None,
                                    s) == nabla.NABLA_ERR_INVALID
     assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 128, 2, 48, ctypes.c_float(0.0), fake, None,

@@ -70,6 +70,30 @@ def test_small_layers_end_to_end(w):
     assert np.array_equal(o_grid.cpu().view(torch.int16).numpy().view(np.uint16), ref)
 
 
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_fused_flatten_pool_and_pooled_mask(w):
+    """nabla_flatten_pool_qk writes the oracle's flattening (bit-exact) and its
+    pooled means (bit-exact, same fp32 order); nabla_build_mask_pooled on that
+    workspace gives the same block lists as nabla_build_mask."""
+    q, k, _ = inputs.make_qkv(w)
+    qd, kd = q.cuda(), k.cuda()
+    qf, kf, ws = nabla.flatten_pool_qk(qd, kd, w.T, w.H, w.W, thr=w.thr, sta=w.sta)
+    cnt, idx = nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta)
+    torch.cuda.synchronize()
+    assert nabla.get_status() == 0
+    qf_ref = oracle.flatten(q, w.T, w.H, w.W).reshape(q.shape)
+    kf_ref = oracle.flatten(k, w.T, w.H, w.W).reshape(k.shape)
+    assert np.array_equal(qf.cpu().view(torch.int16).numpy().view(np.uint16), qf_ref)
+    assert np.array_equal(kf.cpu().view(torch.int16).numpy().view(np.uint16), kf_ref)
+    qg, kg = nabla.pooled_from_workspace(ws, w.B, w.Hh, w.Nb, w.D)
+    assert np.array_equal(qg.cpu().numpy(), oracle.pool(qf_ref))
+    assert np.array_equal(kg.cpu().numpy(), oracle.pool(kf_ref))
+    cnt2, idx2, _ = nabla.build_mask(qf, kf, w.T, w.H, w.W, w.thr, w.sta)
+    assert torch.equal(cnt, cnt2)
+    valid = torch.arange(w.Nb, device="cuda").view(1, 1, 1, -1) < cnt.unsqueeze(-1)
+    assert torch.equal(torch.where(valid, idx, -1), torch.where(valid, idx2, -1))
+
+
 def dense_grid(q, k, v, scale):
     qd, kd, vd = q.double(), k.double(), v.double()
     B, S, Hh, D = qd.shape
