@@ -177,17 +177,21 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tma_prefetch_desc(&tmV);
     }
   }
-  // The counts and the first kAttnThreads entries of every list are loaded
-  // together (entries past a row's count are read and ignored; a row has Nb
-  // entries), so the list set-up waits for one memory latency, not two.
-  int cnt[4], first[4];
+  // The counts of the lists and their first 32 entries (warp h reads list
+  // h, one cache line) are loaded together, so the common case of lists of
+  // at most 32 blocks waits for one memory latency.  Entries past a row's
+  // count are read and ignored (a row has Nb entries); reading further ahead
+  // would touch lines the mask never wrote, which come from DRAM.
+  int cnt[4];
 #pragma unroll
   for (int h = 0; h < 4; ++h) {
     const bool have = h < nlists && cand[h] >= 0;
-    const int64_t row = bh * Nb + (have ? cand[h] : 0);
-    cnt[h] = have ? __ldg(a.kv_count + row) : 0;
-    first[h] = (have && tid < Nb) ? __ldg(a.kv_idx + row * Nb + tid) : 0;
+    cnt[h] = have ? __ldg(a.kv_count + bh * Nb + (have ? cand[h] : 0)) : 0;
   }
+  int first = 0;
+  const int my_cand = warp == 0 ? cand[0] : warp == 1 ? cand[1] : warp == 2 ? cand[2] : warp == 3 ? cand[3] : -1;
+  const bool first_list = warp < nlists && my_cand >= 0 && lane < Nb;
+  if (first_list) first = __ldg(a.kv_idx + (bh * Nb + my_cand) * static_cast<int64_t>(Nb) + lane);
   for (int w = tid; w < 4 * words; w += kAttnThreads) bm[w] = 0u;
   __syncthreads();
 #pragma unroll
@@ -199,8 +203,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     uint32_t* bmh = bm + h * words;
     const int32_t* src = a.kv_idx + (bh * Nb + (cand[h] >= 0 ? cand[h] : 0)) * static_cast<int64_t>(Nb);
-    for (int e = tid; e < c; e += kAttnThreads) {
-      const int j = e == tid ? first[h] : src[e];
+    if (warp == h && lane < c && first_list) {
+      if (first < 0 || first >= Nb) report(NABLA_ERR_DEVICE_BOUNDS);
+      else atomicOr(bmh + (first >> 5), 1u << (first & 31));
+    }
+    for (int e = 32 + tid; e < c; e += kAttnThreads) {
+      const int j = src[e];
       if (j < 0 || j >= Nb) {
         report(NABLA_ERR_DEVICE_BOUNDS);
         continue;
@@ -209,32 +217,67 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    int x_half0 = 0, x_half1 = 1;  // which candidate (bitmap) each half holds
-    if (grouped) {
-      // Split along t when the two unions along t hold fewer blocks in total
-      // than the two along w.
-      int cw = 0, ct = 0;
-      for (int w = lane; w < words; w += 32) {
-        const uint32_t b0 = bm[w], b1 = bm[words + w], b2 = bm[2 * words + w], b3 = bm[3 * words + w];
-        cw += __popc(b0 | b1) + __popc(b2 | b3);
-        ct += __popc(b0 | b2) + __popc(b1 | b3);
-      }
+  // Which candidate list each half of the tile holds.  Group mode: split
+  // along t when the two unions along t hold fewer blocks in total than the
+  // two along w.  Evaluated by a whole warp; every warp that calls it gets
+  // the same answer.
+  auto halves = [&](int& x_half0, int& x_half1, bool& along_t) {
+    x_half0 = 0;
+    x_half1 = 1;
+    along_t = false;
+    if (!grouped) return;
+    int cw = 0, ct = 0;
+    for (int w = lane; w < words; w += 32) {
+      const uint32_t b0 = bm[w], b1 = bm[words + w], b2 = bm[2 * words + w], b3 = bm[3 * words + w];
+      cw += __popc(b0 | b1) + __popc(b2 | b3);
+      ct += __popc(b0 | b2) + __popc(b1 | b3);
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        cw += __shfl_xor_sync(0xffffffffu, cw, o);
-        ct += __shfl_xor_sync(0xffffffffu, ct, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      cw += __shfl_xor_sync(0xffffffffu, cw, o);
+      ct += __shfl_xor_sync(0xffffffffu, ct, o);
+    }
+    along_t = ct < cw;
+    x_half0 = slot == 0 ? 0 : (along_t ? 1 : 2);
+    x_half1 = slot == 0 ? (along_t ? 2 : 1) : 3;
+  };
+  bool k0_early = false;  // producer: K of the first listed block already requested
+  if (warp == 4) {
+    // The producer finds the first block of the merged list from the
+    // bitmaps and requests its K now, while warp 0 builds the list.
+    int x0, x1;
+    bool along_t;
+    halves(x0, x1, along_t);
+    int j0 = -1;
+    for (int w0 = 0; w0 < words && j0 < 0; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t u = w < words ? (bm[x0 * words + w] | bm[x1 * words + w]) : 0u;
+      const unsigned bal = __ballot_sync(0xffffffffu, u != 0u);
+      if (bal != 0u) {
+        const int src_lane = __ffs(bal) - 1;
+        const uint32_t uw = __shfl_sync(0xffffffffu, u, src_lane);
+        j0 = (w0 + src_lane) * 32 + __ffs(uw) - 1;
       }
-      const bool along_t = ct < cw;
-      x_half0 = slot == 0 ? 0 : (along_t ? 1 : 2);
-      x_half1 = slot == 0 ? (along_t ? 2 : 1) : 3;
+    }
+    if (j0 >= 0) {
+      k0_early = true;
       if (lane == 0) {
-        // the other half of Q; q_full already expects its bytes
-        const int other = slot ? x_half0 : x_half1;
+        mbar_arrive_expect_tx(k_full, L::kKVBytes);
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sm + L::kQ + c * 128 * 128 + (slot ? 0 : 64 * 128), &tmQ, q_full, c * 64, hd,
-                      cand[other] * 64, b);
+          tma_load_4d(sm + L::kK + c * 64 * 128, &tmK, k_full, c * 64, hd, j0 * 64, b);
       }
+    }
+  }
+  if (warp == 0) {
+    int x_half0, x_half1;
+    bool along_t;
+    halves(x_half0, x_half1, along_t);
+    if (grouped && lane == 0) {
+      // the other half of Q; q_full already expects its bytes
+      const int other = slot ? x_half0 : x_half1;
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_4d(sm + L::kQ + c * 128 * 128 + (slot ? 0 : 64 * 128), &tmQ, q_full, c * 64, hd, cand[other] * 64,
+                    b);
     }
     if (lane == 0) {
       half_blk[0] = cand[x_half0];
@@ -287,7 +330,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int n = 0; ok && n <= L_n; ++n) {
-        if (n < L_n) {
+        if (n < L_n && !(n == 0 && k0_early)) {
           const int s = n % kStages;
           if (n >= kStages && !mbar_wait(k_empty + s, ((n / kStages) - 1) & 1, abort_flag)) {
             ok = false;
@@ -297,8 +340,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_4d(sm + L::kK + s * L::kKVBytes + c * 64 * 128, &tmK, k_full + s, c * 64, hd, j * 64, b);
-          k_issued = n + 1;
         }
+        if (n < L_n) k_issued = n + 1;
         if (n >= 1) {
           const int m = n - 1, s = m % kStages;
           if (m >= kStages && !mbar_wait(v_empty + s, ((m / kStages) - 1) & 1, abort_flag)) {

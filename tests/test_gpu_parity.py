@@ -170,6 +170,34 @@ def test_hand_built_lists_pairs_disagree(D, Nb_t, logit_scale):
     assert np.abs(lse.double().cpu().numpy() - ref_lse).max() <= LSE_ABS * max(1.0, logit_scale)
 
 
+@pytest.mark.parametrize("grid", [None, (12, 16, 64)], ids=["pairs", "grid"])
+def test_long_lists(grid):
+    """Lists longer than the 32 entries the kernel reads ahead of their count
+    (and longer than a CTA's thread count), with the two paired halves
+    disagreeing."""
+    rng = np.random.default_rng(77)
+    T, H, W, Hh, B, D = 12, 16, 64, 1, 1, 64  # Nb = 192
+    S = T * H * W
+    Nb = S // 64
+    g = torch.Generator().manual_seed(78)
+    q, k, v = (torch.randn(B, S, Hh, D, generator=g).to(torch.bfloat16) for _ in range(3))
+    cnt = np.zeros((B, Hh, Nb), dtype=np.int32)
+    idx = np.full((B, Hh, Nb, Nb), -1, dtype=np.int32)
+    for i in range(Nb):
+        n = int(rng.choice([5, 33, 64, 150, Nb]))
+        sel = np.sort(rng.choice(Nb, size=n, replace=False))
+        cnt[0, 0, i] = n
+        idx[0, 0, i, :n] = sel
+    out, lse = nabla.sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cnt).cuda(),
+                                     torch.from_numpy(idx).cuda(), grid=grid)
+    torch.cuda.synchronize()
+    assert nabla.get_status() == 0
+    ref, ref_lse = oracle.attention(q, k, v, cnt, idx, 1.0 / math.sqrt(D))
+    err = np.abs(out.double().cpu().numpy() - ref)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    assert np.abs(lse.double().cpu().numpy() - ref_lse).max() <= LSE_ABS
+
+
 def grouped_lists(T, nbh, nbw, Hh, rng):
     """Block lists on a T x nbh x nbw block grid whose 2 x 2 (w, t) groups
     push the grid-aware pairing both ways: in 'w' groups the two horizontal
