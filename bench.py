@@ -1,19 +1,25 @@
 """Benchmark: one NABLA attention layer per step on B200, through the C ABI.
 
 A step is the whole hot path on one batch of synthetic input already
-resident in HBM: fractal flattening of Q, K and V, the adaptive block mask
-(pooling + reduced attention + CDF + compaction), block-sparse attention on
-the kept tiles, and unflattening of the output.  L2 is flushed (a 256 MB
-write) between timed steps, outside the timed events.
+resident in HBM, in three timed stages:
+  1. fractal flattening of Q and K fused with the mask's pooling
+     (nabla_flatten_pool_qk), and flattening of V (nabla_flatten);
+  2. the adaptive block mask from the pooled workspace: reduced attention,
+     CDF threshold, STA union, compaction (nabla_build_mask_pooled);
+  3. block-sparse attention on the kept tiles with the output stored back in
+     grid order, i.e. the unflattening fused into its stores
+     (nabla_sparse_attn_fwd_grid).
+L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan13b]
     python bench.py --impl reference ...   # the CPU oracle, same metric
 
 Prints one JSON line (rank 0).  `value` is kept-tile attention TFLOP/s over
-the whole step (4*64*64*D FLOP per kept 64x64 tile); the per-stage figures
-(ms per layer = mask + attention, mask-build GB/s, attention TFLOP/s) are
-extra keys.  With --gpus N > 1 each rank runs an independent replica of the
-layer (the method runs on one GPU; there is no exchange between ranks).
+the whole step (4*64*64*D FLOP per kept 64x64 tile); per-stage times,
+attention TFLOP/s with its roofline, the mask's score-phase roofline and the
+flatten stage's GB/s are extra keys.  With --gpus N > 1 each rank runs an
+independent replica of the layer (the method runs on one GPU; there is no
+exchange between ranks).
 """
 from __future__ import annotations
 
@@ -159,7 +165,7 @@ def run_gpu(args, rank, world, local_rank):
     # device-resident inputs and outputs (allocated once; the library allocates nothing)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     qf, kf, vf = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    of, og = torch.empty_like(qd), torch.empty_like(qd)
+    og = torch.empty_like(qd)  # attention output, grid order
     kv_count = torch.empty((w.B, w.Hh, w.Nb), dtype=torch.int32, device=dev)
     kv_idx = torch.empty((w.B, w.Hh, w.Nb, w.Nb), dtype=torch.int32, device=dev)
     prm = nabla.params(w.thr, w.sta)
@@ -178,14 +184,12 @@ def run_gpu(args, rank, world, local_rank):
         nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx)
         if ev is not None:
             ev[2].record(stream)
-        nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=of, lse=lse, grid=(w.T, w.H, w.W))
+        # attention with the output stored in grid order (un-flattening fused)
+        nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W))
         if ev is not None:
             ev[3].record(stream)
-        nabla.unflatten(of, w.T, w.H, w.W, out=og)
-        if ev is not None:
-            ev[4].record(stream)
 
-    launches_per_step = 2 + 1 + 1 + 1  # flatten+pool, flatten V, mask rows, attention, unflatten
+    launches_per_step = 2 + 1 + 1  # flatten+pool, flatten V, mask rows, attention (stores O un-flattened)
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -195,7 +199,7 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError(f"device status after warm-up: {nabla.strerror(status)}")
     total_kept = float(kv_count.double().sum().item())
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     if world > 1:
         torch.distributed.barrier()
@@ -215,8 +219,8 @@ def run_gpu(args, rank, world, local_rank):
     def stage(a, b):
         return [events[s][a].elapsed_time(events[s][b]) for s in range(args.steps)]
 
-    step_ms = stage(0, 4)
-    flat_ms, mask_ms, attn_ms, unflat_ms = stage(0, 1), stage(1, 2), stage(2, 3), stage(3, 4)
+    step_ms = stage(0, 3)
+    flat_ms, mask_ms, attn_ms = stage(0, 1), stage(1, 2), stage(2, 3)
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -270,8 +274,8 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic",
         "config": config_dict(w),
-        "stages_ms": {"flatten_pool_qkv": statistics.mean(flat_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg,
-                      "unflatten_o": statistics.mean(unflat_ms)},
+        "stages_ms": {"flatten_pool_qkv": statistics.mean(flat_ms), "mask_rows": mask_avg,
+                      "sparse_attn_unflatten": attn_avg},
         "attn_tflops_kept": achieved,
         "flatten_pool_gbs": flatten_pool_bytes(w) / (statistics.mean(flat_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),

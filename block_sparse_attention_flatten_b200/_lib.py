@@ -257,8 +257,9 @@ def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_cou
     """Block-sparse attention on the kept tiles; returns (out, lse or None).
 
     grid = (T, H, W) of the flattened tokens calls nabla_sparse_attn_fwd_grid,
-    which pairs query blocks by their lists' overlap; None calls
-    nabla_sparse_attn_fwd (pairs 2p, 2p+1)."""
+    which pairs query blocks by their lists' overlap and returns out and lse
+    in GRID order (un-flattened by the kernel's stores); None calls
+    nabla_sparse_attn_fwd (pairs 2p, 2p+1; out and lse in flattened order)."""
     B, S, Hh, D = qf.shape
     if out is None:
         out = torch.empty_like(qf)

@@ -79,6 +79,7 @@ struct AttnArgs {
   int S, Hh, Nb;
   int grp_F;                // query blocks per frame for 2 x 2 (w, t) grouping, 0 = pairs 2p, 2p+1
   int grp_nbw;              // blocks per patch row (W / 8) when grp_F > 0
+  int out_H, out_W;         // > 0: O and LSE rows are stored in grid order of a T x H x W grid
   float scale_log2;         // scale * log2(e)
 };
 
@@ -500,7 +501,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // ---------------------------------------------------------------- epilogue
     const int qblk = half_blk[r >> 6];
     const bool row_valid = qblk >= 0;
-    const int64_t row_g = static_cast<int64_t>(row_valid ? qblk : 0) * 64 + (r & 63);
+    int64_t row_g = static_cast<int64_t>(row_valid ? qblk : 0) * 64 + (r & 63);
+    if (a.out_W > 0) {
+      // store in grid order (the inverse fractal flattening, fused): row r of
+      // block qblk is pixel (r / 8, r % 8) of the block's 8 x 8 patch
+      const int nbw = a.out_W >> 3, per_t = (a.out_H >> 3) * nbw;
+      const int blk = row_valid ? qblk : 0;
+      const int t = blk / per_t, rem = blk - t * per_t, bhh = rem / nbw, bww = rem - bhh * nbw;
+      row_g = (static_cast<int64_t>(t) * a.out_H + bhh * 8 + ((r & 63) >> 3)) * a.out_W + bww * 8 + (r & 7);
+    }
     if (ok && L_n > 0) ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((L_n - 1) & 1), ((L_n - 1) >> 1) & 1, abort_flag));
     tc_fence_after();
     __syncwarp();

@@ -234,7 +234,7 @@ void* g_noalloc_ptr[kMaxDevices] = {};
 // (w, t) grouping of query blocks (grp_F blocks per frame, grp_nbw per row).
 int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                        const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
-                       int grp_F, int grp_nbw, cudaStream_t stream) {
+                       int grp_F, int grp_nbw, int out_H, int out_W, cudaStream_t stream) {
   if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
   if (static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
   if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
@@ -266,6 +266,8 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   a.Nb = Nb;
   a.grp_F = grp_F;
   a.grp_nbw = grp_nbw;
+  a.out_H = out_H;
+  a.out_W = out_W;
   a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
   const dim3 grid((Nb + 1) / 2, Hh, B);
   if (D == 128) {
@@ -353,7 +355,7 @@ int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, 
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
                           nabla_stream_t stream) {
-  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, S, Hh, D, scale, out, lse, 0, 0,
+  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, S, Hh, D, scale, out, lse, 0, 0, 0, 0,
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -366,7 +368,7 @@ int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, c
   const int nbw = W / 8, F = (H / 8) * nbw;
   const bool groups = T % 2 == 0 && nbw % 2 == 0;
   return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
-                            groups ? F : 0, groups ? nbw : 0, reinterpret_cast<cudaStream_t>(stream));
+                            groups ? F : 0, groups ? nbw : 0, H, W, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,

@@ -156,15 +156,19 @@ int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const 
                           float* lse, nabla_stream_t stream);
 
 /* nabla_sparse_attn_fwd for a flattened T x H x W token grid (S = T*H*W,
- * P = 8): same arguments, layouts, results and errors, plus NABLA_ERR_INVALID
- * unless H and W are multiples of 8.  Knowing the grid lets the kernel choose
- * which two query blocks share one 128-row tile: when T and W/8 are even,
- * each 2 x 2 group of patch positions {(t, w), (t, w+1), (t+1, w), (t+1, w+1)}
- * (same patch row) is split along w or along t, whichever leaves fewer key
- * blocks listed by only one of the two (those run as half-masked tiles).
- * The pairing changes the work done, never which keys a query attends to:
- * every query block still attends exactly to its own kv_idx list.  With T or
- * W/8 odd it behaves as nabla_sparse_attn_fwd. */
+ * P = 8), with the output un-flattened: same inputs, lists, arithmetic and
+ * errors, plus NABLA_ERR_INVALID unless H and W are multiples of 8, but
+ *   out   device bf16 [B][S][Hh][D] in GRID order (the row of token
+ *         (t, h, w) is (t*H + h)*W + w), i.e. nabla_unflatten of the output
+ *         of nabla_sparse_attn_fwd, written directly by the kernel;
+ *   lse   fp32 [B][Hh][S] in grid order too (or NULL).
+ * Knowing the grid also lets the kernel choose which two query blocks share
+ * one 128-row tile: when T and W/8 are even, each 2 x 2 group of patch
+ * positions {(t, w), (t, w+1), (t+1, w), (t+1, w+1)} (same patch row) is
+ * split along w or along t, whichever leaves fewer key blocks listed by
+ * only one of the two (those run as half-masked tiles).  The pairing changes
+ * the work done, never which keys a query attends to.  With T or W/8 odd
+ * the pairs are 2p, 2p+1 as in nabla_sparse_attn_fwd. */
 int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                                const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
                                void* out, float* lse, nabla_stream_t stream);

@@ -22,6 +22,20 @@ MEAN_ABS = 2e-3
 LSE_ABS = 2e-3
 
 
+def flat_order(T: int, H: int, W: int, P: int = 8) -> np.ndarray:
+    """g[f] = grid row (t*H + h)*W + w of flattened row f: 8 x 8 patches of
+    each frame, patch-row-major, pixels row-major inside a patch."""
+    t, bh, bw, ph, pw = np.meshgrid(np.arange(T), np.arange(H // P), np.arange(W // P), np.arange(P), np.arange(P),
+                                    indexing="ij")
+    return ((t * H + bh * P + ph) * W + bw * P + pw).reshape(-1)
+
+
+def grid_to_flat_rows(x: torch.Tensor, T: int, H: int, W: int, dim: int) -> torch.Tensor:
+    """Rows of x along `dim` taken from grid order to flattened order."""
+    idx = torch.as_tensor(flat_order(T, H, W), device=x.device)
+    return x.index_select(dim, idx)
+
+
 class Case:
     """One workload on the device, flattened, with its mask and attention."""
 
@@ -43,10 +57,14 @@ class Case:
 
     def attention(self, grid: bool = True):
         """grid=True calls the grid-aware entry point (the one bench.py times),
-        grid=False the plain one."""
+        whose out and lse come in grid order; they are returned permuted back
+        to flattened order, so both paths compare against the oracle alike.
+        grid=False calls the plain entry point."""
         w = self.w
         out, lse = nabla.sparse_attn_fwd(self.qf, self.kf, self.vf, self.kv_count, self.kv_idx,
                                          grid=(w.T, w.H, w.W) if grid else None)
+        if grid:
+            out, lse = grid_to_flat_rows(out, w.T, w.H, w.W, 1), grid_to_flat_rows(lse, w.T, w.H, w.W, 2)
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
         return out, lse

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from _parity import Case, LSE_ABS, MAX_ABS, MEAN_ABS, check_attention, compare_masks, oracle_masks
+from _parity import Case, LSE_ABS, MAX_ABS, MEAN_ABS, check_attention, compare_masks, grid_to_flat_rows, oracle_masks
 from block_sparse_attention_flatten_b200 import inputs
 from block_sparse_attention_flatten_b200 import nabla
 
@@ -192,6 +192,8 @@ def test_long_lists(grid):
                                      torch.from_numpy(idx).cuda(), grid=grid)
     torch.cuda.synchronize()
     assert nabla.get_status() == 0
+    if grid is not None:
+        out, lse = grid_to_flat_rows(out, *grid, 1), grid_to_flat_rows(lse, *grid, 2)
     ref, ref_lse = oracle.attention(q, k, v, cnt, idx, 1.0 / math.sqrt(D))
     err = np.abs(out.double().cpu().numpy() - ref)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
@@ -256,6 +258,8 @@ def test_grid_pairing_takes_both_decisions(D):
         out, lse = nabla.sparse_attn_fwd(qd, kd, vd, cnt_d, idx_d, grid=grid)
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
+        if grid is not None:  # grid-order output: back to the flattened rows the lists index
+            out, lse = grid_to_flat_rows(out, T, H, W, 1), grid_to_flat_rows(lse, T, H, W, 2)
         err = np.abs(out.double().cpu().numpy() - ref)
         assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (grid, err.max(), err.mean())
         got_lse = lse.double().cpu().numpy()

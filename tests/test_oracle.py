@@ -423,3 +423,14 @@ def test_band_marks_a_rounding_tied_arg_max(oracle_lib):
     p2 = np.array([0.2, 0.39, 0.41, 0.0001], dtype=np.float32)  # clear arg-max: nothing band
     _, _, band2, _ = oracle_lib.cdf_keep(p2, 0.0)
     assert not band2.any()
+
+
+def test_parity_helper_flat_order_matches_oracle_flatten(oracle_lib):
+    """The tests' own flat->grid row index (used to compare grid-order
+    attention outputs) agrees with the oracle's flattening."""
+    from _parity import flat_order
+    for T, H, W in ((1, 8, 8), (2, 16, 24), (3, 24, 16)):
+        S = T * H * W
+        ids = np.arange(S, dtype=np.uint16).reshape(1, S, 1)
+        flat = oracle_lib.flatten(ids, T, H, W).reshape(-1)
+        assert np.array_equal(flat, flat_order(T, H, W).astype(np.uint16))
