@@ -1,14 +1,15 @@
 """Benchmark: one NABLA attention layer per step on B200, through the C ABI.
 
 A step is the whole hot path on one batch of synthetic input already
-resident in HBM, in three timed stages:
-  1. fractal flattening of Q and K fused with the mask's pooling
-     (nabla_flatten_pool_qk), and flattening of V (nabla_flatten);
-  2. the adaptive block mask from the pooled workspace: reduced attention,
-     CDF threshold, STA union, compaction (nabla_build_mask_pooled);
-  3. block-sparse attention on the kept tiles with the output stored back in
-     grid order, i.e. the unflattening fused into its stores
-     (nabla_sparse_attn_fwd_grid).
+resident in HBM, Q, K, V in grid order, in three timed stages:
+  1. pooling of Q and K straight from grid order: each block's 64 tokens
+     gathered in the fractal (flattened) order (nabla_flatten_pool_qk
+     without flattened copies);
+  2. the adaptive block mask on the pooled workspace: reduced attention, CDF
+     threshold, STA union, compaction (nabla_build_mask_pooled);
+  3. block-sparse attention on the kept tiles reading Q, K, V in grid order
+     through 5-D TMA boxes (the flattening done by the copy) and storing O
+     and the LSE in grid order (nabla_sparse_attn_fwd_grid).
 L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan13b]
@@ -80,10 +81,10 @@ def kept_flops(w, total_kept):
     return 4.0 * 64 * 64 * w.D * total_kept
 
 
-def flatten_pool_bytes(w):
-    """Compulsory bytes of the flatten stage: Q, K, V read and written once,
-    plus the pooled Q and K (fp32)."""
-    return 6.0 * w.B * w.S * w.Hh * w.D * 2 + 2.0 * 4 * w.B * w.Hh * w.Nb * w.D
+def pool_bytes(w):
+    """Compulsory bytes of the pooling stage: Q and K read once, the pooled
+    Q and K (fp32) written."""
+    return 2.0 * w.B * w.S * w.Hh * w.D * 2 + 2.0 * 4 * w.B * w.Hh * w.Nb * w.D
 
 
 def score_flops(w):
@@ -164,7 +165,6 @@ def run_gpu(args, rank, world, local_rank):
 
     # device-resident inputs and outputs (allocated once; the library allocates nothing)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    qf, kf, vf = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     og = torch.empty_like(qd)  # attention output, grid order
     kv_count = torch.empty((w.B, w.Hh, w.Nb), dtype=torch.int32, device=dev)
     kv_idx = torch.empty((w.B, w.Hh, w.Nb, w.Nb), dtype=torch.int32, device=dev)
@@ -176,20 +176,22 @@ def run_gpu(args, rank, world, local_rank):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        # Q and K: flattening fused with the mask's pooling; V: flattening
-        nabla.flatten_pool_qk(qd, kd, w.T, w.H, w.W, qf=qf, kf=kf, workspace=ws, thr=w.thr, sta=w.sta)
-        nabla.flatten(vd, w.T, w.H, w.W, out=vf)
+        # 1. pooling of Q and K straight from grid order (each block's 64
+        #    tokens gathered in flattened order; no flattened copies)
+        nabla.flatten_pool_qk(qd, kd, w.T, w.H, w.W, workspace=ws, thr=w.thr, sta=w.sta, write_flat=False)
         if ev is not None:
             ev[1].record(stream)
+        # 2. mask rows on the pooled workspace
         nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx)
         if ev is not None:
             ev[2].record(stream)
-        # attention with the output stored in grid order (un-flattening fused)
-        nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W))
+        # 3. attention reading Q, K, V in grid order through 5-D TMA boxes
+        #    and storing O in grid order
+        nabla.sparse_attn_fwd(qd, kd, vd, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W))
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 2 + 1 + 1  # flatten+pool, flatten V, mask rows, attention (stores O un-flattened)
+    launches_per_step = 3  # pooling, mask rows, attention
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -220,7 +222,7 @@ def run_gpu(args, rank, world, local_rank):
         return [events[s][a].elapsed_time(events[s][b]) for s in range(args.steps)]
 
     step_ms = stage(0, 3)
-    flat_ms, mask_ms, attn_ms = stage(0, 1), stage(1, 2), stage(2, 3)
+    pool_ms, mask_ms, attn_ms = stage(0, 1), stage(1, 2), stage(2, 3)
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -274,10 +276,9 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic",
         "config": config_dict(w),
-        "stages_ms": {"flatten_pool_qkv": statistics.mean(flat_ms), "mask_rows": mask_avg,
-                      "sparse_attn_unflatten": attn_avg},
+        "stages_ms": {"pool_qk": statistics.mean(pool_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg},
         "attn_tflops_kept": achieved,
-        "flatten_pool_gbs": flatten_pool_bytes(w) / (statistics.mean(flat_ms) * 1e-3) / 1e9,
+        "pool_gbs": pool_bytes(w) / (statistics.mean(pool_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",

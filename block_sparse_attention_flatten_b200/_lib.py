@@ -36,6 +36,7 @@ EXPORTS = (
     "nabla_build_mask_noalloc",
     "nabla_flatten_pool_qk",
     "nabla_build_mask_pooled",
+    "nabla_build_mask_grid",
     "nabla_sparse_attn_fwd",
     "nabla_sparse_attn_fwd_grid",
     "nabla_get_status",
@@ -84,6 +85,7 @@ def lib():
         L.nabla_build_mask_noalloc.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp]
         L.nabla_flatten_pool_qk.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, pp, vp, vp]
         L.nabla_build_mask_pooled.argtypes = [vp, i, i, i, i, i, i, pp, vp, vp, vp]
+        L.nabla_build_mask_grid.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
@@ -179,26 +181,54 @@ def build_mask(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: 
 
 
 def flatten_pool_qk(q: torch.Tensor, k: torch.Tensor, T: int, H: int, W: int, qf=None, kf=None, workspace=None,
-                    thr: float = 0.0, sta=(0, 0, 0), stream=None, P: int = 8):
+                    thr: float = 0.0, sta=(0, 0, 0), stream=None, P: int = 8, write_flat: bool = True):
     """Flatten Q and K (grid order [B, T*H*W, Hh, D], bf16, CUDA) and pool
-    them into a mask workspace in one pass (nabla_flatten_pool_qk).
-    Returns (qf, kf, workspace); finish the mask with :func:`build_mask_pooled`."""
+    them into a mask workspace in one pass (nabla_flatten_pool_qk); with
+    write_flat=False only the pooled vectors are written.
+    Returns (qf, kf, workspace) (qf, kf None without write_flat); finish the
+    mask with :func:`build_mask_pooled`."""
     B, S, Hh, D = q.shape
     prm = params(thr, sta, 0.0, P)
-    if qf is None:
+    if write_flat and qf is None:
         qf = torch.empty_like(q)
-    if kf is None:
+    if write_flat and kf is None:
         kf = torch.empty_like(k)
     if workspace is None:
         nbytes = mask_workspace_bytes(B, Hh, D, T, H, W, prm)
         if nbytes == 0:
             raise NablaError(NABLA_ERR_INVALID, "nabla_mask_workspace_bytes")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
-    _check(lib().nabla_flatten_pool_qk(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
-                                       _dev(qf, torch.bfloat16, "qf"), _dev(kf, torch.bfloat16, "kf"), B, Hh, D, T, H,
-                                       W, ctypes.byref(prm), _dev(workspace, torch.uint8, "workspace"),
+    qf_p = _dev(qf, torch.bfloat16, "qf") if write_flat else None
+    kf_p = _dev(kf, torch.bfloat16, "kf") if write_flat else None
+    _check(lib().nabla_flatten_pool_qk(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), qf_p, kf_p, B, Hh,
+                                       D, T, H, W, ctypes.byref(prm), _dev(workspace, torch.uint8, "workspace"),
                                        _stream(stream)), "nabla_flatten_pool_qk")
     return qf, kf, workspace
+
+
+def build_mask_grid(q: torch.Tensor, k: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),
+                    scale: float = 0.0, kv_count=None, kv_idx=None, workspace=None, stream=None, P: int = 8):
+    """:func:`build_mask` on Q, K in grid order [B, T*H*W, Hh, D] (no
+    flattened copies; nabla_build_mask_grid).  Returns (kv_count, kv_idx,
+    workspace)."""
+    B, S, Hh, D = q.shape
+    Nb = S // BLOCK
+    prm = params(thr, sta, scale, P)
+    dev = q.device
+    if kv_count is None:
+        kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)
+    if workspace is None:
+        nbytes = mask_workspace_bytes(B, Hh, D, T, H, W, prm)
+        if nbytes == 0:
+            raise NablaError(NABLA_ERR_INVALID, "nabla_mask_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(lib().nabla_build_mask_grid(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), B, Hh, D, T, H, W,
+                                       ctypes.byref(prm), _dev(kv_count, torch.int32, "kv_count"),
+                                       _dev(kv_idx, torch.int32, "kv_idx"), _dev(workspace, torch.uint8, "workspace"),
+                                       _stream(stream)), "nabla_build_mask_grid")
+    return kv_count, kv_idx, workspace
 
 
 def build_mask_pooled(workspace: torch.Tensor, B: int, Hh: int, D: int, T: int, H: int, W: int, thr: float,
@@ -256,10 +286,12 @@ def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_cou
                     stream=None, grid=None):
     """Block-sparse attention on the kept tiles; returns (out, lse or None).
 
-    grid = (T, H, W) of the flattened tokens calls nabla_sparse_attn_fwd_grid,
-    which pairs query blocks by their lists' overlap and returns out and lse
-    in GRID order (un-flattened by the kernel's stores); None calls
-    nabla_sparse_attn_fwd (pairs 2p, 2p+1; out and lse in flattened order)."""
+    grid = None: qf, kf, vf are flattened; nabla_sparse_attn_fwd (pairs 2p,
+    2p+1; out and lse in flattened order).
+    grid = (T, H, W): the three tensors are in GRID order (token (t, h, w) at
+    row (t*H + h)*W + w); nabla_sparse_attn_fwd_grid reads the blocks through
+    5-D TMA boxes, pairs query blocks by their lists' overlap and returns out
+    and lse in grid order."""
     B, S, Hh, D = qf.shape
     if out is None:
         out = torch.empty_like(qf)

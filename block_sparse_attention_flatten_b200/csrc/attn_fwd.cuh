@@ -80,6 +80,8 @@ struct AttnArgs {
   int grp_F;                // query blocks per frame for 2 x 2 (w, t) grouping, 0 = pairs 2p, 2p+1
   int grp_nbw;              // blocks per patch row (W / 8) when grp_F > 0
   int out_H, out_W;         // > 0: O and LSE rows are stored in grid order of a T x H x W grid
+  int in_T, in_nbw, in_per_t;  // in_nbw > 0: Q, K, V are in grid order, read through 5-D maps
+  uint32_t in_inv_per_t, in_inv_nbw;  // floor(2^32 / d) + 1 (0 for d = 1): j / d = umulhi(j, inv) for j, d < 2^14
   float scale_log2;         // scale * log2(e)
 };
 
@@ -113,6 +115,28 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int p = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
+  // One 64-token block j of Q, K or V, 64 columns (chunk c) of one head, as
+  // 64 rows of 128 bytes.  Flattened input: rows 64j..64j+63 (4-D map).
+  // Grid-order input: block j is the 8 x 8 patch (bh, bw) of frame t, read
+  // through a 5-D map (d, head, w, h, frame) whose box lists its pixels row
+  // by row, i.e. in the flattened order inside the block: the fractal
+  // flattening happens in the copy.
+  // All kChunks column chunks of block j; the block's patch coordinates are
+  // derived once, with multiply-high reciprocals (the producer is a single
+  // thread on the critical path, where integer divisions would cost).
+  auto load_block = [&](unsigned char* dst, const CUtensorMap* map, uint64_t* bar, int j, int chunk_stride) {
+    if (a.in_nbw > 0) {
+      // (an inverse of 0 stands for the divisor 1, whose reciprocal 2^32 does not fit)
+      const int t = a.in_inv_per_t ? static_cast<int>(__umulhi(static_cast<uint32_t>(j), a.in_inv_per_t)) : j;
+      const int rem = j - t * a.in_per_t;
+      const int bhh = a.in_inv_nbw ? static_cast<int>(__umulhi(static_cast<uint32_t>(rem), a.in_inv_nbw)) : rem;
+      const int bww = rem - bhh * a.in_nbw;
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_5d(dst + c * chunk_stride, map, bar, c * 64, hd, bww * 8, bhh * 8, b * a.in_T + t);
+    } else {
+      for (int c = 0; c < L::kChunks; ++c) tma_load_4d(dst + c * chunk_stride, map, bar, c * 64, hd, j * 64, b);
+    }
+  };
 
   // Candidate query blocks.  Group mode: cand = {(t,w), (t,w+1), (t+1,w),
   // (t+1,w+1)}; CTA slot 0 owns cand[0] in half 0 and slot 1 owns cand[3] in
@@ -159,15 +183,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tma_prefetch_desc(&tmQ);
     mbar_arrive_expect_tx(q_full, L::kQBytes);
     if (grouped) {
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_4d(sm + L::kQ + c * 128 * 128 + slot * 64 * 128, &tmQ, q_full, c * 64, hd,
-                    cand[slot ? 3 : 0] * 64, b);
+      load_block(sm + L::kQ + slot * 64 * 128, &tmQ, q_full, cand[slot ? 3 : 0], 128 * 128);
     } else {
       const int q1 = cand[1] >= 0 ? cand[1] : cand[0];
-      for (int c = 0; c < L::kChunks; ++c) {
-        tma_load_4d(sm + L::kQ + c * 128 * 128, &tmQ, q_full, c * 64, hd, cand[0] * 64, b);
-        tma_load_4d(sm + L::kQ + c * 128 * 128 + 64 * 128, &tmQ, q_full, c * 64, hd, q1 * 64, b);
-      }
+      load_block(sm + L::kQ, &tmQ, q_full, cand[0], 128 * 128);
+      load_block(sm + L::kQ + 64 * 128, &tmQ, q_full, q1, 128 * 128);
     }
   }
   if (warp == 4) {
@@ -264,8 +284,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       k0_early = true;
       if (lane == 0) {
         mbar_arrive_expect_tx(k_full, L::kKVBytes);
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(sm + L::kK + c * 64 * 128, &tmK, k_full, c * 64, hd, j0 * 64, b);
+        load_block(sm + L::kK, &tmK, k_full, j0, 64 * 128);
       }
     }
   }
@@ -276,9 +295,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (grouped && lane == 0) {
       // the other half of Q; q_full already expects its bytes
       const int other = slot ? x_half0 : x_half1;
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_4d(sm + L::kQ + c * 128 * 128 + (slot ? 0 : 64 * 128), &tmQ, q_full, c * 64, hd, cand[other] * 64,
-                    b);
+      load_block(sm + L::kQ + (slot ? 0 : 64 * 128), &tmQ, q_full, cand[other], 128 * 128);
     }
     if (lane == 0) {
       half_blk[0] = cand[x_half0];
@@ -339,8 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           }
           const int j = static_cast<int>(list[n] & 0x3FFFu);
           mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(sm + L::kK + s * L::kKVBytes + c * 64 * 128, &tmK, k_full + s, c * 64, hd, j * 64, b);
+          load_block(sm + L::kK + s * L::kKVBytes, &tmK, k_full + s, j, 64 * 128);
         }
         if (n < L_n) k_issued = n + 1;
         if (n >= 1) {
@@ -351,8 +367,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           }
           const int j = static_cast<int>(list[m] & 0x3FFFu);
           mbar_arrive_expect_tx(v_full + s, L::kKVBytes);
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_load_4d(sm + L::kV + s * L::kKVBytes + c * 64 * 128, &tmV, v_full + s, c * 64, hd, j * 64, b);
+          load_block(sm + L::kV + s * L::kKVBytes, &tmV, v_full + s, j, 64 * 128);
           v_issued = m + 1;
         }
       }

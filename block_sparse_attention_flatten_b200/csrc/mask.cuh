@@ -33,9 +33,9 @@ namespace nabla {
 // Thread c handles elements 8c..8c+7 of a token row (Hh*D elements), summing
 // the block's 64 rows in ascending flattened order in fp32.
 // kFlatten = false: q, k are already flattened.  kFlatten = true: q, k are in
-// grid order; the kernel also writes the block's 64 rows, permuted, to
-// qf_out / kf_out (fractal flattening fused with the pooling, so Q and K are
-// read once).  Flattened rows 8u..8u+7 of a block are one run of 8
+// grid order and the block's 64 rows are gathered in flattened order; if
+// qf_out / kf_out are given the kernel also writes them there (fractal
+// flattening fused with the pooling, so Q and K are read once).  Flattened rows 8u..8u+7 of a block are one run of 8
 // consecutive grid rows (patch row u).
 template <bool kFlatten>
 __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restrict__ q,
@@ -57,9 +57,10 @@ __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restri
     src0 = batch_rows + (static_cast<int64_t>(t) * H + bh * 8) * W + bw * 8;
   }
   const uint4* base = reinterpret_cast<const uint4*>(x) + src0 * chunks;
-  uint4* dst = kFlatten ? reinterpret_cast<uint4*>(blockIdx.z == 0 ? qf_out : kf_out) +
-                              (batch_rows + static_cast<int64_t>(i) * 64) * chunks
-                        : nullptr;
+  __nv_bfloat16* flat_out = blockIdx.z == 0 ? qf_out : kf_out;
+  uint4* dst = (kFlatten && flat_out != nullptr)
+                   ? reinterpret_cast<uint4*>(flat_out) + (batch_rows + static_cast<int64_t>(i) * 64) * chunks
+                   : nullptr;
   for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
     float acc[8];
 #pragma unroll
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restri
 #pragma unroll
       for (int u = 0; u < 8; ++u)
         v[u] = kFlatten ? __ldcs(base + (src_row + u) * chunks + c) : __ldg(base + (src_row + u) * chunks + c);
-      if (kFlatten) {
+      if (kFlatten && dst != nullptr) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) dst[static_cast<int64_t>(r0 + u) * chunks + c] = v[u];
       }

@@ -93,6 +93,24 @@ bool make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int Hh, int D
   return r == CUDA_SUCCESS;
 }
 
+// Grid-order BSHD tensor [B][T][H][W][Hh][D] seen as 5-D (d, head, w, h,
+// frame = b*T + t); the box (64, 1, 8, 8, 1) is one 64-token block of one
+// head (an 8 x 8 patch), its pixels row by row, 128-byte swizzled.
+bool make_grid_map(CUtensorMap* m, const void* base, int B, int T, int H, int W, int Hh, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(Hh) * D * 2;  // bytes per token
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hh), static_cast<cuuint64_t>(W),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T) * B};
+  const cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * 2, row, row * W, row * W * H};
+  const cuuint32_t box[5] = {64, 1, 8, 8, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int check_grid(int B, int T, int H, int W, int P) {
   if (B <= 0 || T <= 0 || H <= 0 || W <= 0) return NABLA_ERR_INVALID;
   if (P != 8 || H % P != 0 || W % P != 0) return NABLA_ERR_INVALID;
@@ -234,7 +252,7 @@ void* g_noalloc_ptr[kMaxDevices] = {};
 // (w, t) grouping of query blocks (grp_F blocks per frame, grp_nbw per row).
 int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                        const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
-                       int grp_F, int grp_nbw, int out_H, int out_W, cudaStream_t stream) {
+                       int grp_F, int grp_nbw, int grid_T, int out_H, int out_W, cudaStream_t stream) {
   if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
   if (static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
   if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
@@ -252,10 +270,16 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   if (Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
   const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
 
+  // grid_T > 0: q, k, v are in grid order of a grid_T x out_H x out_W grid
   CUtensorMap tq, tk, tv;
-  if (!make_bshd_map(&tq, qf, B, S, Hh, D, 64) || !make_bshd_map(&tk, kf, B, S, Hh, D, 64) ||
-      !make_bshd_map(&tv, vf, B, S, Hh, D, 64))
+  if (grid_T > 0) {
+    if (!make_grid_map(&tq, qf, B, grid_T, out_H, out_W, Hh, D) || !make_grid_map(&tk, kf, B, grid_T, out_H, out_W, Hh, D) ||
+        !make_grid_map(&tv, vf, B, grid_T, out_H, out_W, Hh, D))
+      return NABLA_ERR_CUDA;
+  } else if (!make_bshd_map(&tq, qf, B, S, Hh, D, 64) || !make_bshd_map(&tk, kf, B, S, Hh, D, 64) ||
+             !make_bshd_map(&tv, vf, B, S, Hh, D, 64)) {
     return NABLA_ERR_CUDA;
+  }
   AttnArgs a;
   a.kv_count = kv_count;
   a.kv_idx = kv_idx;
@@ -268,6 +292,13 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   a.grp_nbw = grp_nbw;
   a.out_H = out_H;
   a.out_W = out_W;
+  a.in_T = grid_T;
+  a.in_nbw = grid_T > 0 ? out_W / 8 : 0;
+  a.in_per_t = grid_T > 0 ? (out_H / 8) * (out_W / 8) : 0;
+  // exact quotients by multiply-high for block indices and divisors < 2^14
+  auto inv = [](int d) -> uint32_t { return d > 1 ? static_cast<uint32_t>((uint64_t{1} << 32) / d + 1) : 0u; };
+  a.in_inv_per_t = inv(a.in_per_t);
+  a.in_inv_nbw = inv(a.in_nbw);
   a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
   const dim3 grid((Nb + 1) / 2, Hh, B);
   if (D == 128) {
@@ -333,11 +364,25 @@ int nabla_flatten_pool_qk(const void* q, const void* k, void* qf, void* kf, int 
   MaskPlan mp;
   int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, nullptr, nullptr, &mp);
   if (rc != NABLA_OK) return rc;
-  if (q == nullptr || k == nullptr || qf == nullptr || kf == nullptr) return NABLA_ERR_INVALID;
-  if (q == qf || q == kf || k == qf || k == kf || qf == kf) return NABLA_ERR_INVALID;
+  if (q == nullptr || k == nullptr || (qf == nullptr) != (kf == nullptr)) return NABLA_ERR_INVALID;
+  if (qf != nullptr && (q == qf || q == kf || k == qf || k == kf || qf == kf)) return NABLA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(qf) || !aligned16(kf)) return NABLA_ERR_ALIGN;
   if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
   return launch_pool<true>(mp, B, q, k, qf, kf, stream);
+}
+
+int nabla_build_mask_grid(const void* q, const void* k, int B, int Hh, int D, int T, int H, int W,
+                          const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, void* workspace,
+                          nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  MaskPlan mp;
+  int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, kv_count, kv_idx, &mp);
+  if (rc != NABLA_OK) return rc;
+  if (q == nullptr || k == nullptr || kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
+  if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
+  if ((rc = launch_pool<true>(mp, B, q, k, nullptr, nullptr, stream)) != NABLA_OK) return rc;
+  return launch_mask_rows(mp, B, stream);
 }
 
 int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, int H, int W,
@@ -355,11 +400,11 @@ int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, 
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
                           nabla_stream_t stream) {
-  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, S, Hh, D, scale, out, lse, 0, 0, 0, 0,
+  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, S, Hh, D, scale, out, lse, 0, 0, 0, 0, 0,
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
-int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, const int32_t* kv_count,
                                const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
                                void* out, float* lse, nabla_stream_t stream) {
   if (T <= 0 || H <= 0 || W <= 0 || H % 8 != 0 || W % 8 != 0) return NABLA_ERR_INVALID;
@@ -367,8 +412,8 @@ int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, c
   if (S > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
   const int nbw = W / 8, F = (H / 8) * nbw;
   const bool groups = T % 2 == 0 && nbw % 2 == 0;
-  return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
-                            groups ? F : 0, groups ? nbw : 0, H, W, reinterpret_cast<cudaStream_t>(stream));
+  return sparse_attn_launch(q, k, v, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
+                            groups ? F : 0, groups ? nbw : 0, T, H, W, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,

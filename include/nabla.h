@@ -123,10 +123,21 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
  *   q, k        device bf16 [B][T*H*W][Hh][D], grid order.
  *   qf, kf      device bf16 [B][T*H*W][Hh][D] outputs, flattened order.
  *   workspace   as for nabla_build_mask.
- * The four tensors must not alias.  Errors: as nabla_build_mask (params are
- * validated the same way although only P is used here). */
+ * qf and kf may both be NULL: then only the pooled vectors are written (the
+ * pooling stage of nabla_build_mask_grid on its own).  The tensors must not
+ * alias.  Errors: as nabla_build_mask (params are validated the same way
+ * although only P is used here). */
 int nabla_flatten_pool_qk(const void* q, const void* k, void* qf, void* kf, int B, int Hh, int D, int T, int H,
                           int W, const nabla_params* params, void* workspace, nabla_stream_t stream);
+
+/* nabla_build_mask on Q and K in GRID order ([B][T*H*W][Hh][D], row of
+ * token (t, h, w) = (t*H + h)*W + w): the pooling gathers each block's 64
+ * tokens in the flattened order (identical bits to pooling the flattened
+ * tensors), then stages 2-4 run as in nabla_build_mask.  Same arguments,
+ * results and errors as nabla_build_mask with q, k in place of qf, kf. */
+int nabla_build_mask_grid(const void* q, const void* k, int B, int Hh, int D, int T, int H, int W,
+                          const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, void* workspace,
+                          nabla_stream_t stream);
 
 /* Stages 2-4 of nabla_build_mask (reduced attention, CDF threshold, STA
  * union, compaction) on a workspace that already holds the pooled queries
@@ -155,21 +166,30 @@ int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const 
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out,
                           float* lse, nabla_stream_t stream);
 
-/* nabla_sparse_attn_fwd for a flattened T x H x W token grid (S = T*H*W,
- * P = 8), with the output un-flattened: same inputs, lists, arithmetic and
- * errors, plus NABLA_ERR_INVALID unless H and W are multiples of 8, but
- *   out   device bf16 [B][S][Hh][D] in GRID order (the row of token
- *         (t, h, w) is (t*H + h)*W + w), i.e. nabla_unflatten of the output
- *         of nabla_sparse_attn_fwd, written directly by the kernel;
- *   lse   fp32 [B][Hh][S] in grid order too (or NULL).
- * Knowing the grid also lets the kernel choose which two query blocks share
- * one 128-row tile: when T and W/8 are even, each 2 x 2 group of patch
- * positions {(t, w), (t, w+1), (t+1, w), (t+1, w+1)} (same patch row) is
- * split along w or along t, whichever leaves fewer key blocks listed by
- * only one of the two (those run as half-masked tiles).  The pairing changes
- * the work done, never which keys a query attends to.  With T or W/8 odd
- * the pairs are 2p, 2p+1 as in nabla_sparse_attn_fwd. */
-int nabla_sparse_attn_fwd_grid(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
+/* Block-sparse attention on tensors in GRID order: the fractal flattening
+ * and its inverse happen inside the kernel, so no flattened copy of Q, K, V
+ * or O is ever materialised.  For a T x H x W grid (S = T*H*W, P = 8):
+ *   q, k, v   device bf16 [B][S][Hh][D] in grid order: the row of token
+ *             (t, h, w) is (t*H + h)*W + w.  Block j of the flattened order
+ *             (the 8 x 8 patch (bh, bw) of frame t, j = t*(H/8)*(W/8) +
+ *             bh*(W/8) + bw) is fetched by one 5-D TMA box (d, head, w, h,
+ *             frame) whose rows come out in the flattened order inside the
+ *             block.
+ *   kv_count, kv_idx   block lists over flattened block indices, as
+ *             written by any of the mask entry points.
+ *   out       device bf16 [B][S][Hh][D] in grid order;
+ *   lse       fp32 [B][Hh][S] in grid order (or NULL).
+ * Results equal nabla_unflatten of nabla_sparse_attn_fwd run on the
+ * flattened tensors (up to the summation order of the online softmax, see
+ * the pairing below).  Knowing the grid also lets the kernel choose which
+ * two query blocks share one 128-row tile: when T and W/8 are even, each
+ * 2 x 2 group of patch positions {(t, w), (t, w+1), (t+1, w), (t+1, w+1)}
+ * (same patch row) is split along w or along t, whichever leaves fewer key
+ * blocks listed by only one of the two (those run as half-masked tiles);
+ * with T or W/8 odd the pairs are 2p, 2p+1.  Errors: as
+ * nabla_sparse_attn_fwd, plus NABLA_ERR_INVALID unless H and W are
+ * multiples of 8. */
+int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, const int32_t* kv_count,
                                const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
                                void* out, float* lse, nabla_stream_t stream);
 

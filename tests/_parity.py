@@ -36,6 +36,12 @@ def grid_to_flat_rows(x: torch.Tensor, T: int, H: int, W: int, dim: int) -> torc
     return x.index_select(dim, idx)
 
 
+def flat_to_grid_rows(x: torch.Tensor, T: int, H: int, W: int, dim: int) -> torch.Tensor:
+    """Rows of x along `dim` taken from flattened order to grid order."""
+    idx = torch.as_tensor(flat_order(T, H, W), device=x.device)
+    return torch.empty_like(x).index_copy_(dim, idx, x)
+
+
 class Case:
     """One workload on the device, flattened, with its mask and attention."""
 
@@ -56,15 +62,18 @@ class Case:
         assert nabla.get_status() == 0
 
     def attention(self, grid: bool = True):
-        """grid=True calls the grid-aware entry point (the one bench.py times),
-        whose out and lse come in grid order; they are returned permuted back
-        to flattened order, so both paths compare against the oracle alike.
-        grid=False calls the plain entry point."""
+        """grid=True calls the grid entry point (the one bench.py times) on the
+        grid-order tensors; its out and lse, in grid order, are returned
+        permuted back to flattened order, so both paths compare against the
+        oracle alike.  grid=False calls the plain entry point on the
+        flattened tensors."""
         w = self.w
-        out, lse = nabla.sparse_attn_fwd(self.qf, self.kf, self.vf, self.kv_count, self.kv_idx,
-                                         grid=(w.T, w.H, w.W) if grid else None)
-        if grid:
+        if grid:  # grid-order inputs and outputs
+            out, lse = nabla.sparse_attn_fwd(self.qd, self.kd, self.vd, self.kv_count, self.kv_idx,
+                                             grid=(w.T, w.H, w.W))
             out, lse = grid_to_flat_rows(out, w.T, w.H, w.W, 1), grid_to_flat_rows(lse, w.T, w.H, w.W, 2)
+        else:
+            out, lse = nabla.sparse_attn_fwd(self.qf, self.kf, self.vf, self.kv_count, self.kv_idx)
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
         return out, lse

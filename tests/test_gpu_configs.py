@@ -29,16 +29,17 @@ def run_config(w: inputs.Workload, n_blocks: int = N_SAMPLED_BLOCKS):
     bad, in_band, nband = compare_masks(case, status)
     kept = float(case.kv_count.double().sum().item()) / (w.B * w.Hh * w.Nb * w.Nb)
     del status
-    # the fused path bench.py times (flatten + pool in one pass, mask from the
-    # pooled workspace) must give the same flattened tensors and block lists
-    qf2, kf2, ws2 = nabla.flatten_pool_qk(case.qd, case.kd, w.T, w.H, w.W, thr=w.thr, sta=w.sta)
-    cnt2, idx2 = nabla.build_mask_pooled(ws2, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta)
+    # the mask path bench.py times (pooling straight from grid order) must
+    # give the same pooled vectors and block lists
+    cnt2, idx2, ws2 = nabla.build_mask_grid(case.qd, case.kd, w.T, w.H, w.W, w.thr, w.sta)
     torch.cuda.synchronize()
-    assert torch.equal(qf2, case.qf) and torch.equal(kf2, case.kf)
+    for a_, b_ in zip(nabla.pooled_from_workspace(ws2, w.B, w.Hh, w.Nb, w.D),
+                      nabla.pooled_from_workspace(case.ws, w.B, w.Hh, w.Nb, w.D)):
+        assert torch.equal(a_, b_)
     assert torch.equal(cnt2, case.kv_count)
     valid = torch.arange(w.Nb, device=cnt2.device).view(1, 1, 1, -1) < cnt2.unsqueeze(-1)
     assert torch.equal(torch.where(valid, idx2, -1), torch.where(valid, case.kv_idx, -1))
-    del qf2, kf2, ws2, cnt2, idx2, valid
+    del ws2, cnt2, idx2, valid
     out, lse = case.attention()
     qblocks = inputs.sample_query_blocks(w.Nb, n_blocks, seed=1234)
     mx, mean, lse_err = check_attention(case, out, lse, qblocks, host)

@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import oracle
-from _parity import Case, LSE_ABS, MAX_ABS, MEAN_ABS, check_attention, compare_masks, grid_to_flat_rows, oracle_masks
+from _parity import (Case, LSE_ABS, MAX_ABS, MEAN_ABS, check_attention, compare_masks, flat_to_grid_rows,
+                     grid_to_flat_rows, oracle_masks)
 from block_sparse_attention_flatten_b200 import inputs
 from block_sparse_attention_flatten_b200 import nabla
 
@@ -89,9 +90,14 @@ def test_fused_flatten_pool_and_pooled_mask(w):
     assert np.array_equal(qg.cpu().numpy(), oracle.pool(qf_ref))
     assert np.array_equal(kg.cpu().numpy(), oracle.pool(kf_ref))
     cnt2, idx2, _ = nabla.build_mask(qf, kf, w.T, w.H, w.W, w.thr, w.sta)
-    assert torch.equal(cnt, cnt2)
+    cnt3, idx3, ws3 = nabla.build_mask_grid(qd, kd, w.T, w.H, w.W, w.thr, w.sta)  # straight from grid order
+    torch.cuda.synchronize()
+    for a_, b_ in zip(nabla.pooled_from_workspace(ws3, w.B, w.Hh, w.Nb, w.D), (qg, kg)):
+        assert torch.equal(a_, b_)  # the pooled vectors (the workspace's padding columns are never written)
     valid = torch.arange(w.Nb, device="cuda").view(1, 1, 1, -1) < cnt.unsqueeze(-1)
-    assert torch.equal(torch.where(valid, idx, -1), torch.where(valid, idx2, -1))
+    for c_, i_ in ((cnt2, idx2), (cnt3, idx3)):
+        assert torch.equal(cnt, c_)
+        assert torch.equal(torch.where(valid, idx, -1), torch.where(valid, i_, -1))
 
 
 def dense_grid(q, k, v, scale):
@@ -188,12 +194,16 @@ def test_long_lists(grid):
         sel = np.sort(rng.choice(Nb, size=n, replace=False))
         cnt[0, 0, i] = n
         idx[0, 0, i, :n] = sel
-    out, lse = nabla.sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cnt).cuda(),
-                                     torch.from_numpy(idx).cuda(), grid=grid)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    cnt_d, idx_d = torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda()
+    if grid is None:
+        out, lse = nabla.sparse_attn_fwd(qd, kd, vd, cnt_d, idx_d)
+    else:
+        qg, kg, vg = (flat_to_grid_rows(x, *grid, 1) for x in (qd, kd, vd))
+        out, lse = nabla.sparse_attn_fwd(qg, kg, vg, cnt_d, idx_d, grid=grid)
+        out, lse = grid_to_flat_rows(out, *grid, 1), grid_to_flat_rows(lse, *grid, 2)
     torch.cuda.synchronize()
     assert nabla.get_status() == 0
-    if grid is not None:
-        out, lse = grid_to_flat_rows(out, *grid, 1), grid_to_flat_rows(lse, *grid, 2)
     ref, ref_lse = oracle.attention(q, k, v, cnt, idx, 1.0 / math.sqrt(D))
     err = np.abs(out.double().cpu().numpy() - ref)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
@@ -255,11 +265,14 @@ def test_grid_pairing_takes_both_decisions(D):
     idx_d = torch.from_numpy(idx).cuda()
     ref, ref_lse = oracle.attention(q, k, v, cnt, idx, 1.0 / math.sqrt(D))
     for grid in (None, (T, H, W)):
-        out, lse = nabla.sparse_attn_fwd(qd, kd, vd, cnt_d, idx_d, grid=grid)
+        if grid is None:  # q, k, v taken as flattened tensors
+            out, lse = nabla.sparse_attn_fwd(qd, kd, vd, cnt_d, idx_d)
+        else:  # the same tensors in grid order; outputs back to flattened rows
+            qg, kg, vg = (flat_to_grid_rows(x, T, H, W, 1) for x in (qd, kd, vd))
+            out, lse = nabla.sparse_attn_fwd(qg, kg, vg, cnt_d, idx_d, grid=grid)
+            out, lse = grid_to_flat_rows(out, T, H, W, 1), grid_to_flat_rows(lse, T, H, W, 2)
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
-        if grid is not None:  # grid-order output: back to the flattened rows the lists index
-            out, lse = grid_to_flat_rows(out, T, H, W, 1), grid_to_flat_rows(lse, T, H, W, 2)
         err = np.abs(out.double().cpu().numpy() - ref)
         assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (grid, err.max(), err.mean())
         got_lse = lse.double().cpu().numpy()
