@@ -240,14 +240,27 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     unsigned long long best = 0;  // (bits(e) << 32) | j; max = arg-max, ties to the larger j
     unsigned long long total = 0;
     int n_tiny = 0;  // blocks with e < 2^-63
+    // first pass of the boundary search (step 3), on the way: masses and
+    // counts of the quarters [2^-63, 2^-47), [2^-47, 2^-31), [2^-31, 2^-15)
+    // of the starting range [2^-63, 2)
+    unsigned long long fm0 = 0, fm1 = 0, fm2 = 0;
+    int fc0 = 0, fc1 = 0, fc2 = 0;
     for (int j = lane; j < Nb; j += 32) {
       const float e = expf(row[j] - m);
       row[j] = e;
       const uint32_t u = __float_as_uint(e);
       const unsigned long long key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
       best = key > best ? key : best;
-      total += mass_bits(u);
+      const unsigned long long w = mass_bits(u);
+      total += w;
       n_tiny += u < 0x20000000u;
+      const uint32_t q = (u - 0x20000000u) >> 27;  // 0..3 for u in [0x20000000, 0x40000000)
+      fm0 += q == 0 ? w : 0ull;
+      fm1 += q == 1 ? w : 0ull;
+      fm2 += q == 2 ? w : 0ull;
+      fc0 += q == 0;
+      fc1 += q == 1;
+      fc2 += q == 2;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -279,6 +292,44 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
       int span = 29;
       unsigned long long below = 0;  // mass(bits(e) < prefix)
       int n_lo = n_tiny, n_hi = Nb;  // blocks below prefix, below prefix + 2^span
+      // Narrows [prefix, prefix + 2^span) to the quarter (of width 2^lo) that
+      // holds bits(e*), given the masses and counts of its first three
+      // quarters.
+      auto narrow = [&](unsigned long long m0, unsigned long long m1, unsigned long long m2, int c0, int c1, int c2,
+                        int lo) {
+        const unsigned long long s1 = below + m0, s2 = s1 + m1, s3 = s2 + m2;
+        if (s3 <= tau_m) {
+          prefix += 3u << lo;
+          below = s3;
+          n_lo += c0 + c1 + c2;
+        } else if (s2 <= tau_m) {
+          prefix += 2u << lo;
+          below = s2;
+          n_lo += c0 + c1;
+          n_hi = n_lo + c2;
+        } else if (s1 <= tau_m) {
+          prefix += 1u << lo;
+          below = s1;
+          n_lo += c0;
+          n_hi = n_lo + c1;
+        } else {
+          n_hi = n_lo + c0;
+        }
+        span = lo;
+      };
+      if (n_hi - n_lo > 32) {
+        // the first pass was done with the exponentials
+        fm0 = warp_sum_u64(fm0);
+        fm1 = warp_sum_u64(fm1);
+        fm2 = warp_sum_u64(fm2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          fc0 += __shfl_xor_sync(0xffffffffu, fc0, o);
+          fc1 += __shfl_xor_sync(0xffffffffu, fc1, o);
+          fc2 += __shfl_xor_sync(0xffffffffu, fc2, o);
+        }
+        narrow(fm0, fm1, fm2, fc0, fc1, fc2, 27);
+      }
       while (span > 0 && n_hi - n_lo > 32) {
         const int lo = span > 2 ? span - 2 : 0;
         const uint32_t range = 1u << span;
@@ -307,25 +358,7 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
           c1 += __shfl_xor_sync(0xffffffffu, c1, o);
           c2 += __shfl_xor_sync(0xffffffffu, c2, o);
         }
-        const unsigned long long s1 = below + m0, s2 = s1 + m1, s3 = s2 + m2;
-        if (s3 <= tau_m) {
-          prefix += 3u << lo;
-          below = s3;
-          n_lo += c0 + c1 + c2;
-        } else if (s2 <= tau_m) {
-          prefix += 2u << lo;
-          below = s2;
-          n_lo += c0 + c1;
-          n_hi = n_lo + c2;
-        } else if (s1 <= tau_m) {
-          prefix += 1u << lo;
-          below = s1;
-          n_lo += c0;
-          n_hi = n_lo + c1;
-        } else {
-          n_hi = n_lo + c0;
-        }
-        span = lo;
+        narrow(m0, m1, m2, c0, c1, c2, lo);
       }
       const uint32_t range = 1u << span;
       if (n_hi - n_lo <= 32) {
