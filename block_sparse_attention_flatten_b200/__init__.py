@@ -4,10 +4,18 @@ The compute path is libnabla.so (hand-written CUDA, C ABI in
 include/nabla.h); this package is its thin Python binding.  PyTorch only
 provides device memory and streams.
 
+Grid-order tensors (token (t, h, w) at row (t*H + h)*W + w), no flattened
+copies -- the fractal flattening happens inside the kernels:
+
     from block_sparse_attention_flatten_b200 import nabla
-    qf = nabla.flatten(q, T, H, W)                       # per tensor, once per sequence
+    kv_count, kv_idx, _ = nabla.build_mask_grid(q, k, T, H, W, thr=0.9, sta=(3, 3, 3))
+    o, lse = nabla.sparse_attn_fwd(q, k, v, kv_count, kv_idx, grid=(T, H, W))
+
+Flattened tensors (e.g. flattened once per sequence):
+
+    qf = nabla.flatten(q, T, H, W)                       # per tensor
     kv_count, kv_idx, _ = nabla.build_mask(qf, kf, T, H, W, thr=0.9, sta=(3, 3, 3))
-    of, lse = nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx, grid=(T, H, W))
+    of, lse = nabla.sparse_attn_fwd(qf, kf, vf, kv_count, kv_idx)
     o = nabla.unflatten(of, T, H, W)
 """
 from . import _lib as nabla  # noqa: F401
