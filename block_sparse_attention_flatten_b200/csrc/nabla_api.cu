@@ -223,8 +223,11 @@ int launch_mask_rows(const MaskPlan& mp, int B, cudaStream_t stream) {
   if (16 * per_row <= 64u * 1024u) return launch_mask<16>(mp.a, B, mp.di, stream);
   const size_t fit = (64u * 1024u) / per_row;
   if (fit >= 8) return launch_mask<8>(mp.a, B, mp.di, stream);
-  if (fit >= 4) return launch_mask<4>(mp.a, B, mp.di, stream);
-  if (mask_smem_bytes(2, D, Nb) <= static_cast<size_t>(mp.di.max_smem_optin)) return launch_mask<2>(mp.a, B, mp.di, stream);
+  // beyond ~4,096 blocks: 4 rows while they fit the SM's shared memory
+  // (then one CTA per SM), else 2
+  const size_t optin = static_cast<size_t>(mp.di.max_smem_optin);
+  if (fit >= 4 || mask_smem_bytes(4, D, Nb) <= optin) return launch_mask<4>(mp.a, B, mp.di, stream);
+  if (mask_smem_bytes(2, D, Nb) <= optin) return launch_mask<2>(mp.a, B, mp.di, stream);
   return NABLA_ERR_INVALID;
 }
 
