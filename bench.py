@@ -51,6 +51,22 @@ CONFIGS.update({f"sweep-a{w.alpha}-t{w.thr}": w for w in inputs.sweep_points()})
 L2_FLUSH_BYTES = 256 << 20
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks (x itself on one rank): a step is timed
+    on every rank's device and the slowest rank sets the job's time."""
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized() and \
+            torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flop_per_step_per_rank: float, steps: int, max_ms: float) -> float:
+    """Units all ranks processed over the slowest rank's time: each of the
+    `world` replicas runs `steps` steps of flop_per_step_per_rank FLOP."""
+    return world * flop_per_step_per_rank * steps / (max_ms * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -223,11 +239,7 @@ def run_gpu(args, rank, world, local_rank):
 
     step_ms = stage(0, 3)
     pool_ms, mask_ms, attn_ms = stage(0, 1), stage(1, 2), stage(2, 3)
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms_max = float(t.item())
+    total_ms_max = max_over_ranks(sum(step_ms), dev)
 
     # end to end through the public API: pinned host inputs in, result out
     e2e = None
@@ -248,14 +260,12 @@ def run_gpu(args, rank, world, local_rank):
             torch.cuda.synchronize()
             if s > 0:
                 e2e_ms.append(e0.elapsed_time(e1))
-        te = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+        te = max_over_ranks(sum(e2e_ms), dev)
         bi = 3 * qd.numel() * qd.element_size()
         bo = og.numel() * og.element_size()
-        e2e = {"value": world * kept_flops(w, total_kept) * len(e2e_ms) / (float(te.item()) * 1e-3) / 1e12,
+        e2e = {"value": whole_job_tflops(world, kept_flops(w, total_kept), len(e2e_ms), te),
                "unit": "TFLOP/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
-               "ms_per_step": float(te.item()) / len(e2e_ms)}
+               "ms_per_step": te / len(e2e_ms)}
 
     peak_tf, peak_gbs, peak_kind = load_peaks()
     attn_avg = statistics.mean(attn_ms)
@@ -264,7 +274,7 @@ def run_gpu(args, rank, world, local_rank):
     traffic = load_traffic(args.config)
     result = {
         "metric": METRIC,
-        "value": world * kept_flops(w, total_kept) * args.steps / (total_ms_max * 1e-3) / 1e12,
+        "value": whole_job_tflops(world, kept_flops(w, total_kept), args.steps, total_ms_max),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
