@@ -97,6 +97,12 @@ def kept_flops(w, total_kept):
     return 4.0 * 64 * 64 * w.D * total_kept
 
 
+def mask_bytes(w, total_kept):
+    """Compulsory bytes of the whole mask build: Q and K read once, the
+    block counts and the kept list entries written."""
+    return 2.0 * w.B * w.S * w.Hh * w.D * 2 + 4.0 * w.B * w.Hh * w.Nb + 4.0 * total_kept
+
+
 def pool_bytes(w):
     """Compulsory bytes of the pooling stage: Q and K read once, the pooled
     Q and K (fp32) written."""
@@ -286,7 +292,13 @@ def run_gpu(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic",
         "config": config_dict(w),
+        # per layer: the whole step, since Q, K, V, O stay in grid order (the
+        # flattening and its inverse happen inside the pooling and attention)
+        "ms_per_layer": statistics.mean(pool_ms) + mask_avg + attn_avg,
         "stages_ms": {"pool_qk": statistics.mean(pool_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg},
+        # mask build = pooling + rows: Q and K read once, kv_count and the kept
+        # kv_idx entries written, over its time
+        "mask_build_gbs": mask_bytes(w, total_kept) / ((statistics.mean(pool_ms) + mask_avg) * 1e-3) / 1e9,
         "attn_tflops_kept": achieved,
         "pool_gbs": pool_bytes(w) / (statistics.mean(pool_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
