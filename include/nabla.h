@@ -4,16 +4,26 @@
  *
  * The method (page "Resumo Tecnico: NABLA - Atencao de Bloco Adaptativa de
  * Vizinhanca para Geracao de Video Eficiente", gist.science paper 2507.13546,
- * section "Metodologia: NABLA") has three stages, each an entry point here:
- *   1. fractal flattening of the T x H x W token grid   -> nabla_flatten
- *   2. adaptive block mask (pool, reduced attention, CDF
- *      threshold, optional STA union)                   -> nabla_build_mask
- *   3. attention on the kept 64 x 64 tiles               -> nabla_sparse_attn_fwd
+ * section "Metodologia: NABLA") has three stages:
+ *   1. fractal flattening of the T x H x W token grid
+ *   2. adaptive block mask (pool, reduced attention, CDF threshold, optional
+ *      STA union)
+ *   3. attention on the kept 64 x 64 tiles
+ * Two ways to run them:
+ *   - on tensors in grid order, without any flattened copy (the flattening
+ *     happens in the kernels' loads and stores):
+ *       nabla_build_mask_grid (or nabla_flatten_pool_qk in pool-only mode +
+ *       nabla_build_mask_pooled), then nabla_sparse_attn_fwd_grid;
+ *   - on materialised flattened tensors:
+ *       nabla_flatten, nabla_build_mask (or nabla_build_mask_noalloc),
+ *       nabla_sparse_attn_fwd, nabla_unflatten.
  *
  * Conventions shared by every call
  *   - Tensors are bf16 in BSHD layout [B][S][Hh][D] (D contiguous), S = T*H*W
  *     tokens, Hh heads, head dimension D in {64, 128}.  A block is P*P = 64
- *     consecutive tokens of the flattened order (P = 8); Nb = S / 64.
+ *     consecutive tokens of the flattened order (P = 8), i.e. one 8 x 8 patch
+ *     of one frame; Nb = S / 64.  Block lists always index blocks in the
+ *     flattened order.
  *   - Every pointer argument is a DEVICE pointer owned by the caller, who
  *     allocates it (the library allocates no device memory) and keeps it alive
  *     until the stream has executed the call.  Inputs and outputs never alias.
@@ -141,7 +151,8 @@ int nabla_build_mask_grid(const void* q, const void* k, int B, int Hh, int D, in
 
 /* Stages 2-4 of nabla_build_mask (reduced attention, CDF threshold, STA
  * union, compaction) on a workspace that already holds the pooled queries
- * and keys (written by nabla_flatten_pool_qk or nabla_build_mask).  Same
+ * and keys (written by nabla_flatten_pool_qk, nabla_build_mask or
+ * nabla_build_mask_grid).  Same
  * arguments, results and errors as nabla_build_mask without qf and kf. */
 int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, int H, int W,
                             const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream);
