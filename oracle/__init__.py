@@ -59,6 +59,7 @@ def _load():
         lib.oracle_cdf_keep.restype = i
         lib.oracle_sta.argtypes = [i, i, i, i, i, i, i]
         lib.oracle_sta.restype = i
+        lib.oracle_sta_lists.argtypes = [i, i, i, i, i, i, P, P]
         lib.oracle_num_threads.restype = i
         _lib = lib
     return _lib
@@ -133,6 +134,17 @@ def cdf_keep(p: np.ndarray, thr: float, band: float = BAND):
 
 def sta(i: int, j: int, nbh: int, nbw: int, window=(3, 3, 3)) -> bool:
     return bool(_load().oracle_sta(i, j, nbh, nbw, *window))
+
+
+def sta_lists(nbt: int, nbh: int, nbw: int, window=(3, 3, 3)):
+    """The static window alone as block lists for one (b, head):
+    kv_count int32 [Nb], kv_idx int32 [Nb, Nb] (ascending, -1 past the count)."""
+    Nb = nbt * nbh * nbw
+    kv_count = np.zeros(Nb, dtype=np.int32)
+    kv_idx = np.full((Nb, Nb), -1, dtype=np.int32)
+    _load().oracle_sta_lists(Nb, nbh, nbw, int(window[0]), int(window[1]), int(window[2]),
+                             _ptr(kv_count), _ptr(kv_idx))
+    return kv_count, kv_idx
 
 
 def build_mask(qbar: np.ndarray, kbar: np.ndarray, thr: float, scale: float, nbh: int, nbw: int,

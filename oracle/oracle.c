@@ -385,3 +385,26 @@ int oracle_cdf_keep(const float* p, int Nb, float thr, uint8_t* keep, double* cu
 int oracle_sta(int i, int j, int nbh, int nbw, int sta_t, int sta_h, int sta_w) {
   return sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w);
 }
+
+/* ------------------------------------------------------------------------ */
+/* The static window on its own, M_STA (Metodologia item 3 without the      */
+/* content-adaptive term; the "pure STA" configurations the summary compares */
+/* NABLA with under "Comparacao com Metodos Estaticos"): for every query     */
+/* block i, the blocks j with sta_keep(i, j) in ascending order.  The lists  */
+/* depend only on the grid, so this fills one (b, head):                     */
+/*   kv_count[i], kv_idx[i*Nb + 0..kv_count[i])                              */
+/* Entries past the count are left as they are.  Pinned by the closed-form   */
+/* per-row counts (any window), the identity lists of a 1x1x1 window, the    */
+/* full lists of a window covering the grid, and an enumeration of the       */
+/* window by coordinates written independently in the tests.                 */
+/* ------------------------------------------------------------------------ */
+void oracle_sta_lists(int Nb, int nbh, int nbw, int sta_t, int sta_h, int sta_w, int32_t* kv_count,
+                      int32_t* kv_idx) {
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int i = 0; i < Nb; ++i) {
+    int n = 0;
+    for (int j = 0; j < Nb; ++j)
+      if (sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w)) kv_idx[(int64_t)i * Nb + n++] = j;
+    kv_count[i] = n;
+  }
+}

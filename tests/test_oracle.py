@@ -302,6 +302,57 @@ def test_sta_union_is_superset(oracle_lib):
         [[oracle_lib.sta(i, j, w.nbh, w.nbw) for j in range(w.Nb)] for i in range(w.Nb)])[None, None])
 
 
+def sta_window_by_coordinates(i, nt, nh, nw, window):
+    """Independent formulation of one row of the static window: walk the
+    window's (frame, patch row, patch column) offsets in nested order, keep
+    those inside the grid and map them to flattened block indices."""
+    rt, rh, rw = (x // 2 for x in window)
+    t, h, w_ = i // (nh * nw), (i // nw) % nh, i % nw
+    out = []
+    for tt in range(t - rt, t + rt + 1):
+        for hh in range(h - rh, h + rh + 1):
+            for ww in range(w_ - rw, w_ + rw + 1):
+                if 0 <= tt < nt and 0 <= hh < nh and 0 <= ww < nw:
+                    out.append((tt * nh + hh) * nw + ww)
+    return out
+
+
+@pytest.mark.parametrize("nt,nh,nw,total", read_sta_counts())
+def test_sta_lists_golden_totals(oracle_lib, nt, nh, nw, total):
+    cnt, idx = oracle_lib.sta_lists(nt, nh, nw, (3, 3, 3))
+    assert int(cnt.sum()) == total
+    Nb = nt * nh * nw
+    for i in (range(Nb) if Nb <= 200 else range(0, Nb, 13)):
+        assert list(idx[i, :cnt[i]]) == sta_window_by_coordinates(i, nt, nh, nw, (3, 3, 3))
+        assert np.all(idx[i, cnt[i]:] == -1)
+
+
+@pytest.mark.parametrize("window", [(1, 3, 5), (5, 1, 3), (3, 5, 1), (7, 7, 7)])
+def test_sta_lists_other_windows(oracle_lib, window):
+    nt, nh, nw = 5, 4, 6
+    cnt, idx = oracle_lib.sta_lists(nt, nh, nw, window)
+    rt, rh, rw = (x // 2 for x in window)
+
+    def axis(x, n, r):
+        return min(x + r, n - 1) - max(x - r, 0) + 1
+    for i in range(nt * nh * nw):
+        t, h, w_ = i // (nh * nw), (i // nw) % nh, i % nw
+        assert cnt[i] == axis(t, nt, rt) * axis(h, nh, rh) * axis(w_, nw, rw)
+        assert list(idx[i, :cnt[i]]) == sta_window_by_coordinates(i, nt, nh, nw, window)
+
+
+def test_sta_lists_degenerate_windows(oracle_lib):
+    nt, nh, nw = 3, 2, 5
+    Nb = nt * nh * nw
+    # 1x1x1: every block attends to itself only (tile-local attention)
+    cnt, idx = oracle_lib.sta_lists(nt, nh, nw, (1, 1, 1))
+    assert np.all(cnt == 1) and np.array_equal(idx[:, 0], np.arange(Nb))
+    # a window reaching across the whole grid from any block: dense lists
+    cnt, idx = oracle_lib.sta_lists(nt, nh, nw, (2 * nt - 1, 2 * nh - 1, 2 * nw - 1))
+    assert np.all(cnt == Nb)
+    assert np.array_equal(idx, np.broadcast_to(np.arange(Nb), (Nb, Nb)))
+
+
 # ----------------------------------------------------------------------------
 # Attention on kept tiles
 # ----------------------------------------------------------------------------
