@@ -11,6 +11,8 @@ resident in HBM, Q, K, V in grid order, in three timed stages:
      through 5-D TMA boxes (the flattening done by the copy) and storing O
      and the LSE in grid order (nabla_sparse_attn_fwd_grid).
 L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
+With --config hunyuan-sta the mask is the static sliding-tile window alone
+(nabla_build_mask_sta replaces stages 1 and 2; Q and K are not read for it).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan13b]
     python bench.py --impl reference ...   # the CPU oracle, same metric
@@ -46,6 +48,7 @@ CONFIGS = {
     "wan13b": inputs.WAN13B,
     "hunyuan": inputs.HUNYUAN,
     "long": inputs.LONG,
+    "hunyuan-sta": inputs.HUNYUAN_STA,
 }
 CONFIGS.update({f"sweep-a{w.alpha}-t{w.thr}": w for w in inputs.sweep_points()})
 L2_FLUSH_BYTES = 256 << 20
@@ -85,7 +88,9 @@ def config_dict(w: inputs.Workload):
         "grid_THW": [w.T, w.H, w.W],
         "tokens": w.S,
         "blocks": w.Nb,
-        "thr": w.thr,
+        "mask": "adaptive (CDF)" + (" OR static STA window" if any(w.sta) else "") if w.mask == "nabla"
+                else "static STA window only",
+        "thr": w.thr if w.mask == "nabla" else None,
         "sta": list(w.sta) if any(w.sta) else None,
         "locality_amplitude": w.alpha,
         "seed": w.seed,
@@ -190,30 +195,40 @@ def run_gpu(args, rank, world, local_rank):
     og = torch.empty_like(qd)  # attention output, grid order
     kv_count = torch.empty((w.B, w.Hh, w.Nb), dtype=torch.int32, device=dev)
     kv_idx = torch.empty((w.B, w.Hh, w.Nb, w.Nb), dtype=torch.int32, device=dev)
+    static = w.mask == "sta"  # the static window alone: no pooling, no scores
     prm = nabla.params(w.thr, w.sta)
-    ws = torch.empty(nabla.mask_workspace_bytes(w.B, w.Hh, w.D, w.T, w.H, w.W, prm), dtype=torch.uint8, device=dev)
+    ws = None if static else torch.empty(nabla.mask_workspace_bytes(w.B, w.Hh, w.D, w.T, w.H, w.W, prm),
+                                         dtype=torch.uint8, device=dev)
     lse = torch.empty((w.B, w.Hh, w.S), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        # 1. pooling of Q and K straight from grid order (each block's 64
-        #    tokens gathered in flattened order; no flattened copies)
-        nabla.flatten_pool_qk(qd, kd, w.T, w.H, w.W, workspace=ws, thr=w.thr, sta=w.sta, write_flat=False)
-        if ev is not None:
-            ev[1].record(stream)
-        # 2. mask rows on the pooled workspace
-        nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count, kv_idx=kv_idx)
-        if ev is not None:
-            ev[2].record(stream)
+        if static:
+            # 1-2. the window's block lists (nothing read)
+            nabla.build_mask_sta(w.B, w.Hh, w.T, w.H, w.W, w.sta, kv_count=kv_count, kv_idx=kv_idx)
+            if ev is not None:
+                ev[1].record(stream)
+                ev[2].record(stream)
+        else:
+            # 1. pooling of Q and K straight from grid order (each block's 64
+            #    tokens gathered in flattened order; no flattened copies)
+            nabla.flatten_pool_qk(qd, kd, w.T, w.H, w.W, workspace=ws, thr=w.thr, sta=w.sta, write_flat=False)
+            if ev is not None:
+                ev[1].record(stream)
+            # 2. mask rows on the pooled workspace
+            nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count,
+                                    kv_idx=kv_idx)
+            if ev is not None:
+                ev[2].record(stream)
         # 3. attention reading Q, K, V in grid order through 5-D TMA boxes
         #    and storing O in grid order
         nabla.sparse_attn_fwd(qd, kd, vd, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W))
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 3  # pooling, mask rows, attention
+    launches_per_step = 2 if static else 3  # (window lists | pooling, mask rows), attention
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -277,9 +292,13 @@ def run_gpu(args, rank, world, local_rank):
                 vd_.copy_(vh, non_blocking=True)
                 v_in[b_].record(up)
             stream.wait_event(qk_in[b_])
-            nabla.flatten_pool_qk(qd_, kd_, w.T, w.H, w.W, workspace=ws, thr=w.thr, sta=w.sta, write_flat=False)
-            nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count,
-                                    kv_idx=kv_idx)
+            if static:
+                nabla.build_mask_sta(w.B, w.Hh, w.T, w.H, w.W, w.sta, kv_count=kv_count, kv_idx=kv_idx)
+            else:
+                nabla.flatten_pool_qk(qd_, kd_, w.T, w.H, w.W, workspace=ws, thr=w.thr, sta=w.sta,
+                                      write_flat=False)
+                nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count,
+                                        kv_idx=kv_idx)
             stream.wait_event(v_in[b_])
             if s_ >= 2:
                 stream.wait_event(out[b_])  # step s-2's output has been downloaded
@@ -333,17 +352,20 @@ def run_gpu(args, rank, world, local_rank):
         # per layer: the whole step, since Q, K, V, O stay in grid order (the
         # flattening and its inverse happen inside the pooling and attention)
         "ms_per_layer": statistics.mean(pool_ms) + mask_avg + attn_avg,
-        "stages_ms": {"pool_qk": statistics.mean(pool_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg},
+        "stages_ms": ({"sta_lists": statistics.mean(pool_ms), "sparse_attn": attn_avg} if static else
+                      {"pool_qk": statistics.mean(pool_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg}),
         # mask build = pooling + rows: Q and K read once, kv_count and the kept
-        # kv_idx entries written, over its time
-        "mask_build_gbs": mask_bytes(w, total_kept) / ((statistics.mean(pool_ms) + mask_avg) * 1e-3) / 1e9,
+        # kv_idx entries written, over its time (the static window reads
+        # nothing: only the lists are written)
+        "mask_build_gbs": (mask_bytes(w, total_kept) - (0 if not static else 4.0 * w.B * w.S * w.Hh * w.D)) /
+                          ((statistics.mean(pool_ms) + mask_avg) * 1e-3) / 1e9,
         "attn_tflops_kept": achieved,
-        "pool_gbs": pool_bytes(w) / (statistics.mean(pool_ms) * 1e-3) / 1e9,
+        "pool_gbs": None if static else pool_bytes(w) / (statistics.mean(pool_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": traffic},
-        "mask_roofline": {"bound": "alu", "kernel": "mask_rows_kernel", "achieved": score_flops(w) / (mask_avg * 1e-3) / 1e12,
+        "mask_roofline": None if static else {"bound": "alu", "kernel": "mask_rows_kernel", "achieved": score_flops(w) / (mask_avg * 1e-3) / 1e12,
                           "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
                           "frac": score_flops(w) / (mask_avg * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
                           "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"},
@@ -385,9 +407,14 @@ def oracle_sample(w, q, k, v, n_blocks, total_kept=None):
     kf = oracle.flatten(k, w.T, w.H, w.W).reshape(k.shape)
     vf = oracle.flatten(v, w.T, w.H, w.W).reshape(v.shape)
     t1 = time.perf_counter()
-    qbar, kbar = oracle.pool(qf), oracle.pool(kf)
-    cnt, idx, _, _ = oracle.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, sta_window=w.sta,
-                                       want_status=False)
+    if w.mask == "sta":
+        c1, i1 = oracle.sta_lists(w.T, w.nbh, w.nbw, w.sta)
+        cnt = np.broadcast_to(c1, (w.B, w.Hh, w.Nb))
+        idx = np.broadcast_to(i1, (w.B, w.Hh, w.Nb, w.Nb))
+    else:
+        qbar, kbar = oracle.pool(qf), oracle.pool(kf)
+        cnt, idx, _, _ = oracle.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, sta_window=w.sta,
+                                           want_status=False)
     t2 = time.perf_counter()
     qblocks = inputs.sample_query_blocks(w.Nb, n_blocks, seed=1234)
     oracle.attention(qf, kf, vf, cnt, idx, w.scale, qblocks=qblocks)
@@ -401,7 +428,7 @@ def oracle_sample(w, q, k, v, n_blocks, total_kept=None):
         "unit": "TFLOP/s",
         "cores": oracle.num_threads(),
         "kind": "oracle",
-        "sample": (f"flatten+pool+full mask ({t2 - t0:.2f} s) and attention on {len(qblocks)} seeded query blocks x "
+        "sample": (f"flatten+{'window lists' if w.mask == 'sta' else 'pool+full mask'} ({t2 - t0:.2f} s) and attention on {len(qblocks)} seeded query blocks x "
                    f"{w.Hh} heads ({t3 - t2:.2f} s), attention extrapolated to all {w.Nb} blocks by kept-tile count"),
         "ms_per_step_extrapolated": step_s * 1e3,
     }

@@ -37,6 +37,7 @@ EXPORTS = (
     "nabla_flatten_pool_qk",
     "nabla_build_mask_pooled",
     "nabla_build_mask_grid",
+    "nabla_build_mask_sta",
     "nabla_sparse_attn_fwd",
     "nabla_sparse_attn_fwd_grid",
     "nabla_get_status",
@@ -86,6 +87,7 @@ def lib():
         L.nabla_flatten_pool_qk.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, pp, vp, vp]
         L.nabla_build_mask_pooled.argtypes = [vp, i, i, i, i, i, i, pp, vp, vp, vp]
         L.nabla_build_mask_grid.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
+        L.nabla_build_mask_sta.argtypes = [i, i, i, i, i, i, i, i, i, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
@@ -246,6 +248,23 @@ def build_mask_pooled(workspace: torch.Tensor, B: int, Hh: int, D: int, T: int, 
                                          ctypes.byref(prm), _dev(kv_count, torch.int32, "kv_count"),
                                          _dev(kv_idx, torch.int32, "kv_idx"), _stream(stream)),
            "nabla_build_mask_pooled")
+    return kv_count, kv_idx
+
+
+def build_mask_sta(B: int, Hh: int, T: int, H: int, W: int, sta=(3, 3, 3), kv_count=None, kv_idx=None,
+                   device=None, stream=None, P: int = 8):
+    """The static sliding-tile window alone as block lists (nabla_build_mask_sta;
+    reads no Q or K).  Returns (kv_count int32 [B,Hh,Nb], kv_idx int32
+    [B,Hh,Nb,Nb])."""
+    Nb = T * H * W // BLOCK
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if kv_count is None:
+        kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)
+    _check(lib().nabla_build_mask_sta(B, Hh, T, H, W, P, int(sta[0]), int(sta[1]), int(sta[2]),
+                                      _dev(kv_count, torch.int32, "kv_count"), _dev(kv_idx, torch.int32, "kv_idx"),
+                                      _stream(stream)), "nabla_build_mask_sta")
     return kv_count, kv_idx
 
 

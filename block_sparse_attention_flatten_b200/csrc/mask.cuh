@@ -286,7 +286,11 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     //    prefix sums.  Every block with positive mass has e >= 2^-40, so e*
     //    does too and the search starts at [2^-63, 2): bits(e*) has bit 29
     //    set and bit 30 clear, and nothing below 2^-63 carries mass.
-    unsigned long long kstar = ~0ull;
+    //    When no finite element qualifies (thr = 0: the mass never exceeds
+    //    tau_m = total) the boundary is the smallest key of an STA-marked
+    //    block, +inf: the CDF then keeps nothing but the arg-max, and the
+    //    window is still kept.
+    unsigned long long kstar = 0x7F800000ull << 32;
     if (!a.keep_all && total > tau_m) {
       uint32_t prefix = 0x20000000u;
       int span = 29;
@@ -460,6 +464,40 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
       count += __popc(bal);
     }
     if (lane == 0) a.kv_count[bh * Nb + i] = count;
+  }
+}
+
+// ------------------------------------------------ static sliding-tile lists
+// The window mask M_STA on its own ("Integracao Hibrida com STA" without the
+// content-adaptive term): row i lists the blocks of the window centred on
+// block i and truncated at the grid border, ascending.  The truncated window
+// is a box [t0,t1] x [h0,h1] x [w0,w1] of block coordinates, and walking it
+// frame, patch row, patch column in nested order visits the flattened
+// indices (t*nbh + h)*nbw + w in ascending order, so entry e of the list is
+// the box's e-th block.  Nothing depends on the data: one warp computes row
+// i and writes it into every (b, head) copy blockIdx.y, blockIdx.y +
+// gridDim.y, ...; lane e writes entries e, e + 32, ... (coalesced).
+__global__ void __launch_bounds__(256) sta_lists_kernel(int32_t* __restrict__ kv_count,
+                                                        int32_t* __restrict__ kv_idx, int copies, int Nb,
+                                                        int nbh, int nbw, int rt, int rh, int rw) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (i >= Nb) return;
+  const int per_t = nbh * nbw;
+  const int nbt = Nb / per_t;
+  const int ti = i / per_t, hi = (i - ti * per_t) / nbw, wi = i - ti * per_t - hi * nbw;
+  const int t0 = max(ti - rt, 0), t1 = min(ti + rt, nbt - 1);
+  const int h0 = max(hi - rh, 0), h1 = min(hi + rh, nbh - 1);
+  const int w0 = max(wi - rw, 0), w1 = min(wi + rw, nbw - 1);
+  const int nh = h1 - h0 + 1, nw = w1 - w0 + 1, plane = nh * nw;
+  const int count = (t1 - t0 + 1) * plane;
+  for (int c = blockIdx.y; c < copies; c += gridDim.y) {
+    int32_t* out = kv_idx + (static_cast<int64_t>(c) * Nb + i) * Nb;
+    for (int e = lane; e < count; e += 32) {
+      const int et = e / plane, r = e - et * plane, eh = r / nw;
+      out[e] = ((t0 + et) * nbh + h0 + eh) * nbw + w0 + (r - eh * nw);
+    }
+    if (lane == 0) kv_count[static_cast<int64_t>(c) * Nb + i] = count;
   }
 }
 

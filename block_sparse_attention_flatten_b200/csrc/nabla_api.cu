@@ -402,6 +402,26 @@ int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, 
   return launch_mask_rows(mp, B, stream);
 }
 
+int nabla_build_mask_sta(int B, int Hh, int T, int H, int W, int P, int sta_t, int sta_h, int sta_w,
+                         int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int rc = check_grid(B, T, H, W, P);
+  if (rc != NABLA_OK) return rc;
+  if (Hh <= 0 || static_cast<int64_t>(B) * Hh > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
+  for (const int s : {sta_t, sta_h, sta_w})
+    if (s < 1 || s > 65535 || s % 2 == 0) return NABLA_ERR_INVALID;
+  if (kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != NABLA_OK) return rc;
+  const int Nb = T * H * W / 64;
+  const int copies = B * Hh;
+  const dim3 grid((Nb + 7) / 8, copies < 65535 ? copies : 65535);
+  sta_lists_kernel<<<grid, 256, 0, stream>>>(kv_count, kv_idx, copies, Nb, H / 8, W / 8, sta_t / 2, sta_h / 2,
+                                             sta_w / 2);
+  return launch_status();
+}
+
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
                           nabla_stream_t stream) {

@@ -41,6 +41,9 @@ class Workload:
     sta: tuple = (0, 0, 0)
     seed: int = 0
     P: int = 8
+    # "nabla": the adaptive mask (OR the window when sta is set); "sta": the
+    # static window alone (thr unused)
+    mask: str = "nabla"
 
     @property
     def S(self) -> int:
@@ -68,6 +71,10 @@ TINY = Workload("tiny: B1 Hh2 D64 grid 4x16x16, thr 0.9, no STA", 1, 2, 64, 4, 1
 WAN13B = Workload("Wan-1.3B-like: B1 Hh12 D128 grid 16x48x80, thr 0.7, no STA", 1, 12, 128, 16, 48, 80, 1.0, 0.7, seed=2)
 HUNYUAN = Workload("HunyuanVideo-like: B1 Hh24 D128 grid 32x48x80, thr 0.9 OR STA 3x3x3", 1, 24, 128, 32, 48, 80, 1.0, 0.9,
                    sta=(3, 3, 3), seed=3)
+# The same layer under the static window alone: the pure-STA configuration
+# the method is compared with.
+HUNYUAN_STA = Workload("HunyuanVideo-like, static STA 3x3x3 only: B1 Hh24 D128 grid 32x48x80", 1, 24, 128, 32, 48,
+                       80, 1.0, 1.0, sta=(3, 3, 3), seed=3, mask="sta")
 LONG = Workload("long video: B1 Hh24 D128 grid 64x48x80, thr 0.9 OR STA 3x3x3", 1, 24, 128, 64, 48, 80, 1.0, 0.9,
                 sta=(3, 3, 3), seed=5)
 

@@ -17,6 +17,9 @@
  *   - on materialised flattened tensors:
  *       nabla_flatten, nabla_build_mask (or nabla_build_mask_noalloc),
  *       nabla_sparse_attn_fwd, nabla_unflatten.
+ * The block lists are plain device buffers: one mask may serve several
+ * attention calls (rebuilt every few steps), and nabla_build_mask_sta
+ * writes the static window alone, without reading Q or K.
  *
  * Conventions shared by every call
  *   - Tensors are bf16 in BSHD layout [B][S][Hh][D] (D contiguous), S = T*H*W
@@ -156,6 +159,23 @@ int nabla_build_mask_grid(const void* q, const void* k, int B, int Hh, int D, in
  * arguments, results and errors as nabla_build_mask without qf and kf. */
 int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, int H, int W,
                             const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream);
+
+/* The static Sliding-Tile window on its own, M_STA of "Integracao Hibrida
+ * com STA" without the content-adaptive term (the pure-STA configuration the
+ * summary compares NABLA with, "Comparacao com Metodos Estaticos").  No Q or
+ * K is read: row i of every (b, head) lists the blocks j whose frame, patch
+ * row and patch column each differ from block i's by at most sta_t/2,
+ * sta_h/2, sta_w/2 (window centred on block i, truncated at the grid
+ * border), ascending; the lists are the STA part of nabla_build_mask's union
+ * with the same window.
+ *   P           must be 8; H and W multiples of 8.
+ *   sta_t, sta_h, sta_w   odd window sizes in [1, 65535] (in frames, patch
+ *               rows, patch columns).
+ *   kv_count, kv_idx      as for nabla_build_mask (16-byte aligned).
+ * Errors: NABLA_ERR_INVALID (grid, Hh, window sizes, NULL lists);
+ * NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
+int nabla_build_mask_sta(int B, int Hh, int T, int H, int W, int P, int sta_t, int sta_h, int sta_w,
+                         int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream);
 
 /* Block-sparse attention forward on the kept tiles ("Expansao": only the
  * listed N x N blocks are computed; a dropped block is in neither the

@@ -92,6 +92,15 @@ def test_invalid_arguments_rejected_before_launch(lib):
                                      s) == nabla.NABLA_ERR_INVALID
     assert L.nabla_build_mask_pooled(ctypes.c_void_p(0x1004), 1, 2, 64, 4, 16, 16, ctypes.byref(prm), fake, fake,
                                      s) == nabla.NABLA_ERR_ALIGN
+    # static window: odd sizes in [1, 65535], lists present and aligned
+    assert L.nabla_build_mask_sta(1, 2, 4, 16, 16, 8, 3, 2, 3, a1, a2, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_sta(1, 2, 4, 16, 16, 8, 0, 3, 3, a1, a2, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_sta(1, 2, 4, 16, 16, 8, 3, 3, 65537, a1, a2, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_sta(1, 2, 4, 12, 16, 8, 3, 3, 3, a1, a2, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_sta(1, 0, 4, 16, 16, 8, 3, 3, 3, a1, a2, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_sta(1, 2, 4, 16, 16, 8, 3, 3, 3, None, a2, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_build_mask_sta(1, 2, 4, 16, 16, 8, 3, 3, 3, a1, ctypes.c_void_p(0x2004),
+                                  s) == nabla.NABLA_ERR_ALIGN
     assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 100, 2, 64, ctypes.c_float(0.0), fake, None,
                                    s) == nabla.NABLA_ERR_INVALID
     assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 128, 2, 48, ctypes.c_float(0.0), fake, None,

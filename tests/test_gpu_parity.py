@@ -40,6 +40,7 @@ SMALL = [
     inputs.Workload("Nb=24 D64 dense", 1, 4, 64, 2, 16, 48, 1.0, 1.0, seed=35),
     inputs.Workload("Nb=24 thr0", 1, 2, 128, 2, 16, 48, 1.0, 0.0, seed=36),
     inputs.Workload("Nb=35 D64 STA 5x3x1", 1, 2, 64, 5, 8, 56, 1.0, 0.6, sta=(5, 3, 1), seed=37),
+    inputs.Workload("Nb=45 D64 thr0 STA", 1, 2, 64, 5, 24, 24, 1.0, 0.0, sta=(3, 3, 3), seed=38),
 ]
 
 
