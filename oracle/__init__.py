@@ -60,6 +60,7 @@ def _load():
         lib.oracle_sta.argtypes = [i, i, i, i, i, i, i]
         lib.oracle_sta.restype = i
         lib.oracle_sta_lists.argtypes = [i, i, i, i, i, i, P, P]
+        lib.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, P, P]
         lib.oracle_num_threads.restype = i
         _lib = lib
     return _lib
@@ -199,3 +200,19 @@ def attention(qf, kf, vf, kv_count: np.ndarray, kv_idx: np.ndarray, scale: float
     _load().oracle_attention(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(kv_count), _ptr(kv_idx), B, S, Hh, D,
                              scale, _ptr(qblocks), nq, _ptr(out), _ptr(lse))
     return out, lse
+
+
+def attention_bwd(qf, kf, vf, dof, kv_count: np.ndarray, kv_idx: np.ndarray, scale: float):
+    """Gradients (dq, dk, dv), fp64 [B, S, Hh, D], of sum(dO * O) for the
+    attention on the kept tiles (flattened order; full lists)."""
+    qf, kf, vf, dof = _bits(qf), _bits(kf), _bits(vf), _bits(dof)
+    B, S, Hh, D = qf.shape
+    kv_count = np.ascontiguousarray(kv_count, dtype=np.int32)
+    kv_idx = np.ascontiguousarray(kv_idx, dtype=np.int32)
+    assert kv_count.shape == (B, Hh, S // BLOCK) and kv_idx.shape == (B, Hh, S // BLOCK, S // BLOCK)
+    dq = np.empty((B, S, Hh, D), dtype=np.float64)
+    dk = np.empty_like(dq)
+    dv = np.empty_like(dq)
+    _load().oracle_attention_bwd(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(dof), _ptr(kv_count), _ptr(kv_idx),
+                                 B, S, Hh, D, scale, _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv

@@ -408,3 +408,102 @@ void oracle_sta_lists(int Nb, int nbh, int nbw, int sta_t, int sta_h, int sta_w,
     kv_count[i] = n;
   }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Gradient of the attention on the kept tiles (the backward pass a training  */
+/* step needs: the summary states that NABLA speeds up both pre-training /   */
+/* fine-tuning and inference, "Principais Contribuicoes", "Aceleracao de     */
+/* Dupla Fase", and reports pre-training iteration times, "Resultados        */
+/* Experimentais" item 2).  It is the exact derivative of oracle_attention   */
+/* on the same lists, written out with the chain rule, in fp64: for query    */
+/* token a of block i and every token c of the kept blocks of its row,       */
+/*   P_ac  = softmax_c(l_ac),  l_ac = (q_a . k_c) * scale                    */
+/*   dP_ac = dO_a . v_c                                                      */
+/*   dS_ac = P_ac * (dP_ac - sum_c' P_ac' dP_ac')     (softmax Jacobian)     */
+/*   dV_c += P_ac dO_a,  dQ_a += scale dS_ac k_c,  dK_c += scale dS_ac q_a.  */
+/* A dropped tile contributes nothing; a token kept by no row gets dK = dV = */
+/* 0; a row with no kept block gets dQ = 0.                                  */
+/* qf, kf, vf, dof: bf16 bits [B][S][Hh][D] (flattened order); lists as for  */
+/* nabla's forward ([B][Hh][Nb], [B][Hh][Nb][Nb]).  dq, dk, dv: fp64         */
+/* [B][S][Hh][D], overwritten.  OpenMP over (b, head): each head's dK, dV    */
+/* are accumulated by one thread in query order.                             */
+/* Pinned by: autograd (fp64) of a token-level masked softmax attention      */
+/* built from the lists; sum_c dK_c = 0 and sum_c dV_c = sum_a dO_a over     */
+/* rows with kept blocks; zero gradients for unkept key blocks and empty     */
+/* rows.                                                                     */
+/* ------------------------------------------------------------------------ */
+void oracle_attention_bwd(const uint16_t* qf, const uint16_t* kf, const uint16_t* vf, const uint16_t* dof,
+                          const int32_t* kv_count, const int32_t* kv_idx, int B, int S, int Hh, int D,
+                          double scale, double* dq, double* dk, double* dv) {
+  int Nb = S / ORACLE_BLOCK;
+  int64_t n_all = (int64_t)B * S * Hh * D;
+  for (int64_t x = 0; x < n_all; ++x) dq[x] = dk[x] = dv[x] = 0.0;
+#pragma omp parallel
+  {
+    double* pr = (double*)malloc(sizeof(double) * (size_t)S);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)S);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < (int64_t)B * Hh; ++bh) {
+      int b = (int)(bh / Hh), hd = (int)(bh % Hh);
+#define ORACLE_AT(base, tok) ((base) + (((int64_t)b * S + (tok)) * Hh + hd) * D)
+      for (int i = 0; i < Nb; ++i) {
+        int64_t row = bh * Nb + i;
+        int cnt = kv_count[row];
+        const int32_t* lst = kv_idx + row * Nb;
+        for (int r = 0; r < ORACLE_BLOCK; ++r) {
+          int64_t a = (int64_t)i * ORACLE_BLOCK + r;
+          const uint16_t* q = ORACLE_AT(qf, a);
+          const uint16_t* g = ORACLE_AT(dof, a);
+          /* probabilities of the row */
+          double mx = -INFINITY, den = 0.0;
+          int64_t n = 0;
+          for (int e = 0; e < cnt; ++e)
+            for (int c = 0; c < ORACLE_BLOCK; ++c) {
+              const uint16_t* k = ORACLE_AT(kf, (int64_t)lst[e] * ORACLE_BLOCK + c);
+              double dot = 0.0;
+              for (int d = 0; d < D; ++d) dot += (double)bf16_bits_to_f32(q[d]) * (double)bf16_bits_to_f32(k[d]);
+              pr[n] = dot * scale;
+              if (pr[n] > mx) mx = pr[n];
+              ++n;
+            }
+          for (int64_t c = 0; c < n; ++c) {
+            pr[c] = exp(pr[c] - mx);
+            den += pr[c];
+          }
+          for (int64_t c = 0; c < n; ++c) pr[c] /= den;
+          /* dP and the softmax Jacobian's row term sum_c P dP */
+          double pdp = 0.0;
+          n = 0;
+          for (int e = 0; e < cnt; ++e)
+            for (int c = 0; c < ORACLE_BLOCK; ++c) {
+              const uint16_t* v = ORACLE_AT(vf, (int64_t)lst[e] * ORACLE_BLOCK + c);
+              double dot = 0.0;
+              for (int d = 0; d < D; ++d) dot += (double)bf16_bits_to_f32(g[d]) * (double)bf16_bits_to_f32(v[d]);
+              dp[n] = dot;
+              pdp += pr[n] * dot;
+              ++n;
+            }
+          double* dqa = ORACLE_AT(dq, a);
+          n = 0;
+          for (int e = 0; e < cnt; ++e)
+            for (int c = 0; c < ORACLE_BLOCK; ++c) {
+              int64_t tok = (int64_t)lst[e] * ORACLE_BLOCK + c;
+              const uint16_t* k = ORACLE_AT(kf, tok);
+              double* dkc = ORACLE_AT(dk, tok);
+              double* dvc = ORACLE_AT(dv, tok);
+              double ds = pr[n] * (dp[n] - pdp);
+              for (int d = 0; d < D; ++d) {
+                dvc[d] += pr[n] * (double)bf16_bits_to_f32(g[d]);
+                dqa[d] += scale * ds * (double)bf16_bits_to_f32(k[d]);
+                dkc[d] += scale * ds * (double)bf16_bits_to_f32(q[d]);
+              }
+              ++n;
+            }
+        }
+      }
+#undef ORACLE_AT
+    }
+    free(pr);
+    free(dp);
+  }
+}

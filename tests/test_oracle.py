@@ -432,6 +432,83 @@ def test_attention_special_cases(oracle_lib):
     assert np.all(out4 == 0) and np.all(np.isneginf(lse4))
 
 
+# ----------------------------------------------------------------------------
+# Gradient of the attention on kept tiles (backward pass for training)
+# ----------------------------------------------------------------------------
+def random_lists(rng, B, Hh, Nb, p_keep, empty_rows=(), unkept_col=None):
+    cnt = np.zeros((B, Hh, Nb), dtype=np.int32)
+    idx = np.full((B, Hh, Nb, Nb), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hh):
+            for i in range(Nb):
+                if i in empty_rows:
+                    continue
+                keep = np.nonzero(rng.random(Nb) < p_keep)[0]
+                if unkept_col is not None:
+                    keep = keep[keep != unkept_col]
+                if keep.size == 0:
+                    keep = np.array([i if i != unkept_col else (i + 1) % Nb])
+                cnt[b, h, i] = keep.size
+                idx[b, h, i, :keep.size] = np.sort(keep)
+    return cnt, idx
+
+
+def autograd_masked_attention(q, k, v, do, cnt, idx, scale):
+    """Independent formulation: token-level masked softmax attention in fp64
+    torch, differentiated by autograd.  Rows with no kept block are left out
+    of the loss (their output is defined as 0)."""
+    B, S, Hh, D = q.shape
+    Nb = S // BLOCK
+    blk = np.zeros((B, Hh, Nb, Nb), dtype=bool)
+    for b in range(B):
+        for h in range(Hh):
+            for i in range(Nb):
+                blk[b, h, i, idx[b, h, i, :cnt[b, h, i]]] = True
+    tok = torch.from_numpy(blk).repeat_interleave(BLOCK, 2).repeat_interleave(BLOCK, 3)  # [B,Hh,S,S]
+    qt, kt, vt = (x.to(torch.float64).permute(0, 2, 1, 3).clone().requires_grad_(True) for x in (q, k, v))
+    logits = (qt @ kt.transpose(-1, -2)) * scale
+    rows = tok.any(-1)
+    p = torch.softmax(logits.masked_fill(~tok, float("-inf")), -1)
+    p = torch.where(rows.unsqueeze(-1), p, torch.zeros_like(p))
+    out = p @ vt
+    (out * do.to(torch.float64).permute(0, 2, 1, 3)).sum().backward()
+    return tuple(x.grad.permute(0, 2, 1, 3).numpy() for x in (qt, kt, vt))
+
+
+@pytest.mark.parametrize("D,p_keep,empty", [(64, 0.5, ()), (128, 0.3, (2,)), (64, 1.0, ())])
+def test_attention_bwd_equals_autograd(oracle_lib, D, p_keep, empty):
+    rng = np.random.default_rng(7 + D)
+    B, Hh, Nb = 2, 2, 5
+    S = Nb * BLOCK
+    q, k, v, do = (inputs.randn_bf16((B, S, Hh, D), seed=s) for s in (11, 12, 13, 14))
+    cnt, idx = random_lists(rng, B, Hh, Nb, p_keep, empty_rows=empty, unkept_col=3 if p_keep < 1 else None)
+    scale = 1.0 / math.sqrt(D)
+    dq, dk, dv = oracle_lib.attention_bwd(q, k, v, do, cnt, idx, scale)
+    rq, rk, rv = autograd_masked_attention(q, k, v, do, cnt, idx, scale)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        assert np.abs(got - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+
+
+def test_attention_bwd_invariants(oracle_lib):
+    rng = np.random.default_rng(3)
+    B, Hh, Nb, D = 1, 3, 6, 64
+    S = Nb * BLOCK
+    q, k, v, do = (inputs.randn_bf16((B, S, Hh, D), seed=s) for s in (21, 22, 23, 24))
+    cnt, idx = random_lists(rng, B, Hh, Nb, 0.4, empty_rows=(4,), unkept_col=1)
+    dq, dk, dv = oracle_lib.attention_bwd(q, k, v, do, cnt, idx, 0.125)
+    # the softmax Jacobian's rows sum to zero, so the key gradients of one
+    # head sum to zero over all key tokens
+    assert np.abs(dk.sum(axis=1)).max() < 1e-9
+    # each kept row's probabilities sum to one: the value gradients sum to
+    # the output gradients of the rows that keep anything
+    live = np.repeat(cnt > 0, BLOCK, axis=2).transpose(0, 2, 1)  # [B,S,Hh]
+    dof = do.to(torch.float64).numpy() * live[..., None]
+    assert np.abs(dv.sum(axis=1) - dof.sum(axis=1)).max() < 1e-9
+    # a key block no row keeps, and a row that keeps nothing, get zeros
+    assert not np.any(dk[:, 64:128]) and not np.any(dv[:, 64:128])
+    assert not np.any(dq[:, 4 * 64:5 * 64])
+
+
 def test_generator_is_deterministic_and_shaped():
     w = inputs.Workload("g", 1, 2, 64, 2, 8, 16, 1.0, 0.9, seed=3)
     a = inputs.make_qkv(w)
