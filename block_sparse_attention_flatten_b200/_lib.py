@@ -40,6 +40,9 @@ EXPORTS = (
     "nabla_build_mask_sta",
     "nabla_sparse_attn_fwd",
     "nabla_sparse_attn_fwd_grid",
+    "nabla_transpose_lists",
+    "nabla_sparse_attn_bwd",
+    "nabla_sparse_attn_bwd_grid",
     "nabla_get_status",
     "nabla_validate_mask",
     "nabla_selftest_wait_timeout",
@@ -90,6 +93,9 @@ def lib():
         L.nabla_build_mask_sta.argtypes = [i, i, i, i, i, i, i, i, i, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
+        L.nabla_transpose_lists.argtypes = [vp, vp, i, i, i, vp, vp, vp]
+        L.nabla_sparse_attn_bwd.argtypes = [vp] * 10 + [i, i, i, i, f, vp, vp, vp, vp, vp]
+        L.nabla_sparse_attn_bwd_grid.argtypes = [vp] * 10 + [i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
         L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
         L.nabla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
@@ -331,6 +337,54 @@ def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_cou
                                                 _stream(stream)),
                "nabla_sparse_attn_fwd_grid")
     return out, lse
+
+
+def transpose_lists(kv_count: torch.Tensor, kv_idx: torch.Tensor, q_count=None, q_idx=None, stream=None):
+    """Column lists of the block lists (nabla_transpose_lists): for every key
+    block the query blocks that keep it, ascending.  Returns (q_count,
+    q_idx), shaped like (kv_count, kv_idx)."""
+    B, Hh, Nb = kv_count.shape
+    if q_count is None:
+        q_count = torch.empty_like(kv_count)
+    if q_idx is None:
+        q_idx = torch.empty_like(kv_idx)
+    _check(lib().nabla_transpose_lists(_dev(kv_count, torch.int32, "kv_count"), _dev(kv_idx, torch.int32, "kv_idx"),
+                                       B, Hh, Nb, _dev(q_count, torch.int32, "q_count"),
+                                       _dev(q_idx, torch.int32, "q_idx"), _stream(stream)), "nabla_transpose_lists")
+    return q_count, q_idx
+
+
+def sparse_attn_bwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+                    lse: torch.Tensor, kv_count: torch.Tensor, kv_idx: torch.Tensor, q_lists=None,
+                    scale: float = 0.0, dq=None, dk=None, dv=None, delta=None, stream=None, grid=None):
+    """Gradients (dq, dk, dv) of sum(dout * out) for the attention on the kept
+    tiles.  q_lists = (q_count, q_idx) from :func:`transpose_lists` (computed
+    here when None).  grid = None: flattened tensors (nabla_sparse_attn_bwd);
+    grid = (T, H, W): grid-order tensors, LSE and outputs as
+    :func:`sparse_attn_fwd` with a grid (nabla_sparse_attn_bwd_grid)."""
+    B, S, Hh, D = qf.shape
+    if q_lists is None:
+        q_lists = transpose_lists(kv_count, kv_idx, stream=stream)
+    q_count, q_idx = q_lists
+    dq = torch.empty_like(qf) if dq is None else dq
+    dk = torch.empty_like(kf) if dk is None else dk
+    dv = torch.empty_like(vf) if dv is None else dv
+    if delta is None:
+        delta = torch.empty((B, Hh, S), dtype=torch.float32, device=qf.device)
+    ptrs = [_dev(x, torch.bfloat16, n) for x, n in ((qf, "q"), (kf, "k"), (vf, "v"), (out, "out"), (dout, "dout"))]
+    ptrs += [_dev(lse, torch.float32, "lse"), _dev(kv_count, torch.int32, "kv_count"), _dev(kv_idx, torch.int32, "kv_idx"),
+             _dev(q_count, torch.int32, "q_count"), _dev(q_idx, torch.int32, "q_idx")]
+    outs = [_dev(dq, torch.bfloat16, "dq"), _dev(dk, torch.bfloat16, "dk"), _dev(dv, torch.bfloat16, "dv"),
+            _dev(delta, torch.float32, "delta"), _stream(stream)]
+    if grid is None:
+        _check(lib().nabla_sparse_attn_bwd(*ptrs, B, S, Hh, D, float(scale), *outs), "nabla_sparse_attn_bwd")
+    else:
+        T, H, W = (int(x) for x in grid)
+        if T * H * W != S:
+            raise ValueError(f"grid {grid} does not hold {S} tokens")
+        _check(lib().nabla_sparse_attn_bwd_grid(*ptrs, B, Hh, D, T, H, W, float(scale), *outs),
+               "nabla_sparse_attn_bwd_grid")
+    return dq, dk, dv
 
 
 def get_status(stream=None) -> int:

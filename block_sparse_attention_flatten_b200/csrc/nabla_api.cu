@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "common.cuh"
 #include "flatten.cuh"
@@ -324,6 +325,69 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   return launch_status();
 }
 
+// Backward launches: Delta, then dQ over the row lists, then dK and dV over
+// the column lists.
+template <int D>
+int launch_bwd(const BwdArgs& a, const void* out, int B, const DeviceInfo& di, cudaStream_t stream) {
+  const size_t smem = BwdTile<D>::kSmemBytes;
+  if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
+  if (cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return NABLA_ERR_CUDA;
+  const int64_t rows = static_cast<int64_t>(B) * a.S;
+  bwd_delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(out), a.dout, const_cast<float*>(a.delta), rows, a.S, a.Hh, D);
+  const dim3 grid(a.Nb, a.Hh, B);
+  bwd_dq_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a);
+  bwd_dkdv_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a);
+  return launch_status();
+}
+
+int sparse_attn_bwd(const void* qf, const void* kf, const void* vf, const void* out, const void* dout,
+                    const float* lse, const int32_t* kv_count, const int32_t* kv_idx, const int32_t* q_count,
+                    const int32_t* q_idx, int B, int S, int Hh, int D, float scale, void* dq, void* dk, void* dv,
+                    float* delta, int H, int W, cudaStream_t stream) {
+  if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
+  if (B > 65535 || Hh > 65535 || static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
+  if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
+  const void* ptrs[] = {qf, kf, vf, out, dout, lse, kv_count, kv_idx, q_count, q_idx, dq, dk, dv, delta};
+  for (const void* p : ptrs)
+    if (p == nullptr) return NABLA_ERR_INVALID;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc != NABLA_OK) return rc;
+  if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
+  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  BwdArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(qf);
+  a.k = static_cast<const __nv_bfloat16*>(kf);
+  a.v = static_cast<const __nv_bfloat16*>(vf);
+  a.dout = static_cast<const __nv_bfloat16*>(dout);
+  a.lse = lse;
+  a.delta = delta;
+  a.kv_count = kv_count;
+  a.kv_idx = kv_idx;
+  a.q_count = q_count;
+  a.q_idx = q_idx;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.S = S;
+  a.Hh = Hh;
+  a.Nb = S / 64;
+  a.scale = sc;
+  a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
+  a.H = H;
+  a.W = W;
+  a.nbw = W / 8;
+  a.per_t = (H / 8) * (W / 8);
+  return D == 128 ? launch_bwd<128>(a, out, B, di, stream) : launch_bwd<64>(a, out, B, di, stream);
+}
+
 }  // namespace
 }  // namespace nabla
 
@@ -439,6 +503,37 @@ int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, cons
   const bool groups = T % 2 == 0 && nbw % 2 == 0;
   return sparse_attn_launch(q, k, v, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
                             groups ? F : 0, groups ? nbw : 0, T, H, W, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int nabla_transpose_lists(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb, int32_t* q_count,
+                          int32_t* q_idx, nabla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B <= 0 || Hh <= 0 || Nb <= 0 || Nb > (1 << 24) || static_cast<int64_t>(B) * Hh > 65535) return NABLA_ERR_INVALID;
+  if (kv_count == nullptr || kv_idx == nullptr || q_count == nullptr || q_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(kv_count) || !aligned16(kv_idx) || !aligned16(q_count) || !aligned16(q_idx)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  int rc = device_info(&di);
+  if (rc != NABLA_OK) return rc;
+  transpose_lists_kernel<<<dim3((Nb + 7) / 8, B * Hh), 256, 0, stream>>>(kv_count, kv_idx, q_count, q_idx, Nb);
+  return launch_status();
+}
+
+int nabla_sparse_attn_bwd(const void* qf, const void* kf, const void* vf, const void* out, const void* dout,
+                          const float* lse, const int32_t* kv_count, const int32_t* kv_idx, const int32_t* q_count,
+                          const int32_t* q_idx, int B, int S, int Hh, int D, float scale, void* dq, void* dk,
+                          void* dv, float* delta, nabla_stream_t stream) {
+  return sparse_attn_bwd(qf, kf, vf, out, dout, lse, kv_count, kv_idx, q_count, q_idx, B, S, Hh, D, scale, dq, dk,
+                         dv, delta, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int nabla_sparse_attn_bwd_grid(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                               const float* lse, const int32_t* kv_count, const int32_t* kv_idx,
+                               const int32_t* q_count, const int32_t* q_idx, int B, int Hh, int D, int T, int H,
+                               int W, float scale, void* dq, void* dk, void* dv, float* delta,
+                               nabla_stream_t stream) {
+  if (check_grid(B, T, H, W, 8) != NABLA_OK) return NABLA_ERR_INVALID;
+  return sparse_attn_bwd(q, k, v, out, dout, lse, kv_count, kv_idx, q_count, q_idx, B, T * H * W, Hh, D, scale, dq,
+                         dk, dv, delta, H, W, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,

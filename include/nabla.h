@@ -224,6 +224,59 @@ int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, cons
                                const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
                                void* out, float* lse, nabla_stream_t stream);
 
+/* Column (transposed) block lists for the backward pass: for key block j of
+ * (b, hd), the query blocks i whose row kv_idx[b,hd,i,0..kv_count) lists j,
+ * ascending.
+ *   kv_count, kv_idx   row lists as written by the mask entry points
+ *               ([B][Hh][Nb], [B][Hh][Nb][Nb], rows ascending).
+ *   q_count     device int32 [B][Hh][Nb] output: query blocks per key block.
+ *   q_idx       device int32 [B][Hh][Nb][Nb] output: entries [0, q_count)
+ *               of row (b,hd,j); later entries are not written.
+ * A row whose count is outside [0, Nb] is taken as empty and recorded as
+ * NABLA_ERR_DEVICE_BOUNDS.  Errors: NABLA_ERR_INVALID (sizes, B*Hh > 65535,
+ * NULL); NABLA_ERR_ALIGN (pointers not 16-byte aligned); NABLA_ERR_CUDA. */
+int nabla_transpose_lists(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb, int32_t* q_count,
+                          int32_t* q_idx, nabla_stream_t stream);
+
+/* Backward pass of nabla_sparse_attn_fwd over the same kept tiles: the
+ * gradients of sum(dO * O) with respect to Q, K and V, for training (the
+ * summary's "Aceleracao de Dupla Fase": the method also speeds up
+ * pre-training and fine-tuning).  With P the forward's probabilities
+ * (recomputed from lse), for query token a and the tokens c of its kept
+ * blocks:
+ *   Delta_a = dO_a . O_a,  dS_ac = P_ac (dO_a . v_c - Delta_a),
+ *   dQ_a = scale sum_c dS_ac k_c,  dK_c = scale sum_a dS_ac q_a,
+ *   dV_c = sum_a P_ac dO_a;
+ * a key block kept by no row gets dK = dV = 0, an empty row dQ = 0.
+ *   qf, kf, vf, out, dout   device bf16 [B][S][Hh][D], flattened order: the
+ *               forward's inputs, its output O and the output gradient.
+ *   lse         device fp32 [B][Hh][S]: the forward's LSE.
+ *   kv_count, kv_idx   the forward's row lists; q_count, q_idx their
+ *               transpose (nabla_transpose_lists).
+ *   scale       0 selects 1/sqrt(D) (must match the forward).
+ *   dq, dk, dv  device bf16 [B][S][Hh][D] outputs (every element written).
+ *   delta       device fp32 [B][Hh][S] workspace, written with Delta.
+ * Each output element is computed by one CTA in a fixed order: results are
+ * deterministic.  Errors: as nabla_sparse_attn_fwd (every pointer required,
+ * B and Hh at most 65535); list faults are recorded as for the forward. */
+int nabla_sparse_attn_bwd(const void* qf, const void* kf, const void* vf, const void* out, const void* dout,
+                          const float* lse, const int32_t* kv_count, const int32_t* kv_idx, const int32_t* q_count,
+                          const int32_t* q_idx, int B, int S, int Hh, int D, float scale, void* dq, void* dk,
+                          void* dv, float* delta, nabla_stream_t stream);
+
+/* nabla_sparse_attn_bwd on tensors in GRID order (as nabla_sparse_attn_fwd_grid
+ * reads and writes them): q, k, v, out, dout, dq, dk, dv [B][T*H*W][Hh][D]
+ * and lse, delta [B][Hh][T*H*W] indexed by the grid row (t*H + h)*W + w;
+ * the block lists index blocks in the flattened order.  Results equal
+ * nabla_sparse_attn_bwd on the flattened tensors, permuted back.  Errors:
+ * as nabla_sparse_attn_bwd, plus NABLA_ERR_INVALID unless H and W are
+ * multiples of 8. */
+int nabla_sparse_attn_bwd_grid(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                               const float* lse, const int32_t* kv_count, const int32_t* kv_idx,
+                               const int32_t* q_count, const int32_t* q_idx, int B, int Hh, int D, int T, int H,
+                               int W, float scale, void* dq, void* dk, void* dv, float* delta,
+                               nabla_stream_t stream);
+
 /* Same mask as nabla_build_mask, for callers that cannot allocate device
  * memory.  This entry point has no counterpart in the paper; it exists for
  * code that hands the library only its input and output buffers: a plug-in

@@ -103,6 +103,19 @@ def test_invalid_arguments_rejected_before_launch(lib):
                                   s) == nabla.NABLA_ERR_ALIGN
     assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 100, 2, 64, ctypes.c_float(0.0), fake, None,
                                    s) == nabla.NABLA_ERR_INVALID
+    # backward: lists transposed need aligned buffers; every pointer required
+    assert L.nabla_transpose_lists(a1, a2, 1, 2, 0, a3, fake, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_transpose_lists(a1, a2, 1, 2, 4, None, fake, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_transpose_lists(a1, a2, 1, 2, 4, a3, ctypes.c_void_p(0x4004), s) == nabla.NABLA_ERR_ALIGN
+    p10 = [ctypes.c_void_p(0x1000 * (n + 1)) for n in range(10)]
+    o4 = [ctypes.c_void_p(0x20000 + 0x1000 * n) for n in range(4)]
+    f0 = ctypes.c_float(0.0)
+    assert L.nabla_sparse_attn_bwd(*p10, 1, 100, 2, 64, f0, *o4, s) == nabla.NABLA_ERR_INVALID  # S % 64
+    assert L.nabla_sparse_attn_bwd(*p10, 1, 128, 2, 96, f0, *o4, s) == nabla.NABLA_ERR_INVALID  # D
+    assert L.nabla_sparse_attn_bwd(*p10[:5], None, *p10[6:], 1, 128, 2, 64, f0, *o4, s) == nabla.NABLA_ERR_INVALID
+    assert L.nabla_sparse_attn_bwd(*p10, 1, 128, 2, 64, f0, *o4[:3], ctypes.c_void_p(0x30004),
+                                   s) == nabla.NABLA_ERR_ALIGN
+    assert L.nabla_sparse_attn_bwd_grid(*p10, 1, 2, 64, 2, 12, 16, f0, *o4, s) == nabla.NABLA_ERR_INVALID  # H % 8
     assert L.nabla_sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 128, 2, 48, ctypes.c_float(0.0), fake, None,
                                    s) == nabla.NABLA_ERR_INVALID
 
