@@ -330,6 +330,48 @@ def run_gpu(args, rank, world, local_rank):
                "unit": "TFLOP/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                "ms_per_step": te / len(e2e_ms)}
 
+    # backward pass over the same lists (training), timed on its own: the
+    # column lists, then Delta, dQ and dK/dV; not part of `value`
+    backward = None
+    if args.backward_steps > 0:
+        do = inputs.randn_bf16(tuple(qd.shape), seed=w.seed + 1000).to(dev)  # output gradient
+        q_count, q_idx = torch.empty_like(kv_count), torch.empty_like(kv_idx)
+        dq_, dk_, dv_ = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+        delta = torch.empty_like(lse)
+        nabla.sparse_attn_fwd(qd, kd, vd, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W))
+
+        def bstep(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            nabla.transpose_lists(kv_count, kv_idx, q_count=q_count, q_idx=q_idx)
+            if ev is not None:
+                ev[1].record(stream)
+            nabla.sparse_attn_bwd(qd, kd, vd, og, do, lse, kv_count, kv_idx, q_lists=(q_count, q_idx), dq=dq_,
+                                  dk=dk_, dv=dv_, delta=delta, grid=(w.T, w.H, w.W))
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(3):
+            flush.zero_()
+            bstep()
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.backward_steps)]
+        for s in range(args.backward_steps):
+            flush.zero_()
+            bstep(bev[s])
+        torch.cuda.synchronize()
+        status = nabla.get_status()
+        if status != 0:
+            raise RuntimeError(f"device status after the backward: {nabla.strerror(status)}")
+        t_tr = statistics.mean(e[0].elapsed_time(e[1]) for e in bev)
+        t_bw = statistics.mean(e[1].elapsed_time(e[2]) for e in bev)
+        bwd_flops = 2.5 * kept_flops(w, total_kept)  # S, dP, dV, dK, dQ: five 64x64xD products per tile
+        backward = {"ms": t_tr + t_bw, "transpose_lists_ms": t_tr, "attn_bwd_ms": t_bw,
+                    "tflops_kept": bwd_flops / ((t_tr + t_bw) * 1e-3) / 1e12,
+                    "flop_count": "10*64*64*D per kept tile (five products; the kernels recompute S and dP "
+                                  "in both passes, 14*64*64*D executed)",
+                    "steps": args.backward_steps, "launches_per_step": 4}
+        del do, q_count, q_idx, dq_, dk_, dv_, delta
+
     peak_tf, peak_gbs, peak_kind = load_peaks()
     attn_avg = statistics.mean(attn_ms)
     mask_avg = statistics.mean(mask_ms)
@@ -370,6 +412,7 @@ def run_gpu(args, rank, world, local_rank):
                           "frac": score_flops(w) / (mask_avg * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
                           "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"},
         "e2e": e2e,
+        "backward": backward,
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
@@ -476,6 +519,7 @@ def main():
     ap.add_argument("--config", default="wan13b", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--backward-steps", type=int, default=20, help="timed steps of the backward pass (0: skip)")
     ap.add_argument("--cpu-blocks", type=int, default=8, help="query blocks in the CPU-baseline sample")
     ap.add_argument("--ref-blocks", type=int, default=4, help="query blocks per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -17,8 +17,8 @@
 //                     dK and dV accumulated in registers.
 // The tile products use the warp-level bf16 tensor-core MMA (m16n8k16, fp32
 // accumulation) on operands staged in padded shared memory: four warps, 16
-// rows of the 64-row block each.  P and dS are rounded to bf16 for the
-// products, as the forward rounds P.  No thread ever waits on another
+// rows of the 64-row block each, operand fragments loaded by ldmatrix.  P
+// and dS are rounded to bf16 for the products, as the forward rounds P.  No thread ever waits on another
 // except at __syncthreads.
 #pragma once
 
@@ -128,19 +128,25 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Two bf16 of one shared-memory row, adjacent columns (32-bit load).
-__device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
-
-// Two bf16 of one column, rows r and r+1 (two 16-bit loads).
-__device__ __forceinline__ uint32_t ld_col_pair(const __nv_bfloat16* p, int stride) {
-  const uint32_t lo = *reinterpret_cast<const uint16_t*>(p);
-  const uint32_t hi = *reinterpret_cast<const uint16_t*>(p + stride);
-  return lo | (hi << 16);
+// Four 8 x 8 bf16 matrices from shared memory; lanes 8m..8m+7 give the row
+// addresses of matrix m (16-byte aligned) and register m receives it:
+// without .trans lane (g, t) gets row g, columns 2t and 2t+1 (an A or a
+// row-indexed B fragment); with .trans it gets rows 2t and 2t+1 of column g
+// (a B fragment of a matrix stored with k along rows).
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const __nv_bfloat16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const __nv_bfloat16* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
 }
 
 // Shared-memory row stride of a staged 64 x D tile: D + 8 elements, so rows
-// start 16 bytes apart modulo 128 and neither the row-pair nor the
-// column-pair fragment loads of a warp hit one bank twice.
+// start 16 bytes apart modulo 128 and the eight 16-byte rows of every
+// ldmatrix matrix fall in distinct banks.
 template <int D>
 struct BwdTile {
   static constexpr int kStride = D + 8;
@@ -172,20 +178,26 @@ __device__ __forceinline__ void stage_tile(__nv_bfloat16* dst, const __nv_bfloat
 // from row0) times B^T where B is the 64 x D tile sb (column n of the result
 // is row n of sb): the "row . row" product used for S = Q K^T and dP = dO V^T
 // and their transposes.
+// Fragment loads by ldmatrix (lane l, m = l / 8, r = l % 8): A's matrices
+// are (rows lo, k lo), (rows hi, k lo), (rows lo, k hi), (rows hi, k hi); a
+// B pair covers two column tiles, each (k lo), (k hi).
 template <int D>
 __device__ __forceinline__ void mma_rows_rows(float (&acc)[8][4], const __nv_bfloat16* sa, int row0,
-                                              const __nv_bfloat16* sb, int g, int t) {
+                                              const __nv_bfloat16* sb, int lane) {
   constexpr int ST = BwdTile<D>::kStride;
+  const int m = lane >> 3, r = lane & 7;
 #pragma unroll
   for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
-    const __nv_bfloat16* ar = sa + (row0 + g) * ST + ks * 16 + 2 * t;
-    const uint32_t a0 = ld_pair(ar), a1 = ld_pair(ar + 8 * ST), a2 = ld_pair(ar + 8), a3 = ld_pair(ar + 8 * ST + 8);
+    uint32_t a[4];
+    ldsm_x4(a, sa + (row0 + r + 8 * (m & 1)) * ST + ks * 16 + 8 * (m >> 1));
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      const __nv_bfloat16* br = sb + (n * 8 + g) * ST + ks * 16 + 2 * t;
-      mma_bf16_16816(acc[n], a0, a1, a2, a3, ld_pair(br), ld_pair(br + 8));
+    for (int np = 0; np < 4; ++np) {
+      uint32_t bb[4];
+      ldsm_x4(bb, sb + ((2 * np + (m >> 1)) * 8 + r) * ST + ks * 16 + 8 * (m & 1));
+      mma_bf16_16816(acc[2 * np], a[0], a[1], a[2], a[3], bb[0], bb[1]);
+      mma_bf16_16816(acc[2 * np + 1], a[0], a[1], a[2], a[3], bb[2], bb[3]);
     }
   }
 }
@@ -194,18 +206,22 @@ __device__ __forceinline__ void mma_rows_rows(float (&acc)[8][4], const __nv_bfl
 // the 8 column tiles, rounded to bf16 here) times the 64 x D tile sb.
 template <int D>
 __device__ __forceinline__ void mma_p_tile(float (&out)[D / 8][4], const float (&p)[8][4],
-                                           const __nv_bfloat16* sb, int g, int t) {
+                                           const __nv_bfloat16* sb, int lane) {
   constexpr int ST = BwdTile<D>::kStride;
+  const int m = lane >> 3, r = lane & 7;
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {  // 16 of the 64 columns of P per step
     const uint32_t a0 = pack2_bf16(p[2 * ks][0], p[2 * ks][1]);
     const uint32_t a1 = pack2_bf16(p[2 * ks][2], p[2 * ks][3]);
     const uint32_t a2 = pack2_bf16(p[2 * ks + 1][0], p[2 * ks + 1][1]);
     const uint32_t a3 = pack2_bf16(p[2 * ks + 1][2], p[2 * ks + 1][3]);
-    const __nv_bfloat16* bc = sb + (ks * 16 + 2 * t) * ST + g;
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-      mma_bf16_16816(out[n], a0, a1, a2, a3, ld_col_pair(bc + n * 8, ST), ld_col_pair(bc + n * 8 + 8 * ST, ST));
+    for (int np = 0; np < D / 16; ++np) {
+      uint32_t bb[4];
+      ldsm_x4_trans(bb, sb + (ks * 16 + r + 8 * (m & 1)) * ST + (2 * np + (m >> 1)) * 8);
+      mma_bf16_16816(out[2 * np], a0, a1, a2, a3, bb[0], bb[1]);
+      mma_bf16_16816(out[2 * np + 1], a0, a1, a2, a3, bb[2], bb[3]);
+    }
   }
 }
 
@@ -277,8 +293,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdArgs a) {
     stage_tile<D>(sv, a.v + ktok * row_elems + hd * D, row_elems, a.W);
     __syncthreads();
     float s[8][4], dp[8][4];
-    mma_rows_rows<D>(s, sq, warp * 16, sk, g, t);   // S = Q K^T
-    mma_rows_rows<D>(dp, sdo, warp * 16, sv, g, t);  // dP = dO V^T
+    mma_rows_rows<D>(s, sq, warp * 16, sk, lane);   // S = Q K^T
+    mma_rows_rows<D>(dp, sdo, warp * 16, sv, lane);  // dP = dO V^T
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const float p0 = exp2f(s[n][0] * a.scale_log2 - L0), p1 = exp2f(s[n][1] * a.scale_log2 - L0);
@@ -288,7 +304,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdArgs a) {
       s[n][2] = p2 * (dp[n][2] - d1);
       s[n][3] = p3 * (dp[n][3] - d1);
     }
-    mma_p_tile<D>(dq, s, sk, g, t);  // dQ += dS K
+    mma_p_tile<D>(dq, s, sk, lane);  // dQ += dS K
   }
   __nv_bfloat16* out0 = a.dq + (tok0 + o0) * row_elems + hd * D;
   __nv_bfloat16* out1 = a.dq + (tok0 + o1) * row_elems + hd * D;
@@ -352,8 +368,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdArgs a) 
     }
     __syncthreads();
     float s[8][4], dp[8][4];
-    mma_rows_rows<D>(s, sk, warp * 16, sq, g, t);   // S^T = K Q^T
-    mma_rows_rows<D>(dp, sv, warp * 16, sdo, g, t);  // dP^T = V dO^T
+    mma_rows_rows<D>(s, sk, warp * 16, sq, lane);   // S^T = K Q^T
+    mma_rows_rows<D>(dp, sv, warp * 16, sdo, lane);  // dP^T = V dO^T
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const int c = n * 8 + 2 * t;  // query columns c, c+1
@@ -369,8 +385,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdArgs a) 
       dp[n][2] = p2 * (dp[n][2] - d0);
       dp[n][3] = p3 * (dp[n][3] - d1);
     }
-    mma_p_tile<D>(dv, s, sdo, g, t);  // dV += P^T dO
-    mma_p_tile<D>(dk, dp, sq, g, t);  // dK += dS^T Q
+    mma_p_tile<D>(dv, s, sdo, lane);  // dV += P^T dO
+    mma_p_tile<D>(dk, dp, sq, lane);  // dK += dS^T Q
   }
   const int r0 = warp * 16 + g;
   const int64_t o0 = (tok0 + block_row(r0, a.W)) * row_elems + hd * D;
