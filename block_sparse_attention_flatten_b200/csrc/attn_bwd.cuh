@@ -150,9 +150,10 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const __nv_bfloa
 template <int D>
 struct BwdTile {
   static constexpr int kStride = D + 8;
-  // dynamic shared memory of the dQ and dK/dV kernels: four staged tiles,
-  // then the 64 LSE and Delta values of the dK/dV kernel
-  static constexpr size_t kSmemBytes = 4u * 64u * kStride * 2u + 2u * 64u * 4u;
+  // dynamic shared memory of the dQ and dK/dV kernels: the CTA's own two
+  // tiles, two buffers of the two tiles it walks over, then two buffers of
+  // the 64 LSE and Delta values of the dK/dV kernel
+  static constexpr size_t kSmemBytes = 6u * 64u * kStride * 2u + 2u * 2u * 64u * 4u;
 };
 
 // Row of the r-th token (flattened order inside the block) of a block,
@@ -160,6 +161,31 @@ struct BwdTile {
 // tensors in grid order (W > 0) row r/8 of the 8 x 8 patch, column r%8.
 __device__ __forceinline__ int64_t block_row(int r, int W) {
   return W > 0 ? static_cast<int64_t>(r >> 3) * W + (r & 7) : r;
+}
+
+// Asynchronous global -> shared copies (cp.async): the data lands after the
+// committing thread's cp.async.wait_group, and is visible to the CTA after
+// the __syncthreads that follows.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until at most one committed group of this thread is still in flight
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// stage_tile with asynchronous copies.
+template <int D>
+__device__ __forceinline__ void stage_tile_async(__nv_bfloat16* dst, const __nv_bfloat16* src_row0, int row_elems,
+                                                 int W) {
+  constexpr int kChunks = D / 8;
+  for (int x = threadIdx.x; x < 64 * kChunks; x += kBwdThreads) {
+    const int r = x / kChunks, c = x - r * kChunks;
+    cp_async16(dst + r * BwdTile<D>::kStride + c * 8,
+               reinterpret_cast<const uint4*>(src_row0 + block_row(r, W) * row_elems) + c);
+  }
 }
 
 // Copies a 64-token x D tile of one head (rows of Hh*D elements; first token
@@ -255,8 +281,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdArgs a) {
   extern __shared__ __align__(16) unsigned char bwd_smem[];
   __nv_bfloat16* sq = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
   __nv_bfloat16* sdo = sq + 64 * ST;
-  __nv_bfloat16* sk = sdo + 64 * ST;
-  __nv_bfloat16* sv = sk + 64 * ST;
+  __nv_bfloat16* skv = sdo + 64 * ST;  // two buffers of (K, V)
   const int i = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int row_elems = a.Hh * D;
@@ -281,17 +306,35 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdArgs a) {
   float dq[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.f;
-  for (int e = 0; e < cnt; ++e) {
+  // K, V of list entry e go to buffer e & 1: the copies of entry e + 1 are
+  // in flight while entry e is multiplied.  A bad entry is reported, not
+  // fetched and skipped.
+  auto fetch = [&](int e) -> bool {
     const int j = list[e];
     if (j < 0 || j >= a.Nb) {
       if (threadIdx.x == 0) report(NABLA_ERR_DEVICE_BOUNDS);
+      return false;
+    }
+    const int64_t ktok = static_cast<int64_t>(b) * a.S + block_first_token(a, j);
+    __nv_bfloat16* bk = skv + (e & 1) * 2 * 64 * ST;
+    stage_tile_async<D>(bk, a.k + ktok * row_elems + hd * D, row_elems, a.W);
+    stage_tile_async<D>(bk + 64 * ST, a.v + ktok * row_elems + hd * D, row_elems, a.W);
+    return true;
+  };
+  bool ok = cnt > 0 && fetch(0);
+  cp_async_commit();
+  for (int e = 0; e < cnt; ++e) {
+    const bool ok_next = e + 1 < cnt && fetch(e + 1);
+    cp_async_commit();
+    cp_async_wait_one();  // entry e's copies have landed
+    __syncthreads();
+    if (!ok) {
+      __syncthreads();
+      ok = ok_next;
       continue;
     }
-    __syncthreads();  // every warp is done with the previous K, V
-    const int64_t ktok = static_cast<int64_t>(b) * a.S + block_first_token(a, j);
-    stage_tile<D>(sk, a.k + ktok * row_elems + hd * D, row_elems, a.W);
-    stage_tile<D>(sv, a.v + ktok * row_elems + hd * D, row_elems, a.W);
-    __syncthreads();
+    const __nv_bfloat16* sk = skv + (e & 1) * 2 * 64 * ST;
+    const __nv_bfloat16* sv = sk + 64 * ST;
     float s[8][4], dp[8][4];
     mma_rows_rows<D>(s, sq, warp * 16, sk, lane);   // S = Q K^T
     mma_rows_rows<D>(dp, sdo, warp * 16, sv, lane);  // dP = dO V^T
@@ -305,6 +348,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdArgs a) {
       s[n][3] = p3 * (dp[n][3] - d1);
     }
     mma_p_tile<D>(dq, s, sk, lane);  // dQ += dS K
+    __syncthreads();  // every warp is done with buffer e & 1 before entry e + 2 is fetched into it
+    ok = ok_next;
   }
   __nv_bfloat16* out0 = a.dq + (tok0 + o0) * row_elems + hd * D;
   __nv_bfloat16* out1 = a.dq + (tok0 + o1) * row_elems + hd * D;
@@ -326,10 +371,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdArgs a) 
   extern __shared__ __align__(16) unsigned char bwd_smem[];
   __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(bwd_smem);
   __nv_bfloat16* sv = sk + 64 * ST;
-  __nv_bfloat16* sq = sv + 64 * ST;
-  __nv_bfloat16* sdo = sq + 64 * ST;
-  float* s_l = reinterpret_cast<float*>(sdo + 64 * ST);
-  float* s_d = s_l + 64;
+  __nv_bfloat16* sqdo = sv + 64 * ST;  // two buffers of (Q, dO)
+  float* s_ld = reinterpret_cast<float*>(sqdo + 4 * 64 * ST);  // two buffers of (LSE, Delta), raw
   const int j = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int row_elems = a.Hh * D;
@@ -349,31 +392,49 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdArgs a) 
     dk[n][0] = dk[n][1] = dk[n][2] = dk[n][3] = 0.f;
     dv[n][0] = dv[n][1] = dv[n][2] = dv[n][3] = 0.f;
   }
-  for (int e = 0; e < cnt; ++e) {
+  // Q, dO, LSE and Delta of list entry e go to buffer e & 1 (as in the dQ
+  // kernel, the next entry's copies overlap this entry's products).
+  auto fetch = [&](int e) -> bool {
     const int i = list[e];
     if (i < 0 || i >= a.Nb) {
       if (threadIdx.x == 0) report(NABLA_ERR_DEVICE_BOUNDS);
-      continue;
+      return false;
     }
-    __syncthreads();  // every warp is done with the previous Q, dO
     const int64_t qfirst = block_first_token(a, i);
     const int64_t qtok = static_cast<int64_t>(b) * a.S + qfirst;
-    stage_tile<D>(sq, a.q + qtok * row_elems + hd * D, row_elems, a.W);
-    stage_tile<D>(sdo, a.dout + qtok * row_elems + hd * D, row_elems, a.W);
-    if (threadIdx.x < 64) {
-      const int64_t lr = bh * a.S + qfirst + block_row(threadIdx.x, a.W);
-      const float l = a.lse[lr];
-      s_l[threadIdx.x] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-      s_d[threadIdx.x] = a.delta[lr];
-    }
+    __nv_bfloat16* bq = sqdo + (e & 1) * 2 * 64 * ST;
+    stage_tile_async<D>(bq, a.q + qtok * row_elems + hd * D, row_elems, a.W);
+    stage_tile_async<D>(bq + 64 * ST, a.dout + qtok * row_elems + hd * D, row_elems, a.W);
+    const int x = threadIdx.x & 63;  // threads 0-63 copy the LSE, 64-127 Delta
+    const int64_t lr = bh * a.S + qfirst + block_row(x, a.W);
+    cp_async4(s_ld + (e & 1) * 128 + threadIdx.x, threadIdx.x < 64 ? a.lse + lr : a.delta + lr);
+    return true;
+  };
+  bool ok = cnt > 0 && fetch(0);
+  cp_async_commit();
+  for (int e = 0; e < cnt; ++e) {
+    const bool ok_next = e + 1 < cnt && fetch(e + 1);
+    cp_async_commit();
+    cp_async_wait_one();  // entry e's copies have landed
     __syncthreads();
+    if (!ok) {
+      __syncthreads();
+      ok = ok_next;
+      continue;
+    }
+    const __nv_bfloat16* sq = sqdo + (e & 1) * 2 * 64 * ST;
+    const __nv_bfloat16* sdo = sq + 64 * ST;
+    const float* s_l = s_ld + (e & 1) * 128;
+    const float* s_d = s_l + 64;
     float s[8][4], dp[8][4];
     mma_rows_rows<D>(s, sk, warp * 16, sq, lane);   // S^T = K Q^T
     mma_rows_rows<D>(dp, sv, warp * 16, sdo, lane);  // dP^T = V dO^T
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const int c = n * 8 + 2 * t;  // query columns c, c+1
-      const float L0 = s_l[c], L1 = s_l[c + 1], d0 = s_d[c], d1 = s_d[c + 1];
+      const float l0 = s_l[c], l1 = s_l[c + 1], d0 = s_d[c], d1 = s_d[c + 1];
+      const float L0 = l0 == -INFINITY ? INFINITY : l0 * 1.4426950408889634f;
+      const float L1 = l1 == -INFINITY ? INFINITY : l1 * 1.4426950408889634f;
       const float p0 = exp2f(s[n][0] * a.scale_log2 - L0), p1 = exp2f(s[n][1] * a.scale_log2 - L1);
       const float p2 = exp2f(s[n][2] * a.scale_log2 - L0), p3 = exp2f(s[n][3] * a.scale_log2 - L1);
       s[n][0] = p0;
@@ -387,6 +448,8 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdArgs a) 
     }
     mma_p_tile<D>(dv, s, sdo, lane);  // dV += P^T dO
     mma_p_tile<D>(dk, dp, sq, lane);  // dK += dS^T Q
+    __syncthreads();  // every warp is done with buffer e & 1 before entry e + 2 is fetched into it
+    ok = ok_next;
   }
   const int r0 = warp * 16 + g;
   const int64_t o0 = (tok0 + block_row(r0, a.W)) * row_elems + hd * D;
