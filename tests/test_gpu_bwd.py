@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from _parity import Case, flat_to_grid_rows, grid_to_flat_rows
+from _parity import Case, grid_to_flat_rows
 from block_sparse_attention_flatten_b200 import inputs
 from block_sparse_attention_flatten_b200 import nabla
 
