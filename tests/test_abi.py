@@ -35,6 +35,24 @@ def test_header_declares_the_boundary():
     assert set(fns) == set(nabla.EXPORTS)
 
 
+def header_prototypes():
+    """name -> number of parameters, from the header's declarations."""
+    text = open(os.path.join(ROOT, "include", "nabla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b(nabla_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text):
+        params = m.group(2).strip()
+        protos[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_argtypes_match_header_prototypes(lib):
+    protos = header_prototypes()
+    assert set(protos) == set(nabla.EXPORTS)
+    for name, n in protos.items():
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in header_functions():
         assert hasattr(lib, name), name
