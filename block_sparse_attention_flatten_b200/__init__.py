@@ -11,6 +11,14 @@ copies -- the fractal flattening happens inside the kernels:
     kv_count, kv_idx, _ = nabla.build_mask_grid(q, k, T, H, W, thr=0.9, sta=(3, 3, 3))
     o, lse = nabla.sparse_attn_fwd(q, k, v, kv_count, kv_idx, grid=(T, H, W))
 
+Backward pass over the same lists (training), grid order as well:
+
+    dq, dk, dv = nabla.sparse_attn_bwd(q, k, v, o, do, lse, kv_count, kv_idx, grid=(T, H, W))
+
+The static sliding-tile window alone, without reading Q or K:
+
+    kv_count, kv_idx = nabla.build_mask_sta(B, Hh, T, H, W, (3, 3, 3))
+
 Flattened tensors (e.g. flattened once per sequence):
 
     qf = nabla.flatten(q, T, H, W)                       # per tensor
