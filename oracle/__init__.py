@@ -61,6 +61,7 @@ def _load():
         lib.oracle_sta.restype = i
         lib.oracle_sta_lists.argtypes = [i, i, i, i, i, i, P, P]
         lib.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, P, P]
+        lib.oracle_attention_bwd_sampled.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, i, P, i, P, P, P]
         lib.oracle_num_threads.restype = i
         _lib = lib
     return _lib
@@ -215,4 +216,25 @@ def attention_bwd(qf, kf, vf, dof, kv_count: np.ndarray, kv_idx: np.ndarray, sca
     dv = np.empty_like(dq)
     _load().oracle_attention_bwd(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(dof), _ptr(kv_count), _ptr(kv_idx),
                                  B, S, Hh, D, scale, _ptr(dq), _ptr(dk), _ptr(dv))
+    return dq, dk, dv
+
+
+def attention_bwd_sampled(qf, kf, vf, dof, kv_count: np.ndarray, kv_idx: np.ndarray, scale: float,
+                          qblocks, kblocks):
+    """:func:`attention_bwd` restricted to listed blocks: dq fp64 [B, nq*64,
+    Hh, D] for the query blocks qblocks, dk and dv fp64 [B, nk*64, Hh, D] for
+    the key blocks kblocks (each list ascending or not, no repeats)."""
+    qf, kf, vf, dof = _bits(qf), _bits(kf), _bits(vf), _bits(dof)
+    B, S, Hh, D = qf.shape
+    kv_count = np.ascontiguousarray(kv_count, dtype=np.int32)
+    kv_idx = np.ascontiguousarray(kv_idx, dtype=np.int32)
+    qblocks = np.ascontiguousarray(qblocks, dtype=np.int32)
+    kblocks = np.ascontiguousarray(kblocks, dtype=np.int32)
+    nq, nk = qblocks.shape[0], kblocks.shape[0]
+    dq = np.empty((B, nq * BLOCK, Hh, D), dtype=np.float64)
+    dk = np.empty((B, nk * BLOCK, Hh, D), dtype=np.float64)
+    dv = np.empty_like(dk)
+    _load().oracle_attention_bwd_sampled(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(dof), _ptr(kv_count), _ptr(kv_idx),
+                                         B, S, Hh, D, scale, _ptr(qblocks), nq, _ptr(kblocks), nk,
+                                         _ptr(dq), _ptr(dk), _ptr(dv))
     return dq, dk, dv

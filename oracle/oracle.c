@@ -507,3 +507,106 @@ void oracle_attention_bwd(const uint16_t* qf, const uint16_t* kf, const uint16_t
     free(dp);
   }
 }
+
+/* ------------------------------------------------------------------------ */
+/* The same gradient as oracle_attention_bwd, restricted to listed blocks so */
+/* that full-size layers can be checked on a sample: dQ for the query blocks */
+/* in qblocks (nq of them) and dK, dV for the key blocks in kblocks (nk).    */
+/* dQ of a query token needs only its own row; dK, dV of a key token need    */
+/* every row that keeps its block, so those rows are evaluated in full (the  */
+/* row's softmax and its sum_c P dP run over all of the row's kept tokens).  */
+/* Arithmetic per row as in oracle_attention_bwd.                            */
+/* dq: fp64 [B][nq*64][Hh][D] (qblocks order); dk, dv: fp64 [B][nk*64][Hh][D] */
+/* (kblocks order); all overwritten.  Either list may be empty (n = 0).      */
+/* Pinned by: autograd of the token-level masked attention on the listed     */
+/* blocks.                                                                   */
+/* ------------------------------------------------------------------------ */
+void oracle_attention_bwd_sampled(const uint16_t* qf, const uint16_t* kf, const uint16_t* vf,
+                                  const uint16_t* dof, const int32_t* kv_count, const int32_t* kv_idx, int B,
+                                  int S, int Hh, int D, double scale, const int32_t* qblocks, int nq,
+                                  const int32_t* kblocks, int nk, double* dq, double* dk, double* dv) {
+  int Nb = S / ORACLE_BLOCK;
+  int* qpos = (int*)malloc(sizeof(int) * (size_t)Nb);
+  int* kpos = (int*)malloc(sizeof(int) * (size_t)Nb);
+  for (int j = 0; j < Nb; ++j) qpos[j] = kpos[j] = -1;
+  for (int x = 0; x < nq; ++x) qpos[qblocks[x]] = x;
+  for (int x = 0; x < nk; ++x) kpos[kblocks[x]] = x;
+  for (int64_t x = 0; x < (int64_t)B * nq * ORACLE_BLOCK * Hh * D; ++x) dq[x] = 0.0;
+  for (int64_t x = 0; x < (int64_t)B * nk * ORACLE_BLOCK * Hh * D; ++x) dk[x] = dv[x] = 0.0;
+#pragma omp parallel
+  {
+    double* pr = (double*)malloc(sizeof(double) * (size_t)S);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)S);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < (int64_t)B * Hh; ++bh) {
+      int b = (int)(bh / Hh), hd = (int)(bh % Hh);
+#define ORACLE_AT(base, tok) ((base) + (((int64_t)b * S + (tok)) * Hh + hd) * D)
+#define ORACLE_OUT(base, n, pos, r) ((base) + (((int64_t)b * (n) * ORACLE_BLOCK + (int64_t)(pos) * ORACLE_BLOCK + (r)) * Hh + hd) * D)
+      for (int i = 0; i < Nb; ++i) {
+        int64_t row = bh * Nb + i;
+        int cnt = kv_count[row];
+        const int32_t* lst = kv_idx + row * Nb;
+        int needed = qpos[i] >= 0;
+        for (int e = 0; e < cnt && !needed; ++e) needed = kpos[lst[e]] >= 0;
+        if (!needed) continue;
+        for (int r = 0; r < ORACLE_BLOCK; ++r) {
+          int64_t a = (int64_t)i * ORACLE_BLOCK + r;
+          const uint16_t* q = ORACLE_AT(qf, a);
+          const uint16_t* g = ORACLE_AT(dof, a);
+          double mx = -INFINITY, den = 0.0, pdp = 0.0;
+          int64_t n = 0;
+          for (int e = 0; e < cnt; ++e)
+            for (int c = 0; c < ORACLE_BLOCK; ++c) {
+              const uint16_t* k = ORACLE_AT(kf, (int64_t)lst[e] * ORACLE_BLOCK + c);
+              double dot = 0.0;
+              for (int d = 0; d < D; ++d) dot += (double)bf16_bits_to_f32(q[d]) * (double)bf16_bits_to_f32(k[d]);
+              pr[n] = dot * scale;
+              if (pr[n] > mx) mx = pr[n];
+              ++n;
+            }
+          for (int64_t c = 0; c < n; ++c) {
+            pr[c] = exp(pr[c] - mx);
+            den += pr[c];
+          }
+          for (int64_t c = 0; c < n; ++c) pr[c] /= den;
+          n = 0;
+          for (int e = 0; e < cnt; ++e)
+            for (int c = 0; c < ORACLE_BLOCK; ++c) {
+              const uint16_t* v = ORACLE_AT(vf, (int64_t)lst[e] * ORACLE_BLOCK + c);
+              double dot = 0.0;
+              for (int d = 0; d < D; ++d) dot += (double)bf16_bits_to_f32(g[d]) * (double)bf16_bits_to_f32(v[d]);
+              dp[n] = dot;
+              pdp += pr[n] * dot;
+              ++n;
+            }
+          double* dqa = qpos[i] >= 0 ? ORACLE_OUT(dq, nq, qpos[i], r) : NULL;
+          n = 0;
+          for (int e = 0; e < cnt; ++e) {
+            int kp = kpos[lst[e]];
+            for (int c = 0; c < ORACLE_BLOCK; ++c) {
+              const uint16_t* k = ORACLE_AT(kf, (int64_t)lst[e] * ORACLE_BLOCK + c);
+              double ds = pr[n] * (dp[n] - pdp);
+              if (dqa)
+                for (int d = 0; d < D; ++d) dqa[d] += scale * ds * (double)bf16_bits_to_f32(k[d]);
+              if (kp >= 0) {
+                double* dkc = ORACLE_OUT(dk, nk, kp, c);
+                double* dvc = ORACLE_OUT(dv, nk, kp, c);
+                for (int d = 0; d < D; ++d) {
+                  dvc[d] += pr[n] * (double)bf16_bits_to_f32(g[d]);
+                  dkc[d] += scale * ds * (double)bf16_bits_to_f32(q[d]);
+                }
+              }
+              ++n;
+            }
+          }
+        }
+      }
+#undef ORACLE_OUT
+#undef ORACLE_AT
+    }
+    free(pr);
+    free(dp);
+  }
+  free(qpos);
+  free(kpos);
+}

@@ -489,6 +489,22 @@ def test_attention_bwd_equals_autograd(oracle_lib, D, p_keep, empty):
         assert np.abs(got - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
 
 
+def test_attention_bwd_sampled_equals_autograd_on_listed_blocks(oracle_lib):
+    rng = np.random.default_rng(5)
+    B, Hh, Nb, D = 2, 2, 6, 64
+    S = Nb * BLOCK
+    q, k, v, do = (inputs.randn_bf16((B, S, Hh, D), seed=s) for s in (31, 32, 33, 34))
+    cnt, idx = random_lists(rng, B, Hh, Nb, 0.45, empty_rows=(1,), unkept_col=4)
+    rq, rk, rv = autograd_masked_attention(q, k, v, do, cnt, idx, 0.125)
+    qb, kb = np.array([5, 0, 1]), np.array([2, 4, 3])
+    dq, dk, dv = oracle_lib.attention_bwd_sampled(q, k, v, do, cnt, idx, 0.125, qb, kb)
+    rows = lambda blocks: np.concatenate([np.arange(j * BLOCK, (j + 1) * BLOCK) for j in blocks])  # noqa: E731
+    for got, ref in ((dq, rq[:, rows(qb)]), (dk, rk[:, rows(kb)]), (dv, rv[:, rows(kb)])):
+        assert np.abs(got - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    empty = oracle_lib.attention_bwd_sampled(q, k, v, do, cnt, idx, 0.125, np.array([], np.int32), kb)
+    assert empty[0].shape == (B, 0, Hh, D)
+
+
 def test_attention_bwd_invariants(oracle_lib):
     rng = np.random.default_rng(3)
     B, Hh, Nb, D = 1, 3, 6, 64

@@ -45,6 +45,7 @@ PINS = {
     "attention_special": lambda m: pins.test_attention_special_cases(m),
     "bwd_autograd": lambda m: [pins.test_attention_bwd_equals_autograd(m, *a) for a in [(64, 0.5, ()), (128, 0.3, (2,))]],
     "bwd_invariants": lambda m: pins.test_attention_bwd_invariants(m),
+    "bwd_sampled": lambda m: pins.test_attention_bwd_sampled_equals_autograd_on_listed_blocks(m),
 }
 
 # (name, text in oracle.c, planted replacement, pins expected to catch it)
@@ -77,6 +78,11 @@ MUTANTS = [
     ("gradient: dQ from q instead of k",
      "dqa[d] += scale * ds * (double)bf16_bits_to_f32(k[d]);",
      "dqa[d] += scale * ds * (double)bf16_bits_to_f32(q[d]);", ["bwd_autograd"]),
+    ("sampled gradient: row term over the sampled block only", "              pdp += pr[n] * dot;\n              ++n;\n            }\n          double* dqa = qpos",
+     "              if (kpos[lst[e]] >= 0) pdp += pr[n] * dot;\n              ++n;\n            }\n          double* dqa = qpos",
+     ["bwd_sampled"]),
+    ("sampled gradient: dK, dV rows limited to sampled query blocks", "int needed = qpos[i] >= 0;\n        for (int e = 0; e < cnt && !needed; ++e) needed = kpos[lst[e]] >= 0;",
+     "int needed = qpos[i] >= 0;", ["bwd_sampled"]),
 ]
 
 
@@ -84,7 +90,9 @@ def build_variant(tmp_path, tag, old=None, new=None):
     with open(os.path.join(ORACLE_DIR, "oracle.c")) as fh:
         src = fh.read()
     if old is not None:
-        assert src.count(old) == 1, f"mutation target not unique or missing: {old!r}"
+        # every occurrence is planted (the gradient's formulas appear in both
+        # the full and the sampled function)
+        assert src.count(old) >= 1, f"mutation target missing: {old!r}"
         src = src.replace(old, new)
     d = tmp_path / tag
     d.mkdir()
