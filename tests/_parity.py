@@ -148,3 +148,21 @@ def check_attention(case: Case, out: torch.Tensor, lse: torch.Tensor, qblocks, h
     assert np.array_equal(finite, np.isfinite(got_lse))
     lse_err = float(np.abs(got_lse[finite] - ref_lse[finite]).max()) if finite.any() else 0.0
     return float(err.max()), float(err.mean()), lse_err
+
+
+def block_rows(blocks) -> np.ndarray:
+    """Flattened token rows of the listed blocks, in list order."""
+    return np.concatenate([np.arange(j * 64, (j + 1) * 64) for j in blocks])
+
+
+def sampled_gradient_errors(dq, dk, dv, ref, qblocks, kblocks):
+    """Relative errors of flattened-order gradients [B,S,Hh,D] (torch, any
+    device) against the oracle's sampled gradient (dq of qblocks, dk and dv
+    of kblocks): per tensor (max|err| / max|ref|, mean|err| / mean|ref|)."""
+    out = []
+    for got, r, blocks in ((dq, ref[0], qblocks), (dk, ref[1], kblocks), (dv, ref[2], kblocks)):
+        rows = torch.as_tensor(block_rows(blocks), device=got.device)
+        g = got.index_select(1, rows).double().cpu().numpy()
+        err = np.abs(g - r)
+        out.append((err.max() / max(np.abs(r).max(), 1e-30), err.mean() / max(np.abs(r).mean(), 1e-30)))
+    return out

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from _parity import Case, grid_to_flat_rows
+from _parity import Case, grid_to_flat_rows, sampled_gradient_errors
 from block_sparse_attention_flatten_b200 import inputs
 from block_sparse_attention_flatten_b200 import nabla
 
@@ -207,3 +207,28 @@ def test_backward_full_size_properties():
     t_bwd = ev[1].elapsed_time(ev[2])
     print(f"\nWan-like backward: transpose {ev[0].elapsed_time(ev[1]):.3f} ms, backward {t_bwd:.3f} ms, "
           f"{10 * 64 * 64 * w.D * kept / (t_bwd * 1e-3) / 1e12:.1f} TFLOP/s (algorithmic, 5 products per tile)")
+
+
+def test_backward_full_size_sampled_against_oracle():
+    """Wan-1.3B-like layer at full size in grid order (the layout bench.py
+    times): dQ of 8 seeded query blocks and dK, dV of 4 seeded key blocks,
+    all heads, element by element against the oracle's gradient restricted
+    to those blocks (evaluated on the GPU's own lists)."""
+    w = inputs.WAN13B
+    q, k, v = inputs.make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    kv_count, kv_idx, _ = nabla.build_mask_grid(qd, kd, w.T, w.H, w.W, w.thr, w.sta)
+    do = inputs.randn_bf16((w.B, w.S, w.Hh, w.D), seed=97)
+    out, lse = nabla.sparse_attn_fwd(qd, kd, vd, kv_count, kv_idx, grid=(w.T, w.H, w.W))
+    dq, dk, dv = nabla.sparse_attn_bwd(qd, kd, vd, out, do.cuda(), lse, kv_count, kv_idx, grid=(w.T, w.H, w.W))
+    torch.cuda.synchronize()
+    assert nabla.get_status() == 0
+    grads = [grid_to_flat_rows(x, w.T, w.H, w.W, 1) for x in (dq, dk, dv)]
+    del out, lse, dq, dk, dv
+    qb = inputs.sample_query_blocks(w.Nb, 8, seed=1234)
+    kb = inputs.sample_query_blocks(w.Nb, 4, seed=4321)
+    flat = [oracle.flatten(x, w.T, w.H, w.W).reshape(x.shape) for x in (q, k, v, do)]
+    ref = oracle.attention_bwd_sampled(*flat, kv_count.cpu().numpy(), kv_idx.cpu().numpy(), w.scale, qb, kb)
+    for name, (mx, mean) in zip(("dq", "dk", "dv"), sampled_gradient_errors(*grads, ref, qb, kb)):
+        print(f"\nWan-like full size, sampled {name}: max/max|ref| {mx:.2e}, mean/mean|ref| {mean:.2e}")
+        assert mx <= MAX_REL and mean <= MEAN_REL, (name, mx, mean)

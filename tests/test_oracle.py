@@ -578,3 +578,25 @@ def test_parity_helper_flat_order_matches_oracle_flatten(oracle_lib):
         ids = np.arange(S, dtype=np.uint16).reshape(1, S, 1)
         flat = oracle_lib.flatten(ids, T, H, W).reshape(-1)
         assert np.array_equal(flat, flat_order(T, H, W).astype(np.uint16))
+
+
+def test_parity_helper_sampled_gradient_errors(oracle_lib):
+    """The GPU tests' sampled-gradient comparison, fed the full oracle
+    gradient in place of the GPU's: zero error on the listed blocks, and a
+    planted error in a listed block is seen."""
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from _parity import sampled_gradient_errors
+    rng = np.random.default_rng(8)
+    B, Hh, Nb, D = 1, 2, 7, 64
+    S = Nb * BLOCK
+    q, k, v, do = (inputs.randn_bf16((B, S, Hh, D), seed=s) for s in (41, 42, 43, 44))
+    cnt, idx = random_lists(rng, B, Hh, Nb, 0.4)
+    full = [torch.from_numpy(x) for x in oracle_lib.attention_bwd(q, k, v, do, cnt, idx, 0.125)]
+    qb, kb = np.array([6, 2]), np.array([0, 5, 3])
+    ref = oracle_lib.attention_bwd_sampled(q, k, v, do, cnt, idx, 0.125, qb, kb)
+    for mx, mean in sampled_gradient_errors(*full, ref, qb, kb):
+        assert mx < 1e-12 and mean < 1e-12
+    full[1][:, 5 * BLOCK + 3, 1, 7] += 1.0  # key block 5 is listed
+    errs = sampled_gradient_errors(*full, ref, qb, kb)
+    assert errs[1][0] > 1e-3 and errs[0][0] < 1e-12 and errs[2][0] < 1e-12
