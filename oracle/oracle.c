@@ -19,6 +19,11 @@
  * with dropped blocks absent from both numerator and normaliser (the
  * AB-Attention news page, section "Onde os esquemas esparsos anteriores
  * falham", second bullet) -> oracle_attention.
+ * Also: the window mask on its own (item 3 without the adaptive term; the
+ * summary's "Comparacao com Metodos Estaticos") -> oracle_sta_lists; and the
+ * gradient of the attention on the kept blocks, for the training the
+ * summary says NABLA also speeds up ("Aceleracao de Dupla Fase")
+ * -> oracle_attention_bwd, oracle_attention_bwd_sampled.
  *
  * Precision: the mask is fp32 (pooled vectors, scores, exponentials,
  * probabilities) with fp64 accumulation of the softmax normaliser and of the
