@@ -55,6 +55,7 @@ def _load():
         lib.oracle_mask.argtypes = [P, P, i, i, i, i, f, f, i, i, i, i, i, d, P, P, P, P]
         lib.oracle_attention.argtypes = [P, P, P, P, P, i, i, i, i, d, P, i, P, P]
         lib.oracle_block_probs_row.argtypes = [P, P, i, i, f, i, P]
+        lib.oracle_block_numerators_row.argtypes = [P, P, i, i, f, i, P]
         lib.oracle_cdf_keep.argtypes = [P, i, f, P, P, P, d]
         lib.oracle_cdf_keep.restype = i
         lib.oracle_sta.argtypes = [i, i, i, i, i, i, i]
@@ -123,9 +124,21 @@ def block_probs_row(qbar_bh: np.ndarray, kbar_bh: np.ndarray, i: int, scale: flo
     return p
 
 
+def block_numerators_row(qbar_bh: np.ndarray, kbar_bh: np.ndarray, i: int, scale: float) -> np.ndarray:
+    """Softmax numerators e = exp(s - max s) (fp32) of query block i for one
+    (b, head): the weights the CDF rule orders and accumulates."""
+    qbar_bh = np.ascontiguousarray(qbar_bh, dtype=np.float32)
+    kbar_bh = np.ascontiguousarray(kbar_bh, dtype=np.float32)
+    Nb, D = kbar_bh.shape
+    e = np.empty(Nb, dtype=np.float32)
+    _load().oracle_block_numerators_row(_ptr(qbar_bh), _ptr(kbar_bh), Nb, D, scale, i, _ptr(e))
+    return e
+
+
 def cdf_keep(p: np.ndarray, thr: float, band: float = BAND):
     """CDF keep flags, per-block cumulative mass, band flags and the arg-max
-    for one probability row."""
+    for one row of weights (probabilities, or the softmax numerators: the
+    rule normalises them by their sum)."""
     p = np.ascontiguousarray(p, dtype=np.float32)
     keep = np.empty(p.shape[0], dtype=np.uint8)
     cum = np.empty(p.shape[0], dtype=np.float64)

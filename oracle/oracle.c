@@ -11,7 +11,7 @@
  * paper 2507.13546), section "Metodologia: NABLA":
  *   item 1  "Reordenacao de Tokens (Fractal Flattening)"       -> oracle_flatten
  *   item 2  "Downsampling"                                     -> oracle_pool
- *           "Atencao Reduzida"                                 -> block_probs
+ *           "Atencao Reduzida"                -> block_numerators, block_probs
  *           "Limiarizacao CDF"                                 -> cdf_keep_row
  *           "Expansao"                                         -> kv lists
  *   item 3  "Integracao Hibrida com STA", M = M_nabla OR M_STA -> sta_keep
@@ -131,96 +131,85 @@ void oracle_pool(const uint16_t* x, float* xbar, int B, int S, int Hh, int D) {
 /*          multiply-adds in ascending d (fmaf), then one fp32 multiply;     */
 /*   m    = max_j s_ij;                                                      */
 /*   e_j  = exp(s_ij - m) correctly rounded to fp32 (s - m in fp32, exp in   */
-/*          fp64, then rounded);                                             */
-/*   Z    = sum_j e_j in fp64;  p_j = fl32(e_j / Z).                          */
+/*          fp64, then rounded): the softmax numerators, 0 < e_j <= 1;       */
+/*   Z    = sum_j e_j in fp64 (j ascending);  p_j = fl32(e_j / Z).           */
+/* block_numerators stops at e; block_probs goes on to p.                    */
 /* Pinned by: scores against the fp64 mean of token logits; sum p = 1 within */
 /* Nb * 2^-24; the all-equal-scores case giving exactly 1/Nb.                */
 /* ------------------------------------------------------------------------ */
-static void block_probs(const float* qbar_i, const float* kbar, int Nb, int D, float scale,
-                        float* p) {
+static void block_numerators(const float* qbar_i, const float* kbar, int Nb, int D, float scale,
+                             float* e) {
   float m = -INFINITY;
   for (int j = 0; j < Nb; ++j) {
     float dot = 0.0f;
     for (int d = 0; d < D; ++d) dot = fmaf(qbar_i[d], kbar[(int64_t)j * D + d], dot);
     float s = dot * scale;
-    p[j] = s;
+    e[j] = s;
     if (s > m) m = s;
   }
+  for (int j = 0; j < Nb; ++j) e[j] = (float)exp((double)(e[j] - m));
+}
+
+static void block_probs(const float* qbar_i, const float* kbar, int Nb, int D, float scale,
+                        float* p) {
+  block_numerators(qbar_i, kbar, Nb, D, scale, p);
   double Z = 0.0;
-  for (int j = 0; j < Nb; ++j) {
-    float e = (float)exp((double)(p[j] - m));
-    p[j] = e;
-    Z += (double)e;
-  }
+  for (int j = 0; j < Nb; ++j) Z += (double)p[j];
   for (int j = 0; j < Nb; ++j) p[j] = (float)((double)p[j] / Z);
 }
 
 typedef struct {
-  float p;
+  float w;
   int j;
-} pj_t;
+} wj_t;
 
-/* Ascending by probability, ties by ascending block index. */
-static int cmp_pj(const void* a, const void* b) {
-  const pj_t* x = (const pj_t*)a;
-  const pj_t* y = (const pj_t*)b;
-  if (x->p < y->p) return -1;
-  if (x->p > y->p) return 1;
+/* Ascending by weight, ties by ascending block index. */
+static int cmp_wj(const void* a, const void* b) {
+  const wj_t* x = (const wj_t*)a;
+  const wj_t* y = (const wj_t*)b;
+  if (x->w < y->w) return -1;
+  if (x->w > y->w) return 1;
   return (x->j > y->j) - (x->j < y->j);
 }
 
-/* Probabilities within this relative distance of each other are treated as  */
-/* tied by rounding when marking band blocks (about 8-16 fp32 ulps).         */
-#define ORACLE_TIE_REL (1.0 / 1048576.0) /* 2^-20 */
-
 /* ------------------------------------------------------------------------ */
 /* CDF thresholding (NABLA summary, "Limiarizacao CDF"): sort the row's       */
-/* probabilities ascending, take the running sum c_k (fp64) and keep the      */
-/* block at position k iff c_k > 1 - thr.  thr >= 1 keeps every block; the    */
-/* arg-max (last position) is always kept.  cum[j] receives c at block j's    */
-/* position.  band[j] (if not NULL) marks blocks whose decision rounding can  */
-/* change: |c - (1-thr)| < band_width, or a run of rounding-tied             */
-/* probabilities (consecutive in the order, each within ORACLE_TIE_REL of the */
-/* next) whose positions straddle 1 - thr, since the order inside such a run */
-/* is set by rounding, not by the method; the same holds for the run that    */
-/* holds the arg-max when it has more than one member (which block is the   */
-/* forced arg-max is then set by rounding).                                  */
-/* Pinned by: an exact-rational top-p (nucleus) restatement on random rows,  */
+/* probabilities ascending, take the running sum c_k and keep the block at   */
+/* position k iff c_k > 1 - thr.  thr >= 1 keeps every block; the arg-max    */
+/* (last position) is always kept.                                           */
+/* The row is given as weights w_j >= 0 whose normalised values w_j / sum(w) */
+/* are the probabilities (the softmax numerators e_j, or the probabilities   */
+/* themselves).  All probabilities of a row share one normaliser, so their   */
+/* ascending order is the ascending order of the weights, ties by ascending  */
+/* block index; rounding each quotient to fp32 first would merge distinct    */
+/* neighbours into ties the method does not have.                            */
+/*   Z = sum_j w_j (fp64, j ascending);  c_k = (w_(0) + ... + w_(k)) / Z,    */
+/* the running sum in fp64 in the sorted order.  cum[j] receives c at block  */
+/* j's position.  band[j] (if not NULL) marks blocks whose cumulative mass   */
+/* lies within band_width of 1 - thr.                                        */
+/* Pinned by: an exact-rational top-p (nucleus) restatement on real rows,    */
 /* kept mass >= thr and minimality, and the uniform Nb=16 case.              */
 /* ------------------------------------------------------------------------ */
-static int cdf_keep_row(const float* p, int Nb, float thr, uint8_t* keep, double* cum,
-                        uint8_t* band, double band_width, pj_t* scratch) {
+static int cdf_keep_row(const float* w, int Nb, float thr, uint8_t* keep, double* cum,
+                        uint8_t* band, double band_width, wj_t* scratch) {
+  double Z = 0.0;
   for (int j = 0; j < Nb; ++j) {
-    scratch[j].p = p[j];
+    scratch[j].w = w[j];
     scratch[j].j = j;
+    Z += (double)w[j];
   }
-  qsort(scratch, (size_t)Nb, sizeof(pj_t), cmp_pj);
+  qsort(scratch, (size_t)Nb, sizeof(wj_t), cmp_wj);
   double tau = 1.0 - (double)thr;
-  double c = 0.0;
+  double run = 0.0;
   for (int k = 0; k < Nb; ++k) {
-    c += (double)scratch[k].p;
+    run += (double)scratch[k].w;
+    double c = run / Z;
     int j = scratch[k].j;
     cum[j] = c;
     keep[j] = (uint8_t)((thr >= 1.0f) || (c > tau) || (k == Nb - 1));
   }
-  if (band) {
-    int a = 0;
-    while (a < Nb) {
-      int b = a;
-      while (b + 1 < Nb && (double)scratch[b + 1].p <= (double)scratch[b].p * (1.0 + ORACLE_TIE_REL)) ++b;
-      double ca = cum[scratch[a].j], cb = cum[scratch[b].j];
-      int flag;
-      if (b == Nb - 1) {
-        flag = b > a; /* the run holding the forced arg-max */
-      } else {
-        int near = 0;
-        for (int k = a; k <= b; ++k) near |= fabs(cum[scratch[k].j] - tau) < band_width;
-        flag = (ca <= tau && cb > tau) || near;
-      }
-      for (int k = a; k <= b; ++k) band[scratch[k].j] = (uint8_t)flag;
-      a = b + 1;
-    }
-  }
+  if (band)
+    for (int j = 0; j < Nb; ++j) band[j] = (uint8_t)(fabs(cum[j] - tau) < band_width);
   return scratch[Nb - 1].j; /* the arg-max block */
 }
 
@@ -246,7 +235,7 @@ static int sta_keep(int i, int j, int nbh, int nbw, int st, int sh, int sw) {
 /*   kv_count[b,hd,i]   number of kept key blocks                            */
 /*   kv_idx[b,hd,i,:]   kept key-block indices ascending (row stride Nb)      */
 /* status (optional, [B,Hh,Nb,Nb] uint8): bit0 = kept, bit1 = band block     */
-/* (decided by the CDF alone and within the band, see cdf_keep_row).         */
+/* (decided by the CDF alone, cumulative mass within `band` of 1 - thr).     */
 /* probs (optional, [B,Hh,Nb,Nb] fp32): the row probabilities p.             */
 /* qbar/kbar: fp32 [B][Hh][Nb][D].  Rows are independent; OpenMP splits them */
 /* without changing any element's arithmetic.                                */
@@ -257,19 +246,21 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
   int64_t rows = (int64_t)B * Hh * Nb;
 #pragma omp parallel
   {
-    float* p = (float*)malloc(sizeof(float) * (size_t)Nb);
+    float* e = (float*)malloc(sizeof(float) * (size_t)Nb);
     uint8_t* keep = (uint8_t*)malloc((size_t)Nb);
     uint8_t* bandf = (uint8_t*)malloc((size_t)Nb);
     double* cum = (double*)malloc(sizeof(double) * (size_t)Nb);
-    pj_t* scratch = (pj_t*)malloc(sizeof(pj_t) * (size_t)Nb);
+    wj_t* scratch = (wj_t*)malloc(sizeof(wj_t) * (size_t)Nb);
 #pragma omp for schedule(dynamic, 4)
     for (int64_t row = 0; row < rows; ++row) {
       int64_t bh = row / Nb;
       int i = (int)(row % Nb);
       const float* qi = qbar + (bh * Nb + i) * D;
       const float* kb = kbar + bh * Nb * D;
-      block_probs(qi, kb, Nb, D, scale, p);
-      int argmax = cdf_keep_row(p, Nb, thr, keep, cum, status ? bandf : NULL, band, scratch);
+      block_numerators(qi, kb, Nb, D, scale, e);
+      double Z = 0.0;
+      for (int j = 0; j < Nb; ++j) Z += (double)e[j];
+      int argmax = cdf_keep_row(e, Nb, thr, keep, cum, status ? bandf : NULL, band, scratch);
       int32_t n = 0;
       for (int j = 0; j < Nb; ++j) {
         int cdf_kept = keep[j];
@@ -278,16 +269,15 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
         if (kept) kv_idx[row * Nb + n++] = j;
         if (status) {
           /* A block is "band" only when the CDF comparison alone decides it. */
-          int forced = sta || thr >= 1.0f;
-          /* the arg-max is forced unless rounding-tied (then bandf marks it) */
+          int forced = sta || thr >= 1.0f || j == argmax;
           int in_band = !forced && bandf[j];
           status[row * Nb + j] = (uint8_t)(kept | (in_band << 1));
         }
-        if (probs) probs[row * Nb + j] = p[j];
+        if (probs) probs[row * Nb + j] = (float)((double)e[j] / Z);
       }
       kv_count[row] = n;
     }
-    free(p);
+    free(e);
     free(keep);
     free(bandf);
     free(cum);
@@ -377,11 +367,17 @@ void oracle_block_probs_row(const float* qbar, const float* kbar, int Nb, int D,
   block_probs(qbar + (int64_t)i * D, kbar, Nb, D, scale, p_out);
 }
 
-/* CDF keep decision for one probability row (see cdf_keep_row). */
-int oracle_cdf_keep(const float* p, int Nb, float thr, uint8_t* keep, double* cum, uint8_t* band,
+/* Softmax numerators e of one (b, head, i) row (see block_numerators). */
+void oracle_block_numerators_row(const float* qbar, const float* kbar, int Nb, int D, float scale,
+                                 int i, float* e_out) {
+  block_numerators(qbar + (int64_t)i * D, kbar, Nb, D, scale, e_out);
+}
+
+/* CDF keep decision for one row of weights (see cdf_keep_row). */
+int oracle_cdf_keep(const float* w, int Nb, float thr, uint8_t* keep, double* cum, uint8_t* band,
                     double band_width) {
-  pj_t* scratch = (pj_t*)malloc(sizeof(pj_t) * (size_t)Nb);
-  int argmax = cdf_keep_row(p, Nb, thr, keep, cum, band, band_width, scratch);
+  wj_t* scratch = (wj_t*)malloc(sizeof(wj_t) * (size_t)Nb);
+  int argmax = cdf_keep_row(w, Nb, thr, keep, cum, band, band_width, scratch);
   free(scratch);
   return argmax;
 }

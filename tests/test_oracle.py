@@ -168,15 +168,17 @@ def test_uniform_worked_case(oracle_lib, thr, kept):
         assert idx[0, 0, i, : cnt[0, 0, i]].tolist() == kept
 
 
-def exact_top_p(p: np.ndarray, thr: float):
-    """Nucleus selection in exact rational arithmetic: the smallest set of the
-    highest-probability blocks (ties: higher index first) whose complement has
-    mass <= 1 - thr; the arg-max always belongs to it."""
-    n = p.shape[0]
-    order = sorted(range(n), key=lambda j: (float(p[j]), j), reverse=True)
-    fr = [Fraction(float(p[j])) for j in order]
-    tau = Fraction(1) - Fraction(float(np.float32(thr)))
-    rest = sum(fr)
+def exact_top_p(w: np.ndarray, thr: float):
+    """Nucleus selection in exact rational arithmetic on a row of weights w
+    (probabilities up to a common factor): the smallest set of the largest
+    weights (ties: higher index first) whose complement holds at most 1 - thr
+    of the total; the arg-max always belongs to it."""
+    n = w.shape[0]
+    order = sorted(range(n), key=lambda j: (float(w[j]), j), reverse=True)
+    fr = [Fraction(float(w[j])) for j in order]
+    total = sum(fr)
+    tau = (Fraction(1) - Fraction(float(np.float32(thr)))) * total
+    rest = total
     kept = set()
     if thr >= 1.0:
         return set(range(n))
@@ -190,16 +192,38 @@ def exact_top_p(p: np.ndarray, thr: float):
 
 @pytest.mark.parametrize("thr", [0.3, 0.5, 0.7, 0.9, 0.95, 0.99])
 def test_cdf_rule_equals_exact_top_p(oracle_lib, thr):
+    """The oracle's CDF rule on the softmax numerators of real rows equals
+    exact top-p selection; rows whose cumulative mass comes within 1e-12 of
+    the threshold (where fp64 rounding could decide) are skipped."""
     w = inputs.Workload("pin", 1, 3, 64, 4, 16, 24, 1.0, thr, seed=21)
     q, k, _ = inputs.make_qkv(w)
     qbar = oracle_lib.pool(oracle_lib.flatten(q, w.T, w.H, w.W).reshape(q.shape))
     kbar = oracle_lib.pool(oracle_lib.flatten(k, w.T, w.H, w.W).reshape(k.shape))
+    checked = 0
     for hd in range(w.Hh):
         for i in range(w.Nb):
+            e = oracle_lib.block_numerators_row(qbar[0, hd], kbar[0, hd], i, w.scale)
+            keep, cum, band, argmax = oracle_lib.cdf_keep(e, thr)
+            if np.any(np.abs(cum - (1.0 - float(np.float32(thr)))) < 1e-12):
+                continue
+            assert set(np.nonzero(keep)[0].tolist()) == exact_top_p(e, thr)
+            assert keep[int(np.argmax(e))]
+            checked += 1
+    assert checked >= w.Hh * w.Nb - 2
+
+
+def test_numerators_are_the_unnormalised_probabilities(oracle_lib, tiny_flat):
+    """e_j = exp(s_j - max s) with the maximum exactly 1, and e / sum(e)
+    rounded to fp32 is the probability row."""
+    w, _, (qf, kf, vf) = tiny_flat
+    qbar, kbar = oracle_lib.pool(qf), oracle_lib.pool(kf)
+    for hd in range(w.Hh):
+        for i in range(w.Nb):
+            e = oracle_lib.block_numerators_row(qbar[0, hd], kbar[0, hd], i, w.scale)
             p = oracle_lib.block_probs_row(qbar[0, hd], kbar[0, hd], i, w.scale)
-            keep, cum, band, argmax = oracle_lib.cdf_keep(p, thr)
-            assert set(np.nonzero(keep)[0].tolist()) == exact_top_p(p, thr)
-            assert keep[int(np.argmax(p))]
+            assert e.max() == np.float32(1.0) and np.all(e > 0)
+            Z = float(np.sum(e.astype(np.float64)))
+            assert np.array_equal((e.astype(np.float64) / Z).astype(np.float32), p)
 
 
 def test_mask_invariants_mass_and_minimality(oracle_lib):
@@ -214,12 +238,15 @@ def test_mask_invariants_mass_and_minimality(oracle_lib):
             assert np.all(np.diff(lst) > 0)
             p = probs[0, hd, i].astype(np.float64)
             kept_mass = math.fsum(p[lst])
-            assert kept_mass >= w.thr - 1e-12
+            # the rule runs on the exact quotients e / Z; p holds them
+            # rounded to fp32, each within 2^-24 relative
+            tol = 2.0 ** -23
+            assert kept_mass >= w.thr - tol
             # arg-max kept
             assert int(np.argmax(p)) in set(lst.tolist())
             # minimality: dropping the smallest kept block leaves less than thr
             if len(lst) > 1:
-                assert kept_mass - p[lst].min() < w.thr + 1e-12
+                assert kept_mass - p[lst].min() < w.thr + tol
             assert np.array_equal(np.nonzero(status[0, hd, i] & 1)[0], lst)
 
 
@@ -536,37 +563,41 @@ def test_generator_is_deterministic_and_shaped():
     assert len(idx) == 64 and len(set(idx.tolist())) == 64 and np.all(np.diff(idx) > 0)
 
 
-def test_band_marks_rounding_ties_straddling_the_threshold(oracle_lib):
-    """Band blocks: within 1e-5 of 1 - thr, or a run of probabilities equal to
-    within fp32 rounding whose positions straddle 1 - thr (their order, and so
-    which of them is kept, is set by rounding)."""
+def test_band_marks_only_blocks_near_the_threshold(oracle_lib):
+    """Band blocks are exactly those whose cumulative mass lies within 1e-5
+    of 1 - thr; probabilities one ulp apart are ordered by value (the larger
+    one is kept), not banded."""
     one_ulp_up = np.nextafter(np.float32(0.06), np.float32(1.0))
-    # ascending: 0.06 (c=0.06 <= 0.1), 0.06+ulp (c=0.12 > 0.1): a tied pair across the threshold
+    # ascending: 0.06 (c = 0.06 <= 0.1), then 0.06 + 1 ulp (c = 0.12 > 0.1)
     p = np.array([0.8, 0.06, one_ulp_up, 0.2], dtype=np.float32)
-    keep, cum, band, argmax = oracle_lib.cdf_keep(p, 0.9)
+    p = p / p.astype(np.float64).sum()  # weights: the rule normalises anyway
+    keep, cum, band, argmax = oracle_lib.cdf_keep(p.astype(np.float32), 0.9)
     assert keep.tolist() == [True, False, True, True]
-    assert band.tolist() == [False, True, True, False]
-    # same masses but clearly ordered: nothing is band
-    p2 = np.array([0.8, 0.06, 0.062, 0.2], dtype=np.float32)
-    keep2, _, band2, _ = oracle_lib.cdf_keep(p2, 0.9)
-    assert keep2.tolist() == [True, False, True, True] and not band2.any()
+    assert not band.any()
+    # the same with the two near-equal weights swapped between blocks
+    p_sw = np.array([0.8, one_ulp_up, 0.06, 0.2], dtype=np.float32)
+    keep_sw, _, band_sw, _ = oracle_lib.cdf_keep(p_sw, 0.9)
+    assert keep_sw.tolist() == [True, True, False, True] and not band_sw.any()
+    # exactly equal weights across the threshold: the higher index is kept
+    p_eq = np.array([0.8, 0.06, 0.06, 0.2], dtype=np.float32)
+    keep_eq, _, band_eq, _ = oracle_lib.cdf_keep(p_eq, 0.9)
+    assert keep_eq.tolist() == [True, False, True, True] and not band_eq.any()
     # a block whose cumulative mass sits 5e-6 above the threshold
     tau = 1.0 - float(np.float32(0.9))
-    p3 = np.array([0.7, np.float32(tau + 5e-6), 0.3], dtype=np.float32)
+    p3 = np.array([0.6, np.float32(tau + 5e-6), 0.3 - 5e-6], dtype=np.float32)  # sums to 1
     keep3, cum3, band3, _ = oracle_lib.cdf_keep(p3, 0.9)
     assert keep3.tolist() == [True, True, True]
     assert band3.tolist() == [False, True, False]
 
 
-def test_band_marks_a_rounding_tied_arg_max(oracle_lib):
+def test_arg_max_of_near_equal_maxima_is_the_larger(oracle_lib):
     top = np.float32(0.4)
-    p = np.array([0.2, top, np.nextafter(top, np.float32(1.0)), 0.0001], dtype=np.float32)
+    p = np.array([0.2, np.nextafter(top, np.float32(1.0)), top, 0.0001], dtype=np.float32)
     keep, cum, band, argmax = oracle_lib.cdf_keep(p, 0.0)  # thr 0: only the arg-max is kept
-    assert argmax == 2 and keep.tolist() == [False, False, True, False]
-    assert band.tolist() == [False, True, True, False]
-    p2 = np.array([0.2, 0.39, 0.41, 0.0001], dtype=np.float32)  # clear arg-max: nothing band
-    _, _, band2, _ = oracle_lib.cdf_keep(p2, 0.0)
-    assert not band2.any()
+    assert argmax == 1 and keep.tolist() == [False, True, False, False]
+    p2 = np.array([0.2, top, top, 0.0001], dtype=np.float32)  # exact tie: the higher index
+    _, _, _, argmax2 = oracle_lib.cdf_keep(p2, 0.0)
+    assert argmax2 == 2
 
 
 def test_parity_helper_flat_order_matches_oracle_flatten(oracle_lib):

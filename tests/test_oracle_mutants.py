@@ -61,8 +61,11 @@ MUTANTS = [
     ("CDF keeps c >= 1 - thr", "(c > tau)", "(c >= tau)", ["uniform_golden"]),
     ("tie order reversed", "return (x->j > y->j) - (x->j < y->j);", "return (x->j < y->j) - (x->j > y->j);",
      ["uniform_golden"]),
-    ("CDF accumulates descending", "c += (double)scratch[k].p;", "c += (double)scratch[Nb - 1 - k].p;",
+    ("CDF accumulates descending", "run += (double)scratch[k].w;", "run += (double)scratch[Nb - 1 - k].w;",
      ["uniform_golden", "top_p"]),
+    ("CDF not normalised", "double c = run / Z;", "double c = run;", ["uniform_golden", "top_p"]),
+    ("CDF orders blocks by index only", "if (x->w < y->w) return -1;\n  if (x->w > y->w) return 1;\n", "",
+     ["top_p", "uniform_golden"]),
     ("arg-max not forced", " || (k == Nb - 1));", ");", ["thr_extremes"]),
     ("STA window exclusive", "abs(ti - tj) <= st / 2", "abs(ti - tj) < st / 2", ["sta_counts"]),
     ("STA lists skip the query block",
