@@ -52,7 +52,7 @@ def _load():
         lib.oracle_flatten.argtypes = [P, P, i, i, i, i, i, i64]
         lib.oracle_unflatten.argtypes = [P, P, i, i, i, i, i, i64]
         lib.oracle_pool.argtypes = [P, P, i, i, i, i]
-        lib.oracle_mask.argtypes = [P, P, i, i, i, i, f, f, i, i, i, i, i, d, P, P, P, P]
+        lib.oracle_mask.argtypes = [P, P, i, i, i, i, f, f, i, i, i, i, i, i, d, P, P, P, P]
         lib.oracle_attention.argtypes = [P, P, P, P, P, i, i, i, i, d, P, i, P, P]
         lib.oracle_block_probs_row.argtypes = [P, P, i, i, f, i, P]
         lib.oracle_block_numerators_row.argtypes = [P, P, i, i, f, i, P]
@@ -61,6 +61,9 @@ def _load():
         lib.oracle_sta.argtypes = [i, i, i, i, i, i, i]
         lib.oracle_sta.restype = i
         lib.oracle_sta_lists.argtypes = [i, i, i, i, i, i, P, P]
+        lib.oracle_radial_lists.argtypes = [i, i, i, i, P, P]
+        lib.oracle_radial.argtypes = [i, i, i, i, i]
+        lib.oracle_radial.restype = i
         lib.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, P, P]
         lib.oracle_attention_bwd_sampled.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, i, P, i, P, P, P]
         lib.oracle_num_threads.restype = i
@@ -162,10 +165,26 @@ def sta_lists(nbt: int, nbh: int, nbw: int, window=(3, 3, 3)):
     return kv_count, kv_idx
 
 
+def radial(i: int, j: int, nbh: int, nbw: int, r0: int) -> bool:
+    return bool(_load().oracle_radial(i, j, nbh, nbw, r0))
+
+
+def radial_lists(nbt: int, nbh: int, nbw: int, r0: int):
+    """The radial window alone as block lists for one (b, head): kv_count
+    int32 [Nb], kv_idx int32 [Nb, Nb] (ascending, -1 past the count)."""
+    Nb = nbt * nbh * nbw
+    kv_count = np.zeros(Nb, dtype=np.int32)
+    kv_idx = np.full((Nb, Nb), -1, dtype=np.int32)
+    _load().oracle_radial_lists(Nb, nbh, nbw, int(r0), _ptr(kv_count), _ptr(kv_idx))
+    return kv_count, kv_idx
+
+
 def build_mask(qbar: np.ndarray, kbar: np.ndarray, thr: float, scale: float, nbh: int, nbw: int,
                sta_window=(0, 0, 0), band: float = BAND, want_status: bool = True,
-               want_probs: bool = False):
-    """Masks for every row.  Returns (kv_count, kv_idx, status, probs).
+               want_probs: bool = False, radial_r0: int = 0):
+    """Masks for every row, the adaptive mask OR-ed with the sliding-tile
+    window (sta_window) and the radial window (radial_r0 > 0).  Returns
+    (kv_count, kv_idx, status, probs).
 
     kv_count int32 [B,Hh,Nb]; kv_idx int32 [B,Hh,Nb,Nb] (ascending, padded
     with -1 past the count); status uint8 [B,Hh,Nb,Nb] (bit0 kept, bit1 band)
@@ -179,7 +198,7 @@ def build_mask(qbar: np.ndarray, kbar: np.ndarray, thr: float, scale: float, nbh
     status = np.zeros((B, Hh, Nb, Nb), dtype=np.uint8) if want_status else None
     probs = np.zeros((B, Hh, Nb, Nb), dtype=np.float32) if want_probs else None
     _load().oracle_mask(_ptr(qbar), _ptr(kbar), B, Hh, Nb, D, scale, thr, nbh, nbw,
-                        int(sta_window[0]), int(sta_window[1]), int(sta_window[2]), band,
+                        int(sta_window[0]), int(sta_window[1]), int(sta_window[2]), int(radial_r0), band,
                         _ptr(kv_count), _ptr(kv_idx),
                         _ptr(status) if status is not None else None,
                         _ptr(probs) if probs is not None else None)

@@ -15,6 +15,8 @@
  *           "Limiarizacao CDF"                                 -> cdf_keep_row
  *           "Expansao"                                         -> kv lists
  *   item 3  "Integracao Hibrida com STA", M = M_nabla OR M_STA -> sta_keep
+ * The Radial Attention article's static decay mask as another OR-term
+ * (aisight.pl, "Zastosowanie zasad rozkladu energii")       -> radial_keep
  * and the attention on the kept N x N blocks (same section, "Expansao"),
  * with dropped blocks absent from both numerator and normaliser (the
  * AB-Attention news page, section "Onde os esquemas esparsos anteriores
@@ -230,8 +232,56 @@ static int sta_keep(int i, int j, int nbh, int nbw, int st, int sh, int sw) {
 }
 
 /* ------------------------------------------------------------------------ */
+/* Radial window in block space (Radial Attention article, aisight.pl,       */
+/* "Radial Attention: Efektywnosc bez kompromisow" and "Zastosowanie zasad   */
+/* rozkladu energii": a static mask that keeps interactions mostly within    */
+/* the spatiotemporal neighbourhood, its window shrinking as the temporal    */
+/* distance grows, the kept attention decaying exponentially in space and   */
+/* time).  The page gives no formula; the reading here: blocks              */
+/* i=(ti,hi,wi) and j=(tj,hj,wj) at temporal distance dt = |ti - tj| fall in */
+/* band r = floor(log2(dt + 1)) (dt 0; 1-2; 3-6; 7-14; ...), whose spatial   */
+/* half-width is rho = floor(r0 / 2^r): the window halves each time the     */
+/* temporal distance doubles.  keep iff |hi - hj| <= rho and                 */
+/* |wi - wj| <= rho (the co-located block of every frame is always kept).    */
+/* r0 <= 0 disables the window.                                              */
+/* Pinned by: the closed-form per-row count (sum over frames of the clipped */
+/* box areas), an enumeration of the window written independently with     */
+/* floating-point log2, symmetry, and monotone shrinking in dt.             */
+/* ------------------------------------------------------------------------ */
+static int radial_band(int dt) {
+  int r = 0;
+  while ((dt + 1) >> (r + 1)) ++r;
+  return r;
+}
+
+static int radial_keep(int i, int j, int nbh, int nbw, int r0) {
+  if (r0 <= 0) return 0;
+  int per_t = nbh * nbw;
+  int ti = i / per_t, hi = (i % per_t) / nbw, wi = i % nbw;
+  int tj = j / per_t, hj = (j % per_t) / nbw, wj = j % nbw;
+  int rho = r0 >> radial_band(abs(ti - tj));
+  return abs(hi - hj) <= rho && abs(wi - wj) <= rho;
+}
+
+/* The radial window on its own as block lists for one (b, head), as        */
+/* oracle_sta_lists does for the sliding-tile window.                        */
+void oracle_radial_lists(int Nb, int nbh, int nbw, int r0, int32_t* kv_count, int32_t* kv_idx) {
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int i = 0; i < Nb; ++i) {
+    int n = 0;
+    for (int j = 0; j < Nb; ++j)
+      if (radial_keep(i, j, nbh, nbw, r0)) kv_idx[(int64_t)i * Nb + n++] = j;
+    kv_count[i] = n;
+  }
+}
+
+/* Radial predicate for one block pair (see radial_keep). */
+int oracle_radial(int i, int j, int nbh, int nbw, int r0) { return radial_keep(i, j, nbh, nbw, r0); }
+
+/* ------------------------------------------------------------------------ */
 /* Full mask construction for every (b, head, query block) row, producing    */
-/* the block-CSR lists consumed by the attention ("Expansao"):               */
+/* the block-CSR lists consumed by the attention ("Expansao"), with the     */
+/* static windows (sliding tile, radial) OR-ed into the adaptive mask:      */
 /*   kv_count[b,hd,i]   number of kept key blocks                            */
 /*   kv_idx[b,hd,i,:]   kept key-block indices ascending (row stride Nb)      */
 /* status (optional, [B,Hh,Nb,Nb] uint8): bit0 = kept, bit1 = band block     */
@@ -241,7 +291,7 @@ static int sta_keep(int i, int j, int nbh, int nbw, int st, int sh, int sw) {
 /* without changing any element's arithmetic.                                */
 /* ------------------------------------------------------------------------ */
 void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, int D, float scale,
-                 float thr, int nbh, int nbw, int sta_t, int sta_h, int sta_w, double band,
+                 float thr, int nbh, int nbw, int sta_t, int sta_h, int sta_w, int radial_r0, double band,
                  int32_t* kv_count, int32_t* kv_idx, uint8_t* status, float* probs) {
   int64_t rows = (int64_t)B * Hh * Nb;
 #pragma omp parallel
@@ -264,7 +314,7 @@ void oracle_mask(const float* qbar, const float* kbar, int B, int Hh, int Nb, in
       int32_t n = 0;
       for (int j = 0; j < Nb; ++j) {
         int cdf_kept = keep[j];
-        int sta = sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w);
+        int sta = sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w) || radial_keep(i, j, nbh, nbw, radial_r0);
         int kept = cdf_kept || sta;
         if (kept) kv_idx[row * Nb + n++] = j;
         if (status) {

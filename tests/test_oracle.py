@@ -552,6 +552,88 @@ def test_attention_bwd_invariants(oracle_lib):
     assert not np.any(dq[:, 4 * 64:5 * 64])
 
 
+# ----------------------------------------------------------------------------
+# Radial window (Radial Attention article, "Zastosowanie zasad rozkladu
+# energii"): half-width floor(r0 / 2^floor(log2(dt + 1))) at temporal
+# distance dt
+# ----------------------------------------------------------------------------
+def radial_rho(dt: int, r0: int) -> int:
+    """Restated with floating-point log2 (independent of the oracle's bit loop)."""
+    return int(r0 // (2 ** math.floor(math.log2(dt + 1))))
+
+
+def radial_enumerate(nbt, nbh, nbw, r0):
+    """Row lists by walking each frame's clipped box in (frame, row, column)
+    order, which is ascending flattened order."""
+    per_t = nbh * nbw
+    rows = []
+    for i in range(nbt * per_t):
+        ti, hi, wi = i // per_t, (i % per_t) // nbw, i % nbw
+        out = []
+        for tj in range(nbt):
+            rho = radial_rho(abs(ti - tj), r0)
+            for hj in range(max(0, hi - rho), min(nbh - 1, hi + rho) + 1):
+                for wj in range(max(0, wi - rho), min(nbw - 1, wi + rho) + 1):
+                    out.append((tj * nbh + hj) * nbw + wj)
+        rows.append(out)
+    return rows
+
+
+RADIAL_GRIDS = [(16, 6, 10, 4), (9, 3, 5, 1), (20, 2, 2, 7), (4, 6, 10, 100), (1, 1, 1, 1), (33, 6, 10, 2)]
+
+
+@pytest.mark.parametrize("nbt,nbh,nbw,r0", RADIAL_GRIDS)
+def test_radial_lists_equal_enumeration_and_closed_form(oracle_lib, nbt, nbh, nbw, r0):
+    cnt, idx = oracle_lib.radial_lists(nbt, nbh, nbw, r0)
+    ref = radial_enumerate(nbt, nbh, nbw, r0)
+    per_t = nbh * nbw
+    for i, lst in enumerate(ref):
+        assert idx[i, : cnt[i]].tolist() == lst
+        ti, hi, wi = i // per_t, (i % per_t) // nbw, i % nbw
+        closed = sum((min(hi + radial_rho(abs(ti - tj), r0), nbh - 1) - max(hi - radial_rho(abs(ti - tj), r0), 0) + 1) *
+                     (min(wi + radial_rho(abs(ti - tj), r0), nbw - 1) - max(wi - radial_rho(abs(ti - tj), r0), 0) + 1)
+                     for tj in range(nbt))
+        assert cnt[i] == closed
+
+
+def test_radial_symmetric_and_shrinking(oracle_lib):
+    nbt, nbh, nbw, r0 = 12, 6, 10, 5
+    per_t = nbh * nbw
+    Nb = nbt * per_t
+    rng = np.random.default_rng(17)
+    for _ in range(3000):
+        i, j = (int(x) for x in rng.integers(0, Nb, size=2))
+        assert oracle_lib.radial(i, j, nbh, nbw, r0) == oracle_lib.radial(j, i, nbh, nbw, r0)
+    # a spatial offset kept at temporal distance dt is kept at every smaller one
+    i = 5 * per_t + 2 * nbw + 4
+    for dh in range(-3, 4):
+        for dw in range(-5, 6):
+            kept = [oracle_lib.radial(i, tj * per_t + (2 + dh) * nbw + 4 + dw, nbh, nbw, r0)
+                    for tj in range(5, nbt) if 0 <= 2 + dh < nbh and 0 <= 4 + dw < nbw]
+            assert kept == sorted(kept, reverse=True)
+    # co-located blocks of every frame are kept; nothing is kept when off
+    assert all(oracle_lib.radial(i, tj * per_t + 2 * nbw + 4, nbh, nbw, r0) for tj in range(nbt))
+    assert not any(oracle_lib.radial(i, j, nbh, nbw, 0) for j in range(Nb))
+
+
+def test_radial_union_is_superset(oracle_lib):
+    w = inputs.Workload("pin", 1, 2, 64, 8, 16, 24, 1.0, 0.7, seed=19)
+    q, k, _ = inputs.make_qkv(w)
+    qbar = oracle_lib.pool(oracle_lib.flatten(q, w.T, w.H, w.W).reshape(q.shape))
+    kbar = oracle_lib.pool(oracle_lib.flatten(k, w.T, w.H, w.W).reshape(k.shape))
+    cnt_a, idx_a, _, _ = oracle_lib.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw)
+    cnt_u, idx_u, status, _ = oracle_lib.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, radial_r0=2)
+    cnt_r, idx_r = oracle_lib.radial_lists(w.T, w.nbh, w.nbw, 2)
+    for hd in range(w.Hh):
+        for i in range(w.Nb):
+            u = set(idx_u[0, hd, i, : cnt_u[0, hd, i]].tolist())
+            a = set(idx_a[0, hd, i, : cnt_a[0, hd, i]].tolist())
+            r = set(idx_r[i, : cnt_r[i]].tolist())
+            assert u == a | r
+            # window blocks are forced, never band
+            assert not any(status[0, hd, i, j] & 2 for j in r)
+
+
 def test_generator_is_deterministic_and_shaped():
     w = inputs.Workload("g", 1, 2, 64, 2, 8, 16, 1.0, 0.9, seed=3)
     a = inputs.make_qkv(w)

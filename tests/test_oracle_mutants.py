@@ -41,6 +41,9 @@ PINS = {
     "sta_counts": lambda m: [pins.test_sta_closed_form_counts(m, *r) for r in pins.read_sta_counts()],
     "sta_lists": lambda m: (pins.test_sta_lists_degenerate_windows(m),
                             [pins.test_sta_lists_other_windows(m, wnd) for wnd in [(1, 3, 5), (7, 7, 7)]]),
+    "radial_lists": lambda m: [pins.test_radial_lists_equal_enumeration_and_closed_form(m, *g)
+                               for g in pins.RADIAL_GRIDS[:3]],
+    "radial_union": lambda m: pins.test_radial_union_is_superset(m),
     "dense_attention": lambda m: pins.test_thr_one_equals_dense_attention(m, tiny_flat(m)),
     "attention_special": lambda m: pins.test_attention_special_cases(m),
     "bwd_autograd": lambda m: [pins.test_attention_bwd_equals_autograd(m, *a) for a in [(64, 0.5, ()), (128, 0.3, (2,))]],
@@ -71,6 +74,12 @@ MUTANTS = [
     ("STA lists skip the query block",
      "if (sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w)) kv_idx",
      "if (j != i && sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w)) kv_idx", ["sta_lists"]),
+    ("radial bands one frame late", "while ((dt + 1) >> (r + 1)) ++r;", "while (dt >> (r + 1)) ++r;",
+     ["radial_lists"]),
+    ("radial window never shrinks", "int rho = r0 >> radial_band(abs(ti - tj));", "int rho = r0;", ["radial_lists"]),
+    ("radial window left out of the union",
+     "sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w) || radial_keep(i, j, nbh, nbw, radial_r0);",
+     "sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w);", ["radial_union"]),
     ("attention scale dropped", "double l = dot * scale;", "double l = dot;", ["dense_attention"]),
     ("attention normaliser dropped", "o[d] = cnt > 0 ? acc[d] / den : 0.0;", "o[d] = cnt > 0 ? acc[d] : 0.0;",
      ["attention_special", "dense_attention"]),
