@@ -41,9 +41,11 @@ class Workload:
     sta: tuple = (0, 0, 0)
     seed: int = 0
     P: int = 8
-    # "nabla": the adaptive mask (OR the window when sta is set); "sta": the
-    # static window alone (thr unused)
+    # "nabla": the adaptive mask (OR the sliding-tile window when sta is set,
+    # OR the radial window when radial > 0); "sta" / "radial": that static
+    # window alone (thr unused)
     mask: str = "nabla"
+    radial: int = 0  # radial window half-width at temporal distance 0 (0: off)
 
     @property
     def S(self) -> int:
@@ -75,6 +77,13 @@ HUNYUAN = Workload("HunyuanVideo-like: B1 Hh24 D128 grid 32x48x80, thr 0.9 OR ST
 # the method is compared with.
 HUNYUAN_STA = Workload("HunyuanVideo-like, static STA 3x3x3 only: B1 Hh24 D128 grid 32x48x80", 1, 24, 128, 32, 48,
                        80, 1.0, 1.0, sta=(3, 3, 3), seed=3, mask="sta")
+# The HunyuanVideo-like layer with the radial decay window (half-width 2
+# patches at temporal distance 0, halving per doubling of the distance) as
+# the OR-term, and the long-video layer under that window alone.
+HUNYUAN_RADIAL = Workload("HunyuanVideo-like: B1 Hh24 D128 grid 32x48x80, thr 0.9 OR radial window r0=2", 1, 24, 128,
+                          32, 48, 80, 1.0, 0.9, seed=3, radial=2)
+LONG_RADIAL = Workload("long video, static radial window r0=2 only: B1 Hh24 D128 grid 64x48x80", 1, 24, 128, 64, 48,
+                       80, 1.0, 1.0, seed=5, mask="radial", radial=2)
 LONG = Workload("long video: B1 Hh24 D128 grid 64x48x80, thr 0.9 OR STA 3x3x3", 1, 24, 128, 64, 48, 80, 1.0, 0.9,
                 sta=(3, 3, 3), seed=5)
 
@@ -127,3 +136,45 @@ def sample_query_blocks(Nb: int, n: int = 64, seed: int = 1234):
 def randn_bf16(shape, seed: int):
     g = torch.Generator().manual_seed(seed)
     return torch.randn(shape, generator=g).to(torch.bfloat16)
+
+
+# ------------------------------------------------------------- AB-Attention
+@dataclass(frozen=True)
+class ABWorkload:
+    """A layer under the AB-Attention scheme: the Q, K, V recipe of
+    `base` (grid order, not permuted), 128-token query blocks, 8 clusters,
+    4-token key blocks, `kmeans_iters` Lloyd iterations, and an expected
+    sample of `budget_frac` of the key blocks per query block."""
+    name: str
+    base: Workload
+    budget_frac: float
+    kmeans_iters: int = 4
+    seed_u: int = 77
+
+    @property
+    def nqb(self) -> int:
+        return self.base.S // 128
+
+    @property
+    def nkb(self) -> int:
+        return self.base.S // 4
+
+    @property
+    def budget(self) -> float:
+        return float(math.ceil(self.budget_frac * self.nkb))
+
+
+def ab_uniforms(w: ABWorkload) -> torch.Tensor:
+    """The sampling's uniform random numbers in [0, 1), one per (batch, head,
+    query block, key block): fp32 [B, Hh, NQB, NKB], seeded."""
+    g = torch.Generator().manual_seed(w.seed_u)
+    return torch.rand((w.base.B, w.base.Hh, w.nqb, w.nkb), generator=g)
+
+
+# The AB-Attention workloads: the Wan-1.3B-like layer with 10% of the key
+# blocks sampled in expectation (the page reports 89-92% of the attention
+# skipped), and a small one the oracle finishes in seconds.
+AB_TINY = ABWorkload("AB tiny: B1 Hh2 D64 grid 4x16x32 (2048 tokens), 10% sampled",
+                     Workload("ab-tiny", 1, 2, 64, 4, 16, 32, 1.0, 1.0, seed=61), 0.10)
+AB_WAN13B = ABWorkload("AB Wan-1.3B-like: B1 Hh12 D128 grid 16x48x80, 10% sampled",
+                       Workload("ab-wan", 1, 12, 128, 16, 48, 80, 1.0, 1.0, seed=2), 0.10)

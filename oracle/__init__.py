@@ -67,6 +67,13 @@ def _load():
         lib.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, P, P]
         lib.oracle_attention_bwd_sampled.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, i, P, i, P, P, P]
         lib.oracle_num_threads.restype = i
+        lib.oracle_ab_key_means.argtypes = [P, i, i, i, i, P]
+        lib.oracle_ab_kmeans.argtypes = [P, i, i, i, i, i, P, P, P]
+        lib.oracle_ab_scores.argtypes = [P, P, P, i, i, i, i, i, f, P]
+        lib.oracle_ab_inclusion.argtypes = [P, i, d, P]
+        lib.oracle_ab_inclusion.restype = d
+        lib.oracle_ab_inclusion_all.argtypes = [P, i64, i, d, P]
+        lib.oracle_ab_attention.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, i, P, P]
         _lib = lib
     return _lib
 
@@ -270,3 +277,106 @@ def attention_bwd_sampled(qf, kf, vf, dof, kv_count: np.ndarray, kv_idx: np.ndar
                                          B, S, Hh, D, scale, _ptr(qblocks), nq, _ptr(kblocks), nk,
                                          _ptr(dq), _ptr(dk), _ptr(dv))
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- AB-Attention
+AB_QBLOCK = 128
+AB_CLUSTERS = 8
+AB_KBLOCK = 4
+
+
+def ab_key_means(k) -> np.ndarray:
+    """Mean key of every 4-token block (grid order): fp32 [B, Hh, S/4, D]."""
+    k = _bits(k)
+    B, S, Hh, D = k.shape
+    out = np.empty((B, Hh, S // AB_KBLOCK, D), dtype=np.float32)
+    _load().oracle_ab_key_means(_ptr(k), B, S, Hh, D, _ptr(out))
+    return out
+
+
+def ab_kmeans(q, iters: int = 4):
+    """IBCS clustering of every 128-query block: (centroids fp32 [B, Hh, NQB,
+    8, D], counts int32 [B, Hh, NQB, 8], assignment int32 [B, Hh, S])."""
+    q = _bits(q)
+    B, S, Hh, D = q.shape
+    nqb = S // AB_QBLOCK
+    cent = np.empty((B, Hh, nqb, AB_CLUSTERS, D), dtype=np.float32)
+    counts = np.empty((B, Hh, nqb, AB_CLUSTERS), dtype=np.int32)
+    assign = np.empty((B, Hh, S), dtype=np.int32)
+    _load().oracle_ab_kmeans(_ptr(q), B, S, Hh, D, iters, _ptr(cent), _ptr(counts), _ptr(assign))
+    return cent, counts, assign
+
+
+def ab_scores(cent: np.ndarray, counts: np.ndarray, kbar: np.ndarray, scale: float) -> np.ndarray:
+    """IBCS block scores, fp64 [B, Hh, NQB, NKB]."""
+    cent = np.ascontiguousarray(cent, dtype=np.float32)
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    kbar = np.ascontiguousarray(kbar, dtype=np.float32)
+    B, Hh, nqb, _, D = cent.shape
+    nkb = kbar.shape[2]
+    out = np.empty((B, Hh, nqb, nkb), dtype=np.float64)
+    _load().oracle_ab_scores(_ptr(cent), _ptr(counts), _ptr(kbar), B, Hh, nqb, nkb, D, scale, _ptr(out))
+    return out
+
+
+def ab_inclusion(score: np.ndarray, budget: float) -> np.ndarray:
+    """SIP inclusion probabilities (fp64) for every row of scores (last axis)."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    pi = np.empty_like(score)
+    n = score.shape[-1]
+    _load().oracle_ab_inclusion_all(_ptr(score), score.size // n, n, float(budget), _ptr(pi))
+    return pi
+
+
+def ab_inclusion_row(score: np.ndarray, budget: float):
+    """(pi, lambda) for one row."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    pi = np.empty_like(score)
+    lam = _load().oracle_ab_inclusion(_ptr(score), score.shape[0], float(budget), _ptr(pi))
+    return pi, lam
+
+
+def ab_sample(pi: np.ndarray, u: np.ndarray):
+    """Poisson sampling: block J of a row is in the sample iff u_J < pi_J.
+    Returns (count int32 [...], idx int32 [..., NKB] ascending and -1 past the
+    count, shift fp64 [..., NKB] = -log(pi) of each listed block)."""
+    inc = u.astype(np.float64) < pi
+    n = pi.shape[-1]
+    count = inc.sum(axis=-1).astype(np.int32)
+    idx = np.full(pi.shape, -1, dtype=np.int32)
+    shift = np.zeros(pi.shape, dtype=np.float64)
+    flat_inc = inc.reshape(-1, n)
+    flat_pi = pi.reshape(-1, n)
+    fi, fs = idx.reshape(-1, n), shift.reshape(-1, n)
+    for r in range(flat_inc.shape[0]):
+        js = np.nonzero(flat_inc[r])[0]
+        fi[r, :js.size] = js
+        fs[r, :js.size] = -np.log(flat_pi[r, js])
+    return count, idx, shift
+
+
+def ab_attention(q, k, v, kcount, kidx, shift, scale: float, qblocks=None):
+    """Attention of the listed 128-token query blocks over their sampled
+    4-token key blocks with the Horvitz-Thompson logit shifts (fp64).
+    kcount/kidx/shift either cover every query block or, when qblocks is
+    given, may already be restricted to them.  Returns (out fp64 [B,
+    nq*128, Hh, D], lse fp64 [B, Hh, nq*128])."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, S, Hh, D = q.shape
+    nqb, nkb = S // AB_QBLOCK, S // AB_KBLOCK
+    if qblocks is None:
+        qblocks = np.arange(nqb, dtype=np.int32)
+    qblocks = np.ascontiguousarray(qblocks, dtype=np.int32)
+    nq = qblocks.shape[0]
+    kcount, kidx, shift = np.asarray(kcount), np.asarray(kidx), np.asarray(shift)
+    if kcount.shape[-1] != nq:
+        kcount, kidx, shift = kcount[:, :, qblocks], kidx[:, :, qblocks], shift[:, :, qblocks]
+    kcount = np.ascontiguousarray(kcount, dtype=np.int32)
+    kidx = np.ascontiguousarray(kidx, dtype=np.int32)
+    shift = np.ascontiguousarray(shift, dtype=np.float64)
+    assert kidx.shape == (B, Hh, nq, nkb) and shift.shape == (B, Hh, nq, nkb)
+    out = np.zeros((B, nq * AB_QBLOCK, Hh, D), dtype=np.float64)
+    lse = np.zeros((B, Hh, nq * AB_QBLOCK), dtype=np.float64)
+    _load().oracle_ab_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(kcount), _ptr(kidx), _ptr(shift), B, S, Hh, D,
+                                scale, _ptr(qblocks), nq, _ptr(out), _ptr(lse))
+    return out, lse

@@ -661,3 +661,287 @@ void oracle_attention_bwd_sampled(const uint16_t* qf, const uint16_t* kf, const 
   free(qpos);
   free(kpos);
 }
+
+/* ======================================================================== */
+/* AB-Attention (news page "AB-Attention acelera a geracao de video em ate  */
+/* 2,23x e pula 92% da atencao", section "Os tres recursos do AB-Attention")*/
+/* as a second workload over the same token tensors, kept in their original */
+/* (grid) order: the page says the tokens are not permuted.                 */
+/*   IBCS: query blocks of 128 tokens, 8 clusters per block, each with a     */
+/*         centroid and a weight = its fraction of the block's queries; a   */
+/*         key block is scored by the weighted attention of the centroids   */
+/*         to its mean key.                                                 */
+/*   SIP:  a key block enters the sample with probability proportional to   */
+/*         its score, the most important ones always; a sampled block counts */
+/*         1 / (inclusion probability) times (Horvitz-Thompson), applied as  */
+/*         a logit shift of -log(pi).                                       */
+/*   Key blocks of 4 tokens, gathered by index.                             */
+/* Readings where the page is silent: k-means starts from the queries at    */
+/* positions 0, 16, ..., 112 of the block and runs `iters` Lloyd iterations  */
+/* (assignment to the nearest centroid by squared distance, ties to the      */
+/* lower cluster; each centroid becomes the mean of its queries, an empty   */
+/* cluster keeps its centroid); the weights come from the last assignment.  */
+/* The score softmax runs over all key blocks of the (b, head), scale       */
+/* 1/sqrt(D).  Inclusion probabilities pi = min(1, lambda * score) with      */
+/* lambda such that sum(pi) equals the sampling budget (the expected number  */
+/* of sampled blocks); a block is sampled iff u < pi for its uniform random */
+/* number u, drawn outside and passed in.                                   */
+/* ======================================================================== */
+#define AB_QBLOCK 128
+#define AB_CLUSTERS 8
+#define AB_KBLOCK 4
+
+/* Mean key of every 4-token block: kbar[b][hd][J][d] = (sum_{r<4} k[b][4J+r]
+ * [hd][d], fp32, r ascending) * 0.25.  k is bf16 [B][S][Hh][D], grid order.
+ * Pinned by: the fp64 block mean. */
+void oracle_ab_key_means(const uint16_t* k, int B, int S, int Hh, int D, float* kbar) {
+  int nkb = S / AB_KBLOCK;
+  for (int b = 0; b < B; ++b)
+    for (int hd = 0; hd < Hh; ++hd)
+      for (int J = 0; J < nkb; ++J)
+        for (int d = 0; d < D; ++d) {
+          float acc = 0.0f;
+          for (int r = 0; r < AB_KBLOCK; ++r)
+            acc = acc + bf16_bits_to_f32(k[(((int64_t)b * S + (int64_t)J * AB_KBLOCK + r) * Hh + hd) * D + d]);
+          kbar[(((int64_t)b * Hh + hd) * nkb + J) * D + d] = acc * 0.25f;
+        }
+}
+
+/* Squared distance, fp32: diff = x - mu rounded, then a fused multiply-add  */
+/* chain over d ascending. */
+static float ab_dist(const float* x, const float* mu, int D) {
+  float acc = 0.0f;
+  for (int d = 0; d < D; ++d) {
+    float diff = x[d] - mu[d];
+    acc = fmaf(diff, diff, acc);
+  }
+  return acc;
+}
+
+/* IBCS clustering of every 128-query block (see the section comment):      */
+/* cent [B][Hh][NQB][8][D] fp32, counts [B][Hh][NQB][8] int32, assign         */
+/* [B][Hh][S] int32 (may be NULL).  Centroid update: fp32 sum of the         */
+/* cluster's queries in ascending token order, divided by the count (one     */
+/* fp32 division).  Pinned by: recovery of well-separated clusters, each    */
+/* centroid the mean of its queries, each query at its nearest centroid of   */
+/* the last assignment, and non-increasing within-cluster sum of squares.   */
+void oracle_ab_kmeans(const uint16_t* q, int B, int S, int Hh, int D, int iters, float* cent, int32_t* counts,
+                      int32_t* assign_out) {
+  int nqb = S / AB_QBLOCK;
+#pragma omp parallel
+  {
+    float* x = (float*)malloc(sizeof(float) * AB_QBLOCK * (size_t)D);
+    float* mu = (float*)malloc(sizeof(float) * AB_CLUSTERS * (size_t)D);
+    float* acc = (float*)malloc(sizeof(float) * (size_t)D);
+    int asg[AB_QBLOCK];
+    int cnt[AB_CLUSTERS];
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t u = 0; u < (int64_t)B * Hh * nqb; ++u) {
+      int I = (int)(u % nqb);
+      int64_t bh = u / nqb;
+      int b = (int)(bh / Hh), hd = (int)(bh % Hh);
+      for (int t = 0; t < AB_QBLOCK; ++t)
+        for (int d = 0; d < D; ++d)
+          x[t * D + d] = bf16_bits_to_f32(q[(((int64_t)b * S + (int64_t)I * AB_QBLOCK + t) * Hh + hd) * D + d]);
+      for (int c = 0; c < AB_CLUSTERS; ++c)
+        for (int d = 0; d < D; ++d) mu[c * D + d] = x[(c * (AB_QBLOCK / AB_CLUSTERS)) * D + d];
+      for (int c = 0; c < AB_CLUSTERS; ++c) cnt[c] = 0;
+      for (int it = 0; it < iters; ++it) {
+        for (int t = 0; t < AB_QBLOCK; ++t) {
+          int best = 0;
+          float bd = ab_dist(x + t * D, mu, D);
+          for (int c = 1; c < AB_CLUSTERS; ++c) {
+            float dd = ab_dist(x + t * D, mu + c * D, D);
+            if (dd < bd) {
+              bd = dd;
+              best = c;
+            }
+          }
+          asg[t] = best;
+        }
+        for (int c = 0; c < AB_CLUSTERS; ++c) {
+          int n = 0;
+          for (int d = 0; d < D; ++d) acc[d] = 0.0f;
+          for (int t = 0; t < AB_QBLOCK; ++t)
+            if (asg[t] == c) {
+              for (int d = 0; d < D; ++d) acc[d] = acc[d] + x[t * D + d];
+              ++n;
+            }
+          cnt[c] = n;
+          if (n > 0)
+            for (int d = 0; d < D; ++d) mu[c * D + d] = acc[d] / (float)n;
+        }
+      }
+      for (int c = 0; c < AB_CLUSTERS; ++c) {
+        counts[u * AB_CLUSTERS + c] = cnt[c];
+        for (int d = 0; d < D; ++d) cent[(u * AB_CLUSTERS + c) * D + d] = mu[c * D + d];
+      }
+      if (assign_out)
+        for (int t = 0; t < AB_QBLOCK; ++t) assign_out[bh * S + (int64_t)I * AB_QBLOCK + t] = asg[t];
+    }
+    free(x);
+    free(mu);
+    free(acc);
+  }
+}
+
+/* IBCS block scores: for query block I and every key block J,              */
+/*   l_cJ = fl32(fmaf chain over d of cent_c . kbar_J) * scale,            */
+/*   a_cJ = exp(l_cJ - max_J l_cJ) / sum_J exp(...)   (fp64),               */
+/*   score_IJ = sum_c (counts_c / 128) * a_cJ        (fp64, c ascending;    */
+/*              empty clusters have weight 0).                              */
+/* score [B][Hh][NQB][NKB] fp64.  Pinned by: an fp64 restatement with numpy, */
+/* sum_J score = 1, and the single-cluster case equal to one softmax.       */
+void oracle_ab_scores(const float* cent, const int32_t* counts, const float* kbar, int B, int Hh, int nqb, int nkb,
+                      int D, float scale, double* score) {
+#pragma omp parallel
+  {
+    float* l = (float*)malloc(sizeof(float) * (size_t)nkb);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t u = 0; u < (int64_t)B * Hh * nqb; ++u) {
+      int64_t bh = u / nqb;
+      const float* kb = kbar + bh * nkb * D;
+      double* s = score + u * nkb;
+      for (int J = 0; J < nkb; ++J) s[J] = 0.0;
+      for (int c = 0; c < AB_CLUSTERS; ++c) {
+        int n = counts[u * AB_CLUSTERS + c];
+        if (n == 0) continue;
+        const float* mu = cent + (u * AB_CLUSTERS + c) * D;
+        float m = -INFINITY;
+        for (int J = 0; J < nkb; ++J) {
+          float dot = 0.0f;
+          for (int d = 0; d < D; ++d) dot = fmaf(mu[d], kb[(int64_t)J * D + d], dot);
+          l[J] = dot * scale;
+          if (l[J] > m) m = l[J];
+        }
+        double Z = 0.0;
+        for (int J = 0; J < nkb; ++J) Z += exp((double)l[J] - (double)m);
+        double w = (double)n / (double)AB_QBLOCK;
+        for (int J = 0; J < nkb; ++J) s[J] += w * (exp((double)l[J] - (double)m) / Z);
+      }
+    }
+    free(l);
+  }
+}
+
+typedef struct {
+  double s;
+  int j;
+} sj_t;
+
+static int cmp_sj_desc(const void* a, const void* b) {
+  const sj_t* x = (const sj_t*)a;
+  const sj_t* y = (const sj_t*)b;
+  if (x->s > y->s) return -1;
+  if (x->s < y->s) return 1;
+  return (x->j > y->j) - (x->j < y->j);
+}
+
+/* SIP inclusion probabilities of one row of n scores for an expected sample */
+/* size `budget`: pi_J = min(1, lambda * s_J) with sum_J pi_J = budget.      */
+/* With the scores sorted descending, the first m blocks are capped at 1,   */
+/* m the smallest count for which lambda = (budget - m) / (sum of the rest)  */
+/* leaves the largest remaining score below 1 / lambda.  A budget at or     */
+/* above the number of positive scores samples every positive-score block.  */
+/* Returns lambda.  Pinned by: sum pi = budget, pi proportional to s below  */
+/* the cap, the capped blocks' lambda * s >= 1, and an exact-rational       */
+/* restatement.                                                             */
+double oracle_ab_inclusion(const double* s, int n, double budget, double* pi) {
+  sj_t* v = (sj_t*)malloc(sizeof(sj_t) * (size_t)n);
+  double* tail = (double*)malloc(sizeof(double) * ((size_t)n + 1));
+  int npos = 0;
+  for (int j = 0; j < n; ++j) {
+    v[j].s = s[j];
+    v[j].j = j;
+    npos += s[j] > 0.0;
+  }
+  qsort(v, (size_t)n, sizeof(sj_t), cmp_sj_desc);
+  tail[n] = 0.0;
+  for (int k = n - 1; k >= 0; --k) tail[k] = tail[k + 1] + v[k].s; /* smallest first */
+  double lambda = 0.0;
+  int m = 0;
+  if (budget >= (double)npos) {
+    m = npos;
+    lambda = INFINITY;
+  } else {
+    while (m < npos) {
+      lambda = (budget - (double)m) / tail[m];
+      if (lambda * v[m].s < 1.0) break;
+      ++m;
+    }
+  }
+  for (int k = 0; k < n; ++k) {
+    int j = v[k].j;
+    pi[j] = v[k].s <= 0.0 ? 0.0 : (k < m ? 1.0 : lambda * v[k].s);
+  }
+  free(v);
+  free(tail);
+  return lambda;
+}
+
+/* Inclusion probabilities for every (b, head, query block) row of scores. */
+void oracle_ab_inclusion_all(const double* score, int64_t rows, int nkb, double budget, double* pi) {
+#pragma omp parallel for schedule(dynamic, 8)
+  for (int64_t r = 0; r < rows; ++r) oracle_ab_inclusion(score + r * nkb, nkb, budget, pi + r * nkb);
+}
+
+/* Attention of the query blocks listed in qblocks (all heads) over their   */
+/* sampled 4-token key blocks, each logit shifted by that block's shift     */
+/* (-log pi for the Horvitz-Thompson weight 1 / pi):                        */
+/*   l = (q_a . k_c) * scale + shift_J(c),  O_a = softmax(l) V,  LSE.       */
+/* kcount [B][Hh][nq], kidx [B][Hh][nq][NKB] (sampled blocks ascending),     */
+/* shift [B][Hh][nq][NKB] fp64 (entry e belongs to kidx entry e); q, k, v    */
+/* bf16 [B][S][Hh][D] in grid order.  out fp64 [B][nq*128][Hh][D], lse fp64  */
+/* [B][Hh][nq*128].  A row with no sampled block gives O = 0, LSE = -inf.   */
+/* Pinned by: unbiasedness of the numerator and the normaliser over every   */
+/* sample of a small case, weighted by its probability (exact enumeration), */
+/* and equality with dense attention when every block is sampled with pi=1. */
+void oracle_ab_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* kcount,
+                         const int32_t* kidx, const double* shift, int B, int S, int Hh, int D, double scale,
+                         const int32_t* qblocks, int nq, double* out, double* lse) {
+  int nkb = S / AB_KBLOCK;
+  int64_t units = (int64_t)B * Hh * nq * AB_QBLOCK;
+#pragma omp parallel
+  {
+    double* logit = (double*)malloc(sizeof(double) * (size_t)S);
+#pragma omp for schedule(dynamic, 16)
+    for (int64_t u = 0; u < units; ++u) {
+      int r = (int)(u % AB_QBLOCK);
+      int64_t t1 = u / AB_QBLOCK;
+      int qn = (int)(t1 % nq);
+      int64_t t2 = t1 / nq;
+      int hd = (int)(t2 % Hh), b = (int)(t2 / Hh);
+      int64_t row = ((int64_t)b * Hh + hd) * nq + qn;
+      int cnt = kcount[row];
+      const int32_t* lst = kidx + row * nkb;
+      const double* sh = shift + row * nkb;
+      int64_t a = (int64_t)qblocks[qn] * AB_QBLOCK + r;
+      const uint16_t* qa = q + (((int64_t)b * S + a) * Hh + hd) * D;
+      double mx = -INFINITY;
+      int64_t n = 0;
+      for (int e = 0; e < cnt; ++e)
+        for (int c = 0; c < AB_KBLOCK; ++c) {
+          const uint16_t* kc = k + (((int64_t)b * S + (int64_t)lst[e] * AB_KBLOCK + c) * Hh + hd) * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d) dot += (double)bf16_bits_to_f32(qa[d]) * (double)bf16_bits_to_f32(kc[d]);
+          logit[n] = dot * scale + sh[e];
+          if (logit[n] > mx) mx = logit[n];
+          ++n;
+        }
+      double* o = out + (((int64_t)b * nq * AB_QBLOCK + (int64_t)qn * AB_QBLOCK + r) * Hh + hd) * D;
+      for (int d = 0; d < D; ++d) o[d] = 0.0;
+      double den = 0.0;
+      n = 0;
+      for (int e = 0; e < cnt; ++e)
+        for (int c = 0; c < AB_KBLOCK; ++c) {
+          const uint16_t* vc = v + (((int64_t)b * S + (int64_t)lst[e] * AB_KBLOCK + c) * Hh + hd) * D;
+          double w = exp(logit[n++] - mx);
+          den += w;
+          for (int d = 0; d < D; ++d) o[d] += w * (double)bf16_bits_to_f32(vc[d]);
+        }
+      for (int d = 0; d < D; ++d) o[d] = cnt > 0 ? o[d] / den : 0.0;
+      if (lse) lse[((int64_t)b * Hh + hd) * nq * AB_QBLOCK + (int64_t)qn * AB_QBLOCK + r] = cnt > 0 ? mx + log(den) : -INFINITY;
+    }
+    free(logit);
+  }
+}

@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 
 import test_oracle as pins
+import test_oracle_ab as ab_pins
 from block_sparse_attention_flatten_b200 import inputs
 
 ORACLE_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle")
@@ -26,6 +27,12 @@ def tiny_flat(mod):
     kf = mod.flatten(k, w.T, w.H, w.W).reshape(k.shape)
     vf = mod.flatten(v, w.T, w.H, w.W).reshape(v.shape)
     return w, (q, k, v), (qf, kf, vf)
+
+
+def ab_tiny(mod):
+    w = inputs.AB_TINY
+    q, k, v = inputs.make_qkv(w.base)
+    return w, q, k, v
 
 
 # pin name -> call with an oracle module
@@ -44,6 +51,14 @@ PINS = {
     "radial_lists": lambda m: [pins.test_radial_lists_equal_enumeration_and_closed_form(m, *g)
                                for g in pins.RADIAL_GRIDS[:3]],
     "radial_union": lambda m: pins.test_radial_union_is_superset(m),
+    "ab_key_means": lambda m: ab_pins.test_key_means_are_block_means(m, ab_tiny(m)),
+    "ab_kmeans": lambda m: (ab_pins.test_kmeans_recovers_separated_clusters(m),
+                            ab_pins.test_kmeans_centroids_assignment_and_descent(m, ab_tiny(m))),
+    "ab_scores": lambda m: ab_pins.test_scores_restated_in_fp64(m, ab_tiny(m)),
+    "ab_inclusion": lambda m: [ab_pins.test_inclusion_probabilities(m, *a)
+                               for a in [(1, 40, 4.0), (2, 64, 10.0), (5, 50, 1.0)]],
+    "ab_unbiased": lambda m: ab_pins.test_horvitz_thompson_unbiased_by_enumeration(m),
+    "ab_dense": lambda m: ab_pins.test_full_sample_equals_dense_attention(m, ab_tiny(m)),
     "dense_attention": lambda m: pins.test_thr_one_equals_dense_attention(m, tiny_flat(m)),
     "attention_special": lambda m: pins.test_attention_special_cases(m),
     "bwd_autograd": lambda m: [pins.test_attention_bwd_equals_autograd(m, *a) for a in [(64, 0.5, ()), (128, 0.3, (2,))]],
@@ -80,6 +95,16 @@ MUTANTS = [
     ("radial window left out of the union",
      "sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w) || radial_keep(i, j, nbh, nbw, radial_r0);",
      "sta_keep(i, j, nbh, nbw, sta_t, sta_h, sta_w);", ["radial_union"]),
+    ("AB key means over 3 tokens", "kbar[(((int64_t)b * Hh + hd) * nkb + J) * D + d] = acc * 0.25f;",
+     "kbar[(((int64_t)b * Hh + hd) * nkb + J) * D + d] = acc * (1.0f / 3.0f);", ["ab_key_means"]),
+    ("AB centroid divides by count + 1", "mu[c * D + d] = acc[d] / (float)n;", "mu[c * D + d] = acc[d] / (float)(n + 1);",
+     ["ab_kmeans"]),
+    ("AB clusters weighted equally", "double w = (double)n / (double)AB_QBLOCK;", "double w = 1.0 / AB_CLUSTERS;",
+     ["ab_scores"]),
+    ("AB inclusion never capped", "if (lambda * v[m].s < 1.0) break;", "break;", ["ab_inclusion"]),
+    ("AB Horvitz-Thompson shift sign flipped", "logit[n] = dot * scale + sh[e];", "logit[n] = dot * scale - sh[e];",
+     ["ab_unbiased"]),
+    ("AB attention scale dropped", "logit[n] = dot * scale + sh[e];", "logit[n] = dot + sh[e];", ["ab_dense"]),
     ("attention scale dropped", "double l = dot * scale;", "double l = dot;", ["dense_attention"]),
     ("attention normaliser dropped", "o[d] = cnt > 0 ? acc[d] / den : 0.0;", "o[d] = cnt > 0 ? acc[d] : 0.0;",
      ["attention_special", "dense_attention"]),
