@@ -14,7 +14,7 @@ L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
 With --config hunyuan-sta the mask is the static sliding-tile window alone
 (nabla_build_mask_sta replaces stages 1 and 2; Q and K are not read for it).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan13b]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long]
     python bench.py --impl reference ...   # the CPU oracle, same metric
 
 Prints one JSON line (rank 0).  `value` is kept-tile attention TFLOP/s over
@@ -49,8 +49,12 @@ CONFIGS = {
     "hunyuan": inputs.HUNYUAN,
     "long": inputs.LONG,
     "hunyuan-sta": inputs.HUNYUAN_STA,
+    "hunyuan-radial": inputs.HUNYUAN_RADIAL,
+    "long-radial": inputs.LONG_RADIAL,
 }
 CONFIGS.update({f"sweep-a{w.alpha}-t{w.thr}": w for w in inputs.sweep_points()})
+# AB-Attention (second workload): sampling plan + attention on the samples
+AB_CONFIGS = {"ab-wan13b": inputs.AB_WAN13B, "ab-tiny": inputs.AB_TINY}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -88,8 +92,9 @@ def config_dict(w: inputs.Workload):
         "grid_THW": [w.T, w.H, w.W],
         "tokens": w.S,
         "blocks": w.Nb,
-        "mask": "adaptive (CDF)" + (" OR static STA window" if any(w.sta) else "") if w.mask == "nabla"
-                else "static STA window only",
+        "mask": ("adaptive (CDF)" + (" OR static STA window" if any(w.sta) else "") +
+                 (f" OR radial window r0={w.radial}" if w.radial else "")) if w.mask == "nabla"
+                else ("static STA window only" if w.mask == "sta" else f"static radial window r0={w.radial} only"),
         "thr": w.thr if w.mask == "nabla" else None,
         "sta": list(w.sta) if any(w.sta) else None,
         "locality_amplitude": w.alpha,
@@ -195,19 +200,25 @@ def run_gpu(args, rank, world, local_rank):
     og = torch.empty_like(qd)  # attention output, grid order
     kv_count = torch.empty((w.B, w.Hh, w.Nb), dtype=torch.int32, device=dev)
     kv_idx = torch.empty((w.B, w.Hh, w.Nb, w.Nb), dtype=torch.int32, device=dev)
-    static = w.mask == "sta"  # the static window alone: no pooling, no scores
-    prm = nabla.params(w.thr, w.sta)
+    static = w.mask in ("sta", "radial")  # a static window alone: no pooling, no scores
+    prm = nabla.params(w.thr, w.sta, radial=w.radial)
     ws = None if static else torch.empty(nabla.mask_workspace_bytes(w.B, w.Hh, w.D, w.T, w.H, w.W, prm),
                                          dtype=torch.uint8, device=dev)
     lse = torch.empty((w.B, w.Hh, w.S), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def static_lists():
+        if w.mask == "sta":
+            nabla.build_mask_sta(w.B, w.Hh, w.T, w.H, w.W, w.sta, kv_count=kv_count, kv_idx=kv_idx)
+        else:
+            nabla.build_mask_radial(w.B, w.Hh, w.T, w.H, w.W, w.radial, kv_count=kv_count, kv_idx=kv_idx)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
         if static:
             # 1-2. the window's block lists (nothing read)
-            nabla.build_mask_sta(w.B, w.Hh, w.T, w.H, w.W, w.sta, kv_count=kv_count, kv_idx=kv_idx)
+            static_lists()
             if ev is not None:
                 ev[1].record(stream)
                 ev[2].record(stream)
@@ -219,7 +230,7 @@ def run_gpu(args, rank, world, local_rank):
                 ev[1].record(stream)
             # 2. mask rows on the pooled workspace
             nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count,
-                                    kv_idx=kv_idx)
+                                    kv_idx=kv_idx, radial=w.radial)
             if ev is not None:
                 ev[2].record(stream)
         # 3. attention reading Q, K, V in grid order through 5-D TMA boxes
@@ -228,7 +239,7 @@ def run_gpu(args, rank, world, local_rank):
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 2 if static else 3  # (window lists | pooling, mask rows), attention
+    launches_per_step = 2 if static else 4  # (window lists | pooling, scores, selection), attention
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -293,12 +304,12 @@ def run_gpu(args, rank, world, local_rank):
                 v_in[b_].record(up)
             stream.wait_event(qk_in[b_])
             if static:
-                nabla.build_mask_sta(w.B, w.Hh, w.T, w.H, w.W, w.sta, kv_count=kv_count, kv_idx=kv_idx)
+                static_lists()
             else:
                 nabla.flatten_pool_qk(qd_, kd_, w.T, w.H, w.W, workspace=ws, thr=w.thr, sta=w.sta,
                                       write_flat=False)
                 nabla.build_mask_pooled(ws, w.B, w.Hh, w.D, w.T, w.H, w.W, w.thr, w.sta, kv_count=kv_count,
-                                        kv_idx=kv_idx)
+                                        kv_idx=kv_idx, radial=w.radial)
             stream.wait_event(v_in[b_])
             if s_ >= 2:
                 stream.wait_event(out[b_])  # step s-2's output has been downloaded
@@ -375,6 +386,8 @@ def run_gpu(args, rank, world, local_rank):
     peak_tf, peak_gbs, peak_kind = load_peaks()
     attn_avg = statistics.mean(attn_ms)
     mask_avg = statistics.mean(mask_ms)
+    mask_gbs = (mask_bytes(w, total_kept) - (0 if not static else 4.0 * w.B * w.S * w.Hh * w.D)) / \
+        ((statistics.mean(pool_ms) + mask_avg) * 1e-3) / 1e9
     achieved = kept_flops(w, total_kept) / (attn_avg * 1e-3) / 1e12
     traffic = load_traffic(args.config)
     result = {
@@ -394,29 +407,127 @@ def run_gpu(args, rank, world, local_rank):
         # per layer: the whole step, since Q, K, V, O stay in grid order (the
         # flattening and its inverse happen inside the pooling and attention)
         "ms_per_layer": statistics.mean(pool_ms) + mask_avg + attn_avg,
-        "stages_ms": ({"sta_lists": statistics.mean(pool_ms), "sparse_attn": attn_avg} if static else
+        "stages_ms": ({"window_lists": statistics.mean(pool_ms), "sparse_attn": attn_avg} if static else
                       {"pool_qk": statistics.mean(pool_ms), "mask_rows": mask_avg, "sparse_attn": attn_avg}),
         # mask build = pooling + rows: Q and K read once, kv_count and the kept
         # kv_idx entries written, over its time (the static window reads
         # nothing: only the lists are written)
-        "mask_build_gbs": (mask_bytes(w, total_kept) - (0 if not static else 4.0 * w.B * w.S * w.Hh * w.D)) /
-                          ((statistics.mean(pool_ms) + mask_avg) * 1e-3) / 1e9,
+        "mask_build_gbs": mask_gbs,
         "attn_tflops_kept": achieved,
         "pool_gbs": None if static else pool_bytes(w) / (statistics.mean(pool_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
                      "traffic": traffic},
-        "mask_roofline": None if static else {"bound": "alu", "kernel": "mask_rows_kernel", "achieved": score_flops(w) / (mask_avg * 1e-3) / 1e12,
-                          "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                          "frac": score_flops(w) / (mask_avg * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
-                          "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"},
+        # the mask build (pooling + rows) against HBM: Q and K read once, the
+        # lists written, over the two stages' time
+        "mask_roofline": None if static else {
+            "bound": "hbm", "kernels": "pool_kernel<true> + score_tile_kernel + select_rows_kernel",
+            "achieved": mask_gbs, "peak": peak_gbs, "unit": "GB/s", "frac": mask_gbs / peak_gbs,
+            "peak_kind": f"{peak_kind} HBM copy", "target_frac": 0.6},
+        # the rows stage alone against the fp32 FMA peak (its scores are an
+        # fp32 GEMM of 2*B*Hh*Nb^2*D FLOP)
+        "mask_score_roofline": None if static else {
+            "bound": "alu", "kernels": "score_tile_kernel + select_rows_kernel",
+            "achieved": score_flops(w) / (mask_avg * 1e-3) / 1e12, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+            "frac": score_flops(w) / (mask_avg * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
+            "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"},
         "e2e": e2e,
         "backward": backward,
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
     return result, (q, k, v, w, total_kept)
+
+
+def run_gpu_ab(args, rank, world, local_rank):
+    """AB-Attention layer: a step is the sampling plan (key means, clusters,
+    centroid logits, scores, inclusion probabilities, the sample) and the
+    attention on the sampled 4-token blocks, Q, K, V in grid order.  value =
+    attention FLOPs on the sampled blocks (4 * 128 * 4 * D per (query block,
+    sampled key block)) over the whole step."""
+    from block_sparse_attention_flatten_b200 import nabla
+    from block_sparse_attention_flatten_b200 import build as nbuild
+
+    nbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = AB_CONFIGS[args.config]
+    base = w.base
+    q, k, v = inputs.make_qkv(base)
+    u = inputs.ab_uniforms(w)
+    stream = torch.cuda.current_stream()
+    qd, kd, vd, ud = q.to(dev), k.to(dev), v.to(dev), u.to(dev)
+    kcount = torch.empty((base.B, base.Hh, w.nqb), dtype=torch.int32, device=dev)
+    kidx = torch.empty((base.B, base.Hh, w.nqb, w.nkb), dtype=torch.int32, device=dev)
+    kshift = torch.empty((base.B, base.Hh, w.nqb, w.nkb), dtype=torch.float32, device=dev)
+    ws = torch.empty(nabla.ab_workspace_bytes(base.B, base.S, base.Hh, base.D), dtype=torch.uint8, device=dev)
+    og = torch.empty_like(qd)
+    lse = torch.empty((base.B, base.Hh, base.S), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        nabla.ab_plan(qd, kd, ud, w.budget, w.kmeans_iters, kcount=kcount, kidx=kidx, kshift=kshift, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        nabla.ab_attn_fwd(qd, kd, vd, kcount, kidx, kshift, out=og, lse=lse)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = nabla.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {nabla.strerror(status)}")
+    sampled = float(kcount.double().sum().item())
+    flop = 4.0 * 128 * 4 * base.D * sampled
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    sampler.start()
+    for s_ in range(args.steps):
+        flush.zero_()
+        step(events[s_])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in events)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
+    total = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in events), dev)
+    peak_tf, peak_gbs, peak_kind = load_peaks()
+    achieved = flop / (attn_ms * 1e-3) / 1e12
+    cfg = config_dict(base)
+    cfg.update({"workload": w.name, "mask": "AB-Attention sample (IBCS clusters + SIP, 4-token key blocks)",
+                "thr": None, "budget_blocks_per_query_block": w.budget, "kmeans_iters": w.kmeans_iters,
+                "query_block": 128, "key_block": 4})
+    return {
+        "metric": METRIC,
+        "value": whole_job_tflops(world, flop, args.steps, total),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": cfg,
+        "stages_ms": {"ab_plan": plan_ms, "ab_attn": attn_ms},
+        "sampled_block_fraction": sampled / (base.B * base.Hh * w.nqb * w.nkb),
+        "attn_tflops_sampled": achieved,
+        "roofline": {"bound": "tensor", "kernel": "ab_attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
+                     "traffic": None},
+        "clocks": clocks,
+        "gpu_launches": 5 * args.steps,
+        "cpu_baseline": None,
+        "e2e": None,
+    }, (q, k, v, u)
 
 
 def load_traffic(config):
@@ -439,52 +550,118 @@ def load_traffic(config):
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_sample(w, q, k, v, n_blocks, total_kept=None):
-    """Time the CPU oracle on a bounded sample of the layer: flattening,
-    pooling and the full mask, plus attention on n_blocks seeded query blocks
-    (all heads).  Returns the dict for `cpu_baseline`."""
+def oracle_sample(w, q, k, v, n_blocks, heads=1):
+    """Time the CPU oracle on a bounded sample of the layer: `heads` seeded
+    heads (all their tokens: flattening, pooling and the full mask of every
+    query block), plus attention on n_blocks seeded query blocks of those
+    heads; the stage times are extrapolated to all heads (flattening,
+    pooling, mask) and to all kept tiles (attention).  Returns the dict for
+    `cpu_baseline`."""
     import oracle
     oracle.build()
+    heads = min(heads, w.Hh)
+    hsel = np.sort(np.random.default_rng(4321).choice(w.Hh, size=heads, replace=False))
+    sub = [np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16)[:, :, hsel]) for x in (q, k, v)]
     t0 = time.perf_counter()
-    qf = oracle.flatten(q, w.T, w.H, w.W).reshape(q.shape)
-    kf = oracle.flatten(k, w.T, w.H, w.W).reshape(k.shape)
-    vf = oracle.flatten(v, w.T, w.H, w.W).reshape(v.shape)
+    qf, kf, vf = (oracle.flatten(x, w.T, w.H, w.W).reshape(x.shape) for x in sub)
     t1 = time.perf_counter()
-    if w.mask == "sta":
-        c1, i1 = oracle.sta_lists(w.T, w.nbh, w.nbw, w.sta)
-        cnt = np.broadcast_to(c1, (w.B, w.Hh, w.Nb))
-        idx = np.broadcast_to(i1, (w.B, w.Hh, w.Nb, w.Nb))
+    if w.mask in ("sta", "radial"):
+        c1, i1 = (oracle.sta_lists(w.T, w.nbh, w.nbw, w.sta) if w.mask == "sta" else
+                  oracle.radial_lists(w.T, w.nbh, w.nbw, w.radial))
+        cnt = np.broadcast_to(c1, (w.B, heads, w.Nb))
+        idx = np.broadcast_to(i1, (w.B, heads, w.Nb, w.Nb))
     else:
         qbar, kbar = oracle.pool(qf), oracle.pool(kf)
         cnt, idx, _, _ = oracle.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, sta_window=w.sta,
-                                           want_status=False)
+                                           want_status=False, radial_r0=w.radial)
     t2 = time.perf_counter()
     qblocks = inputs.sample_query_blocks(w.Nb, n_blocks, seed=1234)
     oracle.attention(qf, kf, vf, cnt, idx, w.scale, qblocks=qblocks)
     t3 = time.perf_counter()
-    all_kept = float(cnt.astype(np.float64).sum())
+    head_kept = float(cnt.astype(np.float64).sum())
     sample_kept = float(cnt[:, :, qblocks].astype(np.float64).sum())
+    all_kept = head_kept * w.Hh / heads  # kept tiles of the whole layer, from the sampled heads
+    mask_full_s = (t2 - t0) * w.Hh / heads
     attn_full_s = (t3 - t2) * all_kept / max(sample_kept, 1.0)
-    step_s = (t1 - t0) + (t2 - t1) + attn_full_s
+    step_s = mask_full_s + attn_full_s
     return {
         "value": kept_flops(w, all_kept) / step_s / 1e12,
         "unit": "TFLOP/s",
         "cores": oracle.num_threads(),
         "kind": "oracle",
-        "sample": (f"flatten+{'window lists' if w.mask == 'sta' else 'pool+full mask'} ({t2 - t0:.2f} s) and attention on {len(qblocks)} seeded query blocks x "
-                   f"{w.Hh} heads ({t3 - t2:.2f} s), attention extrapolated to all {w.Nb} blocks by kept-tile count"),
+        "sample": (f"{heads} of {w.Hh} heads: flatten+{'pool+full mask' if w.mask == 'nabla' else 'window lists'} "
+                   f"({t2 - t0:.2f} s, x{w.Hh / heads:g} for all heads) and attention on {len(qblocks)} seeded "
+                   f"query blocks ({t3 - t2:.2f} s, extrapolated to all {w.Nb} blocks by kept-tile count)"),
+        "ms_per_step_extrapolated": step_s * 1e3,
+        "sample_s": t3 - t0,
+    }
+
+
+def oracle_sample_ab(w, q, k, v, u, n_blocks, heads=1):
+    """The CPU oracle on a bounded sample of an AB-Attention layer: `heads`
+    seeded heads (key means, clustering, scores, inclusion and the sample of
+    every query block) plus attention on n_blocks query blocks of them,
+    extrapolated to all heads and all sampled blocks."""
+    import oracle
+    oracle.build()
+    base = w.base
+    heads = min(heads, base.Hh)
+    hsel = np.sort(np.random.default_rng(4321).choice(base.Hh, size=heads, replace=False))
+    qs, ks, vs = (np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16)[:, :, hsel]) for x in (q, k, v))
+    us = u.numpy()[:, hsel]
+    t0 = time.perf_counter()
+    kbar = oracle.ab_key_means(ks)
+    cent, counts, _ = oracle.ab_kmeans(qs, iters=w.kmeans_iters)
+    score = oracle.ab_scores(cent, counts, kbar, base.scale)
+    pi = oracle.ab_inclusion(score, w.budget)
+    cnt, idx, shift = oracle.ab_sample(pi, us)
+    t1 = time.perf_counter()
+    qblocks = inputs.sample_query_blocks(w.nqb, n_blocks, seed=1234)
+    oracle.ab_attention(qs, ks, vs, cnt, idx, shift, base.scale, qblocks=qblocks)
+    t2 = time.perf_counter()
+    all_sampled = float(cnt.sum()) * base.Hh / heads
+    frac = float(cnt.sum()) / max(float(cnt[:, :, qblocks].sum()), 1.0)
+    step_s = (t1 - t0) * base.Hh / heads + (t2 - t1) * frac * base.Hh / heads
+    return {
+        "value": 4.0 * 128 * 4 * base.D * all_sampled / step_s / 1e12,
+        "unit": "TFLOP/s",
+        "cores": oracle.num_threads(),
+        "kind": "oracle",
+        "sample": (f"{heads} of {base.Hh} heads: sampling plan ({t1 - t0:.2f} s, x{base.Hh / heads:g}) and attention "
+                   f"on {len(qblocks)} query blocks ({t2 - t1:.2f} s, extrapolated by sampled-block count)"),
         "ms_per_step_extrapolated": step_s * 1e3,
     }
 
 
 def run_reference(args):
+    if args.config in AB_CONFIGS:
+        w = AB_CONFIGS[args.config]
+        q, k, v = inputs.make_qkv(w.base)
+        u = inputs.ab_uniforms(w)
+        times, vals, last = [], [], None
+        for s_ in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            last = oracle_sample_ab(w, q, k, v, u, args.ref_blocks, heads=args.ref_heads)
+            if s_ >= args.warmup:
+                times.append(time.perf_counter() - t0)
+                vals.append(last["value"])
+        value = statistics.mean(vals)
+        cfg = config_dict(w.base)
+        cfg["workload"] = w.name
+        return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": last["ms_per_step_extrapolated"],
+                "sample_s_per_step": statistics.mean(times), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
+                                 "sample": last["sample"]},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     w = CONFIGS[args.config]
     q, k, v = inputs.make_qkv(w)
     times, vals = [], []
     last = None
     for s in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        last = oracle_sample(w, q, k, v, args.ref_blocks)
+        last = oracle_sample(w, q, k, v, args.ref_blocks, heads=args.ref_heads)
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             times.append(dt)
@@ -498,7 +675,8 @@ def run_reference(args):
         "n_gpus": 1,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": statistics.mean(times) * 1e3,
+        "ms_per_step": last["ms_per_step_extrapolated"],
+        "sample_s_per_step": statistics.mean(times),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -516,12 +694,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="wan13b", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="long", choices=sorted(CONFIGS) + sorted(AB_CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--backward-steps", type=int, default=20, help="timed steps of the backward pass (0: skip)")
     ap.add_argument("--cpu-blocks", type=int, default=8, help="query blocks in the CPU-baseline sample")
-    ap.add_argument("--ref-blocks", type=int, default=4, help="query blocks per reference-arm step")
+    ap.add_argument("--ref-blocks", type=int, default=2, help="query blocks per reference-arm step")
+    ap.add_argument("--ref-heads", type=int, default=1, help="heads per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -542,11 +721,21 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
+    if args.config in AB_CONFIGS:
+        result, (q, k, v, u) = run_gpu_ab(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                result["cpu_baseline"] = oracle_sample_ab(AB_CONFIGS[args.config], q, k, v, u, args.cpu_blocks,
+                                                          heads=args.ref_heads)
+            print(json.dumps(result), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     try:
         result, (q, k, v, w, total_kept) = run_gpu(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                result["cpu_baseline"] = oracle_sample(w, q, k, v, args.cpu_blocks)
+                result["cpu_baseline"] = oracle_sample(w, q, k, v, args.cpu_blocks, heads=args.ref_heads)
             else:
                 result["cpu_baseline"] = None
             print(json.dumps(result), flush=True)

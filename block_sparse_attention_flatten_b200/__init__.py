@@ -19,6 +19,16 @@ The static sliding-tile window alone, without reading Q or K:
 
     kv_count, kv_idx = nabla.build_mask_sta(B, Hh, T, H, W, (3, 3, 3))
 
+A radial decay window, alone or OR-ed into the adaptive mask:
+
+    kv_count, kv_idx = nabla.build_mask_radial(B, Hh, T, H, W, r0=2)
+    kv_count, kv_idx, _ = nabla.build_mask_grid(q, k, T, H, W, thr=0.9, radial=2)
+
+AB-Attention on the same grid-order tensors (u: uniforms [B, Hh, S/128, S/4]):
+
+    kcount, kidx, kshift, _ = nabla.ab_plan(q, k, u, budget=0.1 * S / 4)
+    o, lse = nabla.ab_attn_fwd(q, k, v, kcount, kidx, kshift)
+
 Flattened tensors (e.g. flattened once per sequence):
 
     qf = nabla.flatten(q, T, H, W)                       # per tensor

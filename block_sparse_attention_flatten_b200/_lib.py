@@ -38,11 +38,15 @@ EXPORTS = (
     "nabla_build_mask_pooled",
     "nabla_build_mask_grid",
     "nabla_build_mask_sta",
+    "nabla_build_mask_radial",
     "nabla_sparse_attn_fwd",
     "nabla_sparse_attn_fwd_grid",
     "nabla_transpose_lists",
     "nabla_sparse_attn_bwd",
     "nabla_sparse_attn_bwd_grid",
+    "nabla_ab_workspace_bytes",
+    "nabla_ab_plan",
+    "nabla_ab_attn_fwd",
     "nabla_get_status",
     "nabla_validate_mask",
     "nabla_selftest_wait_timeout",
@@ -65,6 +69,7 @@ class NablaParams(ctypes.Structure):
         ("sta_w", ctypes.c_int),
         ("scale", ctypes.c_float),
         ("flags", ctypes.c_uint),
+        ("radial", ctypes.c_int),
     ]
 
 
@@ -91,18 +96,23 @@ def lib():
         L.nabla_build_mask_pooled.argtypes = [vp, i, i, i, i, i, i, pp, vp, vp, vp]
         L.nabla_build_mask_grid.argtypes = [vp, vp, i, i, i, i, i, i, pp, vp, vp, vp, vp]
         L.nabla_build_mask_sta.argtypes = [i, i, i, i, i, i, i, i, i, vp, vp, vp]
+        L.nabla_build_mask_radial.argtypes = [i, i, i, i, i, i, i, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
         L.nabla_transpose_lists.argtypes = [vp, vp, i, i, i, vp, vp, vp]
         L.nabla_sparse_attn_bwd.argtypes = [vp] * 10 + [i, i, i, i, f, vp, vp, vp, vp, vp]
         L.nabla_sparse_attn_bwd_grid.argtypes = [vp] * 10 + [i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
+        L.nabla_ab_workspace_bytes.argtypes = [i, i, i, i]
+        L.nabla_ab_workspace_bytes.restype = sz
+        L.nabla_ab_plan.argtypes = [vp, vp, vp, i, i, i, i, i, ctypes.c_double, f, vp, vp, vp, vp, vp]
+        L.nabla_ab_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_get_status.argtypes = [vp]
         L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
         L.nabla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
         L.nabla_strerror.argtypes = [i]
         L.nabla_strerror.restype = ctypes.c_char_p
         for name in EXPORTS:
-            if name not in ("nabla_mask_workspace_bytes", "nabla_strerror"):
+            if name not in ("nabla_mask_workspace_bytes", "nabla_ab_workspace_bytes", "nabla_strerror"):
                 getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -132,8 +142,8 @@ def _dev(t: torch.Tensor, dtype, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def params(thr: float, sta=(0, 0, 0), scale: float = 0.0, P: int = 8) -> NablaParams:
-    return NablaParams(P, float(thr), int(sta[0]), int(sta[1]), int(sta[2]), float(scale), 0)
+def params(thr: float, sta=(0, 0, 0), scale: float = 0.0, P: int = 8, radial: int = 0) -> NablaParams:
+    return NablaParams(P, float(thr), int(sta[0]), int(sta[1]), int(sta[2]), float(scale), 0, int(radial))
 
 
 def _permute(fn, x: torch.Tensor, T: int, H: int, W: int, out, stream, P: int):
@@ -161,16 +171,17 @@ def mask_workspace_bytes(B: int, Hh: int, D: int, T: int, H: int, W: int, prm: N
 
 
 def build_mask(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),
-               scale: float = 0.0, kv_count=None, kv_idx=None, workspace=None, stream=None, P: int = 8):
+               scale: float = 0.0, kv_count=None, kv_idx=None, workspace=None, stream=None, P: int = 8,
+               radial: int = 0):
     """Adaptive block mask from flattened Q, K [B, S, Hh, D] (bf16, CUDA).
 
     Returns (kv_count int32 [B,Hh,Nb], kv_idx int32 [B,Hh,Nb,Nb], workspace
-    uint8 holding the pooled qbar [B,Hh,Nb,D] then kbar^T [B,Hh,D,Nbp], fp32;
-    see :func:`pooled_from_workspace`).
+    uint8 holding the pooled qbar^T and kbar^T [B,Hh,D,Nbp] (fp32, see
+    :func:`pooled_from_workspace`) and the score scratch).
     """
     B, S, Hh, D = qf.shape
     Nb = S // BLOCK
-    prm = params(thr, sta, scale, P)
+    prm = params(thr, sta, scale, P, radial)
     dev = qf.device
     if kv_count is None:
         kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
@@ -215,13 +226,14 @@ def flatten_pool_qk(q: torch.Tensor, k: torch.Tensor, T: int, H: int, W: int, qf
 
 
 def build_mask_grid(q: torch.Tensor, k: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),
-                    scale: float = 0.0, kv_count=None, kv_idx=None, workspace=None, stream=None, P: int = 8):
+                    scale: float = 0.0, kv_count=None, kv_idx=None, workspace=None, stream=None, P: int = 8,
+                    radial: int = 0):
     """:func:`build_mask` on Q, K in grid order [B, T*H*W, Hh, D] (no
     flattened copies; nabla_build_mask_grid).  Returns (kv_count, kv_idx,
     workspace)."""
     B, S, Hh, D = q.shape
     Nb = S // BLOCK
-    prm = params(thr, sta, scale, P)
+    prm = params(thr, sta, scale, P, radial)
     dev = q.device
     if kv_count is None:
         kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
@@ -240,11 +252,12 @@ def build_mask_grid(q: torch.Tensor, k: torch.Tensor, T: int, H: int, W: int, th
 
 
 def build_mask_pooled(workspace: torch.Tensor, B: int, Hh: int, D: int, T: int, H: int, W: int, thr: float,
-                      sta=(0, 0, 0), scale: float = 0.0, kv_count=None, kv_idx=None, stream=None, P: int = 8):
+                      sta=(0, 0, 0), scale: float = 0.0, kv_count=None, kv_idx=None, stream=None, P: int = 8,
+                      radial: int = 0):
     """The mask from a workspace that already holds the pooled Q and K
     (nabla_build_mask_pooled).  Returns (kv_count, kv_idx)."""
     Nb = T * H * W // BLOCK
-    prm = params(thr, sta, scale, P)
+    prm = params(thr, sta, scale, P, radial)
     dev = workspace.device
     if kv_count is None:
         kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
@@ -274,15 +287,32 @@ def build_mask_sta(B: int, Hh: int, T: int, H: int, W: int, sta=(3, 3, 3), kv_co
     return kv_count, kv_idx
 
 
+def build_mask_radial(B: int, Hh: int, T: int, H: int, W: int, r0: int, kv_count=None, kv_idx=None, device=None,
+                      stream=None, P: int = 8):
+    """The radial decay window alone as block lists (nabla_build_mask_radial;
+    reads no Q or K).  Returns (kv_count int32 [B,Hh,Nb], kv_idx int32
+    [B,Hh,Nb,Nb])."""
+    Nb = T * H * W // BLOCK
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if kv_count is None:
+        kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
+    if kv_idx is None:
+        kv_idx = torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)
+    _check(lib().nabla_build_mask_radial(B, Hh, T, H, W, P, int(r0), _dev(kv_count, torch.int32, "kv_count"),
+                                         _dev(kv_idx, torch.int32, "kv_idx"), _stream(stream)),
+           "nabla_build_mask_radial")
+    return kv_count, kv_idx
+
+
 def build_mask_noalloc(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: int, thr: float, sta=(0, 0, 0),
-                       scale: float = 0.0, kv_count=None, kv_idx=None, stream=None, P: int = 8):
+                       scale: float = 0.0, kv_count=None, kv_idx=None, stream=None, P: int = 8, radial: int = 0):
     """The mask of :func:`build_mask` through nabla_build_mask_noalloc: the
     library keeps the pooled vectors in its own static device buffer (16 MiB)
-    and allocates nothing; calls sharing that buffer must not overlap on the
-    GPU.  Returns (kv_count, kv_idx)."""
+    and allocates nothing (the scores stay in shared memory); calls sharing
+    that buffer must not overlap on the GPU.  Returns (kv_count, kv_idx)."""
     B, S, Hh, D = qf.shape
     Nb = S // BLOCK
-    prm = params(thr, sta, scale, P)
+    prm = params(thr, sta, scale, P, radial)
     dev = qf.device
     if kv_count is None:
         kv_count = torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev)
@@ -296,14 +326,15 @@ def build_mask_noalloc(qf: torch.Tensor, kf: torch.Tensor, T: int, H: int, W: in
 
 
 def pooled_from_workspace(workspace: torch.Tensor, B: int, Hh: int, Nb: int, D: int):
-    """qbar [B,Hh,Nb,D] and kbar [B,Hh,Nb,D] from a mask workspace (kbar is
+    """qbar [B,Hh,Nb,D] and kbar [B,Hh,Nb,D] from a mask workspace.  Both are
     stored transposed, [B,Hh,D,Nbp] with Nbp = Nb rounded up to 4; the
-    returned kbar is a strided view of its first Nb columns)."""
+    returned tensors are strided views of their first Nb columns."""
     f = workspace.view(torch.float32)
-    n = B * Hh * Nb * D
     nbp = (Nb + 3) // 4 * 4
-    kt = f[n:n + B * Hh * D * nbp].view(B, Hh, D, nbp)
-    return f[:n].view(B, Hh, Nb, D), kt[..., :Nb].transpose(2, 3)
+    n = B * Hh * D * nbp
+    qt = f[:n].view(B, Hh, D, nbp)
+    kt = f[n:2 * n].view(B, Hh, D, nbp)
+    return qt[..., :Nb].transpose(2, 3), kt[..., :Nb].transpose(2, 3)
 
 
 def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_count: torch.Tensor,
@@ -385,6 +416,77 @@ def sparse_attn_bwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, out: t
         _check(lib().nabla_sparse_attn_bwd_grid(*ptrs, B, Hh, D, T, H, W, float(scale), *outs),
                "nabla_sparse_attn_bwd_grid")
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- AB-Attention
+AB_QBLOCK = 128
+AB_KBLOCK = 4
+AB_CLUSTERS = 8
+
+
+def ab_workspace_bytes(B: int, S: int, Hh: int, D: int) -> int:
+    return int(lib().nabla_ab_workspace_bytes(B, S, Hh, D))
+
+
+def ab_plan(q: torch.Tensor, k: torch.Tensor, u: torch.Tensor, budget: float, kmeans_iters: int = 4,
+            scale: float = 0.0, kcount=None, kidx=None, kshift=None, workspace=None, stream=None):
+    """The AB-Attention sampling plan (nabla_ab_plan) for Q, K [B, S, Hh, D]
+    in grid order and uniforms u fp32 [B, Hh, S/128, S/4].  Returns (kcount
+    int32 [B,Hh,NQB], kidx int32 [B,Hh,NQB,NKB], kshift fp32 [B,Hh,NQB,NKB],
+    workspace; see :func:`ab_views`)."""
+    B, S, Hh, D = q.shape
+    nqb, nkb = S // AB_QBLOCK, S // AB_KBLOCK
+    dev = q.device
+    kcount = torch.empty((B, Hh, nqb), dtype=torch.int32, device=dev) if kcount is None else kcount
+    kidx = torch.empty((B, Hh, nqb, nkb), dtype=torch.int32, device=dev) if kidx is None else kidx
+    kshift = torch.empty((B, Hh, nqb, nkb), dtype=torch.float32, device=dev) if kshift is None else kshift
+    if workspace is None:
+        nbytes = ab_workspace_bytes(B, S, Hh, D)
+        if nbytes == 0:
+            raise NablaError(NABLA_ERR_INVALID, "nabla_ab_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(lib().nabla_ab_plan(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), _dev(u, torch.float32, "u"),
+                               B, S, Hh, D, int(kmeans_iters), float(budget), float(scale),
+                               _dev(kcount, torch.int32, "kcount"), _dev(kidx, torch.int32, "kidx"),
+                               _dev(kshift, torch.float32, "kshift"), _dev(workspace, torch.uint8, "workspace"),
+                               _stream(stream)), "nabla_ab_plan")
+    return kcount, kidx, kshift, workspace
+
+
+def ab_views(workspace: torch.Tensor, B: int, S: int, Hh: int, D: int):
+    """Views into an AB plan workspace: (kbar [B,Hh,NKB,D], cent [B,Hh,NQB,8,D]
+    (both strided views of the transposed storage), counts int32
+    [B,Hh,NQB,8], logits fp32 [B,Hh,NQB*8,NKB])."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    nkb, nqb = S // AB_KBLOCK, S // AB_QBLOCK
+    R = nqb * AB_CLUSTERS
+    bh = B * Hh
+    o_cent = up(bh * D * nkb * 4)
+    o_counts = o_cent + up(bh * D * R * 4)
+    o_logits = o_counts + up(bh * nqb * AB_CLUSTERS * 4)
+    kt = workspace[:bh * D * nkb * 4].view(torch.float32).view(B, Hh, D, nkb)
+    ct = workspace[o_cent:o_cent + bh * D * R * 4].view(torch.float32).view(B, Hh, D, nqb, AB_CLUSTERS)
+    counts = workspace[o_counts:o_counts + bh * nqb * AB_CLUSTERS * 4].view(torch.int32).view(B, Hh, nqb, AB_CLUSTERS)
+    logits = workspace[o_logits:o_logits + bh * R * nkb * 4].view(torch.float32).view(B, Hh, R, nkb)
+    return kt.transpose(2, 3), ct.permute(0, 1, 3, 4, 2), counts, logits
+
+
+def ab_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kcount: torch.Tensor, kidx: torch.Tensor,
+                kshift: torch.Tensor, scale: float = 0.0, out=None, lse=None, want_lse: bool = True, stream=None):
+    """AB-Attention forward on the sampled 4-token key blocks with their
+    logit shifts (nabla_ab_attn_fwd); grid-order tensors in and out.
+    Returns (out, lse or None)."""
+    B, S, Hh, D = q.shape
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hh, S), dtype=torch.float32, device=q.device)
+    lse_p = _dev(lse, torch.float32, "lse") if lse is not None else None
+    _check(lib().nabla_ab_attn_fwd(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                   _dev(v, torch.bfloat16, "v"), _dev(kcount, torch.int32, "kcount"),
+                                   _dev(kidx, torch.int32, "kidx"), _dev(kshift, torch.float32, "kshift"), B, S, Hh,
+                                   D, float(scale), _dev(out, torch.bfloat16, "out"), lse_p, _stream(stream)),
+           "nabla_ab_attn_fwd")
+    return out, lse
 
 
 def get_status(stream=None) -> int:

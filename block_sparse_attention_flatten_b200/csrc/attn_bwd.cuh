@@ -163,19 +163,6 @@ __device__ __forceinline__ int64_t block_row(int r, int W) {
   return W > 0 ? static_cast<int64_t>(r >> 3) * W + (r & 7) : r;
 }
 
-// Asynchronous global -> shared copies (cp.async): the data lands after the
-// committing thread's cp.async.wait_group, and is visible to the CTA after
-// the __syncthreads that follows.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// waits until at most one committed group of this thread is still in flight
-__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
 // stage_tile with asynchronous copies.
 template <int D>
 __device__ __forceinline__ void stage_tile_async(__nv_bfloat16* dst, const __nv_bfloat16* src_row0, int row_elems,

@@ -1,25 +1,23 @@
 // Adaptive block mask (NABLA technical summary, "Metodologia: NABLA", item 2
 // "Construcao de Mascara Adaptativa" and item 3 "Integracao Hibrida com STA").
 //
-// pool_kernel       Downsampling: per 64-token block the fp32 mean of the
-//                   flattened queries and keys (Q and K read once from HBM),
-//                   optionally fused with their fractal flattening.
-// mask_rows_kernel  Reduced attention, CDF threshold, STA union and block-CSR
-//                   compaction, R query-block rows per CTA:
-//   1. scores s_ij = (qbar_i . kbar_j) * scale (fp32 FMA chain over d) into
-//      shared memory, one row of Nb scores per query block;
-//   2. softmax numerators per row (one warp per row): max, e = expf(s - max);
-//      p = e / sum(e) is never formed: the order of e is the order of p, and
-//      the masses are integers e * 2^40, so every partial sum is exact and
-//      independent of summation order;
-//   3. the CDF rule "keep where the ascending cumulative mass exceeds 1 - thr"
-//      without a full sort: a search over the fp32 bit patterns of e, two
-//      bits per pass, with warp-summed exact masses finds the boundary
-//      element (e*, j*) of the ascending (e, j) order (shared-memory
-//      histograms with atomics serialise on the few bins most masses fall
-//      into);
-//   4. keep = (e, j) >= (e*, j*)  OR arg-max  OR STA window, compacted with
-//      warp ballots into ascending kv_idx and kv_count.
+// pool_kernel         Downsampling: per 64-token block the fp32 mean of the
+//                     flattened queries and keys (Q and K read once from
+//                     HBM), optionally fused with their fractal flattening.
+// score_tile_kernel   Reduced attention scores s_ij = (qbar_i . kbar_j) *
+//                     scale as a tiled fp32 GEMM (128 x 128 tiles, the
+//                     oracle's FMA chain per entry) into a score scratch.
+// select_rows_kernel  Per row (one warp): softmax numerators, the CDF
+//                     threshold, STA union and block-CSR compaction.
+// mask_rows_smem_kernel  Both stages in one kernel with the score rows in
+//                     shared memory (no scratch), for callers without one.
+// sta_lists_kernel, radial_lists_kernel  The static windows alone as lists.
+// The selection (select_row) never forms p = e / sum(e) and never sorts the
+// row: the order of e is the order of p, the masses are integers e * 2^40
+// (every partial sum exact and independent of summation order), and the
+// boundary element (e*, j*) of the ascending (e, j) order is found by
+// 32-way mass histograms over the bit patterns of e, then a warp sort of
+// the last <= 32 candidates; keep = (e, j) >= (e*, j*) OR arg-max OR STA.
 #pragma once
 
 #include "common.cuh"
@@ -88,51 +86,87 @@ __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restri
         }
       }
     }
+    // transposed, xbar^T [B][Hh][D][Nbp]: the score stages read a d-slice of
+    // consecutive blocks as one contiguous run
     const int col = c * 8;
     const int h = col / D, d = col - h * D;
-    if (blockIdx.z == 0) {
-      float4* o = reinterpret_cast<float4*>(out + ((static_cast<int64_t>(b) * Hh + h) * Nb + i) * D + d);
-      o[0] = make_float4(acc[0] * (1.f / 64.f), acc[1] * (1.f / 64.f), acc[2] * (1.f / 64.f), acc[3] * (1.f / 64.f));
-      o[1] = make_float4(acc[4] * (1.f / 64.f), acc[5] * (1.f / 64.f), acc[6] * (1.f / 64.f), acc[7] * (1.f / 64.f));
-    } else {
-      // keys transposed: kbar^T [B][Hh][D][Nbp], so the score phase reads
-      // them coalesced along the key blocks
-      const int Nbp = (Nb + 3) & ~3;
-      float* o = out + ((static_cast<int64_t>(b) * Hh + h) * D + d) * Nbp + i;
+    const int Nbp = (Nb + 3) & ~3;
+    float* o = out + ((static_cast<int64_t>(b) * Hh + h) * D + d) * Nbp + i;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[static_cast<int64_t>(e) * Nbp] = acc[e] * (1.f / 64.f);
-    }
+    for (int e = 0; e < 8; ++e) o[static_cast<int64_t>(e) * Nbp] = acc[e] * (1.f / 64.f);
   }
 }
 
 // -------------------------------------------------------------- mask rows
 struct MaskArgs {
-  const float* qbar;  // [B][Hh][Nb][D]
-  const float* kbar;
+  const float* qbar;  // pooled queries, transposed: [B][Hh][D][Nbp]
+  const float* kbar;  // pooled keys, transposed:    [B][Hh][D][Nbp]
   int32_t* kv_count;  // [B][Hh][Nb]
   int32_t* kv_idx;    // [B][Hh][Nb][Nb]
   int Hh, Nb, D;
   int nbh, nbw;       // blocks per frame row / column
   int sta_rt, sta_rh, sta_rw;  // STA half-widths; sta_on = 0 disables
   int sta_on;
+  int radial_r0;      // radial window half-width at temporal distance 0; 0 disables
   int keep_all;       // thr >= 1
   float scale;
   double tau;         // 1 - thr (exact in double)
 };
 
+// Temporal band of the radial window: floor(log2(dt + 1)); its spatial
+// half-width is r0 >> band (the window halves each time dt + 1 doubles).
+__host__ __device__ __forceinline__ int radial_band(int dt) {
+  int r = 0;
+  while ((dt + 1) >> (r + 1)) ++r;
+  return r;
+}
+
+// Calls f(j) for every block j of the radial window of block i (frame ti,
+// patch row hi, column wi): per frame tj the box of half-width
+// r0 >> radial_band(|ti - tj|) around (hi, wi), clipped to the grid; e runs
+// over the box's entries in (row, column) order.  f receives (j, position
+// in the ascending list).  Returns the window's size.
+template <class F>
+__device__ __forceinline__ int radial_for_each(int ti, int hi, int wi, int nbt, int nbh, int nbw, int r0, int lane,
+                                              const F& f) {
+  int n = 0;
+  for (int tj = 0; tj < nbt; ++tj) {
+    const int rho = r0 >> radial_band(abs(ti - tj));
+    const int h0 = max(hi - rho, 0), h1 = min(hi + rho, nbh - 1);
+    const int w0 = max(wi - rho, 0), w1 = min(wi + rho, nbw - 1);
+    const int nw = w1 - w0 + 1, cnt = (h1 - h0 + 1) * nw;
+    for (int e = lane; e < cnt; e += 32) {
+      const int eh = e / nw;
+      f((tj * nbh + h0 + eh) * nbw + w0 + (e - eh * nw), n + e);
+    }
+    n += cnt;
+  }
+  return n;
+}
+
 constexpr int kMaskThreads = 256;
 constexpr int kMaskWarps = kMaskThreads / 32;
-constexpr int kMaskCols = 4;  // adjacent key blocks per thread in the score phase
+constexpr int kMaskCols = 4;  // adjacent key blocks per thread in the in-shared-memory score phase
 
-// Column count of the transposed pooled keys kbar^T [D][Nbp]: Nb rounded up
-// to a multiple of 4 so every thread's four columns are an aligned 16-byte
-// load.
+// Columns of the transposed pooled vectors and row stride of the score
+// scratch: Nb rounded up to a multiple of 4, so every row starts 16-byte
+// aligned and is read and written as float4.
 __host__ __device__ inline int kbar_cols(int Nb) { return (Nb + 3) & ~3; }
+
+// Shared memory one warp needs to select one row: private mass histograms
+// [32 digits][32 lanes] (u64), 32 candidate slots, the row (Nbp floats).
+__host__ __device__ inline size_t select_warp_bytes(int Nb) {
+  return 32 * 32 * 8 + 32 * 4 + static_cast<size_t>(kbar_cols(Nb)) * 4;
+}
 
 // d = a * b + d on two fp32 lanes at once; each lane is one fmaf (round to
 // nearest even), so a lane's chain of these equals the scalar fmaf chain.
 __device__ __forceinline__ void ffma2(unsigned long long& d, unsigned long long a, unsigned long long b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ unsigned long long dup2(float x) {
+  const unsigned long long u = __float_as_uint(x);
+  return (u << 32) | u;
 }
 
 // Integer mass of an unnormalised probability e in [0, 1], from its bit
@@ -152,37 +186,578 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
-// R query-block rows per CTA, 256 threads.  Shared memory: q pairs [D][R]
-// (each fp32 qbar value twice, the second operand of a two-lane FMA), score
-// rows [R][Nb], per-warp candidate slots.
+// The softmax numerator exp(x) correctly rounded to fp32 (evaluated in
+// fp64, then rounded once), as the mask's reading of the method defines it.
+// CUDA's expf is within 2 ulp of it; the selection below uses expf and
+// switches to this value wherever 2 ulp could change a decision.
+__device__ __forceinline__ float exp_rounded(float x) { return __double2float_rn(exp(static_cast<double>(x))); }
+
+constexpr uint32_t kOneBits = 0x3F800000u;                // 1.0f
+constexpr uint32_t kNearOneBits = kOneBits - 8u;         // within 8 ulp below 1.0
+constexpr uint32_t kDigit0Lo = 0x30800000u;              // 2^-30: start of the first histogram's range
+constexpr int kWindowUlps = 8;                           // > 2 ulp (expf) on either side, with margin
+constexpr unsigned long long kInfKey = 0x7F800000ull << 32;
+
+// Adds mass w to digit dg of this lane's private histogram column, through a
+// one-entry register cache: runs of equal digits (neighbouring blocks) cost
+// one shared-memory update.
+struct HistCache {
+  int d = -1;
+  unsigned long long w = 0;
+  __device__ __forceinline__ void add(unsigned long long* hist, int lane, int dg, unsigned long long m) {
+    if (dg != d) {
+      if (d >= 0) hist[d * 32 + lane] += w;
+      d = dg;
+      w = 0;
+    }
+    w += m;
+  }
+  __device__ __forceinline__ void flush(unsigned long long* hist, int lane) {
+    if (d >= 0) hist[d * 32 + lane] += w;
+    d = -1;
+    w = 0;
+  }
+};
+
+__device__ __forceinline__ void hist_clear(unsigned long long* hist, int lane) {
+#pragma unroll
+  for (int d = 0; d < 32; ++d) hist[d * 32 + lane] = 0ull;
+}
+
+// From a histogram of the range [lo, lo + 32 << sh) (digit = (u - lo) >> sh)
+// and the mass below lo, picks the digit holding the CDF boundary: the first
+// digit whose inclusive cumulative mass exceeds tau_m.  Updates lo and
+// below.  Lane d sums digit d's column, reading the lanes' entries in a
+// rotated order (no bank conflicts beyond the 64-bit pairing).
+__device__ __forceinline__ void hist_choose(const unsigned long long* hist, int lane, int sh, unsigned long long tau_m,
+                                            uint32_t& lo, unsigned long long& below) {
+  __syncwarp();
+  unsigned long long hd = 0;
+#pragma unroll 8
+  for (int k = 0; k < 32; ++k) hd += hist[lane * 32 + ((k + lane) & 31)];
+  unsigned long long incl = hd;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  incl += below;
+  const int dstar = __popc(__ballot_sync(0xffffffffu, incl <= tau_m));  // < 32: the range holds the crossing
+  const unsigned long long prev = __shfl_sync(0xffffffffu, incl, dstar > 0 ? dstar - 1 : 0);
+  if (dstar > 0) below = prev;
+  lo += static_cast<uint32_t>(dstar) << sh;
+}
+
+// Ascending warp bitonic sort of up to 32 (key, mass) pairs (lanes >= n hold
+// key ~0), then the key of the first lane whose cumulative mass, on top of
+// `base`, exceeds tau_m (~0 if none).
+__device__ __forceinline__ unsigned long long sort_and_cross(unsigned long long key, unsigned long long w, int lane,
+                                                             unsigned long long base, unsigned long long tau_m,
+                                                             unsigned long long* lane_key, unsigned long long* lane_w) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const unsigned long long okey = __shfl_xor_sync(0xffffffffu, key, stride);
+      const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
+      const bool up = (lane & size) == 0;
+      const bool lower = (lane & stride) == 0;
+      if (lower == up ? (okey < key) : (okey > key)) {
+        key = okey;
+        w = ow;
+      }
+    }
+  }
+  unsigned long long cw = w;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, cw, o);
+    if (lane >= o) cw += v;
+  }
+  *lane_key = key;
+  *lane_w = w;
+  const unsigned hit = __ballot_sync(0xffffffffu, key != ~0ull && base + cw > tau_m);
+  return hit ? __shfl_sync(0xffffffffu, key, __ffs(hit) - 1) : ~0ull;
+}
+
+// Numerator pass: row[j] <- e_j = exp(s_j - m) for j < Nbp (padding scores
+// are -inf, so their e is 0), with the level-0 histogram of masses over the
+// binades [2^-30, 2) (digit = (bits(e) - bits(2^-30)) >> 23; smaller e go to
+// `low`).  kExact: every e is the correctly rounded value, the scores read
+// through score_of (the row already holds numerators); otherwise e = expf,
+// except within 8 ulp of 1 where the correctly rounded value is used, so
+// the set of blocks with e == 1 (the arg-max ties) is exact.
+// Returns the arg-max (largest j with e == 1) and the warp-total masses.
+template <bool kExact, class ScoreFn>
+__device__ __forceinline__ int numerator_pass(float* row, unsigned long long* hist, int Nb, int Nbp, float m,
+                                              const ScoreFn& score_of, unsigned long long& total,
+                                              unsigned long long& low) {
+  const int lane = threadIdx.x & 31;
+  float4* row4 = reinterpret_cast<float4*>(row);
+  hist_clear(hist, lane);
+  HistCache hc;
+  total = 0;
+  low = 0;
+  int amax = -1;
+  for (int c = lane; c < (Nbp >> 2); c += 32) {
+    float ev[4];
+    if (kExact) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) ev[t] = 4 * c + t < Nb ? score_of(4 * c + t) : -INFINITY;
+    } else {
+      const float4 v = row4[c];
+      ev[0] = v.x;
+      ev[1] = v.y;
+      ev[2] = v.z;
+      ev[3] = v.w;
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float x = __fsub_rn(ev[t], m);
+      float e = kExact ? exp_rounded(x) : expf(x);
+      uint32_t u = __float_as_uint(e);
+      if (!kExact && u >= kNearOneBits) {
+        e = exp_rounded(x);
+        u = __float_as_uint(e);
+      }
+      ev[t] = e;
+      if (u == kOneBits) amax = 4 * c + t;
+      const unsigned long long w = mass_bits(u);
+      total += w;
+      const uint32_t dg = (u - kDigit0Lo) >> 23;
+      if (dg < 32u)
+        hc.add(hist, lane, static_cast<int>(dg), w);
+      else
+        low += w;
+    }
+    row4[c] = make_float4(ev[0], ev[1], ev[2], ev[3]);
+  }
+  hc.flush(hist, lane);
+  total = warp_sum_u64(total);
+  low = warp_sum_u64(low);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  __syncwarp();
+  return amax;
+}
+
+// The CDF boundary of a row of numerators: the element (e*, j*) of the
+// ascending (e, j) order at which the cumulative integer mass first exceeds
+// tau_m (keep (e, j) >= (e*, j*)).  Returns its key (bits(e) << 32 | j).
+// The range holding bits(e*) is narrowed by 32-way mass histograms (one
+// pass over the row each, 5 bits at a time: the first comes with the
+// numerators), gathering the elements of the current range on the way;
+// once at most 32 remain they are sorted in the warp.  More than 32 equal
+// values: the boundary is the need-th smallest index among them.
+// Requires tau_m < total; `low` is the mass below 2^-30.
+__device__ __forceinline__ unsigned long long cdf_boundary(const float* row, unsigned long long* hist, int* cand, int Nbp,
+                                           unsigned long long tau_m, unsigned long long low, uint32_t* range_lo,
+                                           int* range_span, unsigned long long* range_below,
+                                           unsigned long long* lane_key, unsigned long long* lane_w) {
+  const int lane = threadIdx.x & 31;
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+  uint32_t lo;
+  int span;
+  unsigned long long below;
+  if (low > tau_m) {  // the boundary lies below 2^-30: start over on [0, 2^30)
+    lo = 0;
+    span = 30;
+    below = 0;
+  } else {
+    lo = kDigit0Lo;
+    below = low;
+    hist_choose(hist, lane, 23, tau_m, lo, below);
+    span = 23;
+  }
+  int n = 0;
+  while (true) {
+    // one pass: gather the range's elements, histogram them one level down
+    const int sh = span > 5 ? span - 5 : 0;
+    const uint32_t width = 1u << span;
+    hist_clear(hist, lane);
+    HistCache hc;
+    n = 0;
+    for (int c = lane; c - lane < (Nbp >> 2); c += 32) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      const bool live = c < (Nbp >> 2);
+      if (live) v = row4[c];
+      const float ev[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t u = __float_as_uint(ev[t]);
+        const uint32_t d = u - lo;
+        const bool in = live && d < width;
+        const unsigned bal = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const int pos = n + __popc(bal & ((1u << lane) - 1u));
+          if (pos < 32) cand[pos] = 4 * c + t;
+          hc.add(hist, lane, static_cast<int>(d >> sh), mass_bits(u));
+        }
+        n += __popc(bal);
+      }
+    }
+    hc.flush(hist, lane);
+    __syncwarp();
+    if (n <= 32 || span == 0) break;
+    hist_choose(hist, lane, sh, tau_m, lo, below);
+    span = sh;
+  }
+  *range_lo = lo;
+  *range_span = span;
+  *range_below = below;
+  if (n <= 32) {
+    unsigned long long key = ~0ull, w = 0ull;
+    if (lane < n) {
+      const int j = cand[lane];
+      const uint32_t u = __float_as_uint(row[j]);
+      key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
+      w = mass_bits(u);
+    }
+    __syncwarp();
+    return sort_and_cross(key, w, lane, below, tau_m, lane_key, lane_w);
+  }
+  // more than 32 elements share the value lo
+  *lane_key = ~0ull;
+  *lane_w = 0;
+  const unsigned long long wstar = mass_bits(lo);
+  const unsigned long long need = (tau_m - below) / wstar + 1ull;
+  unsigned long long seen = 0;
+  int jstar = -1;
+  for (int base = 0; base < Nbp && jstar < 0; base += 32) {
+    const int j = base + lane;
+    const bool hit = j < Nbp && __float_as_uint(row[j]) == lo;
+    const unsigned bal = __ballot_sync(0xffffffffu, hit);
+    const unsigned c = __popc(bal);
+    if (seen + c >= need) {
+      unsigned bb = bal;
+      for (unsigned long long t = seen + 1; t < need; ++t) bb &= bb - 1;  // drop lower hits
+      jstar = base + __ffs(bb) - 1;
+    }
+    seen += c;
+  }
+  return (static_cast<unsigned long long>(lo) << 32) | static_cast<unsigned>(jstar);
+}
+
+// Selects the kept blocks of query block i from its scores, one warp:
+//   1. m = max_j s_j;
+//   2. e_j = exp(s_j - m) (numerator_pass), the masses floor(e * 2^40) and
+//      their total; the arg-max;
+//   3. the CDF boundary (cdf_boundary) on these e;
+//   4. exactness: e_j differs from the correctly rounded value by at most
+//      2 ulp, so the order statistics shift by at most 2 ulp and only blocks
+//      within 8 ulp of the boundary value B can be ordered differently.
+//      Those (gathered from the last range, or by one more pass) get the
+//      correctly rounded e (scores re-read through score_of) and are sorted
+//      again on top of the mass below B - 8 ulp: the boundary is then the
+//      one of the exact order.  (More than 32 such blocks: the whole row is
+//      recomputed exactly and searched again.)
+//   5. STA window blocks marked +inf, then keep = (e, j) >= (e*, j*), the
+//      arg-max, or the window, compacted ascending with warp ballots.
+// row: Nbp scores in shared memory, -inf past Nb; overwritten.
+template <class ScoreFn>
+__device__ __forceinline__ void select_row(float* row, unsigned long long* hist, int* cand, int Nb, int i, const MaskArgs& a,
+                           int32_t* out, int32_t* count_out, const ScoreFn& score_of) {
+  const int lane = threadIdx.x & 31;
+  const int Nbp = kbar_cols(Nb);
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+  float m = -INFINITY;
+  for (int c = lane; c < (Nbp >> 2); c += 32) {
+    const float4 v = row4[c];
+    m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+
+  unsigned long long total, low;
+  int argmax = numerator_pass<false>(row, hist, Nb, Nbp, m, score_of, total, low);
+  unsigned long long tau_m = static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
+  unsigned long long kstar = kInfKey;  // thr = 0: the CDF keeps nothing but the arg-max
+  if (!a.keep_all && total > tau_m) {
+    uint32_t lo;
+    int span;
+    unsigned long long below, lkey, lw;
+    const unsigned long long kfast = cdf_boundary(row, hist, cand, Nbp, tau_m, low, &lo, &span, &below, &lkey, &lw);
+    const uint32_t B = static_cast<uint32_t>(kfast >> 32);
+    const uint32_t wlo = B - kWindowUlps, whi = B + kWindowUlps;
+    // the window's blocks and the mass below it
+    unsigned long long base = 0;
+    int nw = 0;
+    unsigned long long wkey = ~0ull;
+    if (wlo >= lo && whi - lo < (1u << span)) {
+      // the last range held every block of the window, sorted in lkey/lw
+      const uint32_t u = static_cast<uint32_t>(lkey >> 32);
+      const bool inw = lkey != ~0ull && u >= wlo && u <= whi;
+      base = below + warp_sum_u64(lkey != ~0ull && u < wlo ? lw : 0ull);
+      const unsigned bal = __ballot_sync(0xffffffffu, inw);
+      nw = __popc(bal);
+      if (inw) cand[__popc(bal & ((1u << lane) - 1u))] = static_cast<int>(lkey & 0xffffffffu);
+    } else {
+      unsigned long long ml = 0;
+      for (int base_j = 0; base_j < Nbp; base_j += 32) {
+        const int j = base_j + lane;
+        const uint32_t u = j < Nbp ? __float_as_uint(row[j]) : 0u;
+        if (u < wlo) ml += mass_bits(u);
+        const bool inw = u >= wlo && u <= whi;
+        const unsigned bal = __ballot_sync(0xffffffffu, inw);
+        if (inw && nw + __popc(bal & ((1u << lane) - 1u)) < 32) cand[nw + __popc(bal & ((1u << lane) - 1u))] = j;
+        nw += __popc(bal);
+      }
+      base = warp_sum_u64(ml);
+    }
+    __syncwarp();
+    if (nw <= 32) {
+      unsigned long long w = 0;
+      if (lane < nw) {
+        const int j = cand[lane];
+        const float e = exp_rounded(__fsub_rn(score_of(j), m));
+        row[j] = e;
+        const uint32_t u = __float_as_uint(e);
+        wkey = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
+        w = mass_bits(u);
+      }
+      __syncwarp();
+      unsigned long long k2, w2;
+      kstar = sort_and_cross(wkey, w, lane, base, tau_m, &k2, &w2);
+      if (kstar == ~0ull) kstar = kfast;  // crossing outside the window: a band block, either is allowed
+    } else {
+      // many blocks within a few ulp of the boundary: exact numerators for the
+      // whole row, then the search again (no window step needed)
+      argmax = numerator_pass<true>(row, hist, Nb, Nbp, m, score_of, total, low);
+      tau_m = static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
+      kstar = kInfKey;
+      if (total > tau_m) kstar = cdf_boundary(row, hist, cand, Nbp, tau_m, low, &lo, &span, &below, &lkey, &lw);
+    }
+    __syncwarp();
+  }
+
+  if (a.sta_on) {
+    const int per_t = a.nbh * a.nbw;
+    const int nbt = Nb / per_t;
+    const int ti = i / per_t, hi = (i - ti * per_t) / a.nbw, wi = i - ti * per_t - hi * a.nbw;
+    const int wh = 2 * a.sta_rh + 1, ww = 2 * a.sta_rw + 1, plane = wh * ww;
+    const int nwin = (2 * a.sta_rt + 1) * plane;
+    for (int e = lane; e < nwin; e += 32) {
+      const int et = e / plane, ehw = e - et * plane, eh = ehw / ww;
+      const int tj = ti + et - a.sta_rt, hj = hi + eh - a.sta_rh, wj = wi + (ehw - eh * ww) - a.sta_rw;
+      if (tj >= 0 && tj < nbt && hj >= 0 && hj < a.nbh && wj >= 0 && wj < a.nbw)
+        row[tj * per_t + hj * a.nbw + wj] = __uint_as_float(0x7F800000u);
+    }
+    __syncwarp();
+  }
+  if (a.radial_r0 > 0) {
+    const int per_t = a.nbh * a.nbw;
+    const int ti = i / per_t, hi = (i - ti * per_t) / a.nbw, wi = i - ti * per_t - hi * a.nbw;
+    radial_for_each(ti, hi, wi, Nb / per_t, a.nbh, a.nbw, a.radial_r0, lane,
+                    [row](int j, int) { row[j] = __uint_as_float(0x7F800000u); });
+    __syncwarp();
+  }
+  int count = 0;
+  for (int base_j = 0; base_j < Nb; base_j += 32) {
+    const int j = base_j + lane;
+    bool keep = false;
+    if (j < Nb) {
+      const unsigned long long key =
+          (static_cast<unsigned long long>(__float_as_uint(row[j])) << 32) | static_cast<unsigned>(j);
+      keep = a.keep_all || key >= kstar || j == argmax;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[count + __popc(bal & ((1u << lane) - 1u))] = j;
+    count += __popc(bal);
+  }
+  if (lane == 0) *count_out = count;
+  __syncwarp();
+}
+
+// ------------------------------------------------- scores as a tiled GEMM
+// s_ij = (qbar_i . kbar_j) * scale for a 128 x 128 tile of one (b, head), in
+// the oracle's arithmetic: per (i, j) one fp32 fused multiply-add chain over
+// d ascending (two lanes per fma.rn.f32x2, each rounding like fmaf), then one
+// fp32 multiply.  256 threads; thread (ty, tx) = (tid / 16, tid % 16) owns
+// rows {4ty..4ty+3, 64+4ty..64+4ty+3} and columns {4tx..4tx+3,
+// 64+4tx..64+4tx+3}.  32-deep slices of qbar^T and kbar^T are staged in
+// shared memory by cp.async (two stages, zero fill past Nbp); each d step
+// reads 4 x 16 bytes of shared memory per thread for 64 multiply-adds.
+// Scores go to the scratch, per (b, head) [nrows][out_ld]; for the mask
+// [Nb][Nbp] (columns Nb..Nbp are padding).
+constexpr int kScoreTile = 128;
+constexpr int kScoreKc = 32;
+constexpr int kScoreThreads = 256;
+constexpr int kScoreStageFloats = 2 * kScoreKc * kScoreTile;
+constexpr size_t kScoreSmemBytes = 2 * kScoreStageFloats * sizeof(float);
+
+// Shapes of one score GEMM: rows of A = qT columns, rows of B = kT
+// columns; both operands transposed ([D][ld] per (b, head)), the output
+// [nrows][out_ld] per (b, head).  Leading dimensions are multiples of 4.
+struct ScoreShape {
+  int nrows, ncols, D;
+  int q_ld, k_ld, out_ld;
+  int64_t q_bh, k_bh, out_bh;  // element strides between (b, head) slices
+};
+
+__global__ void __launch_bounds__(kScoreThreads, 2)
+    score_tile_kernel(const float* __restrict__ qT, const float* __restrict__ kT, float* __restrict__ scores,
+                      const ScoreShape sh, float scale) {
+  extern __shared__ __align__(16) float ssm[];
+  const int j0 = blockIdx.x * kScoreTile, i0 = blockIdx.y * kScoreTile;
+  const int64_t bh = blockIdx.z;
+  const int D = sh.D;
+  const float* qs = qT + bh * sh.q_bh;
+  const float* ks = kT + bh * sh.k_bh;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+
+  auto load_stage = [&](int st, int d0) {
+    float* dst = ssm + st * kScoreStageFloats;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = tid + u * kScoreThreads;  // 16-byte chunk: [Q|K][dd][col4]
+      const int which = c >> 10, rem = c & 1023;
+      const int dd = rem >> 5, col = (rem & 31) * 4;
+      const int g = (which ? j0 : i0) + col;
+      const int ld = which ? sh.k_ld : sh.q_ld;
+      const bool ok = g < ld;  // ld % 4 == 0: the chunk is wholly in or out
+      const float* src = (which ? ks : qs) + static_cast<int64_t>(d0 + dd) * ld + (ok ? g : 0);
+      cp_async16_zfill(dst + which * kScoreKc * kScoreTile + dd * kScoreTile + col, src, ok);
+    }
+    cp_async_commit();
+  };
+
+  unsigned long long acc[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0ull;
+
+  const int nk = D / kScoreKc;
+  load_stage(0, 0);
+  if (nk > 1) load_stage(1, kScoreKc);
+  for (int kc = 0; kc < nk; ++kc) {
+    if (kc + 1 < nk)
+      cp_async_wait<1>();
+    else
+      cp_async_wait<0>();
+    __syncthreads();
+    const float* sq = ssm + (kc & 1) * kScoreStageFloats;
+    const float* sk = sq + kScoreKc * kScoreTile;
+#pragma unroll 4
+    for (int dd = 0; dd < kScoreKc; ++dd) {
+      const float4 qa = *reinterpret_cast<const float4*>(sq + dd * kScoreTile + ty * 4);
+      const float4 qb = *reinterpret_cast<const float4*>(sq + dd * kScoreTile + 64 + ty * 4);
+      const ulonglong2 ka = *reinterpret_cast<const ulonglong2*>(sk + dd * kScoreTile + tx * 4);
+      const ulonglong2 kb = *reinterpret_cast<const ulonglong2*>(sk + dd * kScoreTile + 64 + tx * 4);
+      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const unsigned long long qq = dup2(qv[r]);
+        ffma2(acc[r][0], ka.x, qq);
+        ffma2(acc[r][1], ka.y, qq);
+        ffma2(acc[r][2], kb.x, qq);
+        ffma2(acc[r][3], kb.y, qq);
+      }
+    }
+    __syncthreads();
+    if (kc + 2 < nk) load_stage(kc & 1, (kc + 2) * kScoreKc);
+  }
+
+  auto lo32 = [](unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); };
+  auto hi32 = [](unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); };
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int row = i0 + (r < 4 ? ty * 4 + r : 64 + ty * 4 + (r - 4));
+    if (row >= sh.nrows) continue;
+    float* dst = scores + bh * sh.out_bh + static_cast<int64_t>(row) * sh.out_ld;
+    const int ca = j0 + tx * 4, cb = j0 + 64 + tx * 4;
+    if (ca < sh.out_ld)
+      *reinterpret_cast<float4*>(dst + ca) =
+          make_float4(__fmul_rn(lo32(acc[r][0]), scale), __fmul_rn(hi32(acc[r][0]), scale),
+                      __fmul_rn(lo32(acc[r][1]), scale), __fmul_rn(hi32(acc[r][1]), scale));
+    if (cb < sh.out_ld)
+      *reinterpret_cast<float4*>(dst + cb) =
+          make_float4(__fmul_rn(lo32(acc[r][2]), scale), __fmul_rn(hi32(acc[r][2]), scale),
+                      __fmul_rn(lo32(acc[r][3]), scale), __fmul_rn(hi32(acc[r][3]), scale));
+  }
+}
+
+// Launches score_tile_kernel for every (b, head) slice.
+inline cudaError_t launch_score_tiles(const float* qT, const float* kT, float* out, const ScoreShape& sh, int bhs,
+                                      float scale, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(score_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kScoreSmemBytes));
+  if (e != cudaSuccess) return e;
+  const dim3 grid((sh.ncols + kScoreTile - 1) / kScoreTile, (sh.nrows + kScoreTile - 1) / kScoreTile,
+                  static_cast<unsigned>(bhs));
+  score_tile_kernel<<<grid, kScoreThreads, kScoreSmemBytes, stream>>>(qT, kT, out, sh, scale);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------ selection from the scratch
+// One warp per row of the score scratch (rows taken in reverse order of the
+// score kernel's writes, so the first ones read are still in L2).  Shared
+// memory per warp: select_warp_bytes(Nb).
+__global__ void __launch_bounds__(256) select_rows_kernel(const MaskArgs a, const float* __restrict__ scores,
+                                                          int64_t rows_total) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int Nb = a.Nb, Nbp = kbar_cols(Nb);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  unsigned char* mine = smem_raw + static_cast<size_t>(warp) * select_warp_bytes(Nb);
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(mine);
+  int* cand = reinterpret_cast<int*>(mine + 32 * 32 * 8);
+  float* row = reinterpret_cast<float*>(mine + 32 * 32 * 8 + 32 * 4);
+  const int64_t lin = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
+  if (lin >= rows_total) return;
+  const int64_t rid = rows_total - 1 - lin;
+  const int64_t bh = rid / Nb;
+  const int i = static_cast<int>(rid - bh * Nb);
+  const float* src = scores + rid * Nbp;
+  const float4* src4 = reinterpret_cast<const float4*>(src);
+  float4* row4 = reinterpret_cast<float4*>(row);
+  for (int c = lane; c < (Nbp >> 2); c += 32) {
+    float4 v = __ldcs(src4 + c);
+    if (4 * c + 3 >= Nb) {
+      if (4 * c + 0 >= Nb) v.x = -INFINITY;
+      if (4 * c + 1 >= Nb) v.y = -INFINITY;
+      if (4 * c + 2 >= Nb) v.z = -INFINITY;
+      if (4 * c + 3 >= Nb) v.w = -INFINITY;
+    }
+    row4[c] = v;
+  }
+  __syncwarp();
+  select_row(row, hist, cand, Nb, i, a, a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb), a.kv_count + bh * Nb + i,
+             [src](int j) { return src[j]; });
+}
+
+// ------------------------------------- rows with their scores in shared memory
+// The whole mask stage in one kernel, without a score scratch (used where no
+// scratch can be had): R query-block rows per CTA, 256 threads.  Score
+// phase: each thread owns four adjacent key blocks and all R rows; per
+// (row, block) the same fused multiply-add chain as score_tile_kernel, two
+// blocks per fma.rn.f32x2, qbar held in shared memory as duplicated pairs,
+// kbar^T read from global memory two or four d ahead.  Then each warp
+// selects rows warp, warp + 8, ... with select_row (exact numerators near
+// the boundary from a scalar recomputation of the same chain).
+// Shared memory: q pairs [D][R], score rows [R][Nbp], per-warp selection
+// scratch (histograms, candidates; the rows are the score rows).
 template <int R>
-__global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskArgs a) {
+__global__ void __launch_bounds__(kMaskThreads) mask_rows_smem_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int D = a.D, Nb = a.Nb, Nbp = kbar_cols(Nb);
-  unsigned long long* qd = reinterpret_cast<unsigned long long*>(smem_raw);          // [D][R]
-  float* rows = reinterpret_cast<float*>(qd + static_cast<size_t>(R) * D);          // [R][Nb]
-  int* cand_all = reinterpret_cast<int*>(rows + static_cast<size_t>(R) * Nb);      // [warps][32]
+  unsigned long long* qd = reinterpret_cast<unsigned long long*>(smem_raw);  // [D][R]
+  float* rows = reinterpret_cast<float*>(qd + static_cast<size_t>(R) * D);    // [R][Nbp]
+  unsigned char* sel = reinterpret_cast<unsigned char*>(rows + static_cast<size_t>(R) * Nbp);
 
   const int i0 = blockIdx.x * R;
   const int hd = blockIdx.y, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
-  const float* qb = a.qbar + (bh * Nb + i0) * D;
+  const float* qt = a.qbar + bh * static_cast<int64_t>(D) * Nbp;  // qbar^T [D][Nbp]
   const float* kt = a.kbar + bh * static_cast<int64_t>(D) * Nbp;  // kbar^T [D][Nbp]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
 
   for (int e = tid; e < R * D; e += kMaskThreads) {
-    const int r = e / D, d = e - r * D;
-    const uint32_t u = __float_as_uint((i0 + r < Nb) ? qb[e] : 0.f);
-    qd[d * R + r] = (static_cast<unsigned long long>(u) << 32) | u;
+    const int d = e / R, r = e - d * R;
+    qd[d * R + r] = dup2((i0 + r < Nb) ? qt[static_cast<int64_t>(d) * Nbp + i0 + r] : 0.f);
   }
   __syncthreads();
 
-  // 1. scores: thread owns key blocks j..j+3 and all R rows; per (row, block)
-  //    one fused multiply-add chain over d ascending (the oracle's order),
-  //    two blocks per instruction.  kbar^T rows are read coalesced (16 bytes
-  //    a thread), two or four d ahead of use; each q pair loaded from shared memory
-  //    feeds four two-lane FMAs.
-  for (int j = tid * kMaskCols; j < Nb; j += kMaskThreads * kMaskCols) {
+  for (int j = tid * kMaskCols; j < Nbp; j += kMaskThreads * kMaskCols) {
     unsigned long long acc[R][2];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = 0ull;
@@ -200,14 +775,11 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
         kn[u] = more ? __ldg(kp + static_cast<int64_t>(d0 + PF + u) * kstride) : make_ulonglong2(0ull, 0ull);
 #pragma unroll
       for (int u = 0; u < PF; ++u) {
-        const ulonglong2* qrow = reinterpret_cast<const ulonglong2*>(qd + (d0 + u) * R);
+        const unsigned long long* qrow = qd + (d0 + u) * R;
 #pragma unroll
-        for (int r2 = 0; r2 < R / 2; ++r2) {
-          const ulonglong2 qq = qrow[r2];
-          ffma2(acc[2 * r2][0], kv[u].x, qq.x);
-          ffma2(acc[2 * r2][1], kv[u].y, qq.x);
-          ffma2(acc[2 * r2 + 1][0], kv[u].x, qq.y);
-          ffma2(acc[2 * r2 + 1][1], kv[u].y, qq.y);
+        for (int r = 0; r < R; ++r) {
+          ffma2(acc[r][0], kv[u].x, qrow[r]);
+          ffma2(acc[r][1], kv[u].y, qrow[r]);
         }
       }
 #pragma unroll
@@ -215,255 +787,31 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_rows_kernel(const MaskAr
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      float* row = rows + static_cast<size_t>(r) * Nb;
+      float* row = rows + static_cast<size_t>(r) * Nbp;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const unsigned long long v = acc[r][c >> 1];
-        if (j + c < Nb) row[j + c] = __uint_as_float(static_cast<uint32_t>(c & 1 ? v >> 32 : v)) * a.scale;
+        row[j + c] = j + c < Nb ? __fmul_rn(__uint_as_float(static_cast<uint32_t>(c & 1 ? v >> 32 : v)), a.scale)
+                                : -INFINITY;
       }
     }
   }
   __syncthreads();
 
-  int* cand = cand_all + warp * 32;
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(sel + static_cast<size_t>(warp) * (32 * 32 * 8 + 32 * 4));
+  int* cand = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(hist) + 32 * 32 * 8);
   for (int r = warp; r < R; r += kMaskWarps) {
     const int i = i0 + r;
     if (i >= Nb) break;
-    float* row = rows + static_cast<size_t>(r) * Nb;
-
-    // 2. softmax numerators e = exp(s - max) (<= 1), their total integer
-    //    mass and the arg-max, in one pass
-    float m = -INFINITY;
-    for (int j = lane; j < Nb; j += 32) m = fmaxf(m, row[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    unsigned long long best = 0;  // (bits(e) << 32) | j; max = arg-max, ties to the larger j
-    unsigned long long total = 0;
-    int n_tiny = 0;  // blocks with e < 2^-63
-    // first pass of the boundary search (step 3), on the way: masses and
-    // counts of the quarters [2^-63, 2^-47), [2^-47, 2^-31), [2^-31, 2^-15)
-    // of the starting range [2^-63, 2)
-    unsigned long long fm0 = 0, fm1 = 0, fm2 = 0;
-    int fc0 = 0, fc1 = 0, fc2 = 0;
-    for (int j = lane; j < Nb; j += 32) {
-      const float e = expf(row[j] - m);
-      row[j] = e;
-      const uint32_t u = __float_as_uint(e);
-      const unsigned long long key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
-      best = key > best ? key : best;
-      const unsigned long long w = mass_bits(u);
-      total += w;
-      n_tiny += u < 0x20000000u;
-      const uint32_t q = (u - 0x20000000u) >> 27;  // 0..3 for u in [0x20000000, 0x40000000)
-      fm0 += q == 0 ? w : 0ull;
-      fm1 += q == 1 ? w : 0ull;
-      fm2 += q == 2 ? w : 0ull;
-      fc0 += q == 0;
-      fc1 += q == 1;
-      fc2 += q == 2;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long ob = __shfl_xor_sync(0xffffffffu, best, o);
-      best = ob > best ? ob : best;
-    }
-    total = warp_sum_u64(total);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_tiny += __shfl_xor_sync(0xffffffffu, n_tiny, o);
-    const int argmax = static_cast<int>(best & 0xffffffffu);
-    const unsigned long long tau_m =
-        static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
-
-    // 3. CDF boundary: the element (e*, j*) of the ascending (e, j) order at
-    //    which the cumulative mass first exceeds tau_m; keep (e, j) >= it.
-    //    bits(e*) is the largest bit pattern x with mass(bits(e) < x) <= tau_m
-    //    (positive floats order like their bit patterns).  It is narrowed
-    //    inside a range [prefix, prefix + 2^span), two bits per pass: a pass
-    //    sums, per quarter of the range, the exact masses and counts of the
-    //    blocks in it (warp sums, no atomics; blocks outside the range cost a
-    //    compare).  As soon as at most 32 blocks remain in the range they are
-    //    sorted by a warp bitonic sort and the boundary is read off their
-    //    prefix sums.  Every block with positive mass has e >= 2^-40, so e*
-    //    does too and the search starts at [2^-63, 2): bits(e*) has bit 29
-    //    set and bit 30 clear, and nothing below 2^-63 carries mass.
-    //    When no finite element qualifies (thr = 0: the mass never exceeds
-    //    tau_m = total) the boundary is the smallest key of an STA-marked
-    //    block, +inf: the CDF then keeps nothing but the arg-max, and the
-    //    window is still kept.
-    unsigned long long kstar = 0x7F800000ull << 32;
-    if (!a.keep_all && total > tau_m) {
-      uint32_t prefix = 0x20000000u;
-      int span = 29;
-      unsigned long long below = 0;  // mass(bits(e) < prefix)
-      int n_lo = n_tiny, n_hi = Nb;  // blocks below prefix, below prefix + 2^span
-      // Narrows [prefix, prefix + 2^span) to the quarter (of width 2^lo) that
-      // holds bits(e*), given the masses and counts of its first three
-      // quarters.
-      auto narrow = [&](unsigned long long m0, unsigned long long m1, unsigned long long m2, int c0, int c1, int c2,
-                        int lo) {
-        const unsigned long long s1 = below + m0, s2 = s1 + m1, s3 = s2 + m2;
-        if (s3 <= tau_m) {
-          prefix += 3u << lo;
-          below = s3;
-          n_lo += c0 + c1 + c2;
-        } else if (s2 <= tau_m) {
-          prefix += 2u << lo;
-          below = s2;
-          n_lo += c0 + c1;
-          n_hi = n_lo + c2;
-        } else if (s1 <= tau_m) {
-          prefix += 1u << lo;
-          below = s1;
-          n_lo += c0;
-          n_hi = n_lo + c1;
-        } else {
-          n_hi = n_lo + c0;
-        }
-        span = lo;
-      };
-      if (n_hi - n_lo > 32) {
-        // the first pass was done with the exponentials
-        fm0 = warp_sum_u64(fm0);
-        fm1 = warp_sum_u64(fm1);
-        fm2 = warp_sum_u64(fm2);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          fc0 += __shfl_xor_sync(0xffffffffu, fc0, o);
-          fc1 += __shfl_xor_sync(0xffffffffu, fc1, o);
-          fc2 += __shfl_xor_sync(0xffffffffu, fc2, o);
-        }
-        narrow(fm0, fm1, fm2, fc0, fc1, fc2, 27);
-      }
-      while (span > 0 && n_hi - n_lo > 32) {
-        const int lo = span > 2 ? span - 2 : 0;
-        const uint32_t range = 1u << span;
-        unsigned long long m0 = 0, m1 = 0, m2 = 0;
-        int c0 = 0, c1 = 0, c2 = 0;
-        for (int j = lane; j < Nb; j += 32) {
-          const uint32_t u = __float_as_uint(row[j]);
-          const uint32_t d = u - prefix;
-          if (d < range) {
-            const uint32_t q = d >> lo;
-            const unsigned long long w = mass_bits(u);
-            m0 += q == 0 ? w : 0ull;
-            m1 += q == 1 ? w : 0ull;
-            m2 += q == 2 ? w : 0ull;
-            c0 += q == 0;
-            c1 += q == 1;
-            c2 += q == 2;
-          }
-        }
-        m0 = warp_sum_u64(m0);
-        m1 = warp_sum_u64(m1);
-        m2 = warp_sum_u64(m2);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          c0 += __shfl_xor_sync(0xffffffffu, c0, o);
-          c1 += __shfl_xor_sync(0xffffffffu, c1, o);
-          c2 += __shfl_xor_sync(0xffffffffu, c2, o);
-        }
-        narrow(m0, m1, m2, c0, c1, c2, lo);
-      }
-      const uint32_t range = 1u << span;
-      if (n_hi - n_lo <= 32) {
-        // gather the blocks of the range (ascending j), then sort them
-        int ncand = 0;
-        for (int base = 0; base < Nb && ncand < n_hi - n_lo; base += 32) {
-          const int j = base + lane;
-          const bool hit = j < Nb && __float_as_uint(row[j]) - prefix < range;
-          const unsigned bal = __ballot_sync(0xffffffffu, hit);
-          const int pos = ncand + __popc(bal & ((1u << lane) - 1u));
-          if (hit && pos < 32) cand[pos] = j;
-          ncand += __popc(bal);
-        }
-        __syncwarp();
-        unsigned long long key = ~0ull, w = 0ull;
-        if (lane < ncand) {
-          const int j = cand[lane];
-          const uint32_t u = __float_as_uint(row[j]);
-          key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
-          w = mass_bits(u);
-        }
-        // bitonic sort of (key, w) ascending by key across the warp
-#pragma unroll
-        for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-          for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const unsigned long long okey = __shfl_xor_sync(0xffffffffu, key, stride);
-            const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
-            const bool up = (lane & size) == 0;
-            const bool lower = (lane & stride) == 0;
-            if (lower == up ? (okey < key) : (okey > key)) {
-              key = okey;
-              w = ow;
-            }
-          }
-        }
-        unsigned long long cw = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long v = __shfl_up_sync(0xffffffffu, cw, o);
-          if (lane >= o) cw += v;
-        }
-        // below + (mass of the whole range) > tau_m, so some lane qualifies
-        const unsigned hitb = __ballot_sync(0xffffffffu, lane < ncand && below + cw > tau_m);
-        kstar = __shfl_sync(0xffffffffu, key, __ffs(hitb) - 1);
-      } else {
-        // More than 32 blocks share the value e* = prefix: the boundary is
-        // the need-th smallest index among them.
-        const unsigned long long wstar = mass_bits(prefix);
-        const unsigned long long need = (tau_m - below) / wstar + 1ull;
-        unsigned long long seen = 0;
-        int jstar = Nb;
-        for (int base = 0; base < Nb; base += 32) {
-          const int j = base + lane;
-          const bool hit = j < Nb && __float_as_uint(row[j]) == prefix;
-          const unsigned bal = __ballot_sync(0xffffffffu, hit);
-          const unsigned c = __popc(bal);
-          if (seen + c >= need) {
-            unsigned bb = bal;
-            for (unsigned long long t = seen + 1; t < need; ++t) bb &= bb - 1;  // drop lower hits
-            jstar = base + __ffs(bb) - 1;
-            break;
-          }
-          seen += c;
-        }
-        kstar = (static_cast<unsigned long long>(prefix) << 32) | static_cast<unsigned>(jstar);
-      }
-      __syncwarp();
-    }
-
-    // 4. union with the STA window: the window's blocks get e = +inf, which
-    //    orders above every kept key; then compaction of keep = (e, j) >=
-    //    (e*, j*) or arg-max, ascending j
-    if (a.sta_on) {
-      const int per_t = a.nbh * a.nbw;
-      const int nbt = Nb / per_t;
-      const int ti = i / per_t, hi = (i - ti * per_t) / a.nbw, wi = i - ti * per_t - hi * a.nbw;
-      const int wh = 2 * a.sta_rh + 1, ww = 2 * a.sta_rw + 1, plane = wh * ww;
-      const int nwin = (2 * a.sta_rt + 1) * plane;
-      for (int e = lane; e < nwin; e += 32) {
-        const int et = e / plane, ehw = e - et * plane, eh = ehw / ww;
-        const int tj = ti + et - a.sta_rt, hj = hi + eh - a.sta_rh, wj = wi + (ehw - eh * ww) - a.sta_rw;
-        if (tj >= 0 && tj < nbt && hj >= 0 && hj < a.nbh && wj >= 0 && wj < a.nbw)
-          row[tj * per_t + hj * a.nbw + wj] = __uint_as_float(0x7F800000u);
-      }
-      __syncwarp();
-    }
-    int32_t* out = a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb);
-    int count = 0;
-    for (int base = 0; base < Nb; base += 32) {
-      const int j = base + lane;
-      bool keep = false;
-      if (j < Nb) {
-        const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(row[j])) << 32) | static_cast<unsigned>(j);
-        keep = a.keep_all || key >= kstar || j == argmax;
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      if (keep) out[count + __popc(bal & ((1u << lane) - 1u))] = j;
-      count += __popc(bal);
-    }
-    if (lane == 0) a.kv_count[bh * Nb + i] = count;
+    const int rr = r;
+    auto score_of = [&](int j) {
+      float acc = 0.f;
+      for (int d = 0; d < D; ++d)
+        acc = __fmaf_rn(__uint_as_float(static_cast<uint32_t>(qd[d * R + rr])), kt[static_cast<int64_t>(d) * Nbp + j], acc);
+      return __fmul_rn(acc, a.scale);
+    };
+    select_row(rows + static_cast<size_t>(r) * Nbp, hist, cand, Nb, i, a,
+               a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb), a.kv_count + bh * Nb + i, score_of);
   }
 }
 
@@ -498,6 +846,30 @@ __global__ void __launch_bounds__(256) sta_lists_kernel(int32_t* __restrict__ kv
       out[e] = ((t0 + et) * nbh + h0 + eh) * nbw + w0 + (r - eh * nw);
     }
     if (lane == 0) kv_count[static_cast<int64_t>(c) * Nb + i] = count;
+  }
+}
+
+// ------------------------------------------------------ radial window lists
+// The radial decay window on its own (the Radial Attention article's static
+// mask, "Zastosowanie zasad rozkladu energii"): row i lists, ascending, the
+// blocks of every frame tj within r0 >> floor(log2(|ti - tj| + 1)) patch
+// rows and columns of block i.  Walking the frames in order and each
+// frame's clipped box row by row visits the flattened indices in ascending
+// order, so entry positions are running offsets.  One warp per query block
+// writes its row into every (b, head) copy blockIdx.y, blockIdx.y +
+// gridDim.y, ...
+__global__ void __launch_bounds__(256) radial_lists_kernel(int32_t* __restrict__ kv_count,
+                                                           int32_t* __restrict__ kv_idx, int copies, int Nb, int nbh,
+                                                           int nbw, int r0) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (i >= Nb) return;
+  const int per_t = nbh * nbw;
+  const int ti = i / per_t, hi = (i - ti * per_t) / nbw, wi = i - ti * per_t - hi * nbw;
+  for (int c = blockIdx.y; c < copies; c += gridDim.y) {
+    int32_t* out = kv_idx + (static_cast<int64_t>(c) * Nb + i) * Nb;
+    const int n = radial_for_each(ti, hi, wi, Nb / per_t, nbh, nbw, r0, lane, [out](int j, int pos) { out[pos] = j; });
+    if (lane == 0) kv_count[static_cast<int64_t>(c) * Nb + i] = n;
   }
 }
 

@@ -4,13 +4,18 @@
 // the device status word is a single symbol).
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
+#include "ab.cuh"
+#include "ab_attn.cuh"
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_fwd.cuh"
 #include "common.cuh"
 #include "flatten.cuh"
@@ -21,6 +26,15 @@ namespace nabla {
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// NVTX range around one entry point (named after the function), so a
+// profiler's timeline shows which library call launched which kernels; a
+// no-op unless a tool is attached.
+struct NvtxScope {
+  explicit NvtxScope(const char* name) { nvtxRangePushA(name); }
+  ~NvtxScope() { nvtxRangePop(); }
+};
+#define NABLA_NVTX_RANGE() ::nabla::NvtxScope nabla_nvtx_scope_(__func__)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -139,19 +153,21 @@ int permute(const void* in, void* out, int B, int T, int H, int W, int P, int ro
   return launch_status();
 }
 
+// Shared memory of mask_rows_smem_kernel<R>: q pairs, R score rows, the
+// eight warps' selection scratch.
 size_t mask_smem_bytes(int R, int D, int Nb) {
-  return static_cast<size_t>(R) * D * 8 + static_cast<size_t>(R) * Nb * 4 + kMaskWarps * 32 * 4;
+  return static_cast<size_t>(R) * D * 8 + static_cast<size_t>(R) * kbar_cols(Nb) * 4 +
+         static_cast<size_t>(kMaskWarps) * (32 * 32 * 8 + 32 * 4);
 }
 
 template <int R>
-int launch_mask(const MaskArgs& a, int B, const DeviceInfo& di, cudaStream_t stream) {
+int launch_mask_smem(const MaskArgs& a, int B, cudaStream_t stream) {
   const size_t smem = mask_smem_bytes(R, a.D, a.Nb);
-  if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
-  if (cudaFuncSetAttribute(mask_rows_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(mask_rows_smem_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
     return NABLA_ERR_CUDA;
   dim3 grid((a.Nb + R - 1) / R, a.Hh, B);
-  mask_rows_kernel<R><<<grid, kMaskThreads, smem, stream>>>(a);
+  mask_rows_smem_kernel<R><<<grid, kMaskThreads, smem, stream>>>(a);
   return launch_status();
 }
 
@@ -160,7 +176,17 @@ struct MaskPlan {
   MaskArgs a;
   DeviceInfo di;
   int S, H, W;
+  float* scores;  // score scratch [B*Hh][Nb][Nbp] (after the pooled vectors)
 };
+
+// Workspace layout: qbar^T, kbar^T (fp32 [B][Hh][D][Nbp] each), then the
+// score scratch (fp32 [B][Hh][Nb][Nbp]).
+size_t pooled_bytes(int B, int Hh, int D, int Nb) {
+  return 2 * static_cast<size_t>(B) * Hh * D * kbar_cols(Nb) * sizeof(float);
+}
+size_t score_bytes(int B, int Hh, int Nb) {
+  return static_cast<size_t>(B) * Hh * Nb * kbar_cols(Nb) * sizeof(float);
+}
 
 int mask_plan(int B, int Hh, int D, int T, int H, int W, const nabla_params* params, void* workspace,
               int32_t* kv_count, int32_t* kv_idx, MaskPlan* mp) {
@@ -175,6 +201,7 @@ int mask_plan(int B, int Hh, int D, int T, int H, int W, const nabla_params* par
   if (sta_on && (p.sta_t <= 0 || p.sta_h <= 0 || p.sta_w <= 0 || p.sta_t % 2 == 0 || p.sta_h % 2 == 0 ||
                  p.sta_w % 2 == 0))
     return NABLA_ERR_INVALID;
+  if (p.radial < 0 || p.radial > 65535) return NABLA_ERR_INVALID;
   if (workspace == nullptr) return NABLA_ERR_INVALID;
   if (!aligned16(workspace)) return NABLA_ERR_ALIGN;
   if (static_cast<int64_t>(Hh) * D > 3072 * 4) return NABLA_ERR_INVALID;
@@ -182,7 +209,8 @@ int mask_plan(int B, int Hh, int D, int T, int H, int W, const nabla_params* par
   const int Nb = S / 64;
   MaskArgs& a = mp->a;
   a.qbar = static_cast<float*>(workspace);
-  a.kbar = const_cast<float*>(a.qbar) + static_cast<size_t>(B) * Hh * Nb * D;
+  a.kbar = const_cast<float*>(a.qbar) + static_cast<size_t>(B) * Hh * D * kbar_cols(Nb);
+  mp->scores = const_cast<float*>(a.kbar) + static_cast<size_t>(B) * Hh * D * kbar_cols(Nb);
   a.kv_count = kv_count;
   a.kv_idx = kv_idx;
   a.Hh = Hh;
@@ -194,6 +222,7 @@ int mask_plan(int B, int Hh, int D, int T, int H, int W, const nabla_params* par
   a.sta_rt = p.sta_t / 2;
   a.sta_rh = p.sta_h / 2;
   a.sta_rw = p.sta_w / 2;
+  a.radial_r0 = p.radial;
   a.keep_all = p.thr >= 1.f ? 1 : 0;
   a.scale = p.scale > 0.f ? p.scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   a.tau = 1.0 - static_cast<double>(p.thr);  // exact in double
@@ -214,21 +243,45 @@ int launch_pool(const MaskPlan& mp, int B, const void* q, const void* k, void* q
   return launch_status();
 }
 
-int launch_mask_rows(const MaskPlan& mp, int B, cudaStream_t stream) {
-  // Rows per CTA: as many of 16, 8, 4 as keep the score rows within ~64 KB,
-  // so two CTAs (16 warps) share an SM; fewer rows re-read the pooled keys
-  // more often from L2, but one CTA of 8 warps per SM is slower still (16%
-  // on 3,840-block rows, measured).
+// Mask stages 2-4 on pooled vectors.  With the score scratch: the tiled
+// score GEMM, then one warp per row selecting from the scratch.  Without it
+// (the no-allocation entry point): the single kernel holding R score rows in
+// shared memory, R as large as keeps two CTAs per SM, else as fits.
+int launch_mask_rows(const MaskPlan& mp, int B, cudaStream_t stream, bool use_scratch) {
   const int Nb = mp.a.Nb, D = mp.a.D;
-  const size_t per_row = static_cast<size_t>(Nb) * 4;
-  if (16 * per_row <= 64u * 1024u) return launch_mask<16>(mp.a, B, mp.di, stream);
-  const size_t fit = (64u * 1024u) / per_row;
-  if (fit >= 8) return launch_mask<8>(mp.a, B, mp.di, stream);
-  // beyond ~4,096 blocks: 4 rows while they fit the SM's shared memory
-  // (then one CTA per SM), else 2
   const size_t optin = static_cast<size_t>(mp.di.max_smem_optin);
-  if (fit >= 4 || mask_smem_bytes(4, D, Nb) <= optin) return launch_mask<4>(mp.a, B, mp.di, stream);
-  if (mask_smem_bytes(2, D, Nb) <= optin) return launch_mask<2>(mp.a, B, mp.di, stream);
+  if (use_scratch) {
+    const int64_t bhs = static_cast<int64_t>(B) * mp.a.Hh;
+    if (bhs > 65535) return NABLA_ERR_INVALID;
+    const int Nbp = kbar_cols(Nb);
+    ScoreShape sh;
+    sh.nrows = sh.ncols = Nb;
+    sh.D = D;
+    sh.q_ld = sh.k_ld = sh.out_ld = Nbp;
+    sh.q_bh = sh.k_bh = static_cast<int64_t>(D) * Nbp;
+    sh.out_bh = static_cast<int64_t>(Nb) * Nbp;
+    if (launch_score_tiles(mp.a.qbar, mp.a.kbar, mp.scores, sh, static_cast<int>(bhs), mp.a.scale, stream) !=
+        cudaSuccess)
+      return NABLA_ERR_CUDA;
+    const size_t per_warp = select_warp_bytes(Nb);
+    int wpc = static_cast<int>(optin / per_warp);
+    if (wpc < 1) return NABLA_ERR_INVALID;
+    if (wpc > 8) wpc = 8;
+    const size_t smem = per_warp * wpc;
+    if (cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    const int64_t rows = bhs * Nb;
+    select_rows_kernel<<<static_cast<unsigned>((rows + wpc - 1) / wpc), 32 * wpc, smem, stream>>>(mp.a, mp.scores,
+                                                                                                rows);
+    return launch_status();
+  }
+  const size_t two_per_sm = optin / 2;
+  if (mask_smem_bytes(16, D, Nb) <= two_per_sm) return launch_mask_smem<16>(mp.a, B, stream);
+  if (mask_smem_bytes(8, D, Nb) <= two_per_sm) return launch_mask_smem<8>(mp.a, B, stream);
+  if (mask_smem_bytes(4, D, Nb) <= optin) return launch_mask_smem<4>(mp.a, B, stream);
+  if (mask_smem_bytes(2, D, Nb) <= optin) return launch_mask_smem<2>(mp.a, B, stream);
+  if (mask_smem_bytes(1, D, Nb) <= optin) return launch_mask_smem<1>(mp.a, B, stream);
   return NABLA_ERR_INVALID;
 }
 
@@ -249,10 +302,18 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 
 // Scratch of nabla_build_mask_noalloc: the pooled queries then keys.  In host
 // code this name is only a stand-in for the device symbol; its device address
-// comes from cudaGetSymbolAddress, once per device.
+// comes from cudaGetSymbolAddress with the caller's device current.
 __device__ __align__(256) unsigned char g_noalloc_scratch[NABLA_NOALLOC_SCRATCH_BYTES];
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Variant of the attention kernel: QK^T over pairs of listed key blocks (N =
+// 128) when NABLA_ATTN_PAIR_QK=1 in the environment (read once).
+bool attn_pair_qk() {
+  static const bool pair = [] {
+    const char* e = std::getenv("NABLA_ATTN_PAIR_QK");
+    return e != nullptr && e[0] == '1';
+  }();
+  return pair;
+}
 
 // Shared body of the two attention entry points; grp_F > 0 selects the 2 x 2
 // (w, t) grouping of query blocks (grp_F blocks per frame, grp_nbw per row).
@@ -307,22 +368,20 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   a.in_inv_nbw = inv(a.in_nbw);
   a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
   const dim3 grid((Nb + 1) / 2, Hh, B);
-  if (D == 128) {
-    const size_t smem = AttnSmem<128>::bytes(Nb);
+  const bool pair = attn_pair_qk();
+  auto go = [&](auto kernel, size_t smem) -> int {
     if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
       return NABLA_ERR_CUDA;
-    attn_fwd_kernel<128><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
-  } else {
-    const size_t smem = AttnSmem<64>::bytes(Nb);
-    if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return NABLA_ERR_CUDA;
-    attn_fwd_kernel<64><<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
-  }
-  return launch_status();
+    kernel<<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
+    return launch_status();
+  };
+  if (D == 128)
+    return pair ? go(attn_fwd_kernel<128, true>, AttnSmem<128>::bytes(Nb))
+                : go(attn_fwd_kernel<128, false>, AttnSmem<128>::bytes(Nb));
+  return pair ? go(attn_fwd_kernel<64, true>, AttnSmem<64>::bytes(Nb))
+              : go(attn_fwd_kernel<64, false>, AttnSmem<64>::bytes(Nb));
 }
 
 // Backward launches: Delta, then dQ over the row lists, then dK and dV over
@@ -342,6 +401,70 @@ int launch_bwd(const BwdArgs& a, const void* out, int B, const DeviceInfo& di, c
   const dim3 grid(a.Nb, a.Hh, B);
   bwd_dq_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a);
   bwd_dkdv_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a);
+  return launch_status();
+}
+
+// Backward kernels on tcgen05 when NABLA_BWD_TC=1 in the environment (read
+// once; the warp-MMA kernels of attn_bwd.cuh otherwise).
+bool bwd_tc() {
+  static const bool on = [] {
+    const char* e = std::getenv("NABLA_BWD_TC");
+    return e != nullptr && e[0] == '1';
+  }();
+  return on;
+}
+
+// Delta, then the dQ kernel over the row lists and the dK/dV kernel over the
+// column lists, each a CTA per pair of blocks.
+template <int D>
+int launch_bwd_tc(const BwdArgs& ba, const void* qf, const void* kf, const void* vf, const void* out, int B,
+                  const DeviceInfo& di, cudaStream_t stream) {
+  const size_t smem = BwdTcSmem<D>::bytes(ba.Nb);
+  if (smem > static_cast<size_t>(di.max_smem_optin) || ba.Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
+  CUtensorMap tq, tk, tv, tdo;
+  const bool grid = ba.W > 0;
+  const int T = grid ? ba.S / (ba.H * ba.W) : 0;
+  if (grid) {
+    if (!make_grid_map(&tq, qf, B, T, ba.H, ba.W, ba.Hh, D) || !make_grid_map(&tk, kf, B, T, ba.H, ba.W, ba.Hh, D) ||
+        !make_grid_map(&tv, vf, B, T, ba.H, ba.W, ba.Hh, D) ||
+        !make_grid_map(&tdo, ba.dout, B, T, ba.H, ba.W, ba.Hh, D))
+      return NABLA_ERR_CUDA;
+  } else if (!make_bshd_map(&tq, qf, B, ba.S, ba.Hh, D, 64) || !make_bshd_map(&tk, kf, B, ba.S, ba.Hh, D, 64) ||
+             !make_bshd_map(&tv, vf, B, ba.S, ba.Hh, D, 64) || !make_bshd_map(&tdo, ba.dout, B, ba.S, ba.Hh, D, 64)) {
+    return NABLA_ERR_CUDA;
+  }
+  BwdTcArgs a;
+  a.lse = ba.lse;
+  a.delta = ba.delta;
+  a.S = ba.S;
+  a.Hh = ba.Hh;
+  a.Nb = ba.Nb;
+  a.grid_H = grid ? ba.H : 0;
+  a.grid_W = grid ? ba.W : 0;
+  a.in_T = T;
+  a.in_nbw = grid ? ba.W / 8 : 0;
+  a.in_per_t = grid ? (ba.H / 8) * (ba.W / 8) : 0;
+  a.scale = ba.scale;
+  a.scale_log2 = ba.scale_log2;
+  const int64_t rows = static_cast<int64_t>(B) * ba.S;
+  bwd_delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(out), ba.dout, const_cast<float*>(ba.delta), rows, ba.S, ba.Hh, D);
+  if (cudaFuncSetAttribute(bwd_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(bwd_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return NABLA_ERR_CUDA;
+  const dim3 g((ba.Nb + 1) / 2, ba.Hh, B);
+  a.row_count = ba.kv_count;
+  a.row_idx = ba.kv_idx;
+  a.out0 = ba.dq;
+  a.out1 = nullptr;
+  bwd_tc_kernel<D, true><<<g, kBwdTcThreads, smem, stream>>>(tq, tdo, tk, tv, a);
+  a.row_count = ba.q_count;
+  a.row_idx = ba.q_idx;
+  a.out0 = ba.dk;
+  a.out1 = ba.dv;
+  bwd_tc_kernel<D, false><<<g, kBwdTcThreads, smem, stream>>>(tk, tv, tq, tdo, a);
   return launch_status();
 }
 
@@ -385,7 +508,39 @@ int sparse_attn_bwd(const void* qf, const void* kf, const void* vf, const void* 
   a.W = W;
   a.nbw = W / 8;
   a.per_t = (H / 8) * (W / 8);
+  if (bwd_tc()) {
+    if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
+    return D == 128 ? launch_bwd_tc<128>(a, qf, kf, vf, out, B, di, stream)
+                    : launch_bwd_tc<64>(a, qf, kf, vf, out, B, di, stream);
+  }
   return D == 128 ? launch_bwd<128>(a, out, B, di, stream) : launch_bwd<64>(a, out, B, di, stream);
+}
+
+// AB-Attention plan workspace: kbar^T [B*Hh][D][NKB], cent^T [B*Hh][D][R],
+// counts [B*Hh][NQB][8], logits [B*Hh][R][NKB] (R = NQB * 8), each region
+// 256-byte aligned.
+struct ABLayout {
+  size_t kbar, cent, counts, logits, total;
+};
+ABLayout ab_layout(int B, int Hh, int D, int S) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t bh = static_cast<size_t>(B) * Hh, nkb = S / kABKBlock, nqb = S / kABQBlock;
+  const size_t R = nqb * kABClusters;
+  ABLayout l;
+  l.kbar = 0;
+  l.cent = up(bh * D * nkb * 4);
+  l.counts = l.cent + up(bh * D * R * 4);
+  l.logits = l.counts + up(bh * nqb * kABClusters * 4);
+  l.total = l.logits + up(bh * R * nkb * 4);
+  return l;
+}
+
+int ab_check(int B, int S, int Hh, int D) {
+  if (B <= 0 || S <= 0 || Hh <= 0 || S % 128 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
+  if (B > 65535 || Hh > 65535 || static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
+  // the selection holds one row of block scores in shared memory
+  if (ab_select_smem(S / kABKBlock) > 200u * 1024u) return NABLA_ERR_INVALID;
+  return NABLA_OK;
 }
 
 }  // namespace
@@ -397,25 +552,27 @@ extern "C" {
 
 int nabla_flatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
                   nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
   return permute<false>(in, out, B, T, H, W, P, row_elems, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int nabla_unflatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
                     nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
   return permute<true>(in, out, B, T, H, W, P, row_elems, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W, const nabla_params* params) {
   const int P = params ? params->P : 8;
   if (check_grid(B, T, H, W, P) != NABLA_OK || Hh <= 0 || (D != 64 && D != 128)) return 0;
-  const size_t Nb = static_cast<size_t>(T) * H * W / 64;
-  const size_t Nbp = static_cast<size_t>(kbar_cols(static_cast<int>(Nb)));
-  return static_cast<size_t>(B) * Hh * (Nb + Nbp) * D * sizeof(float);
+  const int Nb = static_cast<int>(static_cast<int64_t>(T) * H * W / 64);
+  return pooled_bytes(B, Hh, D, Nb) + score_bytes(B, Hh, Nb);
 }
 
 int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
                      const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, void* workspace,
                      nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   MaskPlan mp;
   int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, kv_count, kv_idx, &mp);
@@ -424,11 +581,12 @@ int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T
   if (!aligned16(qf) || !aligned16(kf) || !aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
   if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
   if ((rc = launch_pool<false>(mp, B, qf, kf, nullptr, nullptr, stream)) != NABLA_OK) return rc;
-  return launch_mask_rows(mp, B, stream);
+  return launch_mask_rows(mp, B, stream, true);
 }
 
 int nabla_flatten_pool_qk(const void* q, const void* k, void* qf, void* kf, int B, int Hh, int D, int T, int H,
                           int W, const nabla_params* params, void* workspace, nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   MaskPlan mp;
   int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, nullptr, nullptr, &mp);
@@ -443,6 +601,7 @@ int nabla_flatten_pool_qk(const void* q, const void* k, void* qf, void* kf, int 
 int nabla_build_mask_grid(const void* q, const void* k, int B, int Hh, int D, int T, int H, int W,
                           const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, void* workspace,
                           nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   MaskPlan mp;
   int rc = mask_plan(B, Hh, D, T, H, W, params, workspace, kv_count, kv_idx, &mp);
@@ -451,11 +610,12 @@ int nabla_build_mask_grid(const void* q, const void* k, int B, int Hh, int D, in
   if (!aligned16(q) || !aligned16(k) || !aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
   if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
   if ((rc = launch_pool<true>(mp, B, q, k, nullptr, nullptr, stream)) != NABLA_OK) return rc;
-  return launch_mask_rows(mp, B, stream);
+  return launch_mask_rows(mp, B, stream, true);
 }
 
 int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, int H, int W,
                             const nabla_params* params, int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   MaskPlan mp;
   int rc = mask_plan(B, Hh, D, T, H, W, params, const_cast<void*>(workspace), kv_count, kv_idx, &mp);
@@ -463,11 +623,12 @@ int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, 
   if (kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
   if (!aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
   if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
-  return launch_mask_rows(mp, B, stream);
+  return launch_mask_rows(mp, B, stream, true);
 }
 
 int nabla_build_mask_sta(int B, int Hh, int T, int H, int W, int P, int sta_t, int sta_h, int sta_w,
                          int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   int rc = check_grid(B, T, H, W, P);
   if (rc != NABLA_OK) return rc;
@@ -486,9 +647,29 @@ int nabla_build_mask_sta(int B, int Hh, int T, int H, int W, int P, int sta_t, i
   return launch_status();
 }
 
+int nabla_build_mask_radial(int B, int Hh, int T, int H, int W, int P, int r0, int32_t* kv_count, int32_t* kv_idx,
+                            nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int rc = check_grid(B, T, H, W, P);
+  if (rc != NABLA_OK) return rc;
+  if (Hh <= 0 || static_cast<int64_t>(B) * Hh > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
+  if (r0 < 1 || r0 > 65535) return NABLA_ERR_INVALID;
+  if (kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != NABLA_OK) return rc;
+  const int Nb = T * H * W / 64;
+  const int copies = B * Hh;
+  const dim3 grid((Nb + 7) / 8, copies < 65535 ? copies : 65535);
+  radial_lists_kernel<<<grid, 256, 0, stream>>>(kv_count, kv_idx, copies, Nb, H / 8, W / 8, r0);
+  return launch_status();
+}
+
 int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                           const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
                           nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
   return sparse_attn_launch(qf, kf, vf, kv_count, kv_idx, B, S, Hh, D, scale, out, lse, 0, 0, 0, 0, 0,
                             reinterpret_cast<cudaStream_t>(stream));
 }
@@ -496,6 +677,7 @@ int nabla_sparse_attn_fwd(const void* qf, const void* kf, const void* vf, const 
 int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, const int32_t* kv_count,
                                const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
                                void* out, float* lse, nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
   if (T <= 0 || H <= 0 || W <= 0 || H % 8 != 0 || W % 8 != 0) return NABLA_ERR_INVALID;
   const int64_t S = static_cast<int64_t>(T) * H * W;
   if (S > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
@@ -507,6 +689,7 @@ int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, cons
 
 int nabla_transpose_lists(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb, int32_t* q_count,
                           int32_t* q_idx, nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (B <= 0 || Hh <= 0 || Nb <= 0 || Nb > (1 << 24) || static_cast<int64_t>(B) * Hh > 65535) return NABLA_ERR_INVALID;
   if (kv_count == nullptr || kv_idx == nullptr || q_count == nullptr || q_idx == nullptr) return NABLA_ERR_INVALID;
@@ -522,6 +705,7 @@ int nabla_sparse_attn_bwd(const void* qf, const void* kf, const void* vf, const 
                           const float* lse, const int32_t* kv_count, const int32_t* kv_idx, const int32_t* q_count,
                           const int32_t* q_idx, int B, int S, int Hh, int D, float scale, void* dq, void* dk,
                           void* dv, float* delta, nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
   return sparse_attn_bwd(qf, kf, vf, out, dout, lse, kv_count, kv_idx, q_count, q_idx, B, S, Hh, D, scale, dq, dk,
                          dv, delta, 0, 0, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -531,6 +715,7 @@ int nabla_sparse_attn_bwd_grid(const void* q, const void* k, const void* v, cons
                                const int32_t* q_count, const int32_t* q_idx, int B, int Hh, int D, int T, int H,
                                int W, float scale, void* dq, void* dk, void* dv, float* delta,
                                nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
   if (check_grid(B, T, H, W, 8) != NABLA_OK) return NABLA_ERR_INVALID;
   return sparse_attn_bwd(q, k, v, out, dout, lse, kv_count, kv_idx, q_count, q_idx, B, T * H * W, Hh, D, scale, dq,
                          dk, dv, delta, H, W, reinterpret_cast<cudaStream_t>(stream));
@@ -538,23 +723,140 @@ int nabla_sparse_attn_bwd_grid(const void* q, const void* k, const void* v, cons
 
 int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
                              const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
-                             nabla_stream_t stream) {
-  const size_t need = nabla_mask_workspace_bytes(B, Hh, D, T, H, W, params);
-  if (params == nullptr || need == 0) return NABLA_ERR_INVALID;
-  if (need > NABLA_NOALLOC_SCRATCH_BYTES) return NABLA_ERR_TOO_LARGE;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NABLA_ERR_CUDA;
+                             nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (params == nullptr || nabla_mask_workspace_bytes(B, Hh, D, T, H, W, params) == 0) return NABLA_ERR_INVALID;
+  const int Nb = static_cast<int>(static_cast<int64_t>(T) * H * W / 64);
+  if (pooled_bytes(B, Hh, D, Nb) > NABLA_NOALLOC_SCRATCH_BYTES) return NABLA_ERR_TOO_LARGE;
+  // The buffer's device address, looked up on every call with the caller's
+  // device current (cheap, host-only): nothing is cached, so a context torn
+  // down and recreated in between cannot leave a stale address behind.
   void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NABLA_ERR_CUDA;
-      g_noalloc_ptr[dev] = p;
-    }
-    scratch = g_noalloc_ptr[dev];
+  if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr) return NABLA_ERR_CUDA;
+  MaskPlan mp;
+  int rc = mask_plan(B, Hh, D, T, H, W, params, scratch, kv_count, kv_idx, &mp);
+  if (rc != NABLA_OK) return rc;
+  if (qf == nullptr || kf == nullptr || kv_count == nullptr || kv_idx == nullptr) return NABLA_ERR_INVALID;
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(kv_count) || !aligned16(kv_idx)) return NABLA_ERR_ALIGN;
+  if ((rc = device_info(&mp.di)) != NABLA_OK) return rc;
+  if ((rc = launch_pool<false>(mp, B, qf, kf, nullptr, nullptr, stream)) != NABLA_OK) return rc;
+  return launch_mask_rows(mp, B, stream, false);
+}
+
+size_t nabla_ab_workspace_bytes(int B, int S, int Hh, int D) {
+  if (ab_check(B, S, Hh, D) != NABLA_OK) return 0;
+  return ab_layout(B, Hh, D, S).total;
+}
+
+int nabla_ab_plan(const void* q, const void* k, const float* u, int B, int S, int Hh, int D, int kmeans_iters,
+                  double budget, float scale, int32_t* kcount, int32_t* kidx, float* kshift, void* workspace,
+                  nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int rc = ab_check(B, S, Hh, D);
+  if (rc != NABLA_OK) return rc;
+  if (kmeans_iters < 0 || kmeans_iters > 64 || !(budget >= 0.0) || std::isinf(budget)) return NABLA_ERR_INVALID;
+  if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
+  const void* ptrs[] = {q, k, u, kcount, kidx, kshift, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr) return NABLA_ERR_INVALID;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != NABLA_OK) return rc;
+  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  const ABLayout lay = ab_layout(B, Hh, D, S);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  float* kbarT = reinterpret_cast<float*>(ws + lay.kbar);
+  float* centT = reinterpret_cast<float*>(ws + lay.cent);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + lay.counts);
+  float* logits = reinterpret_cast<float*>(ws + lay.logits);
+  const int nkb = S / kABKBlock, nqb = S / kABQBlock, R = nqb * kABClusters;
+  ab_key_means_kernel<<<dim3(nkb / 8, B), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), kbarT, S, Hh, D);
+  if ((rc = launch_status()) != NABLA_OK) return rc;
+  const size_t ksm = ab_kmeans_smem(D);
+  if (cudaFuncSetAttribute(ab_kmeans_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ksm)) !=
+      cudaSuccess)
+    return NABLA_ERR_CUDA;
+  ab_kmeans_kernel<<<dim3(nqb, Hh, B), 256, ksm, stream>>>(static_cast<const __nv_bfloat16*>(q), centT, counts, S, Hh,
+                                                           D, kmeans_iters);
+  if ((rc = launch_status()) != NABLA_OK) return rc;
+  ScoreShape sh;
+  sh.nrows = R;
+  sh.ncols = nkb;
+  sh.D = D;
+  sh.q_ld = R;
+  sh.k_ld = sh.out_ld = nkb;
+  sh.q_bh = static_cast<int64_t>(D) * R;
+  sh.k_bh = static_cast<int64_t>(D) * nkb;
+  sh.out_bh = static_cast<int64_t>(R) * nkb;
+  if (launch_score_tiles(centT, kbarT, logits, sh, B * Hh, sc, stream) != cudaSuccess) return NABLA_ERR_CUDA;
+  ABSelectArgs sa;
+  sa.logits = logits;
+  sa.counts = counts;
+  sa.u = u;
+  sa.kcount = kcount;
+  sa.kidx = kidx;
+  sa.kshift = kshift;
+  sa.nqb = nqb;
+  sa.nkb = nkb;
+  sa.budget = budget;
+  const size_t ssm = ab_select_smem(nkb);
+  if (cudaFuncSetAttribute(ab_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssm)) !=
+      cudaSuccess)
+    return NABLA_ERR_CUDA;
+  ab_select_kernel<<<dim3(nqb, B * Hh), 256, ssm, stream>>>(sa);
+  return launch_status();
+}
+
+int nabla_ab_attn_fwd(const void* q, const void* k, const void* v, const int32_t* kcount, const int32_t* kidx,
+                      const float* kshift, int B, int S, int Hh, int D, float scale, void* out, float* lse,
+                      nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int rc = ab_check(B, S, Hh, D);
+  if (rc != NABLA_OK) return rc;
+  if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
+  const void* ptrs[] = {q, k, v, kcount, kidx, kshift, out};
+  for (const void* p : ptrs)
+    if (p == nullptr) return NABLA_ERR_INVALID;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return NABLA_ERR_ALIGN;
+  if (lse != nullptr && !aligned16(lse)) return NABLA_ERR_ALIGN;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != NABLA_OK) return rc;
+  if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
+  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  CUtensorMap tq;
+  if (!make_bshd_map(&tq, q, B, S, Hh, D, 128)) return NABLA_ERR_CUDA;
+  ABAttnArgs a;
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.kcount = kcount;
+  a.kidx = kidx;
+  a.kshift = kshift;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.S = S;
+  a.Hh = Hh;
+  a.nkb = S / kABKBlock;
+  a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
+  const dim3 grid(S / 128, Hh, B);
+  if (D == 128) {
+    const size_t smem = ABAttnSmem<128>::kBytes;
+    if (cudaFuncSetAttribute(ab_attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    ab_attn_fwd_kernel<128><<<grid, kABAttnThreads, smem, stream>>>(tq, a);
+  } else {
+    const size_t smem = ABAttnSmem<64>::kBytes;
+    if (cudaFuncSetAttribute(ab_attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    ab_attn_fwd_kernel<64><<<grid, kABAttnThreads, smem, stream>>>(tq, a);
   }
-  return nabla_build_mask(qf, kf, B, Hh, D, T, H, W, params, kv_count, kv_idx, scratch, stream);
+  return launch_status();
 }
 
 int nabla_selftest_wait_timeout(long long limit_cycles, nabla_stream_t stream_) {
@@ -578,6 +880,7 @@ int nabla_get_status(nabla_stream_t stream_) {
 
 int nabla_validate_mask(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb, int32_t* bad_rows,
                         nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (B <= 0 || Hh <= 0 || Nb <= 0 || kv_count == nullptr || kv_idx == nullptr || bad_rows == nullptr)
     return NABLA_ERR_INVALID;

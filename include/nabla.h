@@ -72,13 +72,22 @@ enum {
  *          com STA", M = M_nabla OR M_STA).  The window is centred on the query
  *          block and truncated at the grid border.
  *   scale  score scale; 0 selects 1/sqrt(D).
- *   flags  reserved, must be 0. */
+ *   flags  reserved, must be 0.
+ *   radial radial decay window OR-ed into the mask, the static mask of the
+ *          Radial Attention article ("Zastosowanie zasad rozkladu energii":
+ *          a neighbourhood window that shrinks as the temporal distance
+ *          grows).  0 disables it; r0 = radial >= 1 keeps block j for block
+ *          i when their patch rows and columns each differ by at most
+ *          r0 >> floor(log2(|ti - tj| + 1)), ti, tj their frames: the
+ *          window halves each time the temporal distance (plus one)
+ *          doubles, and the co-located block of every frame stays. */
 typedef struct {
   int P;
   float thr;
   int sta_t, sta_h, sta_w;
   float scale;
   unsigned flags;
+  int radial;
 } nabla_params;
 
 /* Fractal flattening ("Metodologia: NABLA", item 1, "Reordenacao de Tokens"):
@@ -98,10 +107,11 @@ int nabla_flatten(const void* in, void* out, int B, int T, int H, int W, int P, 
 int nabla_unflatten(const void* in, void* out, int B, int T, int H, int W, int P, int row_elems,
                     nabla_stream_t stream);
 
-/* Bytes of device workspace nabla_build_mask needs: the pooled queries,
- * fp32 [B][Hh][Nb][D], then the pooled keys transposed, fp32
- * [B][Hh][D][Nbp] with Nbp = Nb rounded up to a multiple of 4 (columns
- * >= Nb are padding).  Returns 0 for invalid sizes. */
+/* Bytes of device workspace nabla_build_mask needs: the pooled queries and
+ * the pooled keys, both transposed, fp32 [B][Hh][D][Nbp] each with Nbp = Nb
+ * rounded up to a multiple of 4 (columns >= Nb are padding), then the
+ * block-score scratch, fp32 [B][Hh][Nb][Nbp] (4*B*Hh*Nb*Nbp bytes: 1.4 GB
+ * for 24 heads of 3,840 blocks).  Returns 0 for invalid sizes. */
 size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W,
                                   const nabla_params* params);
 
@@ -119,10 +129,14 @@ size_t nabla_mask_workspace_bytes(int B, int Hh, int D, int T, int H, int W,
  *               blocks ascending in entries [0, kv_count); later entries are
  *               not written.
  *   workspace   device buffer of nabla_mask_workspace_bytes() bytes, 16-byte
- *               aligned; on return it holds qbar then kbar^T (layouts as
- *               for nabla_mask_workspace_bytes).
+ *               aligned; on return it holds qbar^T, kbar^T and the block
+ *               scores s_ij (layouts as for nabla_mask_workspace_bytes).
+ * The scores are computed as a tiled fp32 GEMM with the same rounding as
+ * the definition above (one fused multiply-add chain over d ascending per
+ * entry, then the scale), and each row is thresholded from them. 
  * Errors: NABLA_ERR_INVALID (shape, D not 64/128, thr outside [0,1], even or
- * negative STA sizes, flags != 0); NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
+ * negative STA sizes, radial outside [0, 65535], flags != 0);
+ * NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
 int nabla_build_mask(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
                      const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
                      void* workspace, nabla_stream_t stream);
@@ -176,6 +190,22 @@ int nabla_build_mask_pooled(const void* workspace, int B, int Hh, int D, int T, 
  * NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
 int nabla_build_mask_sta(int B, int Hh, int T, int H, int W, int P, int sta_t, int sta_h, int sta_w,
                          int32_t* kv_count, int32_t* kv_idx, nabla_stream_t stream);
+
+/* The radial decay window on its own (nabla_params.radial without the
+ * content-adaptive term; the static mask the Radial Attention article
+ * describes).  No Q or K is read: row i of every (b, head) lists, ascending,
+ * the blocks j with |patch row difference| <= rho and |patch column
+ * difference| <= rho, rho = r0 >> floor(log2(|ti - tj| + 1)) for frames
+ * ti, tj.  The lists are the radial part of nabla_build_mask's union with
+ * the same r0.
+ *   P           must be 8; H and W multiples of 8.
+ *   r0          spatial half-width (in patches) at temporal distance 0, in
+ *               [1, 65535].
+ *   kv_count, kv_idx   as for nabla_build_mask (16-byte aligned).
+ * Errors: NABLA_ERR_INVALID (grid, Hh, r0, NULL lists); NABLA_ERR_ALIGN;
+ * NABLA_ERR_CUDA. */
+int nabla_build_mask_radial(int B, int Hh, int T, int H, int W, int P, int r0, int32_t* kv_count, int32_t* kv_idx,
+                            nabla_stream_t stream);
 
 /* Block-sparse attention forward on the kept tiles ("Expansao": only the
  * listed N x N blocks are computed; a dropped block is in neither the
@@ -283,16 +313,19 @@ int nabla_sparse_attn_bwd_grid(const void* q, const void* k, const void* v, cons
  * host or serving runtime that owns all device memory and exposes no
  * allocator, or a latency-critical path where cudaMalloc's implicit
  * device-wide synchronisation is not acceptable.
- *   The pooled queries and keys (the workspace of nabla_build_mask) live in
- *   a static device buffer of NABLA_NOALLOC_SCRATCH_BYTES inside the library;
- *   every GPU that loads the library holds that buffer until the process
- *   exits.  The call allocates nothing and frees nothing.
+ *   The pooled queries and keys (the first part of nabla_build_mask's
+ *   workspace, 8*B*Hh*D*Nbp bytes) live in a static device buffer of
+ *   NABLA_NOALLOC_SCRATCH_BYTES inside the library; the block scores are
+ *   kept in shared memory instead of a scratch.  Every GPU that loads the
+ *   library holds that buffer until the process exits.  The call allocates
+ *   nothing and frees nothing.
  *   Arguments, layouts and results are those of nabla_build_mask without the
- *   workspace argument.  A problem whose workspace
- *   (nabla_mask_workspace_bytes) exceeds NABLA_NOALLOC_SCRATCH_BYTES is
- *   rejected with NABLA_ERR_TOO_LARGE before anything is launched.
- *   The first call on a device looks up the buffer's device address (with
- *   that device current); make that first call before any stream capture.
+ *   workspace argument.  A problem whose pooled vectors exceed
+ *   NABLA_NOALLOC_SCRATCH_BYTES is rejected with NABLA_ERR_TOO_LARGE before
+ *   anything is launched.
+ *   Every call looks up the buffer's device address (cudaGetSymbolAddress,
+ *   with the caller's device current), so nothing is cached across a
+ *   context teardown; make a first call before any stream capture.
  *   All calls share the one buffer and each call overwrites it completely:
  *   calls that overlap on the GPU (other streams, other host threads) race
  *   on it, so the caller must order them. */
@@ -300,6 +333,72 @@ int nabla_sparse_attn_bwd_grid(const void* q, const void* k, const void* v, cons
 int nabla_build_mask_noalloc(const void* qf, const void* kf, int B, int Hh, int D, int T, int H, int W,
                              const nabla_params* params, int32_t* kv_count, int32_t* kv_idx,
                              nabla_stream_t stream);
+
+/* ---------------------------------------------------------------------
+ * AB-Attention, a second sparse-attention scheme over the same tensors
+ * (news page "AB-Attention acelera a geracao de video em ate 2,23x e pula
+ * 92% da atencao", section "Os tres recursos do AB-Attention"), on tensors
+ * in their original (grid) order -- the scheme does not permute tokens.
+ * Query blocks are 128 consecutive tokens (NQB = S / 128), key blocks 4
+ * consecutive tokens (NKB = S / 4).  nabla_ab_plan builds the sampling plan
+ * (the page re-plans every few denoising steps); nabla_ab_attn_fwd runs the
+ * attention on it.
+ * --------------------------------------------------------------------- */
+
+/* Bytes of device workspace nabla_ab_plan needs: the mean keys (transposed,
+ * fp32 [B][Hh][D][NKB]), the centroids (transposed, fp32 [B][Hh][D][NQB*8]),
+ * the cluster counts (int32 [B][Hh][NQB][8]) and the centroid logits (fp32
+ * [B][Hh][NQB*8][NKB]), each region 256-byte aligned, in that order
+ * (2.9 GB for 12 heads of 61,440 tokens).  Returns 0 for invalid sizes. */
+size_t nabla_ab_workspace_bytes(int B, int S, int Hh, int D);
+
+/* The sampling plan ("IBCS" and "SIP"):
+ *   1. mean key of every 4-token block (fp32, tokens in order, * 0.25);
+ *   2. per 128-query block, 8 clusters by kmeans_iters Lloyd iterations
+ *      from the queries at positions 0, 16, ..., 112: squared distances as
+ *      an fp32 fused multiply-add chain over d of the rounded differences,
+ *      ties to the lower cluster; each centroid the fp32 mean of its
+ *      queries (empty clusters keep theirs); weight = count / 128;
+ *   3. block scores s_J = sum_c weight_c softmax_J(cent_c . kbar_J * scale);
+ *   4. inclusion probabilities pi_J = min(1, lambda s_J) with
+ *      sum_J pi_J = budget (water-filling); key block J is sampled iff
+ *      u_J < pi_J, and gets the logit shift -log(pi_J) (its
+ *      Horvitz-Thompson weight 1 / pi_J).
+ *   q, k        device bf16 [B][S][Hh][D], S a multiple of 128.
+ *   u           device fp32 [B][Hh][NQB][NKB]: the uniform random numbers
+ *               in [0, 1) of the sampling (the caller draws them).
+ *   kmeans_iters  0 .. 64;  budget  expected sample size per query block;
+ *   scale       0 selects 1/sqrt(D).
+ *   kcount      device int32 [B][Hh][NQB] output: sampled key blocks.
+ *   kidx        device int32 [B][Hh][NQB][NKB] output: sampled blocks
+ *               ascending in entries [0, kcount); later entries unwritten.
+ *   kshift      device fp32 [B][Hh][NQB][NKB] output: entry e's shift.
+ *   workspace   nabla_ab_workspace_bytes() bytes, 16-byte aligned.
+ * Steps 1-2 and the logits of step 3 follow the fp32 definition above
+ * operation for operation; pi is computed with expf and sums in the GPU's
+ * order (within about 1e-7 of the exact value).  The NKB block scores of a
+ * row are held in shared memory (NKB <= about 50,000).
+ * Errors: NABLA_ERR_INVALID (shapes, iterations, budget, scale, NULL);
+ * NABLA_ERR_ALIGN; NABLA_ERR_CUDA. */
+int nabla_ab_plan(const void* q, const void* k, const float* u, int B, int S, int Hh, int D, int kmeans_iters,
+                  double budget, float scale, int32_t* kcount, int32_t* kidx, float* kshift, void* workspace,
+                  nabla_stream_t stream);
+
+/* Attention of every 128-query block over its sampled 4-token key blocks,
+ * each key's logit shifted by its block's kshift:
+ *   O_a = softmax_c((q_a . k_c) * scale + kshift(c)) V, LSE = log of the
+ *   normaliser; the sampled blocks are gathered by index into 64-key
+ *   tensor-core tiles (16 blocks each).
+ *   q, k, v     device bf16 [B][S][Hh][D], grid order, 16-byte aligned.
+ *   kcount, kidx, kshift   as written by nabla_ab_plan (entries in [0, NKB);
+ *               a bad entry is skipped and recorded as
+ *               NABLA_ERR_DEVICE_BOUNDS).
+ *   out         device bf16 [B][S][Hh][D]; lse fp32 [B][Hh][S] or NULL.
+ * A query block with no sampled block gets O = 0, LSE = -inf.
+ * Errors: as nabla_sparse_attn_fwd. */
+int nabla_ab_attn_fwd(const void* q, const void* k, const void* v, const int32_t* kcount, const int32_t* kidx,
+                      const float* kshift, int B, int S, int Hh, int D, float scale, void* out, float* lse,
+                      nabla_stream_t stream);
 
 /* Synchronises the stream, then returns and clears the current device's
  * status word (NABLA_OK, NABLA_ERR_DEVICE_TIMEOUT or NABLA_ERR_DEVICE_BOUNDS),

@@ -57,7 +57,8 @@ class Case:
         self.qf = nabla.flatten(self.qd, w.T, w.H, w.W)
         self.kf = nabla.flatten(self.kd, w.T, w.H, w.W)
         self.vf = nabla.flatten(self.vd, w.T, w.H, w.W)
-        self.kv_count, self.kv_idx, self.ws = nabla.build_mask(self.qf, self.kf, w.T, w.H, w.W, w.thr, w.sta)
+        self.kv_count, self.kv_idx, self.ws = nabla.build_mask(self.qf, self.kf, w.T, w.H, w.W, w.thr, w.sta,
+                                                               radial=w.radial)
         torch.cuda.synchronize()
         assert nabla.get_status() == 0
 
@@ -79,7 +80,18 @@ class Case:
         return out, lse
 
     def host_flat(self):
-        return (self.qf.cpu(), self.kf.cpu(), self.vf.cpu())
+        """The oracle's own flattening of the host inputs (uint16 bf16 bits),
+        computed once: oracle inputs never come from the CUDA path."""
+        if not hasattr(self, "_host_flat"):
+            w = self.w
+            self._host_flat = tuple(oracle.flatten(x, w.T, w.H, w.W).reshape(x.shape)
+                                    for x in (self.q, self.k, self.v))
+        return self._host_flat
+
+    def assert_flatten_matches_oracle(self):
+        """The GPU's flattened Q, K, V equal the oracle's bit for bit."""
+        for xf, ref in zip((self.qf, self.kf, self.vf), self.host_flat()):
+            assert np.array_equal(xf.cpu().view(torch.int16).numpy().view(np.uint16), ref)
 
 
 def keep_matrix_gpu(kv_count: torch.Tensor, kv_idx: torch.Tensor) -> torch.Tensor:
@@ -95,7 +107,9 @@ def keep_matrix_gpu(kv_count: torch.Tensor, kv_idx: torch.Tensor) -> torch.Tenso
 
 def compare_masks(case: Case, status: np.ndarray):
     """Returns (mismatches outside the band, mismatches inside the band,
-    number of band blocks).  status is the oracle's per-block byte."""
+    number of band blocks).  status is the oracle's per-block byte: bit 0
+    kept, bit 1 band (cumulative mass within 1e-5 of 1 - thr, the one class
+    the acceptance rule excuses)."""
     st = torch.from_numpy(status).to(case.kv_count.device)
     kept_o = (st & 1).bool()
     band = (st & 2).bool()
@@ -113,7 +127,8 @@ def oracle_masks(case: Case, qf_host, kf_host):
     w = case.w
     qbar = oracle.pool(qf_host)
     kbar = oracle.pool(kf_host)
-    cnt, idx, status, _ = oracle.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, sta_window=w.sta)
+    cnt, idx, status, _ = oracle.build_mask(qbar, kbar, w.thr, w.scale, w.nbh, w.nbw, sta_window=w.sta,
+                                            radial_r0=w.radial)
     return qbar, kbar, cnt, idx, status
 
 

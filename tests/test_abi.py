@@ -65,13 +65,17 @@ def test_strerror_covers_codes(lib):
 
 
 def test_params_struct_layout_matches_header():
-    assert ctypes.sizeof(nabla.NablaParams) == 28
+    assert ctypes.sizeof(nabla.NablaParams) == 32
     assert nabla.NablaParams.thr.offset == 4 and nabla.NablaParams.flags.offset == 24
+    assert nabla.NablaParams.radial.offset == 28
 
 
 def test_workspace_bytes(lib):
     prm = nabla.params(0.9)
-    assert nabla.mask_workspace_bytes(1, 12, 128, 16, 48, 80, prm) == 2 * 12 * 960 * 128 * 4
+    # pooled queries and keys (transposed), then the block-score scratch
+    assert nabla.mask_workspace_bytes(1, 12, 128, 16, 48, 80, prm) == 2 * 12 * 960 * 128 * 4 + 12 * 960 * 960 * 4
+    # odd block count: rows padded to a multiple of 4 columns (37 -> 40)
+    assert nabla.mask_workspace_bytes(1, 1, 64, 37, 8, 8, prm) == 2 * 64 * 40 * 4 + 37 * 40 * 4
     assert nabla.mask_workspace_bytes(1, 2, 96, 4, 16, 16, prm) == 0  # D not supported
     assert nabla.mask_workspace_bytes(1, 2, 64, 4, 12, 16, prm) == 0  # H not a multiple of 8
 

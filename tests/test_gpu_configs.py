@@ -24,7 +24,8 @@ N_SAMPLED_BLOCKS = 64
 
 def run_config(w: inputs.Workload, n_blocks: int = N_SAMPLED_BLOCKS):
     case = Case(w)
-    host = case.host_flat()
+    host = case.host_flat()  # the oracle's flattening of the host inputs
+    case.assert_flatten_matches_oracle()
     _, _, _, _, status = oracle_masks(case, host[0], host[1])
     bad, in_band, nband = compare_masks(case, status)
     kept = float(case.kv_count.double().sum().item()) / (w.B * w.Hh * w.Nb * w.Nb)

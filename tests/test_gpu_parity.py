@@ -49,9 +49,7 @@ def test_small_layers_end_to_end(w):
     case = Case(w)
     qf_h, kf_h, vf_h = case.host_flat()
     # flattening is bit-exact
-    for x, xf in ((case.q, qf_h), (case.k, kf_h), (case.v, vf_h)):
-        ref = oracle.flatten(x, w.T, w.H, w.W).reshape(x.shape)
-        assert np.array_equal(xf.view(torch.int16).numpy().view(np.uint16), ref)
+    case.assert_flatten_matches_oracle()
     # pooling: same fp32 sum order as the oracle -> bit-exact
     qbar, kbar, cnt_o, idx_o, status = oracle_masks(case, qf_h, kf_h)
     qg, kg = nabla.pooled_from_workspace(case.ws, w.B, w.Hh, w.Nb, w.D)
