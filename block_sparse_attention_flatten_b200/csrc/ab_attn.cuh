@@ -241,20 +241,24 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence16(sv[c]);
-      // logits in log2 units plus the keys' shifts, in place
+      // logits in log2 units plus the keys' shifts, in place, two columns
+      // per two-lane FMA
       const float* shs = shift_s + s * 64;
+      const unsigned long long sc2 = f2_pack(a.scale_log2, a.scale_log2);
       float mc[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         mc[c] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float x = fmaf(__uint_as_float(sv[c][e]), a.scale_log2, shs[c * 16 + e]);
-          sv[c][e] = __float_as_uint(x);
-          mc[c] = fmaxf(mc[c], x);
+        for (int e = 0; e < 16; e += 2) {
+          const unsigned long long sh2 = *reinterpret_cast<const unsigned long long*>(shs + c * 16 + e);
+          const unsigned long long x2 = f2_fma((static_cast<unsigned long long>(sv[c][e + 1]) << 32) | sv[c][e], sc2, sh2);
+          sv[c][e] = static_cast<uint32_t>(x2);
+          sv[c][e + 1] = static_cast<uint32_t>(x2 >> 32);
+          mc[c] = fmax3(mc[c], f2_lo(x2), f2_hi(x2));
         }
       }
-      const float mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+      const float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]);
       float factor = 1.f;
       bool need = false;
       if (mx > m_run + 8.f) {  // also true while m_run is -inf (unless mx is -inf too)
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
       // a row that so far saw only padding keys has m_run = -inf: its
       // probabilities are 0, not exp(-inf - -inf)
       const float mref = m_run == -INFINITY ? 0.f : m_run;
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      unsigned long long rs2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[2][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -273,11 +277,12 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
         for (int e = 0; e < 16; e += 2) {
           const float p0 = ex2_approx(__uint_as_float(sv[c][e]) - mref);
           const float p1 = ex2_approx(__uint_as_float(sv[c][e + 1]) - mref);
-          rs[c] += p0 + p1;
+          rs2[c] = f2_add(rs2[c], f2_pack(p0, p1));
           const int k = c * 8 + e / 2;
           pk[k >> 4][k & 15] = pack_bf16x2(p0, p1);
         }
-      l_run = l_run * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      const unsigned long long rall = f2_add(f2_add(rs2[0], rs2[1]), f2_add(rs2[2], rs2[3]));
+      l_run = l_run * factor + (f2_lo(rall) + f2_hi(rall));
       __syncwarp();
       if (__any_sync(0xffffffffu, need)) {
         if (!__all_sync(0xffffffffu, mbar_wait(pv_done + ((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag))) {

@@ -10,25 +10,27 @@
 //                     walking the union of their row lists (a key block
 //                     listed by one half is masked for the other half's
 //                     rows): S = Q K^T and dP = dO V^T into tensor memory,
-//                     P and dS by 8 elementwise warps, dQ += dS K.
+//                     P and dS by 16 elementwise warps, dQ += dS K.
 // bwd_dkdv_tc_kernel  one CTA per pair of key blocks (128 key rows),
 //                     walking the union of their column lists:
 //                     S^T = K Q^T, dP^T = V dO^T, P^T and dS^T elementwise,
 //                     dV += P^T dO and dK += dS^T Q, both accumulated in
 //                     tensor memory across the walk.
 // Unlike the forward's softmax the elementwise step has no row reduction
-// (the LSE is known), so two threads share a row: warps w and w + 4 read
-// the same 32 tensor-memory lanes (rows), columns 0-31 and 32-63.  Their
-// bf16 results go back into the columns they read (the first 16 of each
-// half), which the next MMA reads as its A operand (K = 16 per step, so the
-// two halves need not be adjacent).
-// Warp roles (352 threads, one CTA per SM: 512 tensor-memory columns):
-//   warps 0-7  elementwise, then the epilogue (row r = 32 (w % 4) + lane,
-//              column half w / 4);
-//   warp 8     TMA producer (one thread; dK/dV kernel: the warp, for the LSE
+// (the LSE is known), so four threads share a row: warps w, w + 4, w + 8,
+// w + 12 read the same 32 tensor-memory lanes (rows), columns 16q .. 16q+15
+// for quarter q = w / 4.  Their bf16 results go back into the first 8 of
+// the columns they read, which the next MMA reads as its A operand (K = 16
+// keys per step = one quarter, so the quarters need not be adjacent).
+// Sixteen elementwise warps keep four per scheduler, so one warp's wait on
+// a tensor-memory load hides behind the others' arithmetic.
+// Warp roles (608 threads, one CTA per SM: 512 tensor-memory columns):
+//   warps 0-15 elementwise, then the epilogue (row r = 32 (w % 4) + lane,
+//              column quarter w / 4);
+//   warp 16    TMA producer (one thread; dK/dV kernel: the warp, for the LSE
 //              and Delta values it copies);
-//   warp 9     MMA issuer of the two products of a tile (S and dP);
-//   warp 10    MMA issuer of the accumulating products (dQ; dV and dK).
+//   warp 17    MMA issuer of the two products of a tile (S and dP);
+//   warp 18    MMA issuer of the accumulating products (dQ; dV and dK).
 // Every wait is bounded (see common.cuh); a timeout raises the CTA's abort
 // flag, every role drains and the tensor memory is freed.
 #pragma once
@@ -39,7 +41,8 @@
 
 namespace nabla {
 
-constexpr int kBwdTcThreads = 352;
+constexpr int kBwdTcThreads = 608;
+constexpr int kBwdTcElemThreads = 512;  // warps 0-15
 
 struct BwdTcArgs {
   const int32_t* row_count;  // lists walked by the CTA: dQ kernel the row lists, dK/dV the column lists
@@ -63,7 +66,7 @@ __device__ __forceinline__ int64_t bwd_tc_row(const BwdTcArgs& a, int j, int r) 
   return (static_cast<int64_t>(t) * a.grid_H + bh * 8 + (r >> 3)) * a.grid_W + bw * 8 + (r & 7);
 }
 
-template <int D>
+template <int D, int WS>
 struct BwdTcSmem {
   static constexpr int kChunks = D / 64;
   static constexpr int kPairBytes = 128 * 128 * kChunks;  // 128 rows x D
@@ -71,13 +74,20 @@ struct BwdTcSmem {
   // fixed pair tiles: (Q, dO) in the dQ kernel, (K, V) in the dK/dV kernel
   static constexpr int kA = 0;
   static constexpr int kB = kA + kPairBytes;
-  // two stages of the walked blocks: (K, V) or (Q, dO), each 64 rows
+  // kWS stages of the walked blocks: (K, V) or (Q, dO), each 64 rows.  A
+  // stage is held from its load until the tile's accumulating MMAs are
+  // done, so with two stages the load of tile n + 2 waited for the whole
+  // chain of tile n (products, elementwise step, accumulation) and its copy
+  // latency sat on the critical path; four stages keep the copies three
+  // tiles ahead (192 KB of shared memory at D = 128, one CTA per SM); the
+  // launcher falls back to two where the block lists leave no room for four.
+  static constexpr int kWS = WS;
   static constexpr int kW0 = kB + kPairBytes;
-  static constexpr int kW1 = kW0 + 2 * kBlkBytes;
-  static constexpr int kLD = kW1 + 2 * kBlkBytes;  // dK/dV: [2 stages][LSE*log2e 64 | Delta 64] fp32
-  static constexpr int kBars = kLD + 2 * 128 * 4;
-  // fixed_full, w_full[2], w0_empty[2], w1_empty[2], s_full[2], e_full[2], acc_done[2], drain
-  static constexpr int kNumBars = 1 + 2 + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kW1 = kW0 + kWS * kBlkBytes;
+  static constexpr int kLD = kW1 + kWS * kBlkBytes;  // dK/dV: [kWS stages][LSE*log2e 64 | Delta 64] fp32
+  static constexpr int kBars = kLD + kWS * 128 * 4;
+  // fixed_full, w_full[kWS], w0_empty[kWS], w1_empty[kWS], s_full[2], e_full[2], acc_done[2], drain
+  static constexpr int kNumBars = 1 + 3 * kWS + 2 + 2 + 2 + 1;
   static constexpr int kMisc = kBars + 8 * kNumBars;
   static constexpr int kList = kMisc + 32;
   __host__ __device__ static size_t list_bytes(int Nb) { return (static_cast<size_t>(Nb) * 2 + 15) & ~size_t(15); }
@@ -90,23 +100,24 @@ struct BwdTcSmem {
 // kDq = true: the dQ kernel; false: the dK/dV kernel.  tmA/tmB are the maps
 // of the CTA's fixed pair tiles (Q, dO or K, V), tmC/tmD those of the
 // walked blocks (K, V or Q, dO).
-template <int D, bool kDq>
+template <int D, bool kDq, int WS>
 __global__ void __launch_bounds__(kBwdTcThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                   const BwdTcArgs a) {
-  using L = BwdTcSmem<D>;
+  using L = BwdTcSmem<D, WS>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint64_t* fixed_full = bars;
-  uint64_t* w_full = bars + 1;     // [2] walked stage landed
-  uint64_t* w0_empty = bars + 3;   // [2] first walked tile (K or Q) free
-  uint64_t* w1_empty = bars + 5;   // [2] second walked tile (V or dO) free
-  uint64_t* s_full = bars + 7;     // [2] the tile's two products are in tensor memory
-  uint64_t* e_full = bars + 9;     // [2] elementwise results written (256 arrivals)
-  uint64_t* acc_done = bars + 11;  // [2] the accumulating products of the tile are done
-  uint64_t* drain = bars + 13;
+  constexpr int kWS = L::kWS;
+  uint64_t* w_full = bars + 1;               // [kWS] walked stage landed
+  uint64_t* w0_empty = w_full + kWS;         // [kWS] first walked tile (K or Q) free
+  uint64_t* w1_empty = w0_empty + kWS;       // [kWS] second walked tile (V or dO) free
+  uint64_t* s_full = w1_empty + kWS;         // [2] the tile's two products are in tensor memory
+  uint64_t* e_full = s_full + 2;             // [2] elementwise results written (512 arrivals)
+  uint64_t* acc_done = e_full + 2;           // [2] the accumulating products of the tile are done
+  uint64_t* drain = acc_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
   int* list_len = reinterpret_cast<int*>(sm + L::kMisc + 8);
@@ -134,12 +145,14 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   // ---- set-up: barriers, tensor memory, the fixed pair tiles, merged list
   if (tid == 0) {
     mbar_init(fixed_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kWS; ++s) {
       mbar_init(w_full + s, 1);
       mbar_init(w0_empty + s, 1);
       mbar_init(w1_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(e_full + s, 256);
+      mbar_init(e_full + s, kBwdTcElemThreads);
       mbar_init(acc_done + s, 1);
     }
     mbar_init(drain, 2);
@@ -154,7 +167,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     load_block(sm + L::kB, &tmB, fixed_full, blk0, 128 * 128);
     load_block(sm + L::kB + 64 * 128, &tmB, fixed_full, b1, 128 * 128);
   }
-  if (warp == 8) {
+  if (warp == 16) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
     if (lane == 0) {
@@ -223,7 +236,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   const uint32_t sA = smem_u32(sm + L::kA), sB = smem_u32(sm + L::kB);
   const uint32_t sW0 = smem_u32(sm + L::kW0), sW1 = smem_u32(sm + L::kW1);
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ------------------------------------------------------------ producer
     // dQ: walked (K, V) of each key block; dK/dV: (Q, dO) of each query
     // block plus its 64 LSE (times log2 e; -inf -> +inf, so P = 0) and
@@ -231,10 +244,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     int issued = 0;
     bool ok = true;
     for (int n = 0; ok && n < L_n; ++n) {
-      const int s = n & 1;
-      if (n >= 2) {
-        const bool w0 = mbar_wait(w0_empty + s, ((n >> 1) - 1) & 1, abort_flag);
-        const bool w1 = mbar_wait(w1_empty + s, ((n >> 1) - 1) & 1, abort_flag);
+      const int s = n % kWS;
+      if (n >= kWS) {
+        const bool w0 = mbar_wait(w0_empty + s, ((n / kWS) - 1) & 1, abort_flag);
+        const bool w1 = mbar_wait(w1_empty + s, ((n / kWS) - 1) & 1, abort_flag);
         if (!__all_sync(0xffffffffu, w0 && w1)) {
           ok = false;
           break;
@@ -259,10 +272,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       issued = n + 1;
     }
     if (lane == 0) {
-      for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n) mbar_wait_drain(w_full + (n & 1), (n >> 1) & 1);
+      for (int n = (issued > kWS ? issued - kWS : 0); n < issued; ++n)
+        mbar_wait_drain(w_full + n % kWS, (n / kWS) & 1);
       mbar_wait_drain(fixed_full, 0);
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // -------------------------------------------- the two products of a tile
     // dQ: S = Q K^T (A = Q pair, B = K block), dP = dO V^T.
     // dK/dV: S^T = K Q^T (A = K pair, B = Q block), dP^T = V dO^T.
@@ -270,13 +284,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       bool ok = mbar_wait(fixed_full, 0, abort_flag);
       tc_fence_after();
       for (int n = 0; ok && n < L_n; ++n) {
-        const int s = n & 1;
-        if (!mbar_wait(w_full + s, (n >> 1) & 1, abort_flag)) { ok = false; break; }
+        const int s = n & 1, ws = n % kWS;
+        if (!mbar_wait(w_full + ws, (n / kWS) & 1, abort_flag)) { ok = false; break; }
         // buffers s hold the previous use's bf16 results until the
         // accumulating MMAs of tile n - 2 have read them
         if (n >= 2 && !mbar_wait(acc_done + s, ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t w0b = sW0 + s * L::kBlkBytes, w1b = sW1 + s * L::kBlkBytes;
+        const uint32_t w0b = sW0 + ws * L::kBlkBytes, w1b = sW1 + ws * L::kBlkBytes;
         const uint32_t tX = tX0 + s * 64, tY = tY0 + s * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -294,27 +308,27 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
         umma_commit(s_full + s);
         // dQ kernel: V is read only here; dK/dV: dO is read again by dV
-        if (kDq) umma_commit(w1_empty + s);
+        if (kDq) umma_commit(w1_empty + ws);
       }
       umma_commit(drain);
       mbar_wait_drain(drain, 0);
     }
-  } else if (warp == 10) {
+  } else if (warp == 18) {
     // ------------------------------------------ the accumulating products
-    // A operands from tensor memory (bf16 pairs: key/query columns 0-31 in
-    // the buffer's columns 0-15, columns 32-63 in columns 32-47), B operands
+    // A operands from tensor memory (bf16 pairs: the 16 key/query columns
+    // of quarter q in the buffer's columns 16q .. 16q+7), B operands
     // MN-major from the walked stage.
     if (lane == 0 && L_n > 0) {
       bool ok = true;
       for (int n = 0; ok && n < L_n; ++n) {
-        const int s = n & 1;
+        const int s = n & 1, ws = n % kWS;
         if (!mbar_wait(e_full + s, (n >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tX = tX0 + s * 64, tY = tY0 + s * 64;
-        const uint32_t w0b = sW0 + s * L::kBlkBytes, w1b = sW1 + s * L::kBlkBytes;
+        const uint32_t w0b = sW0 + ws * L::kBlkBytes, w1b = sW1 + ws * L::kBlkBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t col = kk < 2 ? kk * 8 : 32 + (kk - 2) * 8;
+          const uint32_t col = kk * 16;
           if (kDq) {
             // dQ += dS K
             const uint64_t bd = smem_desc_sw128(w0b + kk * 16 * 128, 64 * 128, 1024);
@@ -328,16 +342,16 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
           }
         }
         umma_commit(acc_done + s);
-        umma_commit(w0_empty + s);
-        if (!kDq) umma_commit(w1_empty + s);
+        umma_commit(w0_empty + ws);
+        if (!kDq) umma_commit(w1_empty + ws);
       }
       umma_commit(drain);
       mbar_wait_drain(drain, 0);
     }
   } else {
-    // ----------------------------------------------------------- elementwise (warps 0-7)
+    // ----------------------------------------------------------- elementwise (warps 0-15)
     const int r = 32 * (warp & 3) + lane;  // tensor-memory lane = row of the pair tile
-    const int ch = warp >> 2;              // column half
+    const int ch = warp >> 2;              // column quarter
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t flag = 0x4000u << (r >> 6);
     // dQ kernel: this row's LSE (log2 units, -inf -> +inf) and Delta
@@ -353,24 +367,23 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     for (int n = 0; n < L_n; ++n) {
       const int s = n & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (n >> 1) & 1, abort_flag))) { ok = false; break; }
-      if (!kDq && !__all_sync(0xffffffffu, mbar_wait(w_full + s, (n >> 1) & 1, abort_flag))) { ok = false; break; }
+      if (!kDq && !__all_sync(0xffffffffu, mbar_wait(w_full + n % kWS, (n / kWS) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      const uint32_t tX = tX0 + s * 64 + ch * 32 + lane_off, tY = tY0 + s * 64 + ch * 32 + lane_off;
-      uint32_t xv[2][16], yv[2][16];
+      const uint32_t tX = tX0 + s * 64 + ch * 16 + lane_off, tY = tY0 + s * 64 + ch * 16 + lane_off;
+      uint32_t xv[1][16], yv[1][16];  // this quarter's 16 columns of X and Y
       tmem_ld16(tX, xv[0]);
-      tmem_ld16(tX + 16, xv[1]);
       tmem_ld16(tY, yv[0]);
-      tmem_ld16(tY + 16, yv[1]);
       tmem_ld_wait();
       reg_fence16(xv[0]);
-      reg_fence16(xv[1]);
       reg_fence16(yv[0]);
-      reg_fence16(yv[1]);
       const bool inc = (static_cast<uint32_t>(list[n]) & flag) != 0u;
-      const float* lq = ld_s + s * 128 + ch * 32;  // dK/dV: the columns' LSE and Delta
-      uint32_t pk[16], dk[16];
+      const float* lq = ld_s + (n % kWS) * 128 + ch * 16;  // dK/dV: the columns' LSE and Delta
+      uint32_t pk[8], dk[8];
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
+      for (int e = 0; e < 16; e += 2) {
         float p0 = 0.f, p1 = 0.f, d0, d1, L0, L1;
         if (kDq) {
           L0 = L1 = L2row;
@@ -391,10 +404,10 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         dk[e >> 1] = pack_bf16x2(ds0, ds1);
       }
       if (kDq) {
-        tmem_st16(tX, dk);  // dS into the S buffer
+        tmem_st8(tX, dk);  // dS into the S buffer
       } else {
-        tmem_st16(tX, pk);  // P^T into the S^T buffer
-        tmem_st16(tY, dk);  // dS^T into the dP^T buffer
+        tmem_st8(tX, pk);  // P^T into the S^T buffer
+        tmem_st8(tY, dk);  // dS^T into the dP^T buffer
       }
       tmem_st_wait();
       tc_fence_before();
@@ -409,12 +422,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     const int64_t trow = static_cast<int64_t>(b) * a.S + (valid ? bwd_tc_row(a, myblk, r & 63) : 0);
     const int nacc = kDq ? 1 : 2;
     for (int which = 0; which < nacc; ++which) {
-      const uint32_t tacc = (which == 0 ? tAcc0 : tAcc1) + lane_off + ch * (D / 2);
+      const uint32_t tacc = (which == 0 ? tAcc0 : tAcc1) + lane_off + ch * (D / 4);
       // dQ kernel: dQ (scaled); dK/dV kernel: which 0 = dV, 1 = dK (scaled)
       const float f = kDq ? a.scale : (which == 0 ? 1.f : a.scale);
-      __nv_bfloat16* orow = (kDq ? a.out0 : (which == 0 ? a.out1 : a.out0)) + (trow * a.Hh + hd) * D + ch * (D / 2);
+      __nv_bfloat16* orow = (kDq ? a.out0 : (which == 0 ? a.out1 : a.out0)) + (trow * a.Hh + hd) * D + ch * (D / 4);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t ov[16];
         if (ok && L_n > 0) {
           tmem_ld16(tacc + c * 16, ov);
@@ -444,7 +457,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 16) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

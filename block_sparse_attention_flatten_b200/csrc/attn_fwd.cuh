@@ -46,6 +46,14 @@ namespace nabla {
 
 constexpr int kAttnThreads = 224;
 constexpr int kMaxListBlocks = 16383;  // list entries hold a 14-bit block index
+// Softmax exponentials: of every 8 column pairs, those whose bit is set here
+// go to the FMA pipe (exp2_poly_f2), the others to the MUFU.  A step of
+// 128 query rows x 64 keys at D = 128 is 4.2 MFLOP of MMAs, about 512
+// clocks of an SM's tensor cores, and 8192 exponentials, 512 clocks of its
+// MUFU (16 per clock): with every exponential on the MUFU the softmax could
+// keep pace with the MMAs only at perfect overlap.  3 of 8 pairs on the FMA
+// pipe leave both pipes with slack.
+constexpr uint32_t kExpPolyPairs = 0x52u;  // pairs 1, 4, 6
 
 template <int D>
 struct AttnSmem {
@@ -85,18 +93,12 @@ struct AttnArgs {
   float scale_log2;         // scale * log2(e)
 };
 
-// kPair: QK^T of two consecutive listed key blocks as one N = 128 MMA into
-// the adjacent score buffers S0 | S1 (the K ring then holds pairs of blocks,
-// 128 rows per 64-column chunk); softmax and PV still run per block.  The
-// next pair's QK^T waits for the PV of the pair's second block.
-template <int D, bool kPair>
+template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using L = AttnSmem<D>;
   constexpr int kStages = L::kStages;
-  constexpr int kPairSlots = kStages / 2;  // K slots of two blocks in pair mode
-  constexpr int kKChunkStride = kPair ? 2 * 64 * 128 : 64 * 128;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
@@ -289,13 +291,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (j0 >= 0) {
       k0_early = true;
       if (lane == 0) {
-        // pair mode: the pair's arrival (with its second block's bytes)
-        // follows once the list is known
-        if (kPair)
-          mbar_expect_tx(k_full, L::kKVBytes);
-        else
-          mbar_arrive_expect_tx(k_full, L::kKVBytes);
-        load_block(sm + L::kK, &tmK, k_full, j0, kKChunkStride);
+        mbar_arrive_expect_tx(k_full, L::kKVBytes);
+        load_block(sm + L::kK, &tmK, k_full, j0, 64 * 128);
       }
     }
   }
@@ -359,40 +356,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int n = 0; ok && n <= L_n; ++n) {
-        if (kPair) {
-          // even n: both blocks of pair n/2 into one slot, one arrival
-          if (n < L_n && (n & 1) == 0) {
-            const int p = n >> 1, s = p % kPairSlots;
-            if (p >= kPairSlots && !mbar_wait(k_empty + s, ((p / kPairSlots) - 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            const int nb = n + 1 < L_n ? 2 : 1;
-            unsigned char* dst = sm + L::kK + s * 2 * L::kKVBytes;
-            if (n == 0 && k0_early) {
-              // block 0 is in flight and its bytes expected already
-              mbar_arrive_expect_tx(k_full + s, (nb - 1) * L::kKVBytes);
-            } else {
-              mbar_arrive_expect_tx(k_full + s, nb * L::kKVBytes);
-              load_block(dst, &tmK, k_full + s, static_cast<int>(list[n] & 0x3FFFu), kKChunkStride);
-            }
-            if (nb == 2) load_block(dst + 64 * 128, &tmK, k_full + s, static_cast<int>(list[n + 1] & 0x3FFFu),
-                                    kKChunkStride);
-            k_issued = n + nb;
+        if (n < L_n && !(n == 0 && k0_early)) {
+          const int s = n % kStages;
+          if (n >= kStages && !mbar_wait(k_empty + s, ((n / kStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
           }
-        } else {
-          if (n < L_n && !(n == 0 && k0_early)) {
-            const int s = n % kStages;
-            if (n >= kStages && !mbar_wait(k_empty + s, ((n / kStages) - 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            const int j = static_cast<int>(list[n] & 0x3FFFu);
-            mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
-            load_block(sm + L::kK + s * L::kKVBytes, &tmK, k_full + s, j, 64 * 128);
-          }
-          if (n < L_n) k_issued = n + 1;
+          const int j = static_cast<int>(list[n] & 0x3FFFu);
+          mbar_arrive_expect_tx(k_full + s, L::kKVBytes);
+          load_block(sm + L::kK + s * L::kKVBytes, &tmK, k_full + s, j, 64 * 128);
         }
+        if (n < L_n) k_issued = n + 1;
         if (n >= 1) {
           const int m = n - 1, s = m % kStages;
           if (m >= kStages && !mbar_wait(v_empty + s, ((m / kStages) - 1) & 1, abort_flag)) {
@@ -407,14 +381,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
       // Drain: wait for the last issued loads of every stage so no copy is in
       // flight when the CTA exits, also on the abort path (time-bounded).
-      if (kPair) {
-        const int pairs = (k_issued + 1) >> 1;
-        for (int p = (pairs > kPairSlots ? pairs - kPairSlots : 0); p < pairs; ++p)
-          mbar_wait_drain(k_full + p % kPairSlots, (p / kPairSlots) & 1);
-      } else {
-        for (int n = (k_issued > kStages ? k_issued - kStages : 0); n < k_issued; ++n)
-          mbar_wait_drain(k_full + n % kStages, (n / kStages) & 1);
-      }
+      for (int n = (k_issued > kStages ? k_issued - kStages : 0); n < k_issued; ++n)
+        mbar_wait_drain(k_full + n % kStages, (n / kStages) & 1);
       for (int n = (v_issued > kStages ? v_issued - kStages : 0); n < v_issued; ++n)
         mbar_wait_drain(v_full + n % kStages, (n / kStages) & 1);
     }
@@ -424,29 +392,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (lane == 0 && L_n > 0) {
       bool ok = mbar_wait(q_full, 0, abort_flag);
       tc_fence_after();
-      if (kPair) {
-        constexpr uint32_t kIdescQK2 = idesc_bf16_f32(128, 128, false, false);
-        for (int p = 0; ok && 2 * p < L_n; ++p) {
-          const int s = p % kPairSlots;
-          if (!mbar_wait(k_full + s, (p / kPairSlots) & 1, abort_flag)) { ok = false; break; }
-          // S0 | S1 hold P of the previous pair until its second PV has read
-          // it (PVs complete in issue order, so the first one has too)
-          if (p >= 1 && !mbar_wait(pv_done + 1, (p - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kb = sK + s * 2 * L::kKVBytes;
-          const uint32_t idesc = 2 * p + 1 < L_n ? kIdescQK2 : kIdescQK;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int c = kk >> 2, off = (kk & 3) * 32;
-            const uint64_t ad = smem_desc_sw128(sQ + c * 128 * 128 + off, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + c * kKChunkStride + off, 16, 1024);
-            umma_bf16_ss(tS0, ad, bd, idesc, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(s_full);
-          umma_commit(k_empty + s);
-        }
-      }
-      for (int n = 0; !kPair && ok && n < L_n; ++n) {
+      for (int n = 0; ok && n < L_n; ++n) {
         const int s = n % kStages;
         if (!mbar_wait(k_full + s, (n / kStages) & 1, abort_flag)) { ok = false; break; }
         // S buffer (n & 1) still holds P(n-2) until PV(n-2) has read it.
@@ -501,9 +447,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int n = 0; n < L_n; ++n) {
-      // pair mode: one score barrier per pair of blocks
-      uint64_t* sbar = kPair ? s_full : s_full + (n & 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(sbar, (n >> 1) & 1, abort_flag))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + (n & 1), (n >> 1) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[4][16];
       const uint32_t tS = ((n & 1) ? tS1 : tS0) + lane_off;
@@ -517,14 +461,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       float factor = 1.f;
       bool need = false;
       if (inc) {
-        float mc[4];  // four independent max chains
+        float mc[4];  // four independent max chains, three inputs per step
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          mc[c] = __uint_as_float(sv[c][0]);
+          mc[c] = fmaxf(__uint_as_float(sv[c][0]), __uint_as_float(sv[c][15]));
 #pragma unroll
-          for (int e = 1; e < 16; ++e) mc[c] = fmaxf(mc[c], __uint_as_float(sv[c][e]));
+          for (int e = 1; e < 15; e += 2) mc[c] = fmax3(mc[c], __uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1]));
         }
-        float mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+        float mx = fmax3(fmaxf(mc[0], mc[1]), mc[2], mc[3]);
         mx *= a.scale_log2;
         if (mx > m_run + 8.f) {  // also true while m_run is -inf
           factor = ex2_approx(m_run - mx);  // 0 when m_run = -inf
@@ -532,22 +476,34 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           m_run = mx;
         }
       }
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
+      // pairs of columns: x = s * scale_log2 - m in one two-lane FMA, two
+      // exponentials, two-lane sums (four independent accumulators)
+      unsigned long long rs2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[2][16];
+      const unsigned long long sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_run, -m_run);
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           float p0 = 0.f, p1 = 0.f;
           if (inc) {
-            p0 = ex2_approx(fmaf(__uint_as_float(sv[c][e]), a.scale_log2, -m_run));
-            p1 = ex2_approx(fmaf(__uint_as_float(sv[c][e + 1]), a.scale_log2, -m_run));
+            const unsigned long long x2 = f2_fma((static_cast<unsigned long long>(sv[c][e + 1]) << 32) | sv[c][e], sc2, nm2);
+            if ((kExpPolyPairs >> (e / 2)) & 1u) {
+              const unsigned long long p2 = exp2_poly_f2(x2);
+              p0 = f2_lo(p2);
+              p1 = f2_hi(p2);
+            } else {
+              p0 = ex2_approx(f2_lo(x2));
+              p1 = ex2_approx(f2_hi(x2));
+            }
           }
-          rs[c] += p0 + p1;
+          rs2[c] = f2_add(rs2[c], f2_pack(p0, p1));
           const int k = c * 8 + e / 2;
           pk[k >> 4][k & 15] = pack_bf16x2(p0, p1);
         }
-      l_run = l_run * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      const unsigned long long r01 = f2_add(rs2[0], rs2[1]), r23 = f2_add(rs2[2], rs2[3]);
+      const unsigned long long rall = f2_add(r01, r23);
+      l_run = l_run * factor + (f2_lo(rall) + f2_hi(rall));
 
       __syncwarp();
       if (__any_sync(0xffffffffu, need)) {

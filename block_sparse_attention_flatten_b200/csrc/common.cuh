@@ -39,12 +39,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// Raises the transaction count the current phase waits for, without an
-// arrival (the phase still needs its arrivals).
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -234,6 +228,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // Ties 16 registers to a point after tmem_ld_wait so the compiler cannot
@@ -245,10 +244,61 @@ __device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
                  "+r"(r[15]));
 }
 
+// Two-lane fp32 arithmetic (each lane rounds like the scalar instruction)
+// and the three-input maximum of sm_100.
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on two fp32 lanes without the special-function unit (the softmax of
+// the attention kernels puts part of its exponentials here so that they
+// share the work between the MUFU and the FMA pipe).  Range reduction
+// x = n + f, n = round-to-nearest(x) by adding and subtracting the shifter
+// 1.5 * 2^23 (then f = x - n is exact, |f| <= 1/2); 2^f by a degree-3
+// polynomial, the relative-error minimax fit on [-1/2, 1/2] (Lawson's
+// iteratively reweighted least squares, reproduced by fit_exp2_poly.py next
+// to this file): relative error below 7.6e-5 including the fp32 Horner
+// steps, far under the bf16 rounding the probabilities get; n is then added
+// to the exponent field (the low bits of the shifted sum hold n).  x is
+// clamped to >= -125 so the result stays normal: below that it returns
+// 2^-125-ish instead of a smaller number, an absolute error under 2^-124.
+// x must be <= 126 (the softmax's x never exceeds its lazy-rescale margin).
+constexpr float kExp2C0 = 0.99992811f, kExp2C1 = 0.69326099f, kExp2C2 = 0.24261054f, kExp2C3 = 0.05517132f;
+__device__ __forceinline__ unsigned long long exp2_poly_f2(unsigned long long x2) {
+  const float shifter = 12582912.f;  // 1.5 * 2^23
+  const unsigned long long xc = f2_pack(fmaxf(f2_lo(x2), -125.f), fmaxf(f2_hi(x2), -125.f));
+  const unsigned long long t = f2_add(xc, f2_pack(shifter, shifter));
+  const unsigned long long n = f2_add(t, f2_pack(-shifter, -shifter));
+  const unsigned long long f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+  unsigned long long q = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
+  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
+  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+  return (static_cast<unsigned long long>(hi) << 32) | lo;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

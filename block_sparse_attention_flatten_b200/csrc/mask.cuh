@@ -13,11 +13,12 @@
 //                     shared memory (no scratch), for callers without one.
 // sta_lists_kernel, radial_lists_kernel  The static windows alone as lists.
 // The selection (select_row) never forms p = e / sum(e) and never sorts the
-// row: the order of e is the order of p, the masses are integers e * 2^40
-// (every partial sum exact and independent of summation order), and the
-// boundary element (e*, j*) of the ascending (e, j) order is found by
-// 32-way mass histograms over the bit patterns of e, then a warp sort of
-// the last <= 32 candidates; keep = (e, j) >= (e*, j*) OR arg-max OR STA.
+// row: the order of e is the order of p, the masses are the e themselves
+// summed in fp64 in a fixed order, and the boundary element (e*, j*) of the
+// ascending (e, j) order is found by threshold masses (register-only
+// predicated sums) narrowing an interval of bit patterns whose elements are
+// compacted into a shrinking candidate set, then a warp sort of the last
+// <= 32; keep = (e, j) >= (e*, j*) OR arg-max OR a static window.
 #pragma once
 
 #include "common.cuh"
@@ -153,11 +154,6 @@ constexpr int kMaskCols = 4;  // adjacent key blocks per thread in the in-shared
 // aligned and is read and written as float4.
 __host__ __device__ inline int kbar_cols(int Nb) { return (Nb + 3) & ~3; }
 
-// Shared memory one warp needs to select one row: private mass histograms
-// [32 digits][32 lanes] (u64), 32 candidate slots, the row (Nbp floats).
-__host__ __device__ inline size_t select_warp_bytes(int Nb) {
-  return 32 * 32 * 8 + 32 * 4 + static_cast<size_t>(kbar_cols(Nb)) * 4;
-}
 
 // d = a * b + d on two fp32 lanes at once; each lane is one fmaf (round to
 // nearest even), so a lane's chain of these equals the scalar fmaf chain.
@@ -169,18 +165,7 @@ __device__ __forceinline__ unsigned long long dup2(float x) {
   return (u << 32) | u;
 }
 
-// Integer mass of an unnormalised probability e in [0, 1], from its bit
-// pattern u: floor(e * 2^40) (exact for e >= 2^-16; smaller masses lose
-// < 2^-40 each).  The row's CDF rule "cumulative p > 1 - thr" becomes, with
-// p = e / sum(e), "cumulative mass > floor((1 - thr) * total mass)" in exact
-// integers, independent of summation order.
-__device__ __forceinline__ unsigned long long mass_bits(uint32_t u) {
-  const int sh = static_cast<int>(u >> 23) - 110;  // biased exponent - (150 - 40)
-  const unsigned long long m24 = (u & 0x7FFFFFu) | 0x800000u;
-  return sh >= 0 ? (m24 << sh) : (sh > -24 ? (m24 >> -sh) : 0ull);
-}
-
-__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+__device__ __forceinline__ double warp_sum_f64(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -192,74 +177,36 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
 // switches to this value wherever 2 ulp could change a decision.
 __device__ __forceinline__ float exp_rounded(float x) { return __double2float_rn(exp(static_cast<double>(x))); }
 
-constexpr uint32_t kOneBits = 0x3F800000u;                // 1.0f
-constexpr uint32_t kNearOneBits = kOneBits - 8u;         // within 8 ulp below 1.0
-constexpr uint32_t kDigit0Lo = 0x30800000u;              // 2^-30: start of the first histogram's range
-constexpr int kWindowUlps = 8;                           // > 2 ulp (expf) on either side, with margin
+constexpr uint32_t kOneBits = 0x3F800000u;         // 1.0f
+constexpr uint32_t kNearOneBits = kOneBits - 8u;  // within 8 ulp below 1.0
+constexpr int kWindowUlps = 8;                    // > 2 ulp (expf) on either side, with margin
 constexpr unsigned long long kInfKey = 0x7F800000ull << 32;
-
-// Adds mass w to digit dg of this lane's private histogram column, through a
-// one-entry register cache: runs of equal digits (neighbouring blocks) cost
-// one shared-memory update.
-struct HistCache {
-  int d = -1;
-  unsigned long long w = 0;
-  __device__ __forceinline__ void add(unsigned long long* hist, int lane, int dg, unsigned long long m) {
-    if (dg != d) {
-      if (d >= 0) hist[d * 32 + lane] += w;
-      d = dg;
-      w = 0;
-    }
-    w += m;
-  }
-  __device__ __forceinline__ void flush(unsigned long long* hist, int lane) {
-    if (d >= 0) hist[d * 32 + lane] += w;
-    d = -1;
-    w = 0;
-  }
-};
-
-__device__ __forceinline__ void hist_clear(unsigned long long* hist, int lane) {
-#pragma unroll
-  for (int d = 0; d < 32; ++d) hist[d * 32 + lane] = 0ull;
+constexpr int kSelCap = 2048;                     // candidate slots per warp
+// First-pass thresholds: the numerators 2^-1, 2^-2, 2^-4, 2^-7, 2^-11, 2^-16
+// (bit patterns descending).
+constexpr int kNThr = 6;
+__host__ __device__ constexpr uint32_t thr_bits(int k) {
+  return static_cast<uint32_t>(127 - (k == 0 ? 1 : k == 1 ? 2 : k == 2 ? 4 : k == 3 ? 7 : k == 4 ? 11 : 16)) << 23;
 }
 
-// From a histogram of the range [lo, lo + 32 << sh) (digit = (u - lo) >> sh)
-// and the mass below lo, picks the digit holding the CDF boundary: the first
-// digit whose inclusive cumulative mass exceeds tau_m.  Updates lo and
-// below.  Lane d sums digit d's column, reading the lanes' entries in a
-// rotated order (no bank conflicts beyond the 64-bit pairing).
-__device__ __forceinline__ void hist_choose(const unsigned long long* hist, int lane, int sh, unsigned long long tau_m,
-                                            uint32_t& lo, unsigned long long& below) {
-  __syncwarp();
-  unsigned long long hd = 0;
-#pragma unroll 8
-  for (int k = 0; k < 32; ++k) hd += hist[lane * 32 + ((k + lane) & 31)];
-  unsigned long long incl = hd;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  incl += below;
-  const int dstar = __popc(__ballot_sync(0xffffffffu, incl <= tau_m));  // < 32: the range holds the crossing
-  const unsigned long long prev = __shfl_sync(0xffffffffu, incl, dstar > 0 ? dstar - 1 : 0);
-  if (dstar > 0) below = prev;
-  lo += static_cast<uint32_t>(dstar) << sh;
+// Shared memory one warp needs to select one row: candidate slots (int32),
+// 32 more for the window, the row (Nbp floats).
+__host__ __device__ inline size_t select_warp_bytes(int Nb) {
+  return kSelCap * 4 + 32 * 4 + static_cast<size_t>(kbar_cols(Nb)) * 4;
 }
 
-// Ascending warp bitonic sort of up to 32 (key, mass) pairs (lanes >= n hold
-// key ~0), then the key of the first lane whose cumulative mass, on top of
-// `base`, exceeds tau_m (~0 if none).
-__device__ __forceinline__ unsigned long long sort_and_cross(unsigned long long key, unsigned long long w, int lane,
-                                                             unsigned long long base, unsigned long long tau_m,
-                                                             unsigned long long* lane_key, unsigned long long* lane_w) {
+// Ascending warp bitonic sort of up to 32 (key, mass) pairs (lanes past the
+// data hold key ~0), then the key of the first lane whose cumulative mass,
+// on top of `base`, exceeds tau_m (~0 if none).
+__device__ __forceinline__ unsigned long long sort_and_cross(unsigned long long key, double w, int lane, double base,
+                                                             double tau_m, unsigned long long* lane_key,
+                                                             double* lane_w) {
 #pragma unroll
   for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       const unsigned long long okey = __shfl_xor_sync(0xffffffffu, key, stride);
-      const unsigned long long ow = __shfl_xor_sync(0xffffffffu, w, stride);
+      const double ow = __shfl_xor_sync(0xffffffffu, w, stride);
       const bool up = (lane & size) == 0;
       const bool lower = (lane & stride) == 0;
       if (lower == up ? (okey < key) : (okey > key)) {
@@ -268,10 +215,10 @@ __device__ __forceinline__ unsigned long long sort_and_cross(unsigned long long 
       }
     }
   }
-  unsigned long long cw = w;
+  double cw = w;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long v = __shfl_up_sync(0xffffffffu, cw, o);
+    const double v = __shfl_up_sync(0xffffffffu, cw, o);
     if (lane >= o) cw += v;
   }
   *lane_key = key;
@@ -281,23 +228,22 @@ __device__ __forceinline__ unsigned long long sort_and_cross(unsigned long long 
 }
 
 // Numerator pass: row[j] <- e_j = exp(s_j - m) for j < Nbp (padding scores
-// are -inf, so their e is 0), with the level-0 histogram of masses over the
-// binades [2^-30, 2) (digit = (bits(e) - bits(2^-30)) >> 23; smaller e go to
-// `low`).  kExact: every e is the correctly rounded value, the scores read
-// through score_of (the row already holds numerators); otherwise e = expf,
-// except within 8 ulp of 1 where the correctly rounded value is used, so
-// the set of blocks with e == 1 (the arg-max ties) is exact.
-// Returns the arg-max (largest j with e == 1) and the warp-total masses.
+// are -inf, so their e is 0), with the total mass and the masses of the
+// numerators at or above each first-pass threshold, all in fp64 in a fixed
+// order.  Per element only register arithmetic (predicated adds, no memory
+// read-modify-write, no divergence in the common case).  kExact: every e
+// is the correctly rounded value, the scores read through score_of (the
+// row already holds numerators); otherwise e = expf, except within 8 ulp of
+// 1 where the correctly rounded value is used, so the blocks with e == 1
+// (the arg-max ties) are exact.  Returns the arg-max (largest j, e == 1).
 template <bool kExact, class ScoreFn>
-__device__ __forceinline__ int numerator_pass(float* row, unsigned long long* hist, int Nb, int Nbp, float m,
-                                              const ScoreFn& score_of, unsigned long long& total,
-                                              unsigned long long& low) {
+__device__ __forceinline__ int numerator_pass(float* row, int Nb, int Nbp, float m, const ScoreFn& score_of,
+                                              double& total, double (&above)[kNThr]) {
   const int lane = threadIdx.x & 31;
   float4* row4 = reinterpret_cast<float4*>(row);
-  hist_clear(hist, lane);
-  HistCache hc;
-  total = 0;
-  low = 0;
+  total = 0.0;
+#pragma unroll
+  for (int k = 0; k < kNThr; ++k) above[k] = 0.0;
   int amax = -1;
   for (int c = lane; c < (Nbp >> 2); c += 32) {
     float ev[4];
@@ -321,142 +267,246 @@ __device__ __forceinline__ int numerator_pass(float* row, unsigned long long* hi
         u = __float_as_uint(e);
       }
       ev[t] = e;
-      if (u == kOneBits) amax = 4 * c + t;
-      const unsigned long long w = mass_bits(u);
+      amax = u == kOneBits ? 4 * c + t : amax;
+      const double w = static_cast<double>(e);
       total += w;
-      const uint32_t dg = (u - kDigit0Lo) >> 23;
-      if (dg < 32u)
-        hc.add(hist, lane, static_cast<int>(dg), w);
-      else
-        low += w;
+      // selects, not branches: lanes disagree on every comparison
+#pragma unroll
+      for (int k = 0; k < kNThr; ++k) above[k] += u >= thr_bits(k) ? w : 0.0;
     }
     row4[c] = make_float4(ev[0], ev[1], ev[2], ev[3]);
   }
-  hc.flush(hist, lane);
-  total = warp_sum_u64(total);
-  low = warp_sum_u64(low);
+  total = warp_sum_f64(total);
+#pragma unroll
+  for (int k = 0; k < kNThr; ++k) above[k] = warp_sum_f64(above[k]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   __syncwarp();
   return amax;
 }
 
-// The CDF boundary of a row of numerators: the element (e*, j*) of the
-// ascending (e, j) order at which the cumulative integer mass first exceeds
-// tau_m (keep (e, j) >= (e*, j*)).  Returns its key (bits(e) << 32 | j).
-// The range holding bits(e*) is narrowed by 32-way mass histograms (one
-// pass over the row each, 5 bits at a time: the first comes with the
-// numerators), gathering the elements of the current range on the way;
-// once at most 32 remain they are sorted in the warp.  More than 32 equal
-// values: the boundary is the need-th smallest index among them.
-// Requires tau_m < total; `low` is the mass below 2^-30.
-__device__ __forceinline__ unsigned long long cdf_boundary(const float* row, unsigned long long* hist, int* cand, int Nbp,
-                                           unsigned long long tau_m, unsigned long long low, uint32_t* range_lo,
-                                           int* range_span, unsigned long long* range_below,
-                                           unsigned long long* lane_key, unsigned long long* lane_w) {
+// Writes, in ascending j, the indices of the elements whose bit pattern lies
+// in [lo, hi) to cbuf (first kSelCap of them) and returns their count.
+// `from_row`: scan the whole row; otherwise cbuf[0..n) (compacted in place:
+// a write never overtakes the reads of its chunk).
+__device__ __forceinline__ int compact_range(const float* row, int* cbuf, int Nbp, bool from_row, int n, uint32_t lo,
+                                             uint32_t hi) {
   const int lane = threadIdx.x & 31;
-  const float4* row4 = reinterpret_cast<const float4*>(row);
-  uint32_t lo;
-  int span;
-  unsigned long long below;
-  if (low > tau_m) {  // the boundary lies below 2^-30: start over on [0, 2^30)
-    lo = 0;
-    span = 30;
-    below = 0;
-  } else {
-    lo = kDigit0Lo;
-    below = low;
-    hist_choose(hist, lane, 23, tau_m, lo, below);
-    span = 23;
-  }
-  int n = 0;
-  while (true) {
-    // one pass: gather the range's elements, histogram them one level down
-    const int sh = span > 5 ? span - 5 : 0;
-    const uint32_t width = 1u << span;
-    hist_clear(hist, lane);
-    HistCache hc;
-    n = 0;
+  int out = 0;
+  if (from_row) {
+    const float4* row4 = reinterpret_cast<const float4*>(row);
     for (int c = lane; c - lane < (Nbp >> 2); c += 32) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      const bool live = c < (Nbp >> 2);
-      if (live) v = row4[c];
-      const float ev[4] = {v.x, v.y, v.z, v.w};
+      uint32_t fl = 0;
+      if (c < (Nbp >> 2)) {
+        const float4 v = row4[c];
+        const float ev[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const uint32_t u = __float_as_uint(ev[t]);
-        const uint32_t d = u - lo;
-        const bool in = live && d < width;
-        const unsigned bal = __ballot_sync(0xffffffffu, in);
-        if (in) {
-          const int pos = n + __popc(bal & ((1u << lane) - 1u));
-          if (pos < 32) cand[pos] = 4 * c + t;
-          hc.add(hist, lane, static_cast<int>(d >> sh), mass_bits(u));
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t u = __float_as_uint(ev[t]);
+          fl |= (u >= lo && u < hi) ? (1u << t) : 0u;
         }
-        n += __popc(bal);
+      }
+      // ascending j = lane-major, then t: exclusive prefix of the lanes' counts
+      const int cnt = __popc(fl);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int pos = out + incl - cnt;
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (fl & (1u << t)) {
+          if (pos < kSelCap) cbuf[pos] = 4 * c + t;
+          ++pos;
+        }
+      out += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  } else {
+    for (int base = 0; base < n; base += 32) {
+      const int x = base + lane;
+      int j = -1;
+      if (x < n) j = cbuf[x];
+      const uint32_t u = j >= 0 ? __float_as_uint(row[j]) : 0u;
+      const bool in = j >= 0 && u >= lo && u < hi;
+      const unsigned bal = __ballot_sync(0xffffffffu, in);
+      __syncwarp();  // every lane has read its slot before any is overwritten
+      if (in) cbuf[out + __popc(bal & ((1u << lane) - 1u))] = j;
+      out += __popc(bal);
+      __syncwarp();
+    }
+  }
+  __syncwarp();
+  return out;
+}
+
+// The CDF boundary of a row of numerators: the element (e*, j*) of the
+// ascending (e, j) order at which the cumulative mass first exceeds tau_m
+// (keep (e, j) >= (e*, j*)); returns its key (bits(e) << 32 | j).  The
+// first pass's threshold masses give an interval [lo, hi) of bit patterns
+// holding bits(e*); its elements are compacted into cbuf, and the interval
+// is narrowed by 8 each round (masses and counts of 7 interior thresholds
+// over the candidates, then compaction) until at most 32 remain, which are
+// sorted in the warp.  More than 32 equal values: the boundary is the
+// need-th smallest index among them.  Requires tau_m < total.  On return
+// [*rlo, *rhi) is the last interval, *rbelow the mass below it, and when at
+// most 32 candidates remained the lanes hold them sorted (lane_key, lane_w).
+__device__ __forceinline__ unsigned long long cdf_boundary(const float* row, int* cbuf, int Nbp, double total,
+                                                           const double (&above)[kNThr], double tau_m, uint32_t* rlo,
+                                                           uint32_t* rhi, double* rbelow, bool* sorted,
+                                                           unsigned long long* lane_key, double* lane_w) {
+  const int lane = threadIdx.x & 31;
+  // the highest threshold with mass below <= tau_m (masses below grow as the
+  // threshold falls: the qualifying thresholds are the lowest ones)
+  uint32_t lo = 0u, hi = thr_bits(kNThr - 1);
+  double below = 0.0;
+  bool found = false;
+#pragma unroll
+  for (int k = 0; k < kNThr; ++k) {
+    const double bl = total - above[k];
+    if (!found && bl <= tau_m) {
+      found = true;
+      lo = thr_bits(k);
+      below = bl;
+      hi = k == 0 ? 0x7F800000u : thr_bits(k > 0 ? k - 1 : 0);
+    }
+  }
+  bool from_row = true;
+  int n = compact_range(row, cbuf, Nbp, true, 0, lo, hi);
+  from_row = n > kSelCap;
+  while (n > 32 && hi - lo > 1u) {
+    // masses and counts at or above 7 interior thresholds of [lo, hi)
+    const uint32_t width = hi - lo;
+    uint32_t th[7];
+#pragma unroll
+    for (int k = 0; k < 7; ++k)
+      th[k] = lo + static_cast<uint32_t>((static_cast<uint64_t>(width) * (k + 1)) >> 3);
+    double ab[7], mi = 0.0;
+    int cab[7], ci = 0;
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+      ab[k] = 0.0;
+      cab[k] = 0;
+    }
+    const int items = from_row ? Nbp : n;
+    for (int x = lane; x < items; x += 32) {
+      const int j = from_row ? x : cbuf[x];
+      const float e = row[j];
+      const uint32_t u = __float_as_uint(e);
+      const bool in = u >= lo && u < hi;
+      const double w = in ? static_cast<double>(e) : 0.0;
+      mi += w;
+      ci += in;
+#pragma unroll
+      for (int k = 0; k < 7; ++k) {
+        const bool ge = u >= th[k];
+        ab[k] += ge ? w : 0.0;
+        cab[k] += (in && ge) ? 1 : 0;
       }
     }
-    hc.flush(hist, lane);
-    __syncwarp();
-    if (n <= 32 || span == 0) break;
-    hist_choose(hist, lane, sh, tau_m, lo, below);
-    span = sh;
+    const double mass_in = warp_sum_f64(mi);  // the interval's mass and count
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ci += __shfl_xor_sync(0xffffffffu, ci, o);
+    const int cnt_in = ci;
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+      ab[k] = warp_sum_f64(ab[k]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cab[k] += __shfl_xor_sync(0xffffffffu, cab[k], o);
+    }
+    // the highest threshold whose mass below stays <= tau_m (mass below
+    // grows with the threshold, so the qualifying ones are a prefix); none:
+    // the first sub-interval [lo, th[0])
+    uint32_t nlo = lo, nhi = th[0];
+    double nbelow = below;
+    int ncnt = cnt_in - cab[0];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+      const double bl = below + (mass_in - ab[k]);
+      if (bl <= tau_m) {
+        nlo = th[k];
+        nbelow = bl;
+        ncnt = cab[k] - (k < 6 ? cab[k < 6 ? k + 1 : 6] : 0);
+        nhi = k < 6 ? th[k < 6 ? k + 1 : 6] : hi;
+      }
+    }
+    lo = nlo;
+    hi = nhi;
+    below = nbelow;
+    if (from_row && ncnt <= kSelCap) {
+      n = compact_range(row, cbuf, Nbp, true, 0, lo, hi);
+      from_row = false;
+    } else if (!from_row) {
+      n = compact_range(row, cbuf, Nbp, false, n, lo, hi);
+    } else {
+      n = ncnt;
+    }
   }
-  *range_lo = lo;
-  *range_span = span;
-  *range_below = below;
+  *rlo = lo;
+  *rhi = hi;
+  *rbelow = below;
+  *sorted = n <= 32;
   if (n <= 32) {
-    unsigned long long key = ~0ull, w = 0ull;
+    unsigned long long key = ~0ull;
+    double w = 0.0;
     if (lane < n) {
-      const int j = cand[lane];
-      const uint32_t u = __float_as_uint(row[j]);
-      key = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
-      w = mass_bits(u);
+      const int j = cbuf[lane];
+      const float e = row[j];
+      key = (static_cast<unsigned long long>(__float_as_uint(e)) << 32) | static_cast<unsigned>(j);
+      w = static_cast<double>(e);
     }
     __syncwarp();
     return sort_and_cross(key, w, lane, below, tau_m, lane_key, lane_w);
   }
-  // more than 32 elements share the value lo
+  // more than 32 elements share the value lo: the boundary is the need-th
+  // smallest index among them (ascending in cbuf when it holds them)
   *lane_key = ~0ull;
-  *lane_w = 0;
-  const unsigned long long wstar = mass_bits(lo);
-  const unsigned long long need = (tau_m - below) / wstar + 1ull;
-  unsigned long long seen = 0;
+  *lane_w = 0.0;
+  const double wstar = static_cast<double>(__uint_as_float(lo));
+  double needd = floor((tau_m - below) / wstar) + 1.0;
+  const int need = needd < 1.0 ? 1 : (needd > static_cast<double>(n) ? n : static_cast<int>(needd));
   int jstar = -1;
-  for (int base = 0; base < Nbp && jstar < 0; base += 32) {
-    const int j = base + lane;
-    const bool hit = j < Nbp && __float_as_uint(row[j]) == lo;
-    const unsigned bal = __ballot_sync(0xffffffffu, hit);
-    const unsigned c = __popc(bal);
-    if (seen + c >= need) {
-      unsigned bb = bal;
-      for (unsigned long long t = seen + 1; t < need; ++t) bb &= bb - 1;  // drop lower hits
-      jstar = base + __ffs(bb) - 1;
+  if (!from_row) {
+    jstar = cbuf[need - 1];
+  } else {
+    int seen = 0;
+    for (int base = 0; base < Nbp && jstar < 0; base += 32) {
+      const int j = base + lane;
+      const bool hit = j < Nbp && __float_as_uint(row[j]) == lo;
+      const unsigned bal = __ballot_sync(0xffffffffu, hit);
+      const int c = __popc(bal);
+      if (seen + c >= need) {
+        unsigned bb = bal;
+        for (int t = seen + 1; t < need; ++t) bb &= bb - 1;  // drop lower hits
+        jstar = base + __ffs(bb) - 1;
+      }
+      seen += c;
     }
-    seen += c;
   }
   return (static_cast<unsigned long long>(lo) << 32) | static_cast<unsigned>(jstar);
 }
 
 // Selects the kept blocks of query block i from its scores, one warp:
 //   1. m = max_j s_j;
-//   2. e_j = exp(s_j - m) (numerator_pass), the masses floor(e * 2^40) and
-//      their total; the arg-max;
+//   2. e_j = exp(s_j - m) (numerator_pass), their total and threshold
+//      masses in fp64; the arg-max;
 //   3. the CDF boundary (cdf_boundary) on these e;
 //   4. exactness: e_j differs from the correctly rounded value by at most
 //      2 ulp, so the order statistics shift by at most 2 ulp and only blocks
 //      within 8 ulp of the boundary value B can be ordered differently.
-//      Those (gathered from the last range, or by one more pass) get the
+//      Those (taken from the last interval, or by one more pass) get the
 //      correctly rounded e (scores re-read through score_of) and are sorted
 //      again on top of the mass below B - 8 ulp: the boundary is then the
 //      one of the exact order.  (More than 32 such blocks: the whole row is
 //      recomputed exactly and searched again.)
-//   5. STA window blocks marked +inf, then keep = (e, j) >= (e*, j*), the
-//      arg-max, or the window, compacted ascending with warp ballots.
-// row: Nbp scores in shared memory, -inf past Nb; overwritten.
+//   5. static windows (STA, radial) marked +inf, then keep = (e, j) >=
+//      (e*, j*), the arg-max, or a window, compacted ascending with ballots.
+// row: Nbp scores in shared memory, -inf past Nb; overwritten.  cbuf:
+// kSelCap candidate slots; cand: 32 slots.
 template <class ScoreFn>
-__device__ __forceinline__ void select_row(float* row, unsigned long long* hist, int* cand, int Nb, int i, const MaskArgs& a,
-                           int32_t* out, int32_t* count_out, const ScoreFn& score_of) {
+__device__ __forceinline__ void select_row(float* row, int* cbuf, int* cand, int Nb, int i, const MaskArgs& a,
+                                           int32_t* out, int32_t* count_out, const ScoreFn& score_of) {
   const int lane = threadIdx.x & 31;
   const int Nbp = kbar_cols(Nb);
   const float4* row4 = reinterpret_cast<const float4*>(row);
@@ -468,64 +518,76 @@ __device__ __forceinline__ void select_row(float* row, unsigned long long* hist,
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
 
-  unsigned long long total, low;
-  int argmax = numerator_pass<false>(row, hist, Nb, Nbp, m, score_of, total, low);
-  unsigned long long tau_m = static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
+  double total, above[kNThr];
+  int argmax = numerator_pass<false>(row, Nb, Nbp, m, score_of, total, above);
+  double tau_m = a.tau * total;
   unsigned long long kstar = kInfKey;  // thr = 0: the CDF keeps nothing but the arg-max
   if (!a.keep_all && total > tau_m) {
-    uint32_t lo;
-    int span;
-    unsigned long long below, lkey, lw;
-    const unsigned long long kfast = cdf_boundary(row, hist, cand, Nbp, tau_m, low, &lo, &span, &below, &lkey, &lw);
+    uint32_t lo, hi;
+    double below, lw;
+    bool sorted;
+    unsigned long long lkey;
+    const unsigned long long kfast =
+        cdf_boundary(row, cbuf, Nbp, total, above, tau_m, &lo, &hi, &below, &sorted, &lkey, &lw);
     const uint32_t B = static_cast<uint32_t>(kfast >> 32);
     const uint32_t wlo = B - kWindowUlps, whi = B + kWindowUlps;
-    // the window's blocks and the mass below it
-    unsigned long long base = 0;
+    double base = 0.0;
     int nw = 0;
     unsigned long long wkey = ~0ull;
-    if (wlo >= lo && whi - lo < (1u << span)) {
-      // the last range held every block of the window, sorted in lkey/lw
-      const uint32_t u = static_cast<uint32_t>(lkey >> 32);
-      const bool inw = lkey != ~0ull && u >= wlo && u <= whi;
-      base = below + warp_sum_u64(lkey != ~0ull && u < wlo ? lw : 0ull);
-      const unsigned bal = __ballot_sync(0xffffffffu, inw);
-      nw = __popc(bal);
-      if (inw) cand[__popc(bal & ((1u << lane) - 1u))] = static_cast<int>(lkey & 0xffffffffu);
-    } else {
-      unsigned long long ml = 0;
-      for (int base_j = 0; base_j < Nbp; base_j += 32) {
-        const int j = base_j + lane;
-        const uint32_t u = j < Nbp ? __float_as_uint(row[j]) : 0u;
-        if (u < wlo) ml += mass_bits(u);
-        const bool inw = u >= wlo && u <= whi;
+    if (kfast != ~0ull) {
+      if (sorted && wlo >= lo && whi < hi) {
+        // the last interval held every block of the window, sorted in lkey/lw
+        const uint32_t u = static_cast<uint32_t>(lkey >> 32);
+        const bool inw = lkey != ~0ull && u >= wlo && u <= whi;
+        base = below + warp_sum_f64(lkey != ~0ull && u < wlo ? lw : 0.0);
         const unsigned bal = __ballot_sync(0xffffffffu, inw);
-        if (inw && nw + __popc(bal & ((1u << lane) - 1u)) < 32) cand[nw + __popc(bal & ((1u << lane) - 1u))] = j;
-        nw += __popc(bal);
+        nw = __popc(bal);
+        if (inw) cand[__popc(bal & ((1u << lane) - 1u))] = static_cast<int>(lkey & 0xffffffffu);
+      } else {
+        double ml = 0.0;
+        for (int base_j = 0; base_j < Nbp; base_j += 32) {
+          const int j = base_j + lane;
+          const float e = j < Nbp ? row[j] : 0.f;
+          const uint32_t u = __float_as_uint(e);
+          if (u < wlo) ml += static_cast<double>(e);
+          const bool inw = j < Nbp && u >= wlo && u <= whi;
+          const unsigned bal = __ballot_sync(0xffffffffu, inw);
+          if (inw && nw + __popc(bal & ((1u << lane) - 1u)) < 32) cand[nw + __popc(bal & ((1u << lane) - 1u))] = j;
+          nw += __popc(bal);
+        }
+        base = warp_sum_f64(ml);
       }
-      base = warp_sum_u64(ml);
     }
     __syncwarp();
-    if (nw <= 32) {
-      unsigned long long w = 0;
+    if (kfast == ~0ull) {
+      // fp64 rounding put the crossing just past the last candidate (a band
+      // case): keep what lies above the interval
+      kstar = static_cast<unsigned long long>(hi) << 32;
+    } else if (nw <= 32) {
+      double w = 0.0;
       if (lane < nw) {
         const int j = cand[lane];
         const float e = exp_rounded(__fsub_rn(score_of(j), m));
         row[j] = e;
         const uint32_t u = __float_as_uint(e);
         wkey = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);
-        w = mass_bits(u);
+        w = static_cast<double>(e);
       }
       __syncwarp();
-      unsigned long long k2, w2;
+      unsigned long long k2;
+      double w2;
       kstar = sort_and_cross(wkey, w, lane, base, tau_m, &k2, &w2);
       if (kstar == ~0ull) kstar = kfast;  // crossing outside the window: a band block, either is allowed
     } else {
       // many blocks within a few ulp of the boundary: exact numerators for the
       // whole row, then the search again (no window step needed)
-      argmax = numerator_pass<true>(row, hist, Nb, Nbp, m, score_of, total, low);
-      tau_m = static_cast<unsigned long long>(floor(a.tau * static_cast<double>(total)));
+      argmax = numerator_pass<true>(row, Nb, Nbp, m, score_of, total, above);
+      tau_m = a.tau * total;
       kstar = kInfKey;
-      if (total > tau_m) kstar = cdf_boundary(row, hist, cand, Nbp, tau_m, low, &lo, &span, &below, &lkey, &lw);
+      if (total > tau_m) {
+        kstar = cdf_boundary(row, cbuf, Nbp, total, above, tau_m, &lo, &hi, &below, &sorted, &lkey, &lw);
+        if (kstar == ~0ull) kstar = static_cast<unsigned long long>(hi) << 32;
+      }
     }
     __syncwarp();
   }
@@ -693,15 +755,15 @@ inline cudaError_t launch_score_tiles(const float* qT, const float* kT, float* o
 // One warp per row of the score scratch (rows taken in reverse order of the
 // score kernel's writes, so the first ones read are still in L2).  Shared
 // memory per warp: select_warp_bytes(Nb).
-__global__ void __launch_bounds__(256) select_rows_kernel(const MaskArgs a, const float* __restrict__ scores,
+__global__ void __launch_bounds__(256, 1) select_rows_kernel(const MaskArgs a, const float* __restrict__ scores,
                                                           int64_t rows_total) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int Nb = a.Nb, Nbp = kbar_cols(Nb);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   unsigned char* mine = smem_raw + static_cast<size_t>(warp) * select_warp_bytes(Nb);
-  unsigned long long* hist = reinterpret_cast<unsigned long long*>(mine);
-  int* cand = reinterpret_cast<int*>(mine + 32 * 32 * 8);
-  float* row = reinterpret_cast<float*>(mine + 32 * 32 * 8 + 32 * 4);
+  int* cbuf = reinterpret_cast<int*>(mine);
+  int* cand = cbuf + kSelCap;
+  float* row = reinterpret_cast<float*>(cand + 32);
   const int64_t lin = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
   if (lin >= rows_total) return;
   const int64_t rid = rows_total - 1 - lin;
@@ -721,7 +783,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const MaskArgs a, cons
     row4[c] = v;
   }
   __syncwarp();
-  select_row(row, hist, cand, Nb, i, a, a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb), a.kv_count + bh * Nb + i,
+  select_row(row, cbuf, cand, Nb, i, a, a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb), a.kv_count + bh * Nb + i,
              [src](int j) { return src[j]; });
 }
 
@@ -735,9 +797,9 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const MaskArgs a, cons
 // selects rows warp, warp + 8, ... with select_row (exact numerators near
 // the boundary from a scalar recomputation of the same chain).
 // Shared memory: q pairs [D][R], score rows [R][Nbp], per-warp selection
-// scratch (histograms, candidates; the rows are the score rows).
+// scratch (candidate slots; the rows are the score rows).
 template <int R>
-__global__ void __launch_bounds__(kMaskThreads) mask_rows_smem_kernel(const MaskArgs a) {
+__global__ void __launch_bounds__(kMaskThreads, 1) mask_rows_smem_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int D = a.D, Nb = a.Nb, Nbp = kbar_cols(Nb);
   unsigned long long* qd = reinterpret_cast<unsigned long long*>(smem_raw);  // [D][R]
@@ -798,8 +860,8 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_smem_kernel(const Mask
   }
   __syncthreads();
 
-  unsigned long long* hist = reinterpret_cast<unsigned long long*>(sel + static_cast<size_t>(warp) * (32 * 32 * 8 + 32 * 4));
-  int* cand = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(hist) + 32 * 32 * 8);
+  int* cbuf = reinterpret_cast<int*>(sel + static_cast<size_t>(warp) * (kSelCap + 32) * 4);
+  int* cand = cbuf + kSelCap;
   for (int r = warp; r < R; r += kMaskWarps) {
     const int i = i0 + r;
     if (i >= Nb) break;
@@ -810,7 +872,7 @@ __global__ void __launch_bounds__(kMaskThreads) mask_rows_smem_kernel(const Mask
         acc = __fmaf_rn(__uint_as_float(static_cast<uint32_t>(qd[d * R + rr])), kt[static_cast<int64_t>(d) * Nbp + j], acc);
       return __fmul_rn(acc, a.scale);
     };
-    select_row(rows + static_cast<size_t>(r) * Nbp, hist, cand, Nb, i, a,
+    select_row(rows + static_cast<size_t>(r) * Nbp, cbuf, cand, Nb, i, a,
                a.kv_idx + (bh * Nb + i) * static_cast<int64_t>(Nb), a.kv_count + bh * Nb + i, score_of);
   }
 }

@@ -8,7 +8,6 @@
 
 #include <cmath>
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -157,7 +156,7 @@ int permute(const void* in, void* out, int B, int T, int H, int W, int P, int ro
 // eight warps' selection scratch.
 size_t mask_smem_bytes(int R, int D, int Nb) {
   return static_cast<size_t>(R) * D * 8 + static_cast<size_t>(R) * kbar_cols(Nb) * 4 +
-         static_cast<size_t>(kMaskWarps) * (32 * 32 * 8 + 32 * 4);
+         static_cast<size_t>(kMaskWarps) * (kSelCap + 32) * 4;
 }
 
 template <int R>
@@ -305,16 +304,6 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 // comes from cudaGetSymbolAddress with the caller's device current.
 __device__ __align__(256) unsigned char g_noalloc_scratch[NABLA_NOALLOC_SCRATCH_BYTES];
 
-// Variant of the attention kernel: QK^T over pairs of listed key blocks (N =
-// 128) when NABLA_ATTN_PAIR_QK=1 in the environment (read once).
-bool attn_pair_qk() {
-  static const bool pair = [] {
-    const char* e = std::getenv("NABLA_ATTN_PAIR_QK");
-    return e != nullptr && e[0] == '1';
-  }();
-  return pair;
-}
-
 // Shared body of the two attention entry points; grp_F > 0 selects the 2 x 2
 // (w, t) grouping of query blocks (grp_F blocks per frame, grp_nbw per row).
 int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
@@ -368,7 +357,6 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   a.in_inv_nbw = inv(a.in_nbw);
   a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
   const dim3 grid((Nb + 1) / 2, Hh, B);
-  const bool pair = attn_pair_qk();
   auto go = [&](auto kernel, size_t smem) -> int {
     if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
@@ -377,41 +365,7 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
     kernel<<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
     return launch_status();
   };
-  if (D == 128)
-    return pair ? go(attn_fwd_kernel<128, true>, AttnSmem<128>::bytes(Nb))
-                : go(attn_fwd_kernel<128, false>, AttnSmem<128>::bytes(Nb));
-  return pair ? go(attn_fwd_kernel<64, true>, AttnSmem<64>::bytes(Nb))
-              : go(attn_fwd_kernel<64, false>, AttnSmem<64>::bytes(Nb));
-}
-
-// Backward launches: Delta, then dQ over the row lists, then dK and dV over
-// the column lists.
-template <int D>
-int launch_bwd(const BwdArgs& a, const void* out, int B, const DeviceInfo& di, cudaStream_t stream) {
-  const size_t smem = BwdTile<D>::kSmemBytes;
-  if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
-  if (cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return NABLA_ERR_CUDA;
-  const int64_t rows = static_cast<int64_t>(B) * a.S;
-  bwd_delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(out), a.dout, const_cast<float*>(a.delta), rows, a.S, a.Hh, D);
-  const dim3 grid(a.Nb, a.Hh, B);
-  bwd_dq_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a);
-  bwd_dkdv_kernel<D><<<grid, kBwdThreads, smem, stream>>>(a);
-  return launch_status();
-}
-
-// Backward kernels on tcgen05 when NABLA_BWD_TC=1 in the environment (read
-// once; the warp-MMA kernels of attn_bwd.cuh otherwise).
-bool bwd_tc() {
-  static const bool on = [] {
-    const char* e = std::getenv("NABLA_BWD_TC");
-    return e != nullptr && e[0] == '1';
-  }();
-  return on;
+  return D == 128 ? go(attn_fwd_kernel<128>, AttnSmem<128>::bytes(Nb)) : go(attn_fwd_kernel<64>, AttnSmem<64>::bytes(Nb));
 }
 
 // Delta, then the dQ kernel over the row lists and the dK/dV kernel over the
@@ -419,8 +373,11 @@ bool bwd_tc() {
 template <int D>
 int launch_bwd_tc(const BwdArgs& ba, const void* qf, const void* kf, const void* vf, const void* out, int B,
                   const DeviceInfo& di, cudaStream_t stream) {
-  const size_t smem = BwdTcSmem<D>::bytes(ba.Nb);
-  if (smem > static_cast<size_t>(di.max_smem_optin) || ba.Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
+  // four walked stages where the lists leave room, else two
+  const size_t optin = static_cast<size_t>(di.max_smem_optin);
+  const bool deep = BwdTcSmem<D, 4>::bytes(ba.Nb) <= optin;
+  const size_t smem = deep ? BwdTcSmem<D, 4>::bytes(ba.Nb) : BwdTcSmem<D, 2>::bytes(ba.Nb);
+  if (smem > optin || ba.Nb > kMaxListBlocks) return NABLA_ERR_INVALID;
   CUtensorMap tq, tk, tv, tdo;
   const bool grid = ba.W > 0;
   const int T = grid ? ba.S / (ba.H * ba.W) : 0;
@@ -449,22 +406,24 @@ int launch_bwd_tc(const BwdArgs& ba, const void* qf, const void* kf, const void*
   const int64_t rows = static_cast<int64_t>(B) * ba.S;
   bwd_delta_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(out), ba.dout, const_cast<float*>(ba.delta), rows, ba.S, ba.Hh, D);
-  if (cudaFuncSetAttribute(bwd_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess ||
-      cudaFuncSetAttribute(bwd_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  auto* kdq = deep ? bwd_tc_kernel<D, true, 4> : bwd_tc_kernel<D, true, 2>;
+  auto* kdkdv = deep ? bwd_tc_kernel<D, false, 4> : bwd_tc_kernel<D, false, 2>;
+  if (cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess)
     return NABLA_ERR_CUDA;
   const dim3 g((ba.Nb + 1) / 2, ba.Hh, B);
   a.row_count = ba.kv_count;
   a.row_idx = ba.kv_idx;
   a.out0 = ba.dq;
   a.out1 = nullptr;
-  bwd_tc_kernel<D, true><<<g, kBwdTcThreads, smem, stream>>>(tq, tdo, tk, tv, a);
+  kdq<<<g, kBwdTcThreads, smem, stream>>>(tq, tdo, tk, tv, a);
   a.row_count = ba.q_count;
   a.row_idx = ba.q_idx;
   a.out0 = ba.dk;
   a.out1 = ba.dv;
-  bwd_tc_kernel<D, false><<<g, kBwdTcThreads, smem, stream>>>(tk, tv, tq, tdo, a);
+  kdkdv<<<g, kBwdTcThreads, smem, stream>>>(tk, tv, tq, tdo, a);
   return launch_status();
 }
 
@@ -508,12 +467,9 @@ int sparse_attn_bwd(const void* qf, const void* kf, const void* vf, const void* 
   a.W = W;
   a.nbw = W / 8;
   a.per_t = (H / 8) * (W / 8);
-  if (bwd_tc()) {
-    if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
-    return D == 128 ? launch_bwd_tc<128>(a, qf, kf, vf, out, B, di, stream)
-                    : launch_bwd_tc<64>(a, qf, kf, vf, out, B, di, stream);
-  }
-  return D == 128 ? launch_bwd<128>(a, out, B, di, stream) : launch_bwd<64>(a, out, B, di, stream);
+  if (!di.sm100) return NABLA_ERR_UNSUPPORTED;
+  return D == 128 ? launch_bwd_tc<128>(a, qf, kf, vf, out, B, di, stream)
+                  : launch_bwd_tc<64>(a, qf, kf, vf, out, B, di, stream);
 }
 
 // AB-Attention plan workspace: kbar^T [B*Hh][D][NKB], cent^T [B*Hh][D][R],
@@ -856,6 +812,28 @@ int nabla_ab_attn_fwd(const void* q, const void* k, const void* v, const int32_t
       return NABLA_ERR_CUDA;
     ab_attn_fwd_kernel<64><<<grid, kABAttnThreads, smem, stream>>>(tq, a);
   }
+  return launch_status();
+}
+
+__global__ void exp2_poly_selftest_kernel(const float2* __restrict__ x, float2* __restrict__ y, int64_t pairs) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < pairs;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float2 v = x[i];
+    const unsigned long long r = exp2_poly_f2(f2_pack(v.x, v.y));
+    y[i] = make_float2(f2_lo(r), f2_hi(r));
+  }
+}
+
+int nabla_selftest_exp2_poly(const float* x, float* y, int64_t n, nabla_stream_t stream_) {
+  NABLA_NVTX_RANGE();
+  if (n < 0 || (n & 1) || (n > 0 && (x == nullptr || y == nullptr))) return NABLA_ERR_INVALID;
+  if (n == 0) return NABLA_OK;
+  if (!aligned16(x) || !aligned16(y)) return NABLA_ERR_ALIGN;
+  const int64_t pairs = n / 2;
+  const int64_t blocks = (pairs + 255) / 256;
+  exp2_poly_selftest_kernel<<<static_cast<unsigned>(blocks < 1184 ? blocks : 1184), 256, 0,
+                              reinterpret_cast<cudaStream_t>(stream_)>>>(reinterpret_cast<const float2*>(x),
+                                                                          reinterpret_cast<float2*>(y), pairs);
   return launch_status();
 }
 
