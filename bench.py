@@ -75,12 +75,28 @@ def whole_job_tflops(world: int, flop_per_step_per_rank: float, steps: int, max_
 
 
 def load_peaks():
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, HBM GB/s, kind): the
+    measured figures, else this pool's earlier measurements."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as fh:
             d = json.load(fh)
-        return float(d["bf16_tflops"]), float(d["hbm_gbs"]), "measured"
-    return 1590.0, 6650.0, "fallback"
+        burst = float(d["bf16_tflops"])
+        return burst, float(d.get("bf16_tflops_sustained", burst)), float(d["hbm_gbs"]), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# A kernel timed inside a timed region at least this long runs under the
+# power cap (the long-video layer's 20 steps take ~1.4 s at ~1.4 GHz), so its
+# roofline takes the sustained bf16 figure; shorter regions take the burst one.
+SUSTAINED_REGION_MS = 500.0
+
+
+def tensor_peak(timed_ms: float):
+    burst, sustained, _, kind = load_peaks()
+    if timed_ms >= SUSTAINED_REGION_MS:
+        return sustained, burst, f"{kind} bf16 sustained (timed region {timed_ms / 1e3:.2f} s, under the power cap)"
+    return burst, burst, f"{kind} bf16 burst"
 
 
 def config_dict(w: inputs.Workload):
@@ -383,7 +399,8 @@ def run_gpu(args, rank, world, local_rank):
                     "steps": args.backward_steps, "launches_per_step": 4}
         del do, q_count, q_idx, dq_, dk_, dv_, delta
 
-    peak_tf, peak_gbs, peak_kind = load_peaks()
+    _, _, peak_gbs, peak_kind = load_peaks()
+    peak_tf, burst_tf, tf_kind = tensor_peak(total_ms_max)
     attn_avg = statistics.mean(attn_ms)
     mask_avg = statistics.mean(mask_ms)
     mask_gbs = (mask_bytes(w, total_kept) - (0 if not static else 4.0 * w.B * w.S * w.Hh * w.D)) / \
@@ -417,8 +434,8 @@ def run_gpu(args, rank, world, local_rank):
         "pool_gbs": None if static else pool_bytes(w) / (statistics.mean(pool_ms) * 1e-3) / 1e9,
         "kept_tile_fraction": total_kept / (w.B * w.Hh * w.Nb * w.Nb),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
-                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
-                     "traffic": traffic},
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": tf_kind,
+                     "frac_of_burst": achieved / burst_tf, "traffic": traffic},
         # the mask build (pooling + rows) against HBM: Q and K read once, the
         # lists written, over the two stages' time
         "mask_roofline": None if static else {
@@ -497,7 +514,7 @@ def run_gpu_ab(args, rank, world, local_rank):
     plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in events)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in events)
     total = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in events), dev)
-    peak_tf, peak_gbs, peak_kind = load_peaks()
+    peak_tf, burst_tf, tf_kind = tensor_peak(total)
     achieved = flop / (attn_ms * 1e-3) / 1e12
     cfg = config_dict(base)
     cfg.update({"workload": w.name, "mask": "AB-Attention sample (IBCS clusters + SIP, 4-token key blocks)",
@@ -521,7 +538,7 @@ def run_gpu_ab(args, rank, world, local_rank):
         "sampled_block_fraction": sampled / (base.B * base.Hh * w.nqb * w.nkb),
         "attn_tflops_sampled": achieved,
         "roofline": {"bound": "tensor", "kernel": "ab_attn_fwd_kernel<128>", "achieved": achieved, "peak": peak_tf,
-                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": f"{peak_kind} bf16 burst",
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "peak_kind": tf_kind, "frac_of_burst": achieved / burst_tf,
                      "traffic": None},
         "clocks": clocks,
         "gpu_launches": 5 * args.steps,

@@ -50,7 +50,6 @@ EXPORTS = (
     "nabla_get_status",
     "nabla_validate_mask",
     "nabla_selftest_wait_timeout",
-    "nabla_selftest_exp2_poly",
     "nabla_strerror",
 )
 
@@ -110,7 +109,6 @@ def lib():
         L.nabla_get_status.argtypes = [vp]
         L.nabla_validate_mask.argtypes = [vp, vp, i, i, i, vp, vp]
         L.nabla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
-        L.nabla_selftest_exp2_poly.argtypes = [vp, vp, ctypes.c_int64, vp]
         L.nabla_strerror.argtypes = [i]
         L.nabla_strerror.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -511,16 +509,6 @@ def selftest_wait_timeout(limit_cycles: int = 2_000_000, stream=None) -> int:
     (synchronises; NABLA_ERR_DEVICE_TIMEOUT when the wait gave up)."""
     _check(lib().nabla_selftest_wait_timeout(int(limit_cycles), _stream(stream)), "nabla_selftest_wait_timeout")
     return get_status(stream)
-
-
-def selftest_exp2_poly(x, stream=None):
-    """2^x by the attention softmax's FMA-pipe exponential (x: CUDA fp32
-    tensor of even length); returns y."""
-    x = x.contiguous()
-    y = torch.empty_like(x)
-    _check(lib().nabla_selftest_exp2_poly(_dev(x, torch.float32, "x"), _dev(y, torch.float32, "y"), x.numel(),
-                                          _stream(stream)), "nabla_selftest_exp2_poly")
-    return y
 
 
 def default_scale(D: int) -> float:

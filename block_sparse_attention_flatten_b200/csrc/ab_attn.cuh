@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, 128);
+      mbar_init(p_full + s, 4);  // one arrival per softmax warp
       mbar_init(pv_done + s, 1);
     }
     mbar_init(mma_drain, 2);
@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
       tmem_st16(tS + 16, pk[1]);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full + (n & 1));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + (n & 1));
     }
     // ---------------------------------------------------------------- epilogue
     if (ok && n_tiles > 0)

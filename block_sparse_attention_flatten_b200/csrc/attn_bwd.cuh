@@ -15,7 +15,8 @@ namespace nabla {
 
 // ------------------------------------------------------- transposed lists
 // Column lists: for key block j of (b, head), the query blocks i whose row
-// lists j, ascending.  One warp per key block; lane l tests rows base + l by
+// lists j, ascending.  Block counts above kTransposeMaxNb: one warp per key
+// block; lane l tests rows base + l by
 // a binary search of the row's (ascending) list, and a ballot compacts the
 // hits in order.  Rows whose count is out of range are treated as empty and
 // reported.
@@ -53,6 +54,63 @@ __global__ void __launch_bounds__(256) transpose_lists_kernel(const int32_t* __r
     n += __popc(bal);
   }
   if (lane == 0) q_count[bh * Nb + j] = n;
+}
+
+// Column lists by 32 x 32 bit-tile transposes: one CTA per (32 key blocks
+// j0 .. j0+31, b, head).  Each thread takes rows i = tid, tid + 256, ...:
+// a binary search for the first entry >= j0 of the row's list, then the
+// entries below j0 + 32 set bits of a 32-bit row mask (shared memory, one
+// word per row).  Then warp w builds columns j0 + w, j0 + w + 8, ...: per
+// group of 32 rows, lane l holds row 32g + l's mask, a ballot of bit (j -
+// j0) gives the group's hits in row order, and their indices are written
+// ascending.  One binary search per (row, 32 columns) instead of per (row,
+// column).  Shared memory: Nb words.
+constexpr int kTransposeMaxNb = 49152;  // 192 KB of row masks
+__global__ void __launch_bounds__(256) transpose_lists_tiled_kernel(const int32_t* __restrict__ kv_count,
+                                                                    const int32_t* __restrict__ kv_idx,
+                                                                    int32_t* __restrict__ q_count,
+                                                                    int32_t* __restrict__ q_idx, int Nb) {
+  extern __shared__ uint32_t rowmask[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j0 = blockIdx.x * 32;
+  const int64_t bh = blockIdx.y;
+  const int32_t* cnt = kv_count + bh * Nb;
+  const int32_t* lists = kv_idx + bh * static_cast<int64_t>(Nb) * Nb;
+  for (int i = threadIdx.x; i < Nb; i += blockDim.x) {
+    int c = __ldg(cnt + i);
+    if (c < 0 || c > Nb) {
+      if (j0 == 0) report(NABLA_ERR_DEVICE_BOUNDS);
+      c = 0;
+    }
+    const int32_t* l = lists + static_cast<int64_t>(i) * Nb;
+    int lo = 0, hi = c;  // first entry >= j0 in [lo, hi)
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(l + mid) < j0) lo = mid + 1; else hi = mid;
+    }
+    uint32_t m = 0u;
+    for (; lo < c; ++lo) {
+      const int j = __ldg(l + lo);
+      if (j >= j0 + 32 || j >= Nb) break;
+      if (j >= j0) m |= 1u << (j - j0);
+    }
+    rowmask[i] = m;
+  }
+  __syncthreads();
+  for (int b = warp; b < 32; b += blockDim.x >> 5) {
+    const int j = j0 + b;
+    if (j >= Nb) break;
+    int32_t* out = q_idx + (bh * Nb + j) * static_cast<int64_t>(Nb);
+    int n = 0;
+    for (int base = 0; base < Nb; base += 32) {
+      const int i = base + lane;
+      const bool hit = i < Nb && ((rowmask[i] >> b) & 1u);
+      const unsigned bal = __ballot_sync(0xffffffffu, hit);
+      if (hit) out[n + __popc(bal & ((1u << lane) - 1u))] = i;
+      n += __popc(bal);
+    }
+    if (lane == 0) q_count[bh * Nb + j] = n;
+  }
 }
 
 // ------------------------------------------------------------------ Delta

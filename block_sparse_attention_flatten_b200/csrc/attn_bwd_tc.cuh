@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   uint64_t* w0_empty = w_full + kWS;         // [kWS] first walked tile (K or Q) free
   uint64_t* w1_empty = w0_empty + kWS;       // [kWS] second walked tile (V or dO) free
   uint64_t* s_full = w1_empty + kWS;         // [2] the tile's two products are in tensor memory
-  uint64_t* e_full = s_full + 2;             // [2] elementwise results written (512 arrivals)
+  uint64_t* e_full = s_full + 2;             // [2] elementwise results written (one arrival per warp)
   uint64_t* acc_done = e_full + 2;           // [2] the accumulating products of the tile are done
   uint64_t* drain = acc_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(e_full + s, kBwdTcElemThreads);
+      mbar_init(e_full + s, kBwdTcElemThreads / 32);  // one arrival per warp
       mbar_init(acc_done + s, 1);
     }
     mbar_init(drain, 2);
@@ -411,7 +411,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(e_full + s);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(e_full + s);
     }
     // ---------------------------------------------------------------- epilogue
     if (ok && L_n > 0)

@@ -46,14 +46,6 @@ namespace nabla {
 
 constexpr int kAttnThreads = 224;
 constexpr int kMaxListBlocks = 16383;  // list entries hold a 14-bit block index
-// Softmax exponentials: of every 8 column pairs, those whose bit is set here
-// go to the FMA pipe (exp2_poly_f2), the others to the MUFU.  A step of
-// 128 query rows x 64 keys at D = 128 is 4.2 MFLOP of MMAs, about 512
-// clocks of an SM's tensor cores, and 8192 exponentials, 512 clocks of its
-// MUFU (16 per clock): with every exponential on the MUFU the softmax could
-// keep pace with the MMAs only at perfect overlap.  3 of 8 pairs on the FMA
-// pipe leave both pipes with slack.
-constexpr uint32_t kExpPolyPairs = 0x52u;  // pairs 1, 4, 6
 
 template <int D>
 struct AttnSmem {
@@ -179,7 +171,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(p_full + s, 128);
+      mbar_init(p_full + s, 4);  // one arrival per softmax warp
       mbar_init(pv_done + s, 1);
     }
     mbar_init(mma_drain, 2);  // one commit from each MMA-issuing thread
@@ -488,14 +480,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           float p0 = 0.f, p1 = 0.f;
           if (inc) {
             const unsigned long long x2 = f2_fma((static_cast<unsigned long long>(sv[c][e + 1]) << 32) | sv[c][e], sc2, nm2);
-            if ((kExpPolyPairs >> (e / 2)) & 1u) {
-              const unsigned long long p2 = exp2_poly_f2(x2);
-              p0 = f2_lo(p2);
-              p1 = f2_hi(p2);
-            } else {
-              p0 = ex2_approx(f2_lo(x2));
-              p1 = ex2_approx(f2_hi(x2));
-            }
+            p0 = ex2_approx(f2_lo(x2));
+            p1 = ex2_approx(f2_hi(x2));
           }
           rs2[c] = f2_add(rs2[c], f2_pack(p0, p1));
           const int k = c * 8 + e / 2;
@@ -530,7 +516,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tmem_st16(tS + 16, pk[1]);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full + (n & 1));
+      // one arrival per warp, after every lane's stores have completed: 128
+      // arrivals on one mbarrier serialised in shared memory on the softmax's
+      // critical path
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + (n & 1));
     }
 
     // ---------------------------------------------------------------- epilogue

@@ -273,34 +273,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on two fp32 lanes without the special-function unit (the softmax of
-// the attention kernels puts part of its exponentials here so that they
-// share the work between the MUFU and the FMA pipe).  Range reduction
-// x = n + f, n = round-to-nearest(x) by adding and subtracting the shifter
-// 1.5 * 2^23 (then f = x - n is exact, |f| <= 1/2); 2^f by a degree-3
-// polynomial, the relative-error minimax fit on [-1/2, 1/2] (Lawson's
-// iteratively reweighted least squares, reproduced by fit_exp2_poly.py next
-// to this file): relative error below 7.6e-5 including the fp32 Horner
-// steps, far under the bf16 rounding the probabilities get; n is then added
-// to the exponent field (the low bits of the shifted sum hold n).  x is
-// clamped to >= -125 so the result stays normal: below that it returns
-// 2^-125-ish instead of a smaller number, an absolute error under 2^-124.
-// x must be <= 126 (the softmax's x never exceeds its lazy-rescale margin).
-constexpr float kExp2C0 = 0.99992811f, kExp2C1 = 0.69326099f, kExp2C2 = 0.24261054f, kExp2C3 = 0.05517132f;
-__device__ __forceinline__ unsigned long long exp2_poly_f2(unsigned long long x2) {
-  const float shifter = 12582912.f;  // 1.5 * 2^23
-  const unsigned long long xc = f2_pack(fmaxf(f2_lo(x2), -125.f), fmaxf(f2_hi(x2), -125.f));
-  const unsigned long long t = f2_add(xc, f2_pack(shifter, shifter));
-  const unsigned long long n = f2_add(t, f2_pack(-shifter, -shifter));
-  const unsigned long long f = f2_fma(n, f2_pack(-1.f, -1.f), xc);
-  unsigned long long q = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
-  q = f2_fma(q, f, f2_pack(kExp2C1, kExp2C1));
-  q = f2_fma(q, f, f2_pack(kExp2C0, kExp2C0));
-  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
-  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
-  return (static_cast<unsigned long long>(hi) << 32) | lo;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -567,7 +567,7 @@ __device__ __forceinline__ void select_row(float* row, int* cbuf, int* cand, int
       double w = 0.0;
       if (lane < nw) {
         const int j = cand[lane];
-        const float e = exp_rounded(__fsub_rn(score_of(j), m));
+        const float e = j < Nb ? exp_rounded(__fsub_rn(score_of(j), m)) : 0.f;  // padding stays 0
         row[j] = e;
         const uint32_t u = __float_as_uint(e);
         wkey = (static_cast<unsigned long long>(u) << 32) | static_cast<unsigned>(j);

@@ -653,7 +653,16 @@ int nabla_transpose_lists(const int32_t* kv_count, const int32_t* kv_idx, int B,
   DeviceInfo di;
   int rc = device_info(&di);
   if (rc != NABLA_OK) return rc;
-  transpose_lists_kernel<<<dim3((Nb + 7) / 8, B * Hh), 256, 0, stream>>>(kv_count, kv_idx, q_count, q_idx, Nb);
+  const size_t smem = static_cast<size_t>(Nb) * 4;
+  if (Nb <= kTransposeMaxNb && smem <= static_cast<size_t>(di.max_smem_optin)) {
+    if (cudaFuncSetAttribute(transpose_lists_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    transpose_lists_tiled_kernel<<<dim3((Nb + 31) / 32, B * Hh), 256, smem, stream>>>(kv_count, kv_idx, q_count,
+                                                                                     q_idx, Nb);
+  } else {
+    transpose_lists_kernel<<<dim3((Nb + 7) / 8, B * Hh), 256, 0, stream>>>(kv_count, kv_idx, q_count, q_idx, Nb);
+  }
   return launch_status();
 }
 
@@ -812,28 +821,6 @@ int nabla_ab_attn_fwd(const void* q, const void* k, const void* v, const int32_t
       return NABLA_ERR_CUDA;
     ab_attn_fwd_kernel<64><<<grid, kABAttnThreads, smem, stream>>>(tq, a);
   }
-  return launch_status();
-}
-
-__global__ void exp2_poly_selftest_kernel(const float2* __restrict__ x, float2* __restrict__ y, int64_t pairs) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < pairs;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float2 v = x[i];
-    const unsigned long long r = exp2_poly_f2(f2_pack(v.x, v.y));
-    y[i] = make_float2(f2_lo(r), f2_hi(r));
-  }
-}
-
-int nabla_selftest_exp2_poly(const float* x, float* y, int64_t n, nabla_stream_t stream_) {
-  NABLA_NVTX_RANGE();
-  if (n < 0 || (n & 1) || (n > 0 && (x == nullptr || y == nullptr))) return NABLA_ERR_INVALID;
-  if (n == 0) return NABLA_OK;
-  if (!aligned16(x) || !aligned16(y)) return NABLA_ERR_ALIGN;
-  const int64_t pairs = n / 2;
-  const int64_t blocks = (pairs + 255) / 256;
-  exp2_poly_selftest_kernel<<<static_cast<unsigned>(blocks < 1184 ? blocks : 1184), 256, 0,
-                              reinterpret_cast<cudaStream_t>(stream_)>>>(reinterpret_cast<const float2*>(x),
-                                                                          reinterpret_cast<float2*>(y), pairs);
   return launch_status();
 }
 

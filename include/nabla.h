@@ -421,15 +421,6 @@ int nabla_validate_mask(const int32_t* kv_count, const int32_t* kv_idx, int B, i
  * range. */
 int nabla_selftest_wait_timeout(long long limit_cycles, nabla_stream_t stream);
 
-/* Numerical self-test of the attention softmax's FMA-pipe exponential (no
- * counterpart in the paper): y[i] = 2^x[i] as the forward kernel computes it
- * for the column pairs it keeps off the MUFU (range reduction to [-1/2, 1/2],
- * degree-3 polynomial, exponent insertion; x clamped to >= -125).  x and y:
- * device fp32 arrays of n elements (n >= 0, even; 16-byte aligned), owned by
- * the caller.  Asynchronous.  NABLA_ERR_INVALID for a null pointer with
- * n > 0 or an odd n, NABLA_ERR_ALIGN for misaligned arrays. */
-int nabla_selftest_exp2_poly(const float* x, float* y, int64_t n, nabla_stream_t stream);
-
 /* Static description of an error code. */
 const char* nabla_strerror(int code);
 

@@ -145,11 +145,6 @@ def test_invalid_arguments_rejected_before_launch(lib):
 def test_selftest_rejects_out_of_range_limits(lib):
     assert lib.nabla_selftest_wait_timeout(10, None) == nabla.NABLA_ERR_INVALID
     assert lib.nabla_selftest_wait_timeout(10 ** 12, None) == nabla.NABLA_ERR_INVALID
-    fake = ctypes.c_void_p(0x1000)
-    assert lib.nabla_selftest_exp2_poly(fake, fake, 3, None) == nabla.NABLA_ERR_INVALID  # odd n
-    assert lib.nabla_selftest_exp2_poly(None, None, 2, None) == nabla.NABLA_ERR_INVALID
-    assert lib.nabla_selftest_exp2_poly(None, None, 0, None) == nabla.NABLA_OK  # nothing to do
-    assert lib.nabla_selftest_exp2_poly(ctypes.c_void_p(0x1004), fake, 2, None) == nabla.NABLA_ERR_ALIGN
 
 
 def test_binding_refuses_cpu_tensors(lib):

@@ -56,3 +56,20 @@ def test_single_rank_is_its_own_maximum():
     import bench
     assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
     assert bench.whole_job_tflops(1, 1.0e12, 4, 2.0) == pytest.approx(1.0e12 * 4 / 2e-3 / 1e12)
+
+
+def test_peak_choice_follows_the_timed_region(tmp_path, monkeypatch):
+    """A kernel timed inside a long (power-capped) region is rated against
+    the sustained bf16 figure, a short burst against the burst figure."""
+    import json
+
+    import bench
+    peaks = {"bf16_tflops": 1615.5, "bf16_tflops_sustained": 1402.0, "hbm_gbs": 6559.0}
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(peaks))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peak, burst, kind = bench.tensor_peak(1360.0)
+    assert (peak, burst) == (1402.0, 1615.5) and "sustained" in kind
+    peak, burst, kind = bench.tensor_peak(22.0)
+    assert (peak, burst) == (1615.5, 1615.5) and "burst" in kind
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "absent"))
+    assert bench.tensor_peak(22.0)[0] == 1590.0 and bench.tensor_peak(2000.0)[0] == 1400.0
