@@ -357,6 +357,27 @@ def run_gpu(args, rank, world, local_rank):
                "unit": "TFLOP/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                "ms_per_step": te / len(e2e_ms)}
 
+    # the materialised fractal flattening (not on the hot path: the pooling
+    # and the attention's loads flatten on the fly), timed over back-to-back
+    # launches so the writes still draining from L2 at a launch's end are
+    # charged to the next one; not part of `value`
+    flatten = None
+    if not static and args.flatten_launches > 0:
+        qflat = torch.empty_like(qd)
+        nabla.flatten(qd, w.T, w.H, w.W, out=qflat)
+        torch.cuda.synchronize()
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        fe[0].record(stream)
+        for _ in range(args.flatten_launches):
+            nabla.flatten(qd, w.T, w.H, w.W, out=qflat)
+        fe[1].record(stream)
+        torch.cuda.synchronize()
+        t_fl = fe[0].elapsed_time(fe[1]) / args.flatten_launches
+        nbytes = 2.0 * qd.numel() * qd.element_size()
+        flatten = {"ms_per_tensor": t_fl, "gbs": nbytes / (t_fl * 1e-3) / 1e9, "bytes_per_launch": nbytes,
+                   "launches": args.flatten_launches, "timing": "back-to-back launches, CUDA events"}
+        del qflat
+
     # backward pass over the same lists (training), timed on its own: the
     # column lists, then Delta, dQ and dK/dV; not part of `value`
     backward = None
@@ -451,6 +472,7 @@ def run_gpu(args, rank, world, local_rank):
             "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"},
         "e2e": e2e,
         "backward": backward,
+        "flatten": flatten,
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
@@ -715,6 +737,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--backward-steps", type=int, default=20, help="timed steps of the backward pass (0: skip)")
+    ap.add_argument("--flatten-launches", type=int, default=10,
+                    help="back-to-back launches of the materialised flattening to time (0: skip)")
     ap.add_argument("--cpu-blocks", type=int, default=8, help="query blocks in the CPU-baseline sample")
     ap.add_argument("--ref-blocks", type=int, default=2, help="query blocks per reference-arm step")
     ap.add_argument("--ref-heads", type=int, default=1, help="heads per reference-arm step")

@@ -26,25 +26,31 @@
 namespace nabla {
 
 // ------------------------------------------------------------------ pooling
-// grid (Nb, B, 2): z = 0 pools Q into qbar [B][Hh][Nb][D], z = 1 pools K
-// into kbar^T [B][Hh][D][Nbp] (Nbp = Nb rounded up to a multiple of 4; the
-// padding columns are never written).
-// Thread c handles elements 8c..8c+7 of a token row (Hh*D elements), summing
-// the block's 64 rows in ascending flattened order in fp32.
+// grid (Nb, B, 2 * slices), kPoolThreads threads: z & 1 = 0 pools Q into
+// qbar^T, 1 pools K into kbar^T, both [B][Hh][D][Nbp] (Nbp = Nb rounded up
+// to a multiple of 4; the padding columns are never written); z >> 1 is the
+// CTA's slice of kPoolThreads 16-byte chunks of a token row.  Thread c of
+// the row handles elements 8c..8c+7 (Hh*D elements), summing the block's 64
+// rows in ascending flattened order in fp32, with the next 8 rows' loads
+// in flight during each 8 rows' sums.  Small CTAs keep many of them per SM
+// (the loads in flight set the bandwidth) and split a layer into enough
+// CTAs that the last wave is a small fraction.
 // kFlatten = false: q, k are already flattened.  kFlatten = true: q, k are in
 // grid order and the block's 64 rows are gathered in flattened order; if
 // qf_out / kf_out are given the kernel also writes them there (fractal
 // flattening fused with the pooling, so Q and K are read once).  Flattened rows 8u..8u+7 of a block are one run of 8
 // consecutive grid rows (patch row u).
+constexpr int kPoolThreads = 64;
 template <bool kFlatten>
-__global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(kPoolThreads, 8) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, __nv_bfloat16* qf_out,
                                                    __nv_bfloat16* kf_out, float* __restrict__ qbar,
                                                    float* __restrict__ kbar, int S, int Hh, int D, int H, int W) {
   const int i = blockIdx.x, b = blockIdx.y;
   const int Nb = S >> 6;
-  const __nv_bfloat16* x = blockIdx.z == 0 ? q : k;
-  float* out = blockIdx.z == 0 ? qbar : kbar;
+  const int which = blockIdx.z & 1;
+  const __nv_bfloat16* x = which == 0 ? q : k;
+  float* out = which == 0 ? qbar : kbar;
   const int row = Hh * D;
   const int chunks = row >> 3;
   const int64_t batch_rows = static_cast<int64_t>(b) * S;
@@ -56,25 +62,29 @@ __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restri
     src0 = batch_rows + (static_cast<int64_t>(t) * H + bh * 8) * W + bw * 8;
   }
   const uint4* base = reinterpret_cast<const uint4*>(x) + src0 * chunks;
-  __nv_bfloat16* flat_out = blockIdx.z == 0 ? qf_out : kf_out;
+  __nv_bfloat16* flat_out = which == 0 ? qf_out : kf_out;
   uint4* dst = (kFlatten && flat_out != nullptr)
                    ? reinterpret_cast<uint4*>(flat_out) + (batch_rows + static_cast<int64_t>(i) * 64) * chunks
                    : nullptr;
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+  // rows r0..r0+7: flattened order; in grid order one run of 8 along w
+  auto load8 = [&](uint4 (&v)[8], int r0, int c) {
+    const int64_t src_row = kFlatten ? static_cast<int64_t>(r0 >> 3) * W : r0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = kFlatten ? __ldcs(base + (src_row + u) * chunks + c) : __ldg(base + (src_row + u) * chunks + c);
+  };
+  {
+    const int c = (blockIdx.z >> 1) * kPoolThreads + threadIdx.x;
+    if (c >= chunks) return;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 1
-    for (int r0 = 0; r0 < 64; r0 += 8) {
-      // rows r0..r0+7: flattened order; in grid order one run of 8 along w
-      const int64_t src_row = kFlatten ? static_cast<int64_t>(r0 >> 3) * W : r0;
-      uint4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        v[u] = kFlatten ? __ldcs(base + (src_row + u) * chunks + c) : __ldg(base + (src_row + u) * chunks + c);
+    // two groups of 8 rows in flight: the next group's loads are issued
+    // before this group's sums (the sums stay in ascending row order)
+    auto consume = [&](const uint4 (&v)[8], int g) {
       if (kFlatten && dst != nullptr) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) dst[static_cast<int64_t>(r0 + u) * chunks + c] = v[u];
+        for (int u = 0; u < 8; ++u) dst[static_cast<int64_t>(8 * g + u) * chunks + c] = v[u];
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -86,6 +96,15 @@ __global__ void __launch_bounds__(384) pool_kernel(const __nv_bfloat16* __restri
           acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], f.y);
         }
       }
+    };
+    uint4 va[8], vb[8];
+    load8(va, 0, c);
+#pragma unroll 1
+    for (int g = 0; g < 8; g += 2) {
+      load8(vb, 8 * (g + 1), c);
+      consume(va, g);
+      if (g + 2 < 8) load8(va, 8 * (g + 2), c);
+      consume(vb, g + 1);
     }
     // transposed, xbar^T [B][Hh][D][Nbp]: the score stages read a d-slice of
     // consecutive blocks as one contiguous run

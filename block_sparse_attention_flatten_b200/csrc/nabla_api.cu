@@ -233,9 +233,10 @@ int mask_plan(int B, int Hh, int D, int T, int H, int W, const nabla_params* par
 
 template <bool kFlatten>
 int launch_pool(const MaskPlan& mp, int B, const void* q, const void* k, void* qf, void* kf, cudaStream_t stream) {
-  const int row = mp.a.Hh * mp.a.D;
-  const int pool_threads = (row / 8) < 384 ? (row / 8) : 384;
-  pool_kernel<kFlatten><<<dim3(mp.a.Nb, B, 2), pool_threads, 0, stream>>>(
+  const int chunks = mp.a.Hh * mp.a.D / 8;
+  const int slices = (chunks + kPoolThreads - 1) / kPoolThreads;
+  if (2 * slices > 65535) return NABLA_ERR_INVALID;
+  pool_kernel<kFlatten><<<dim3(mp.a.Nb, B, 2 * slices), kPoolThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(qf),
       static_cast<__nv_bfloat16*>(kf), const_cast<float*>(mp.a.qbar), const_cast<float*>(mp.a.kbar), mp.S, mp.a.Hh,
       mp.a.D, mp.H, mp.W);
