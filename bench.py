@@ -48,6 +48,7 @@ CONFIGS = {
     "wan13b": inputs.WAN13B,
     "hunyuan": inputs.HUNYUAN,
     "long": inputs.LONG,
+    "long-4h": inputs.LONG_4H,
     "hunyuan-sta": inputs.HUNYUAN_STA,
     "hunyuan-radial": inputs.HUNYUAN_RADIAL,
     "long-radial": inputs.LONG_RADIAL,

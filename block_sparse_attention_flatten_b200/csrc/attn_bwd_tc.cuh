@@ -240,9 +240,23 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
     // ------------------------------------------------------------ producer
     // dQ: walked (K, V) of each key block; dK/dV: (Q, dO) of each query
     // block plus its 64 LSE (times log2 e; -inf -> +inf, so P = 0) and
-    // Delta values, written by the warp's lanes before lane 0 arrives.
+    // Delta values, written by the warp's lanes before lane 0 arrives.  The
+    // lanes load the next block's LSE and Delta into registers before
+    // waiting for its stage, so the loads' latency hides behind the wait.
     int issued = 0;
     bool ok = true;
+    float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};  // rows lane, lane + 32 of the next walked block
+    auto fetch = [&](int n) {
+      if (kDq || n >= L_n) return;
+      const int j = static_cast<int>(list[n] & 0x3FFFu);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = bh * a.S + bwd_tc_row(a, j, lane + 32 * h);
+        nl[h] = __ldg(a.lse + row);
+        nd[h] = __ldg(a.delta + row);
+      }
+    };
+    fetch(0);
     for (int n = 0; ok && n < L_n; ++n) {
       const int s = n % kWS;
       if (n >= kWS) {
@@ -256,13 +270,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       const int j = static_cast<int>(list[n] & 0x3FFFu);
       if (!kDq) {
         float* dst = ld_s + s * 128;
-        for (int x = lane; x < 64; x += 32) {
-          const int64_t row = bh * a.S + bwd_tc_row(a, j, x);
-          const float l = __ldg(a.lse + row);
-          dst[x] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-          dst[64 + x] = __ldg(a.delta + row);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          dst[lane + 32 * h] = nl[h] == -INFINITY ? INFINITY : nl[h] * 1.4426950408889634f;
+          dst[64 + lane + 32 * h] = nd[h];
         }
         __syncwarp();
+        fetch(n + 1);
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(w_full + s, 2 * L::kBlkBytes);

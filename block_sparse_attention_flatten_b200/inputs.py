@@ -86,6 +86,11 @@ LONG_RADIAL = Workload("long video, static radial window r0=2 only: B1 Hh24 D128
                        80, 1.0, 1.0, seed=5, mask="radial", radial=2)
 LONG = Workload("long video: B1 Hh24 D128 grid 64x48x80, thr 0.9 OR STA 3x3x3", 1, 24, 128, 64, 48, 80, 1.0, 0.9,
                 sta=(3, 3, 3), seed=5)
+# The long-video layer with 4 of its 24 heads: the same 3,840 blocks per row
+# and per-head structure at a size a full hardware-counter capture can hold
+# (~2 GB on the device), for profiling the kernels of the long layer.
+LONG_4H = Workload("long video, 4 heads: B1 Hh4 D128 grid 64x48x80, thr 0.9 OR STA 3x3x3", 1, 4, 128, 64, 48, 80,
+                   1.0, 0.9, sta=(3, 3, 3), seed=5)
 
 
 def sweep_points():
