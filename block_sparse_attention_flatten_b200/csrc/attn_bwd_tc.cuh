@@ -84,8 +84,10 @@ struct BwdTcSmem {
   static constexpr int kWS = WS;
   static constexpr int kW0 = kB + kPairBytes;
   static constexpr int kW1 = kW0 + kWS * kBlkBytes;
-  static constexpr int kLD = kW1 + kWS * kBlkBytes;  // dK/dV: [kWS stages][LSE*log2e 64 | Delta 64] fp32
-  static constexpr int kBars = kLD + kWS * 128 * 4;
+  // dK/dV: per elementwise warp two slots of its 16 columns' LSE (log2
+  // units) and Delta, [16 warps][2][32] fp32
+  static constexpr int kLD = kW1 + kWS * kBlkBytes;
+  static constexpr int kBars = kLD + 16 * 64 * 4;
   // fixed_full, w_full[kWS], w0_empty[kWS], w1_empty[kWS], s_full[2], e_full[2], acc_done[2], drain
   static constexpr int kNumBars = 1 + 3 * kWS + 2 + 2 + 2 + 1;
   static constexpr int kMisc = kBars + 8 * kNumBars;
@@ -239,24 +241,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
   if (warp == 16) {
     // ------------------------------------------------------------ producer
     // dQ: walked (K, V) of each key block; dK/dV: (Q, dO) of each query
-    // block plus its 64 LSE (times log2 e; -inf -> +inf, so P = 0) and
-    // Delta values, written by the warp's lanes before lane 0 arrives.  The
-    // lanes load the next block's LSE and Delta into registers before
-    // waiting for its stage, so the loads' latency hides behind the wait.
+    // block.  (The elementwise warps load the walked query blocks' LSE and
+    // Delta themselves: in this thread's loop the loads' latency held the
+    // copies back to about one block ahead of the MMAs.)
     int issued = 0;
     bool ok = true;
-    float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};  // rows lane, lane + 32 of the next walked block
-    auto fetch = [&](int n) {
-      if (kDq || n >= L_n) return;
-      const int j = static_cast<int>(list[n] & 0x3FFFu);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t row = bh * a.S + bwd_tc_row(a, j, lane + 32 * h);
-        nl[h] = __ldg(a.lse + row);
-        nd[h] = __ldg(a.delta + row);
-      }
-    };
-    fetch(0);
     for (int n = 0; ok && n < L_n; ++n) {
       const int s = n % kWS;
       if (n >= kWS) {
@@ -268,16 +257,6 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         }
       }
       const int j = static_cast<int>(list[n] & 0x3FFFu);
-      if (!kDq) {
-        float* dst = ld_s + s * 128;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          dst[lane + 32 * h] = nl[h] == -INFINITY ? INFINITY : nl[h] * 1.4426950408889634f;
-          dst[64 + lane + 32 * h] = nd[h];
-        }
-        __syncwarp();
-        fetch(n + 1);
-      }
       if (lane == 0) {
         mbar_arrive_expect_tx(w_full + s, 2 * L::kBlkBytes);
         load_block(sm + L::kW0 + s * L::kBlkBytes, &tmC, w_full + s, j, 64 * 128);
@@ -377,14 +356,28 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       L2row = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
       drow = __ldg(a.delta + row);
     }
+    // dK/dV: the LSE (log2 units; -inf -> +inf, so P = 0) and Delta of this
+    // warp's 16 columns, one walked block ahead: lanes 0-15 load the LSE of
+    // columns 16 ch + lane, lanes 16-31 the Delta, into a register; the
+    // value is published to the warp's shared slot at the next step
+    float* wslot = ld_s + warp * 64;  // [2][32]
+    float pre = 0.f;
+    auto fetch = [&](int n) {
+      if (kDq || n >= L_n) return;
+      const int j = static_cast<int>(list[n] & 0x3FFFu);
+      const int64_t row = bh * a.S + bwd_tc_row(a, j, ch * 16 + (lane & 15));
+      pre = __ldg((lane < 16 ? a.lse : a.delta) + row);
+    };
+    fetch(0);
     bool ok = true;
     for (int n = 0; n < L_n; ++n) {
       const int s = n & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (n >> 1) & 1, abort_flag))) { ok = false; break; }
-      if (!kDq && !__all_sync(0xffffffffu, mbar_wait(w_full + n % kWS, (n / kWS) & 1, abort_flag))) {
-        ok = false;
-        break;
+      if (!kDq) {
+        wslot[(n & 1) * 32 + lane] = lane < 16 ? (pre == -INFINITY ? INFINITY : pre * 1.4426950408889634f) : pre;
+        __syncwarp();
+        fetch(n + 1);
       }
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full + s, (n >> 1) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
       const uint32_t tX = tX0 + s * 64 + ch * 16 + lane_off, tY = tY0 + s * 64 + ch * 16 + lane_off;
       uint32_t xv[1][16], yv[1][16];  // this quarter's 16 columns of X and Y
@@ -394,7 +387,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
       reg_fence16(xv[0]);
       reg_fence16(yv[0]);
       const bool inc = (static_cast<uint32_t>(list[n]) & flag) != 0u;
-      const float* lq = ld_s + (n % kWS) * 128 + ch * 16;  // dK/dV: the columns' LSE and Delta
+      const float* lq = wslot + (n & 1) * 32;  // dK/dV: the 16 columns' LSE, then their Delta
       uint32_t pk[8], dk[8];
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
@@ -405,8 +398,8 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1)
         } else {
           L0 = lq[e];
           L1 = lq[e + 1];
-          d0 = lq[64 + e];
-          d1 = lq[64 + e + 1];
+          d0 = lq[16 + e];
+          d1 = lq[16 + e + 1];
         }
         if (inc) {
           p0 = ex2_approx(fmaf(__uint_as_float(xv[e >> 4][e & 15]), a.scale_log2, -L0));
