@@ -141,25 +141,44 @@ __host__ __device__ __forceinline__ int radial_band(int dt) {
   return r;
 }
 
-// Calls f(j) for every block j of the radial window of block i (frame ti,
-// patch row hi, column wi): per frame tj the box of half-width
-// r0 >> radial_band(|ti - tj|) around (hi, wi), clipped to the grid; e runs
-// over the box's entries in (row, column) order.  f receives (j, position
-// in the ascending list).  Returns the window's size.
+// Calls f(j, pos) for every block j of the radial window of block i (frame
+// ti, patch row hi, column wi), pos = its position in the ascending list:
+// per frame tj the box of half-width r0 >> radial_band(|ti - tj|) around
+// (hi, wi), clipped to the grid, entries in (row, column) order.  One warp:
+// lane l takes frames l, l + 32, ... (most boxes far from ti are a single
+// block, so a frame per lane keeps the lanes busy), the boxes' sizes give
+// the positions by a warp prefix sum.  Returns the window's size (every
+// lane).
 template <class F>
 __device__ __forceinline__ int radial_for_each(int ti, int hi, int wi, int nbt, int nbh, int nbw, int r0, int lane,
                                               const F& f) {
   int n = 0;
-  for (int tj = 0; tj < nbt; ++tj) {
-    const int rho = r0 >> radial_band(abs(ti - tj));
-    const int h0 = max(hi - rho, 0), h1 = min(hi + rho, nbh - 1);
-    const int w0 = max(wi - rho, 0), w1 = min(wi + rho, nbw - 1);
-    const int nw = w1 - w0 + 1, cnt = (h1 - h0 + 1) * nw;
-    for (int e = lane; e < cnt; e += 32) {
-      const int eh = e / nw;
-      f((tj * nbh + h0 + eh) * nbw + w0 + (e - eh * nw), n + e);
+  for (int t0 = 0; t0 < nbt; t0 += 32) {
+    const int tj = t0 + lane;
+    int cnt = 0, h0 = 0, w0 = 0, nw = 1;
+    if (tj < nbt) {
+      const int rho = r0 >> radial_band(abs(ti - tj));
+      h0 = max(hi - rho, 0);
+      w0 = max(wi - rho, 0);
+      const int h1 = min(hi + rho, nbh - 1), w1 = min(wi + rho, nbw - 1);
+      nw = w1 - w0 + 1;
+      cnt = (h1 - h0 + 1) * nw;
     }
-    n += cnt;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int pos = n + incl - cnt;
+    for (int e = 0, eh = 0, ew = 0; e < cnt; ++e) {
+      f((tj * nbh + h0 + eh) * nbw + w0 + ew, pos + e);
+      if (++ew == nw) {
+        ew = 0;
+        ++eh;
+      }
+    }
+    n += __shfl_sync(0xffffffffu, incl, 31);
   }
   return n;
 }
