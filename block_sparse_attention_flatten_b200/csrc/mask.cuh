@@ -219,7 +219,7 @@ constexpr uint32_t kOneBits = 0x3F800000u;         // 1.0f
 constexpr uint32_t kNearOneBits = kOneBits - 8u;  // within 8 ulp below 1.0
 constexpr int kWindowUlps = 8;                    // > 2 ulp (expf) on either side, with margin
 constexpr unsigned long long kInfKey = 0x7F800000ull << 32;
-constexpr int kSelCap = 2048;                     // candidate slots per warp
+constexpr int kSelCap = 1024;                     // candidate slots per warp
 // First-pass thresholds: the numerators 2^-1, 2^-2, 2^-4, 2^-7, 2^-11, 2^-16
 // (bit patterns descending).
 constexpr int kNThr = 6;

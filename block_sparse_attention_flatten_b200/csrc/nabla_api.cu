@@ -42,6 +42,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sms = 0;
   int max_smem_optin = 0;
+  int smem_per_sm = 0;
 };
 
 std::mutex g_mu;
@@ -59,6 +60,8 @@ int device_info(DeviceInfo* out) {
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return NABLA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NABLA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return NABLA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
       return NABLA_ERR_CUDA;
     d.sm100 = (major == 10 && minor == 0);
     d.ready = true;
@@ -263,10 +266,21 @@ int launch_mask_rows(const MaskPlan& mp, int B, cudaStream_t stream, bool use_sc
     if (launch_score_tiles(mp.a.qbar, mp.a.kbar, mp.scores, sh, static_cast<int>(bhs), mp.a.scale, stream) !=
         cudaSuccess)
       return NABLA_ERR_CUDA;
+    // warps per CTA: the most warps per SM that the per-warp shared memory
+    // allows (each CTA also costs 1 KB of reserved shared memory); on ties
+    // the larger CTA
     const size_t per_warp = select_warp_bytes(Nb);
-    int wpc = static_cast<int>(optin / per_warp);
-    if (wpc < 1) return NABLA_ERR_INVALID;
-    if (wpc > 8) wpc = 8;
+    if (per_warp > optin) return NABLA_ERR_INVALID;
+    int wpc = 1, best = 0;
+    for (int w = 8; w >= 1; w >>= 1) {
+      if (per_warp * w > optin) continue;
+      const int ctas = static_cast<int>(static_cast<size_t>(mp.di.smem_per_sm) / (per_warp * w + 1024));
+      const int warps = ctas * w > 16 ? 16 : ctas * w;
+      if (warps > best) {
+        best = warps;
+        wpc = w;
+      }
+    }
     const size_t smem = per_warp * wpc;
     if (cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
