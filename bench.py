@@ -223,6 +223,9 @@ def run_gpu(args, rank, world, local_rank):
                                          dtype=torch.uint8, device=dev)
     lse = torch.empty((w.B, w.Hh, w.S), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    split = args.attn_split if args.attn_split > 0 else auto_split(w)
+    split_ws = (torch.empty(nabla.attn_split_workspace_bytes(w.B, w.Hh, w.D, w.T, w.H, w.W, split),
+                            dtype=torch.uint8, device=dev) if split > 1 else None)
 
     def static_lists():
         if w.mask == "sta":
@@ -252,11 +255,13 @@ def run_gpu(args, rank, world, local_rank):
                 ev[2].record(stream)
         # 3. attention reading Q, K, V in grid order through 5-D TMA boxes
         #    and storing O in grid order
-        nabla.sparse_attn_fwd(qd, kd, vd, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W))
+        nabla.sparse_attn_fwd(qd, kd, vd, kv_count, kv_idx, out=og, lse=lse, grid=(w.T, w.H, w.W), split=split,
+                              workspace=split_ws)
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 2 if static else 4  # (window lists | pooling, scores, selection), attention
+    # (window lists | pooling, scores, selection), attention (+ the merge of a split walk)
+    launches_per_step = (2 if static else 4) + (1 if split > 1 else 0)
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -330,7 +335,8 @@ def run_gpu(args, rank, world, local_rank):
             stream.wait_event(v_in[b_])
             if s_ >= 2:
                 stream.wait_event(out[b_])  # step s-2's output has been downloaded
-            nabla.sparse_attn_fwd(qd_, kd_, vd_, kv_count, kv_idx, out=og_, lse=lse, grid=(w.T, w.H, w.W))
+            nabla.sparse_attn_fwd(qd_, kd_, vd_, kv_count, kv_idx, out=og_, lse=lse, grid=(w.T, w.H, w.W),
+                                  split=split, workspace=split_ws)
             done[b_].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(done[b_])
@@ -442,7 +448,7 @@ def run_gpu(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": config_dict(w),
+        "config": dict(config_dict(w), attn_key_ranges=split),
         # per layer: the whole step, since Q, K, V, O stay in grid order (the
         # flattening and its inverse happen inside the pooling and attention)
         "ms_per_layer": statistics.mean(pool_ms) + mask_avg + attn_avg,
@@ -568,6 +574,18 @@ def run_gpu_ab(args, rank, world, local_rank):
         "cpu_baseline": None,
         "e2e": None,
     }, (q, k, v, u)
+
+
+# Key ranges of the attention walk when --attn-split is 0: a head's K and V
+# larger than half of the 126 MB L2 (the long-video layer's are 123 MB) do
+# not stay in it while one wave of CTAs walks lists spread over the whole
+# sequence; two ranges halve that working set.  Measured on the long-video
+# layer (20 steps, power-capped): 1 range 59.5 ms at 1.44 GHz, 2 ranges 57.9
+# ms at 1.58 GHz, 4 ranges 59.5 ms, 8 ranges 65.8 ms; on the Wan-like layer
+# (30 MB per head) 4 ranges double the attention time.
+def auto_split(w) -> int:
+    head_kv_bytes = w.Nb * 64 * w.D * 2 * 2
+    return 2 if head_kv_bytes > (63 << 20) else 1
 
 
 def load_traffic(config):
@@ -738,6 +756,9 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--backward-steps", type=int, default=20, help="timed steps of the backward pass (0: skip)")
+    ap.add_argument("--attn-split", type=int, default=0,
+                    help="split each head's attention walk into this many key ranges (1: no split; 0: two ranges "
+                         "when a head's K and V exceed half the L2, else one)")
     ap.add_argument("--flatten-launches", type=int, default=10,
                     help="back-to-back launches of the materialised flattening to time (0: skip)")
     ap.add_argument("--cpu-blocks", type=int, default=8, help="query blocks in the CPU-baseline sample")

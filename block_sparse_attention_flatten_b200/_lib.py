@@ -41,6 +41,8 @@ EXPORTS = (
     "nabla_build_mask_radial",
     "nabla_sparse_attn_fwd",
     "nabla_sparse_attn_fwd_grid",
+    "nabla_sparse_attn_fwd_grid_split",
+    "nabla_attn_split_workspace_bytes",
     "nabla_transpose_lists",
     "nabla_sparse_attn_bwd",
     "nabla_sparse_attn_bwd_grid",
@@ -99,6 +101,9 @@ def lib():
         L.nabla_build_mask_radial.argtypes = [i, i, i, i, i, i, i, vp, vp, vp]
         L.nabla_sparse_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, vp, vp, vp]
         L.nabla_sparse_attn_fwd_grid.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, vp]
+        L.nabla_sparse_attn_fwd_grid_split.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+        L.nabla_attn_split_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+        L.nabla_attn_split_workspace_bytes.restype = sz
         L.nabla_transpose_lists.argtypes = [vp, vp, i, i, i, vp, vp, vp]
         L.nabla_sparse_attn_bwd.argtypes = [vp] * 10 + [i, i, i, i, f, vp, vp, vp, vp, vp]
         L.nabla_sparse_attn_bwd_grid.argtypes = [vp] * 10 + [i, i, i, i, i, i, f, vp, vp, vp, vp, vp]
@@ -112,7 +117,8 @@ def lib():
         L.nabla_strerror.argtypes = [i]
         L.nabla_strerror.restype = ctypes.c_char_p
         for name in EXPORTS:
-            if name not in ("nabla_mask_workspace_bytes", "nabla_ab_workspace_bytes", "nabla_strerror"):
+            if name not in ("nabla_mask_workspace_bytes", "nabla_ab_workspace_bytes", "nabla_attn_split_workspace_bytes",
+                            "nabla_strerror"):
                 getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -339,7 +345,7 @@ def pooled_from_workspace(workspace: torch.Tensor, B: int, Hh: int, Nb: int, D: 
 
 def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_count: torch.Tensor,
                     kv_idx: torch.Tensor, scale: float = 0.0, out=None, lse=None, want_lse: bool = True,
-                    stream=None, grid=None):
+                    stream=None, grid=None, split: int = 1, workspace=None):
     """Block-sparse attention on the kept tiles; returns (out, lse or None).
 
     grid = None: qf, kf, vf are flattened; nabla_sparse_attn_fwd (pairs 2p,
@@ -347,7 +353,10 @@ def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_cou
     grid = (T, H, W): the three tensors are in GRID order (token (t, h, w) at
     row (t*H + h)*W + w); nabla_sparse_attn_fwd_grid reads the blocks through
     5-D TMA boxes, pairs query blocks by their lists' overlap and returns out
-    and lse in grid order."""
+    and lse in grid order.  split > 1 (grid order only): each head's walk
+    split into that many key ranges (nabla_sparse_attn_fwd_grid_split); the
+    workspace (uint8 CUDA tensor of at least attn_split_workspace_bytes) is
+    allocated when not given."""
     B, S, Hh, D = qf.shape
     if out is None:
         out = torch.empty_like(qf)
@@ -364,10 +373,26 @@ def sparse_attn_fwd(qf: torch.Tensor, kf: torch.Tensor, vf: torch.Tensor, kv_cou
         T, H, W = (int(x) for x in grid)
         if T * H * W != S:
             raise ValueError(f"grid {grid} does not hold {S} tokens")
-        _check(lib().nabla_sparse_attn_fwd_grid(*ptrs, B, Hh, D, T, H, W, float(scale), o_p, lse_p,
-                                                _stream(stream)),
-               "nabla_sparse_attn_fwd_grid")
+        if split > 1:
+            if workspace is None:
+                workspace = torch.empty(attn_split_workspace_bytes(B, Hh, D, T, H, W, split), dtype=torch.uint8,
+                                        device=qf.device)
+            _check(lib().nabla_sparse_attn_fwd_grid_split(*ptrs, B, Hh, D, T, H, W, float(scale), int(split),
+                                                          _dev(workspace, torch.uint8, "workspace"), o_p, lse_p,
+                                                          _stream(stream)),
+                   "nabla_sparse_attn_fwd_grid_split")
+        else:
+            _check(lib().nabla_sparse_attn_fwd_grid(*ptrs, B, Hh, D, T, H, W, float(scale), o_p, lse_p,
+                                                    _stream(stream)),
+                   "nabla_sparse_attn_fwd_grid")
     return out, lse
+
+
+def attn_split_workspace_bytes(B: int, Hh: int, D: int, T: int, H: int, W: int, split: int) -> int:
+    n = int(lib().nabla_attn_split_workspace_bytes(B, Hh, D, T, H, W, int(split)))
+    if n == 0:
+        raise ValueError("invalid arguments for the key-range split")
+    return n
 
 
 def transpose_lists(kv_count: torch.Tensor, kv_idx: torch.Tensor, q_count=None, q_idx=None, stream=None):

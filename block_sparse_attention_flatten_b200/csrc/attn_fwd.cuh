@@ -83,6 +83,13 @@ struct AttnArgs {
   int in_T, in_nbw, in_per_t;  // in_nbw > 0: Q, K, V are in grid order, read through 5-D maps
   uint32_t in_inv_per_t, in_inv_nbw;  // floor(2^32 / d) + 1 (0 for d = 1): j / d = umulhi(j, inv) for j, d < 2^14
   float scale_log2;         // scale * log2(e)
+  // Key-range split: blockIdx.y = head * nsplit + split; the CTA walks only
+  // the listed key blocks in [split * split_blocks, (split + 1) *
+  // split_blocks) and stores its O (normalised over that range) and LSE at
+  // out + split * split_out_stride, lse + split * split_lse_stride, for a
+  // merge by attn_combine_kernel.  nsplit = 1: the whole list, one output.
+  int nsplit, split_blocks;
+  int64_t split_out_stride, split_lse_stride;
 };
 
 template <int D>
@@ -113,8 +120,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint32_t* bm = reinterpret_cast<uint32_t*>(sm + L::kList + L::list_bytes(Nb));  // [4][words]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int p = blockIdx.x, hd = blockIdx.y, b = blockIdx.z;
+  const int p = blockIdx.x, hd = blockIdx.y / a.nsplit, split = blockIdx.y - hd * a.nsplit, b = blockIdx.z;
   const int64_t bh = static_cast<int64_t>(b) * a.Hh + hd;
+  const int k0 = split * a.split_blocks, k1 = k0 + a.split_blocks;  // key blocks this CTA walks
   // One 64-token block j of Q, K or V, 64 columns (chunk c) of one head, as
   // 64 rows of 128 bytes.  Flattened input: rows 64j..64j+63 (4-D map).
   // Grid-order input: block j is the 8 x 8 patch (bh, bw) of frame t, read
@@ -226,7 +234,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int32_t* src = a.kv_idx + (bh * Nb + (cand[h] >= 0 ? cand[h] : 0)) * static_cast<int64_t>(Nb);
     if (warp == h && lane < c && first_list) {
       if (first < 0 || first >= Nb) report(NABLA_ERR_DEVICE_BOUNDS);
-      else atomicOr(bmh + (first >> 5), 1u << (first & 31));
+      else if (first >= k0 && first < k1) atomicOr(bmh + (first >> 5), 1u << (first & 31));
     }
     for (int e = 32 + tid; e < c; e += kAttnThreads) {
       const int j = src[e];
@@ -234,7 +242,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         report(NABLA_ERR_DEVICE_BOUNDS);
         continue;
       }
-      atomicOr(bmh + (j >> 5), 1u << (j & 31));
+      if (j >= k0 && j < k1) atomicOr(bmh + (j >> 5), 1u << (j & 31));
     }
   }
   __syncthreads();
@@ -539,7 +547,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tc_fence_after();
     __syncwarp();
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-    __nv_bfloat16* orow = a.out + ((static_cast<int64_t>(b) * a.S + row_g) * a.Hh + hd) * D;
+    __nv_bfloat16* orow =
+        a.out + split * a.split_out_stride + ((static_cast<int64_t>(b) * a.S + row_g) * a.Hh + hd) * D;
 #pragma unroll 1
     for (int c0 = 0; c0 < D / 16; c0 += 4) {
       uint32_t ob[4][16];
@@ -575,7 +584,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
     if (row_valid && a.lse != nullptr)
-      a.lse[bh * a.S + row_g] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      a.lse[split * a.split_lse_stride + bh * a.S + row_g] =
+          l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
   }
 
   // ---- teardown
@@ -586,6 +596,55 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
+}
+
+// Merge of the key-range split: per (token row, head), O = sum over the
+// splits of exp(lse_s - L) O_s and LSE L = log sum exp(lse_s), where O_s is
+// the split's output normalised over its own key range (a split with no
+// kept block there has lse_s = -inf and weight 0).  Thread t handles 8
+// consecutive elements of a row's head (D / 8 threads per row and head).
+__global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
+                                                           const float* __restrict__ part_lse, int nsplit,
+                                                           int64_t o_stride, int64_t lse_stride,
+                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                                                           int64_t rows, int S, int Hh, int D) {
+  const int per = D / 8;
+  const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / per;
+  const int part = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) - item * per);
+  if (item >= rows * Hh) return;
+  const int64_t row = item / Hh;  // b * S + s
+  const int hd = static_cast<int>(item - row * Hh);
+  const int64_t b = row / S, sidx = row - b * S;
+  const int64_t li = (b * Hh + hd) * S + sidx;
+  float m = -INFINITY;
+  for (int t = 0; t < nsplit; ++t) m = fmaxf(m, __ldg(part_lse + t * lse_stride + li));
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  const int64_t oi = item * D + part * 8;
+  if (m != -INFINITY) {
+    for (int t = 0; t < nsplit; ++t) {
+      const float w = __expf(__ldg(part_lse + t * lse_stride + li) - m);
+      wsum += w;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(part_o + t * o_stride + oi));
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint4 o;
+  o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(out + oi) = o;
+  if (part == 0 && lse != nullptr) lse[li] = m == -INFINITY ? -INFINITY : m + __logf(wsum);
 }
 
 }  // namespace nabla

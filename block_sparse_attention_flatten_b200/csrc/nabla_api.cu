@@ -319,11 +319,32 @@ __global__ void wait_timeout_selftest_kernel(long long limit) {
 // comes from cudaGetSymbolAddress with the caller's device current.
 __device__ __align__(256) unsigned char g_noalloc_scratch[NABLA_NOALLOC_SCRATCH_BYTES];
 
+// Workspace of the key-range split: the splits' outputs (bf16, the layout
+// of O, o_stride elements apart) then their LSE (fp32, the layout of the
+// LSE, lse_stride apart), each region 256-byte aligned.
+struct AttnSplitLayout {
+  int64_t o_stride, lse_stride;
+  size_t o_off, lse_off, total;
+};
+AttnSplitLayout attn_split_layout(int B, int64_t S, int Hh, int D, int nsplit) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  AttnSplitLayout l;
+  l.o_stride = static_cast<int64_t>(B) * S * Hh * D;
+  l.lse_stride = static_cast<int64_t>(B) * Hh * S;
+  l.o_off = 0;
+  l.lse_off = up(static_cast<size_t>(l.o_stride) * 2 * nsplit);
+  l.total = l.lse_off + up(static_cast<size_t>(l.lse_stride) * 4 * nsplit);
+  return l;
+}
+
 // Shared body of the two attention entry points; grp_F > 0 selects the 2 x 2
 // (w, t) grouping of query blocks (grp_F blocks per frame, grp_nbw per row).
+// nsplit > 1: the key-range split, partial outputs in `part` (see
+// attn_split_layout), then their merge into out and lse.
 int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int32_t* kv_count,
                        const int32_t* kv_idx, int B, int S, int Hh, int D, float scale, void* out, float* lse,
-                       int grp_F, int grp_nbw, int grid_T, int out_H, int out_W, cudaStream_t stream) {
+                       int grp_F, int grp_nbw, int grid_T, int out_H, int out_W, cudaStream_t stream,
+                       int nsplit = 1, void* part = nullptr) {
   if (B <= 0 || S <= 0 || Hh <= 0 || S % 64 != 0 || (D != 64 && D != 128)) return NABLA_ERR_INVALID;
   if (static_cast<int64_t>(S) * Hh * D >= (int64_t{1} << 40)) return NABLA_ERR_INVALID;
   if (!(scale >= 0.f) || std::isinf(scale)) return NABLA_ERR_INVALID;
@@ -333,6 +354,9 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
       !aligned16(kv_count))
     return NABLA_ERR_ALIGN;
   if (lse != nullptr && !aligned16(lse)) return NABLA_ERR_ALIGN;
+  if (nsplit < 1 || nsplit > 64 || static_cast<int64_t>(Hh) * nsplit > 65535) return NABLA_ERR_INVALID;
+  if (nsplit > 1 && part == nullptr) return NABLA_ERR_INVALID;
+  if (nsplit > 1 && !aligned16(part)) return NABLA_ERR_ALIGN;
   DeviceInfo di;
   int rc = device_info(&di);
   if (rc != NABLA_OK) return rc;
@@ -371,13 +395,28 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
   a.in_inv_per_t = inv(a.in_per_t);
   a.in_inv_nbw = inv(a.in_nbw);
   a.scale_log2 = static_cast<float>(static_cast<double>(sc) * 1.4426950408889634);
-  const dim3 grid((Nb + 1) / 2, Hh, B);
+  const AttnSplitLayout sl = attn_split_layout(B, S, Hh, D, nsplit);
+  a.nsplit = nsplit;
+  a.split_blocks = nsplit > 1 ? ((Nb + nsplit - 1) / nsplit + 31) & ~31 : Nb;
+  a.split_out_stride = nsplit > 1 ? sl.o_stride : 0;
+  a.split_lse_stride = nsplit > 1 ? sl.lse_stride : 0;
+  if (nsplit > 1) {
+    a.out = reinterpret_cast<__nv_bfloat16*>(static_cast<unsigned char*>(part) + sl.o_off);
+    a.lse = reinterpret_cast<float*>(static_cast<unsigned char*>(part) + sl.lse_off);
+  }
+  const dim3 grid((Nb + 1) / 2, Hh * nsplit, B);
   auto go = [&](auto kernel, size_t smem) -> int {
     if (smem > static_cast<size_t>(di.max_smem_optin)) return NABLA_ERR_INVALID;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
       return NABLA_ERR_CUDA;
     kernel<<<grid, kAttnThreads, smem, stream>>>(tq, tk, tv, a);
+    if (nsplit > 1) {
+      const int64_t rows = static_cast<int64_t>(B) * S;
+      const int64_t threads = rows * Hh * (D / 8);
+      attn_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+          a.out, a.lse, nsplit, sl.o_stride, sl.lse_stride, static_cast<__nv_bfloat16*>(out), lse, rows, S, Hh, D);
+    }
     return launch_status();
   };
   return D == 128 ? go(attn_fwd_kernel<128>, AttnSmem<128>::bytes(Nb)) : go(attn_fwd_kernel<64>, AttnSmem<64>::bytes(Nb));
@@ -656,6 +695,27 @@ int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, cons
   const bool groups = T % 2 == 0 && nbw % 2 == 0;
   return sparse_attn_launch(q, k, v, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
                             groups ? F : 0, groups ? nbw : 0, T, H, W, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t nabla_attn_split_workspace_bytes(int B, int Hh, int D, int T, int H, int W, int nsplit) {
+  if (B <= 0 || Hh <= 0 || (D != 64 && D != 128) || T <= 0 || H <= 0 || W <= 0 || nsplit < 2 || nsplit > 64)
+    return 0;
+  return attn_split_layout(B, static_cast<int64_t>(T) * H * W, Hh, D, nsplit).total;
+}
+
+int nabla_sparse_attn_fwd_grid_split(const void* q, const void* k, const void* v, const int32_t* kv_count,
+                                     const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
+                                     int nsplit, void* workspace, void* out, float* lse, nabla_stream_t stream) {
+  NABLA_NVTX_RANGE();
+  if (T <= 0 || H <= 0 || W <= 0 || H % 8 != 0 || W % 8 != 0) return NABLA_ERR_INVALID;
+  const int64_t S = static_cast<int64_t>(T) * H * W;
+  if (S > (int64_t{1} << 30)) return NABLA_ERR_INVALID;
+  if (nsplit < 2 || nsplit > 64 || workspace == nullptr) return NABLA_ERR_INVALID;
+  const int nbw = W / 8, F = (H / 8) * nbw;
+  const bool groups = T % 2 == 0 && nbw % 2 == 0;
+  return sparse_attn_launch(q, k, v, kv_count, kv_idx, B, static_cast<int>(S), Hh, D, scale, out, lse,
+                            groups ? F : 0, groups ? nbw : 0, T, H, W, reinterpret_cast<cudaStream_t>(stream), nsplit,
+                            workspace);
 }
 
 int nabla_transpose_lists(const int32_t* kv_count, const int32_t* kv_idx, int B, int Hh, int Nb, int32_t* q_count,

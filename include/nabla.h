@@ -254,6 +254,32 @@ int nabla_sparse_attn_fwd_grid(const void* q, const void* k, const void* v, cons
                                const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
                                void* out, float* lse, nabla_stream_t stream);
 
+/* The same attention as nabla_sparse_attn_fwd_grid with each head's walk
+ * split by key range ("Metodologia: NABLA", item 2 "Expansao": the kept
+ * tiles are computed, grouped differently): the key blocks are cut into
+ * nsplit ranges of ceil(Nb / nsplit) rounded up to 32 blocks; every query
+ * tile is attended over each range by its own CTA, all ranges of one head
+ * in turn, so the CTAs resident at a time read only one range's K and V
+ * (for a mask whose kept blocks are spread over the whole sequence, the
+ * L2 then holds that range instead of missing on a whole head).  Each
+ * range's output (normalised over the range) and LSE go to the workspace;
+ * a second kernel merges them: O = sum_s exp(lse_s - L) O_s, L = log sum_s
+ * exp(lse_s).  Results equal nabla_sparse_attn_fwd_grid's up to rounding
+ * (the range outputs are stored in bf16 before the merge).
+ *   nsplit     2 .. 64 (Hh * nsplit <= 65535)
+ *   workspace  device, at least nabla_attn_split_workspace_bytes(...)
+ *              bytes, 16-byte aligned, owned by the caller, overwritten.
+ * Other arguments and errors as nabla_sparse_attn_fwd_grid; a null or
+ * misaligned workspace gives NABLA_ERR_INVALID / NABLA_ERR_ALIGN. */
+int nabla_sparse_attn_fwd_grid_split(const void* q, const void* k, const void* v, const int32_t* kv_count,
+                                     const int32_t* kv_idx, int B, int Hh, int D, int T, int H, int W, float scale,
+                                     int nsplit, void* workspace, void* out, float* lse, nabla_stream_t stream);
+
+/* Bytes of workspace nabla_sparse_attn_fwd_grid_split needs: nsplit range
+ * outputs (bf16, B*S*Hh*D each) and their LSE (fp32, B*Hh*S each), S =
+ * T*H*W.  0 for invalid arguments (including nsplit < 2). */
+size_t nabla_attn_split_workspace_bytes(int B, int Hh, int D, int T, int H, int W, int nsplit);
+
 /* Column (transposed) block lists for the backward pass: for key block j of
  * (b, hd), the query blocks i whose row kv_idx[b,hd,i,0..kv_count) lists j,
  * ascending.

@@ -78,6 +78,13 @@ def test_workspace_bytes(lib):
     assert nabla.mask_workspace_bytes(1, 1, 64, 37, 8, 8, prm) == 2 * 64 * 40 * 4 + 37 * 40 * 4
     assert nabla.mask_workspace_bytes(1, 2, 96, 4, 16, 16, prm) == 0  # D not supported
     assert nabla.mask_workspace_bytes(1, 2, 64, 4, 12, 16, prm) == 0  # H not a multiple of 8
+    # key-range split: the ranges' bf16 outputs, then their fp32 LSE, each 256-byte aligned
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    S = 64 * 48 * 80
+    assert nabla.attn_split_workspace_bytes(1, 24, 128, 64, 48, 80, 4) == up(4 * S * 24 * 128 * 2) + up(4 * 24 * S * 4)
+    assert nabla.attn_split_workspace_bytes(2, 3, 64, 3, 8, 24, 2) == up(2 * 2 * 576 * 3 * 64 * 2) + up(2 * 2 * 3 * 576 * 4)
+    assert lib.nabla_attn_split_workspace_bytes(1, 2, 64, 4, 16, 16, 1) == 0  # nsplit < 2
+    assert lib.nabla_attn_split_workspace_bytes(1, 2, 96, 4, 16, 16, 2) == 0  # D not supported
 
 
 def test_invalid_arguments_rejected_before_launch(lib):
