@@ -332,34 +332,26 @@ __device__ __forceinline__ int compact_range(const float* row, int* cbuf, int Nb
   const int lane = threadIdx.x & 31;
   int out = 0;
   if (from_row) {
-    const float4* row4 = reinterpret_cast<const float4*>(row);
-    for (int c = lane; c - lane < (Nbp >> 2); c += 32) {
-      uint32_t fl = 0;
-      if (c < (Nbp >> 2)) {
-        const float4 v = row4[c];
-        const float ev[4] = {v.x, v.y, v.z, v.w};
+    // four 32-element chunks per step, lane l taking element 32u + l of
+    // chunk u: ballots give the ascending positions, the chunks' loads are
+    // independent and only the running count links the steps
+    const unsigned below_me = (1u << lane) - 1u;
+    for (int base = 0; base < Nbp; base += 128) {
+      bool in[4];
+      unsigned bal[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint32_t u = __float_as_uint(ev[t]);
-          fl |= (u >= lo && u < hi) ? (1u << t) : 0u;
-        }
+      for (int u = 0; u < 4; ++u) {
+        const int j = base + 32 * u + lane;
+        const uint32_t v = j < Nbp ? __float_as_uint(row[j]) : 0u;
+        in[u] = j < Nbp && v >= lo && v < hi;
+        bal[u] = __ballot_sync(0xffffffffu, in[u]);
       }
-      // ascending j = lane-major, then t: exclusive prefix of the lanes' counts
-      const int cnt = __popc(fl);
-      int incl = cnt;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+      for (int u = 0; u < 4; ++u) {
+        const int pos = out + __popc(bal[u] & below_me);
+        if (in[u] && pos < kSelCap) cbuf[pos] = base + 32 * u + lane;
+        out += __popc(bal[u]);
       }
-      int pos = out + incl - cnt;
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        if (fl & (1u << t)) {
-          if (pos < kSelCap) cbuf[pos] = 4 * c + t;
-          ++pos;
-        }
-      out += __shfl_sync(0xffffffffu, incl, 31);
     }
   } else {
     for (int base = 0; base < n; base += 32) {
@@ -651,18 +643,29 @@ __device__ __forceinline__ void select_row(float* row, int* cbuf, int* cand, int
                     [row](int j, int) { row[j] = __uint_as_float(0x7F800000u); });
     __syncwarp();
   }
+  // four 32-block chunks per step: their loads and ballots are independent,
+  // only the running count links the steps
   int count = 0;
-  for (int base_j = 0; base_j < Nb; base_j += 32) {
-    const int j = base_j + lane;
-    bool keep = false;
-    if (j < Nb) {
-      const unsigned long long key =
-          (static_cast<unsigned long long>(__float_as_uint(row[j])) << 32) | static_cast<unsigned>(j);
-      keep = a.keep_all || key >= kstar || j == argmax;
+  const unsigned below_me = (1u << lane) - 1u;
+  for (int base_j = 0; base_j < Nb; base_j += 128) {
+    bool keep[4];
+    unsigned bal[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base_j + 32 * u + lane;
+      keep[u] = false;
+      if (j < Nb) {
+        const unsigned long long key =
+            (static_cast<unsigned long long>(__float_as_uint(row[j])) << 32) | static_cast<unsigned>(j);
+        keep[u] = a.keep_all || key >= kstar || j == argmax;
+      }
+      bal[u] = __ballot_sync(0xffffffffu, keep[u]);
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[count + __popc(bal & ((1u << lane) - 1u))] = j;
-    count += __popc(bal);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (keep[u]) out[count + __popc(bal[u] & below_me)] = base_j + 32 * u + lane;
+      count += __popc(bal[u]);
+    }
   }
   if (lane == 0) *count_out = count;
   __syncwarp();
