@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       uint32_t pk[2][16];
       const unsigned long long sc2 = f2_pack(a.scale_log2, a.scale_log2), nm2 = f2_pack(-m_run, -m_run);
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
           float p0 = 0.f, p1 = 0.f;
@@ -495,6 +495,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           const int k = c * 8 + e / 2;
           pk[k >> 4][k & 15] = pack_bf16x2(p0, p1);
         }
+        // the first 32 keys' P go to tensor memory while the last 32 are
+        // computed (S is already in registers)
+        if (c == 1) tmem_st16(((n & 1) ? tS1 : tS0) + lane_off, pk[0]);
+      }
       const unsigned long long r01 = f2_add(rs2[0], rs2[1]), r23 = f2_add(rs2[2], rs2[3]);
       const unsigned long long rall = f2_add(r01, r23);
       l_run = l_run * factor + (f2_lo(rall) + f2_hi(rall));
@@ -519,8 +523,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           tmem_st16(tO + lane_off + c * 16, ov);
         }
       }
-      // P(n): bf16 pairs into the first 32 columns of the score buffer.
-      tmem_st16(tS, pk[0]);
+      // P(n): bf16 pairs into the first 32 columns of the score buffer (the
+      // first half was stored above).
       tmem_st16(tS + 16, pk[1]);
       tmem_st_wait();
       tc_fence_before();
