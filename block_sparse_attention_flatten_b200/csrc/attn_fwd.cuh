@@ -607,6 +607,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 // the split's output normalised over its own key range (a split with no
 // kept block there has lse_s = -inf and weight 0).  Thread t handles 8
 // consecutive elements of a row's head (D / 8 threads per row and head).
+// NS > 0: exactly NS splits, every load issued before the first use (one
+// memory latency per thread); NS = 0: any nsplit, split by split.
+template <int NS>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
                                                            const float* __restrict__ part_lse, int nsplit,
                                                            int64_t o_stride, int64_t lse_stride,
@@ -620,24 +623,45 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const __nv_bfloat16* 
   const int hd = static_cast<int>(item - row * Hh);
   const int64_t b = row / S, sidx = row - b * S;
   const int64_t li = (b * Hh + hd) * S + sidx;
-  float m = -INFINITY;
-  for (int t = 0; t < nsplit; ++t) m = fmaxf(m, __ldg(part_lse + t * lse_stride + li));
+  const int64_t oi = item * D + part * 8;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  const int64_t oi = item * D + part * 8;
-  if (m != -INFINITY) {
-    for (int t = 0; t < nsplit; ++t) {
-      const float w = __expf(__ldg(part_lse + t * lse_stride + li) - m);
-      wsum += w;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(part_o + t * o_stride + oi));
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+  float m = -INFINITY, wsum = 0.f;
+  auto accumulate = [&](float w, const uint4& v) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+    }
+  };
+  if constexpr (NS > 0) {
+    float l[NS];
+    uint4 v[NS];
+#pragma unroll
+    for (int t = 0; t < NS; ++t) {
+      l[t] = __ldg(part_lse + t * lse_stride + li);
+      v[t] = __ldg(reinterpret_cast<const uint4*>(part_o + t * o_stride + oi));
+    }
+#pragma unroll
+    for (int t = 0; t < NS; ++t) m = fmaxf(m, l[t]);
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int t = 0; t < NS; ++t) {
+        const float w = __expf(l[t] - m);
+        wsum += w;
+        accumulate(w, v[t]);
+      }
+    }
+  } else {
+    for (int t = 0; t < nsplit; ++t) m = fmaxf(m, __ldg(part_lse + t * lse_stride + li));
+    if (m != -INFINITY) {
+      for (int t = 0; t < nsplit; ++t) {
+        const float w = __expf(__ldg(part_lse + t * lse_stride + li) - m);
+        wsum += w;
+        accumulate(w, __ldg(reinterpret_cast<const uint4*>(part_o + t * o_stride + oi)));
       }
     }
   }

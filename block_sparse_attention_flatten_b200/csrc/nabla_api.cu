@@ -414,8 +414,11 @@ int sparse_attn_launch(const void* qf, const void* kf, const void* vf, const int
     if (nsplit > 1) {
       const int64_t rows = static_cast<int64_t>(B) * S;
       const int64_t threads = rows * Hh * (D / 8);
-      attn_combine_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-          a.out, a.lse, nsplit, sl.o_stride, sl.lse_stride, static_cast<__nv_bfloat16*>(out), lse, rows, S, Hh, D);
+      const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+      auto combine = nsplit == 2 ? attn_combine_kernel<2> : nsplit == 3 ? attn_combine_kernel<3>
+                   : nsplit == 4 ? attn_combine_kernel<4> : attn_combine_kernel<0>;
+      combine<<<blocks, 256, 0, stream>>>(a.out, a.lse, nsplit, sl.o_stride, sl.lse_stride,
+                                          static_cast<__nv_bfloat16*>(out), lse, rows, S, Hh, D);
     }
     return launch_status();
   };

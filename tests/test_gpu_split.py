@@ -2,8 +2,8 @@
 outputs and LSE against the fp64 oracle on the GPU's own block lists, and
 against the unsplit kernel, on hand-built lists that put kept blocks in
 every range, rows whose kept blocks all fall in one range (the others have
-no block: weight 0), empty rows, odd block counts and batch 2; plus the
-argument checks."""
+no block: weight 0), empty rows, odd block counts and batch 2; repeated
+runs on one workspace; plus the argument checks."""
 import math
 
 import numpy as np
@@ -98,6 +98,35 @@ def test_split_against_oracle_and_unsplit(B, Hh, D, grid, split, kind):
     fin = torch.isfinite(lse_1)
     assert torch.equal(fin, torch.isfinite(lse_s))
     assert float((lse_s[fin] - lse_1[fin]).abs().max()) <= LSE_ABS
+
+
+@pytest.mark.parametrize("grid,split", [((4, 32, 48), 2), ((2, 64, 64), 4), ((12, 48, 80), 2)])
+def test_split_is_deterministic_on_a_reused_workspace(grid, split):
+    """Five runs on one workspace, filled with 0xFF before each (stale range
+    outputs and LSE), give bit-identical O and LSE, equal to the unsplit
+    kernel's up to the rounding of the range outputs."""
+    T, H, W = grid
+    B, Hh, D = 1, 2, 128
+    S = T * H * W
+    Nb = S // 64
+    rng = np.random.default_rng(7)
+    g = torch.Generator().manual_seed(8)
+    q, k, v = (torch.randn(B, S, Hh, D, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    cnt, idx = _lists(B, Hh, Nb, rng, "spread")
+    cnt_d, idx_d = torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda()
+    ws = torch.empty(nabla.attn_split_workspace_bytes(B, Hh, D, T, H, W, split), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(5):
+        ws.fill_(255)
+        outs.append(nabla.sparse_attn_fwd(q, k, v, cnt_d, idx_d, grid=grid, split=split, workspace=ws))
+    torch.cuda.synchronize()
+    assert nabla.get_status() == 0
+    for o, l in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(l.view(torch.int32), outs[0][1].view(torch.int32))
+    out_1, _ = nabla.sparse_attn_fwd(q, k, v, cnt_d, idx_d, grid=grid)
+    d = (outs[0][0].float() - out_1.float()).abs()
+    assert float(d.max()) <= MAX_ABS and float(d.mean()) <= MEAN_ABS
 
 
 def test_split_on_the_adaptive_mask_of_a_layer():
