@@ -61,6 +61,7 @@ def _lists(B, Hh, Nb, rng, kind):
     (1, 1, 128, (6, 32, 32), 3, "with_empty"),
     (1, 3, 64, (5, 24, 48), 2, "spread"),
     (1, 2, 128, (3, 16, 16), 2, "spread"),
+    (1, 2, 128, (4, 48, 64), 5, "spread"),  # the merge's any-count path; ranges 4 and 5 empty
 ])
 def test_split_against_oracle_and_unsplit(B, Hh, D, grid, split, kind):
     T, H, W = grid
