@@ -427,6 +427,35 @@ def run_gpu(args, rank, world, local_rank):
                     "steps": args.backward_steps, "launches_per_step": 4}
         del do, q_count, q_idx, dq_, dk_, dv_, delta
 
+    # the same step captured once in a CUDA graph and replayed: the calls
+    # allocate nothing and never synchronise, so one graph holds the whole
+    # layer and its replay pays one launch instead of one per kernel.  Each
+    # replay is timed with events on the launching stream, the L2 flushed
+    # before it; not part of `value`
+    graph = None
+    if args.graph_steps > 0:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            flush.zero_()
+            g.replay()
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.graph_steps)]
+        for s in range(args.graph_steps):
+            flush.zero_()
+            gev[s][0].record(stream)
+            g.replay()
+            gev[s][1].record(stream)
+        torch.cuda.synchronize()
+        status = nabla.get_status()
+        if status != 0:
+            raise RuntimeError(f"device status after the graph replays: {nabla.strerror(status)}")
+        t_g = statistics.mean(e[0].elapsed_time(e[1]) for e in gev)
+        graph = {"ms_per_step": t_g, "value": kept_flops(w, total_kept) / (t_g * 1e-3) / 1e12, "unit": "TFLOP/s",
+                 "eager_ms_per_step": total_ms_max / args.steps, "replays": args.graph_steps,
+                 "kernels_per_replay": launches_per_step}
+        del g
+
     _, _, peak_gbs, peak_kind = load_peaks()
     peak_tf, burst_tf, tf_kind = tensor_peak(total_ms_max)
     attn_avg = statistics.mean(attn_ms)
@@ -480,6 +509,7 @@ def run_gpu(args, rank, world, local_rank):
         "e2e": e2e,
         "backward": backward,
         "flatten": flatten,
+        "graph": graph,
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
@@ -756,6 +786,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--backward-steps", type=int, default=20, help="timed steps of the backward pass (0: skip)")
+    ap.add_argument("--graph-steps", type=int, default=0,
+                    help="timed replays of the step captured in a CUDA graph (0: skip)")
     ap.add_argument("--attn-split", type=int, default=0,
                     help="split each head's attention walk into this many key ranges (1: no split; 0: two ranges "
                          "when a head's K and V exceed half the L2, else one)")
