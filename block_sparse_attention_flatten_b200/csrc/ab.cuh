@@ -197,46 +197,91 @@ __device__ __forceinline__ int block_sum_int(int v, double* red) {
 }
 
 // grid (NQB, B*Hh), 256 threads (8 warps).  Shared memory: the row's block
-// scores (NKB fp32) and per-warp reductions.
-//   1. warp c (centroid c, count n_c > 0): max and sum_J exp(l_cJ - max)
-//      (expf, fp64 sums);
+// scores (NKB fp32), per-warp partial maxima and sums, reductions.  The row's
+// 8 x NKB centroid logits are read twice, as float4 with the 8 centroids'
+// loads independent (NKB is a multiple of 32):
+//   1. one pass for every centroid's max and normaliser: each thread keeps a
+//      running max m and sum z = sum_J exp(l_cJ - m) (expf terms, fp64 sum),
+//      rescaled by exp(m_old - m_new) when m grows; the partial (m, z) pairs
+//      are merged over the warp, then over the CTA, the same way;
 //   2. s_J = sum_c (n_c / 128) exp(l_cJ - max_c) / Z_c, and sum_J s_J;
 //   3. lambda by water-filling: start from lambda = budget / sum(s), then
 //      repeatedly cap the blocks with lambda s >= 1 and set lambda =
 //      (budget - capped) / (sum of the uncapped scores) until the capped
 //      set stops growing (it only grows; at most 64 rounds);
-//   4. block J is sampled iff u_J < min(1, lambda s_J); the sample is
-//      compacted ascending with its shifts -log(pi).
-__global__ void __launch_bounds__(256) ab_select_kernel(const ABSelectArgs a) {
+//   4. block J is sampled iff u_J < min(1, lambda s_J); each warp owns a
+//      contiguous range of J, counts its sample, and after one exchange of
+//      the counts writes it ascending with its shifts -log(pi).
+constexpr int kABSelectWarps = 8;
+__global__ void __launch_bounds__(kABSelectWarps * 32, 3) ab_select_kernel(const ABSelectArgs a) {
   extern __shared__ __align__(16) float sel_sm[];
-  float* sc = sel_sm;                                         // [NKB]
+  float* sc = sel_sm;                                                // [NKB]
   double* red = reinterpret_cast<double*>(sc + ((a.nkb + 3) & ~3));  // [8]
-  float* cmax = reinterpret_cast<float*>(red + 8);            // [8]
-  float* cinv = cmax + 8;                                     // [8]: (n_c / 128) / Z_c
-  int* woff = reinterpret_cast<int*>(cinv + 8);               // [8]
+  double* wsum = red + 8;                                            // [warps][8]
+  float* cmax = reinterpret_cast<float*>(wsum + kABSelectWarps * kABClusters);  // [8]
+  float* cinv = cmax + 8;                                            // [8]: (n_c / 128) / Z_c
+  float* wmax = cinv + 8;                                            // [warps][8]
+  int* woff = reinterpret_cast<int*>(wmax + kABSelectWarps * kABClusters);  // [warps]
   const int I = blockIdx.x;
   const int64_t bh = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nkb = a.nkb;
+  const int nkb = a.nkb, nkb4 = nkb >> 2;
   const int64_t row = bh * a.nqb + I;
   const float* lg = a.logits + (bh * a.nqb * kABClusters + static_cast<int64_t>(I) * kABClusters) * nkb;
-  // 1. per centroid (one warp each): max and normaliser
+  const float4* lg4 = reinterpret_cast<const float4*>(lg);
+  // 1. max and normaliser of every centroid's row
   {
-    const int c = warp;
-    const int n = a.counts[row * kABClusters + c];
-    const float* l = lg + static_cast<int64_t>(c) * nkb;
-    float m = -INFINITY;
-    for (int J = lane; J < nkb; J += 32) m = fmaxf(m, l[J]);
+    float m[kABClusters];
+    double z[kABClusters];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    double z = 0.0;
-    for (int J = lane; J < nkb; J += 32) z += static_cast<double>(expf(l[J] - m));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) {
-      cmax[c] = m;
-      cinv[c] = n > 0 ? static_cast<float>(static_cast<double>(n) / kABQBlock / z) : 0.f;
+    for (int c = 0; c < kABClusters; ++c) {
+      m[c] = -INFINITY;
+      z[c] = 0.0;
     }
+    for (int J4 = tid; J4 < nkb4; J4 += blockDim.x) {
+      float4 x[kABClusters];
+#pragma unroll
+      for (int c = 0; c < kABClusters; ++c) x[c] = __ldg(lg4 + static_cast<int64_t>(c) * nkb4 + J4);
+#pragma unroll
+      for (int c = 0; c < kABClusters; ++c) {
+        const float mn = fmaxf(m[c], fmaxf(fmaxf(x[c].x, x[c].y), fmaxf(x[c].z, x[c].w)));
+        double zc = mn > m[c] ? z[c] * static_cast<double>(expf(m[c] - mn)) : z[c];
+        zc += static_cast<double>(expf(x[c].x - mn));
+        zc += static_cast<double>(expf(x[c].y - mn));
+        zc += static_cast<double>(expf(x[c].z - mn));
+        zc += static_cast<double>(expf(x[c].w - mn));
+        z[c] = zc;
+        m[c] = mn;
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < kABClusters; ++c) {
+      float mw = m[c];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+      // a lane that saw no element (m = -inf) adds nothing
+      double t = m[c] == -INFINITY ? 0.0 : z[c] * static_cast<double>(expf(m[c] - mw));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) {
+        wmax[warp * kABClusters + c] = mw;
+        wsum[warp * kABClusters + c] = t;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < kABClusters) {
+    const int c = tid;
+    float M = -INFINITY;
+    for (int w = 0; w < kABSelectWarps; ++w) M = fmaxf(M, wmax[w * kABClusters + c]);
+    double Z = 0.0;
+    for (int w = 0; w < kABSelectWarps; ++w) {
+      const float mw = wmax[w * kABClusters + c];
+      if (mw != -INFINITY) Z += wsum[w * kABClusters + c] * static_cast<double>(expf(mw - M));
+    }
+    const int n = a.counts[row * kABClusters + c];
+    cmax[c] = M;
+    cinv[c] = n > 0 ? static_cast<float>(static_cast<double>(n) / kABQBlock / Z) : 0.f;
   }
   __syncthreads();
   // 2. block scores
@@ -247,15 +292,27 @@ __global__ void __launch_bounds__(256) ab_select_kernel(const ABSelectArgs a) {
     wloc[c] = cinv[c];
   }
   double tot = 0.0;
-  for (int J = tid; J < nkb; J += blockDim.x) {
-    float s = 0.f;
+  float4* sc4 = reinterpret_cast<float4*>(sc);
+  for (int J4 = tid; J4 < nkb4; J4 += blockDim.x) {
+    float4 x[kABClusters];
+#pragma unroll
+    for (int c = 0; c < kABClusters; ++c) x[c] = __ldg(lg4 + static_cast<int64_t>(c) * nkb4 + J4);
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int c = 0; c < kABClusters; ++c)
-      if (wloc[c] > 0.f) s = __fmaf_rn(wloc[c], expf(lg[static_cast<int64_t>(c) * nkb + J] - mloc[c]), s);
-    sc[J] = s;
-    tot += s;
+      if (wloc[c] > 0.f) {
+        s.x = __fmaf_rn(wloc[c], expf(x[c].x - mloc[c]), s.x);
+        s.y = __fmaf_rn(wloc[c], expf(x[c].y - mloc[c]), s.y);
+        s.z = __fmaf_rn(wloc[c], expf(x[c].z - mloc[c]), s.z);
+        s.w = __fmaf_rn(wloc[c], expf(x[c].w - mloc[c]), s.w);
+      }
+    sc4[J4] = s;
+    tot += s.x;
+    tot += s.y;
+    tot += s.z;
+    tot += s.w;
   }
-  tot = block_sum_f64(tot, red);
+  tot = block_sum_f64(tot, red);  // begins with a barrier: every score is written
   int npos = 0;
   for (int J = tid; J < nkb; J += blockDim.x) npos += sc[J] > 0.f;
   npos = block_sum_int(npos, red);
@@ -285,38 +342,49 @@ __global__ void __launch_bounds__(256) ab_select_kernel(const ABSelectArgs a) {
       lambda = (a.budget - c1) / rest;
     }
   }
-  // 4. sampling and compaction (ascending J, 256 at a time)
+  // 4. sampling and compaction: warp w owns J in [w * seg, (w + 1) * seg)
   const float* u = a.u + row * nkb;
   int32_t* oidx = a.kidx + row * nkb;
   float* osh = a.kshift + row * nkb;
-  int base = 0;
-  for (int J0 = 0; J0 < nkb; J0 += blockDim.x) {
-    const int J = J0 + tid;
-    bool inc = false;
+  const int seg = (nkb + kABSelectWarps * 32 - 1) / (kABSelectWarps * 32) * 32;
+  const int j0 = warp * seg, j1 = min(nkb, j0 + seg);
+  auto sampled = [&](int J, double& pi) {
+    const double s = sc[J];
+    pi = s <= 0.0 ? 0.0 : fmin(1.0, lambda * s);
+    return static_cast<double>(u[J]) < pi;
+  };
+  int mine = 0;
+  for (int b0 = j0; b0 < j1; b0 += 32) {
+    const int J = b0 + lane;
     double pi = 0.0;
-    if (J < nkb) {
-      const double s = sc[J];
-      pi = s <= 0.0 ? 0.0 : fmin(1.0, lambda * s);
-      inc = static_cast<double>(u[J]) < pi;
-    }
+    const bool inc = J < j1 && sampled(J, pi);
+    mine += __popc(__ballot_sync(0xffffffffu, inc));
+  }
+  if (lane == 0) woff[warp] = mine;
+  __syncthreads();
+  int base = 0, total = 0;
+  for (int w = 0; w < kABSelectWarps; ++w) {
+    base += w < warp ? woff[w] : 0;
+    total += woff[w];
+  }
+  for (int b0 = j0; b0 < j1; b0 += 32) {
+    const int J = b0 + lane;
+    double pi = 0.0;
+    const bool inc = J < j1 && sampled(J, pi);
     const unsigned bal = __ballot_sync(0xffffffffu, inc);
-    if (lane == 0) woff[warp] = __popc(bal);
-    __syncthreads();
-    int before = base;
-    for (int w = 0; w < warp; ++w) before += woff[w];
-    int total = base;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) total += woff[w];
     if (inc) {
-      const int pos = before + __popc(bal & ((1u << lane) - 1u));
+      const int pos = base + __popc(bal & ((1u << lane) - 1u));
       oidx[pos] = J;
       osh[pos] = static_cast<float>(-log(pi));
     }
-    __syncthreads();
-    base = total;
+    base += __popc(bal);
   }
-  if (tid == 0) a.kcount[row] = base;
+  if (tid == 0) a.kcount[row] = total;
 }
 
-inline size_t ab_select_smem(int nkb) { return static_cast<size_t>((nkb + 3) & ~3) * 4 + 8 * 8 + 8 * 4 * 2 + 8 * 4; }
+inline size_t ab_select_smem(int nkb) {
+  return static_cast<size_t>((nkb + 3) & ~3) * 4 + 8 * 8 + kABSelectWarps * kABClusters * 8 + 8 * 4 * 2 +
+         kABSelectWarps * kABClusters * 4 + kABSelectWarps * 4;
+}
 
 }  // namespace nabla

@@ -849,7 +849,7 @@ int nabla_ab_plan(const void* q, const void* k, const float* u, int B, int S, in
   if (cudaFuncSetAttribute(ab_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(ssm)) !=
       cudaSuccess)
     return NABLA_ERR_CUDA;
-  ab_select_kernel<<<dim3(nqb, B * Hh), 256, ssm, stream>>>(sa);
+  ab_select_kernel<<<dim3(nqb, B * Hh), kABSelectWarps * 32, ssm, stream>>>(sa);
   return launch_status();
 }
 
