@@ -831,6 +831,16 @@ def main():
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 result["cpu_baseline"] = oracle_sample(w, q, k, v, args.cpu_blocks, heads=args.ref_heads)
+                if w is inputs.TINY:
+                    # the tiny layer's oracle also on one core (its loops are
+                    # over independent rows, so the results are the same)
+                    import oracle
+                    cores = oracle.num_threads()
+                    oracle.set_num_threads(1)
+                    one = oracle_sample(w, q, k, v, args.cpu_blocks, heads=args.ref_heads)
+                    oracle.set_num_threads(cores)
+                    result["cpu_baseline"]["single_core"] = {"value": one["value"], "unit": one["unit"], "cores": 1,
+                                                             "sample_s": one["sample_s"]}
             else:
                 result["cpu_baseline"] = None
             print(json.dumps(result), flush=True)

@@ -67,6 +67,7 @@ def _load():
         lib.oracle_attention_bwd.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, P, P]
         lib.oracle_attention_bwd_sampled.argtypes = [P, P, P, P, P, P, i, i, i, i, d, P, i, P, i, P, P, P]
         lib.oracle_num_threads.restype = i
+        lib.oracle_set_num_threads.argtypes = [i]
         lib.oracle_ab_key_means.argtypes = [P, i, i, i, i, P]
         lib.oracle_ab_kmeans.argtypes = [P, i, i, i, i, i, P, P, P]
         lib.oracle_ab_scores.argtypes = [P, P, P, i, i, i, i, i, f, P]
@@ -85,6 +86,11 @@ def _ptr(a: np.ndarray):
 
 def num_threads() -> int:
     return _load().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops (results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _bits(x: np.ndarray) -> np.ndarray:

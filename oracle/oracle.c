@@ -61,6 +61,17 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the OpenMP loops from now on (n >= 1).  Every loop is over
+ * independent rows, so results do not depend on it; the benchmark uses it
+ * to time the oracle on one core as well as on all of them. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------ */
 /* Fractal flattening (NABLA summary, Metodologia item 1).                   */
 /* Grid order s = (t*H + h)*W + w.  Flattened order: frame-major, then the   */
