@@ -32,14 +32,16 @@
  *     until the stream has executed the call.  Inputs and outputs never alias.
  *   - Calls are asynchronous on the given stream (0 = legacy default stream)
  *     and never synchronise, except nabla_get_status.
- *   - CUDA graphs: the calls of the grid-order path (nabla_flatten_pool_qk,
- *     nabla_build_mask_pooled, nabla_sparse_attn_fwd_grid and its _split
- *     form, nabla_transpose_lists, nabla_sparse_attn_bwd_grid) launch only
- *     on the given stream and allocate nothing, so a sequence of them can be
- *     captured into one CUDA graph; replaying it on new data in the same
- *     buffers gives the same bits as making the calls directly.  Make the
- *     library's first call on a device outside a capture (it looks up the
- *     device's attributes and the driver's tensor-map encoder).
+ *   - CUDA graphs: nabla_flatten, nabla_unflatten, nabla_build_mask,
+ *     nabla_build_mask_grid, nabla_flatten_pool_qk, nabla_build_mask_pooled,
+ *     nabla_build_mask_sta, nabla_build_mask_radial, the nabla_sparse_attn_fwd
+ *     calls (flattened, grid order, key-range split), nabla_transpose_lists,
+ *     both nabla_sparse_attn_bwd calls, nabla_ab_plan and nabla_ab_attn_fwd
+ *     launch only on the given stream and allocate nothing, so a sequence
+ *     of them can be captured into one CUDA graph; replaying it on new data
+ *     in the same buffers gives the same bits as making the calls directly.
+ *     Make the library's first call on a device outside a capture (it looks
+ *     up the device's attributes and the driver's tensor-map encoder).
  *   - Return value: NABLA_OK, or an error code; on error nothing is launched.
  *     Device-side faults of the data (an out-of-range block index, a wait that
  *     ran out of time) are recorded in a per-device status word that

@@ -2,14 +2,17 @@
 
 A serving loop or a training step that replays a CUDA graph per layer needs
 every call it captures to allocate nothing, never synchronise and launch only
-on the caller's stream.  The hot path's entry points are written that way:
-the pooling from grid order, the mask on the pooled workspace, the
-attention (one key range, and two ranges with their merge), the column lists
-and the backward pass.  Here they are captured once on static buffers, and
-every replay on new inputs must give the same bits as the same calls run
-eagerly on those inputs (the kernels are deterministic: no atomics, fixed
-summation orders).  nabla_get_status synchronises and stays outside the
-graph."""
+on the caller's stream.  The entry points are written that way.  Captured
+here once on static buffers: the grid-order hot path (pooling, mask on the
+pooled workspace, attention with one key range and with two plus their
+merge, column lists, backward), and in a second graph the other paths (the
+materialised flattening, the mask and attention on flattened tensors, the
+unflattening and the flattened backward, the one-call grid-order mask, the
+static sliding-tile and radial windows, the AB-Attention plan and
+attention).  Every replay on new inputs must give the same bits as the same
+calls run eagerly on those inputs (the kernels are deterministic: no
+atomics, fixed summation orders).  nabla_get_status synchronises and stays
+outside the graphs."""
 import numpy as np
 import pytest
 import torch
@@ -128,4 +131,100 @@ def test_graph_replay_equals_eager(B, Hh, D, grid, thr, sta, split):
             torch.cuda.synchronize()
             assert nabla.get_status() == 0
             _same(layer.results(), eager[s], f"replay {rep} on input set {s}")
+    del graph
+
+
+def _masked(cnt, idx):
+    """Host copies of block lists with the entries past each count cleared."""
+    c, x = cnt.cpu().numpy(), idx.cpu().numpy().copy()
+    x[np.arange(x.shape[-1])[None, None, None, :] >= c[..., None]] = -1
+    return c, x
+
+
+def _bits(t):
+    return (t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)).cpu().numpy()
+
+
+def test_graph_replay_other_paths():
+    B, Hh, D, grid, thr, sta, r0 = 1, 2, 128, (4, 32, 64), 0.9, (3, 3, 3), 2
+    T, H, W = grid
+    S, Nb = T * H * W, T * H * W // 64
+    ab = inputs.ABWorkload("graph AB", inputs.Workload("graph-ab", B, Hh, D, T, H, W, 1.0, 1.0, seed=71), 0.1)
+    dev = torch.device("cuda")
+    q, k, v, do = (torch.empty((B, S, Hh, D), dtype=torch.bfloat16, device=dev) for _ in range(4))
+    u = torch.empty((B, Hh, ab.nqb, ab.nkb), dtype=torch.float32, device=dev)
+    qf, kf, vf, of, og, dq, dk, dv = (torch.empty_like(q) for _ in range(8))
+    lse, delta = (torch.empty((B, Hh, S), dtype=torch.float32, device=dev) for _ in range(2))
+    ws = torch.empty(nabla.mask_workspace_bytes(B, Hh, D, T, H, W, nabla.params(thr, sta)), dtype=torch.uint8,
+                     device=dev)
+    lists = {n: (torch.empty((B, Hh, Nb), dtype=torch.int32, device=dev),
+                 torch.empty((B, Hh, Nb, Nb), dtype=torch.int32, device=dev)) for n in ("flat", "grid", "sta", "rad", "t")}
+    ab_ws = torch.empty(nabla.ab_workspace_bytes(B, S, Hh, D), dtype=torch.uint8, device=dev)
+    kcount = torch.empty((B, Hh, ab.nqb), dtype=torch.int32, device=dev)
+    kidx = torch.empty((B, Hh, ab.nqb, ab.nkb), dtype=torch.int32, device=dev)
+    kshift = torch.empty((B, Hh, ab.nqb, ab.nkb), dtype=torch.float32, device=dev)
+    oab, lse_ab = torch.empty_like(q), torch.empty((B, Hh, S), dtype=torch.float32, device=dev)
+
+    def step():
+        for src, dst in ((q, qf), (k, kf), (v, vf)):
+            nabla.flatten(src, T, H, W, out=dst)
+        cf, xf = lists["flat"]
+        nabla.build_mask(qf, kf, T, H, W, thr, sta, kv_count=cf, kv_idx=xf, workspace=ws)
+        nabla.sparse_attn_fwd(qf, kf, vf, cf, xf, out=of, lse=lse)
+        nabla.unflatten(of, T, H, W, out=og)
+        ct, xt = lists["t"]
+        nabla.transpose_lists(cf, xf, q_count=ct, q_idx=xt)
+        nabla.sparse_attn_bwd(qf, kf, vf, of, do, lse, cf, xf, q_lists=(ct, xt), dq=dq, dk=dk, dv=dv, delta=delta)
+        cg, xg = lists["grid"]
+        nabla.build_mask_grid(q, k, T, H, W, thr, sta, kv_count=cg, kv_idx=xg, workspace=ws)
+        nabla.build_mask_sta(B, Hh, T, H, W, sta, kv_count=lists["sta"][0], kv_idx=lists["sta"][1])
+        nabla.build_mask_radial(B, Hh, T, H, W, r0, kv_count=lists["rad"][0], kv_idx=lists["rad"][1])
+        nabla.ab_plan(q, k, u, ab.budget, ab.kmeans_iters, kcount=kcount, kidx=kidx, kshift=kshift, workspace=ab_ws)
+        nabla.ab_attn_fwd(q, k, v, kcount, kidx, kshift, out=oab, lse=lse_ab)
+
+    def results():
+        out = {}
+        for n, (c, x) in lists.items():
+            out[n + "_count"], out[n + "_idx"] = _masked(c, x)
+        kc, ki = _masked(kcount, kidx)
+        ks = kshift.cpu().numpy().copy()
+        ks[np.arange(ab.nkb)[None, None, None, :] >= kc[..., None]] = 0.0
+        out.update(kcount=kc, kidx=ki, kshift=ks.view(np.int32))
+        for name, t in (("of", of), ("og", og), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("oab", oab),
+                        ("lse_ab", lse_ab)):
+            out[name] = _bits(t)
+        return out
+
+    sets = []
+    for seed in (401, 402):
+        tensors = _inputs(B, Hh, D, grid, seed)
+        g = torch.Generator().manual_seed(seed + 50)
+        tensors.append(torch.rand((B, Hh, ab.nqb, ab.nkb), generator=g).cuda())
+        sets.append(tensors)
+
+    def load(tensors):
+        for dst, src in zip((q, k, v, do, u), tensors):
+            dst.copy_(src)
+
+    eager = []
+    for tensors in sets:
+        load(tensors)
+        step()
+        torch.cuda.synchronize()
+        assert nabla.get_status() == 0
+        eager.append(results())
+    assert not np.array_equal(eager[0]["oab"], eager[1]["oab"])
+    assert not np.array_equal(eager[0]["of"], eager[1]["of"])
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    for rep in range(2):
+        for s in (1, 0):
+            load(sets[s])
+            graph.replay()
+            torch.cuda.synchronize()
+            assert nabla.get_status() == 0
+            _same(results(), eager[s], f"replay {rep} on input set {s}")
     del graph
