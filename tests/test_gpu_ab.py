@@ -13,7 +13,6 @@ acelera a geracao de video em ate 2,23x e pula 92% da atencao", section
   pi = 1, i.e. dense attention), a tiny budget (mostly one or two blocks),
   D = 64, batch 2, a list entry out of range (skipped and reported).
 """
-import math
 
 import numpy as np
 import pytest

@@ -9,7 +9,6 @@ against the oracle's own mask.
 """
 import gc
 
-import numpy as np
 import pytest
 import torch
 

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from _parity import Case, LSE_ABS, MAX_ABS, MEAN_ABS, check_attention, compare_masks, oracle_masks
+from _parity import Case, LSE_ABS, MAX_ABS, MEAN_ABS, check_attention, compare_masks
 from block_sparse_attention_flatten_b200 import inputs
 from block_sparse_attention_flatten_b200 import nabla
 
