@@ -9,18 +9,23 @@
 // is the full M = 128 of tcgen05.mma).  A tile of keys is 16 sampled blocks
 // = 64 keys; tile n holds sample entries 16n .. 16n+15, the last one padded
 // with zero rows whose shift is -inf (probability 0).
-// Warp roles (224 threads, two CTAs per SM):
+// Warp roles (256 threads, two CTAs per SM):
 //   warps 0-3  softmax: thread t = query row t = TMEM lane t; scores of the
 //              tile plus the keys' shifts, online max/sum with the lazy O
 //              rescale, bf16 P written back into the score buffer's TMEM;
 //              epilogue O / l and the LSE.
-//   warp 4     gather (all 32 lanes): each lane copies 16-byte pieces of the
-//              tile's K and V rows with cp.async into the 128-byte-swizzled
-//              layout a TMA box would produce, and writes the tile's shifts;
-//              then waits for its copies, fences them for the tensor core's
-//              (async) proxy and arrives on the stage's full barrier.
+//   warp 4     K gather (all 32 lanes): each lane copies 16-byte pieces of
+//              the tile's K rows with cp.async into the 128-byte-swizzled
+//              layout a TMA box would produce, then waits for its copies,
+//              fences them for the tensor core's (async) proxy and arrives
+//              on the K stage's full barrier.
+//   warp 7     V gather, the same for V, and the tile's shifts.
 //   warp 5     QK^T issuer (one thread): S = Q K^T (M 128, N 64, K = D).
 //   warp 6     PV issuer (one thread): O += P V (M 128, N = D, K 64).
+// K and V have rings of their own: a K stage is refilled as soon as its
+// QK^T is done, so the gather of tile n+2's keys runs while tile n is in
+// the softmax; a V stage (with the tile's shifts, which the softmax reads)
+// is refilled once its PV is done.
 // Tensor memory per CTA: S0 | S1 (64 columns each, P in their first 32) |
 // O (D columns).  Every wait is bounded; see attn_fwd.cuh.
 #pragma once
@@ -29,7 +34,7 @@
 
 namespace nabla {
 
-constexpr int kABAttnThreads = 224;
+constexpr int kABAttnThreads = 256;
 
 template <int D>
 struct ABAttnSmem {
@@ -40,10 +45,11 @@ struct ABAttnSmem {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kQBytes;
   static constexpr int kV = kK + kStages * kKVBytes;
-  static constexpr int kShift = kV + kStages * kKVBytes;  // [stages][64] fp32, log2 units
+  static constexpr int kShift = kV + kStages * kKVBytes;  // [stages][64] fp32, log2 units (with V)
   static constexpr int kBars = kShift + kStages * 64 * 4;
-  // q_full, kv_full[stages], kv_empty[stages], s_full[2], p_full[2], pv_done[2], mma_drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 6 + 1;
+  // q_full, k_full[stages], k_empty[stages], v_full[stages], v_empty[stages],
+  // s_full[2], p_full[2], pv_done[2], mma_drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 6 + 1;
   static constexpr int kMisc = kBars + 8 * kNumBars;
   static constexpr size_t kBytes = 1024 + kMisc + 32;
 };
@@ -70,9 +76,11 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;  // [2]
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kStages;
+  uint64_t* v_full = k_empty + kStages;
+  uint64_t* v_empty = v_full + kStages;
+  uint64_t* s_full = v_empty + kStages;  // [2]
   uint64_t* p_full = s_full + 2;          // [2]
   uint64_t* pv_done = p_full + 2;         // [2]
   uint64_t* mma_drain = pv_done + 2;
@@ -94,8 +102,10 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
   if (tid == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(kv_full + s, 32);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(k_full + s, 32);  // one arrival per gathering lane
+      mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 32);
+      mbar_init(v_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
@@ -124,52 +134,54 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
   const uint32_t sQ = smem_u32(sm + L::kQ), sK = smem_u32(sm + L::kK), sV = smem_u32(sm + L::kV);
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ gather
+  if (warp == 4 || warp == 7) {
+    // ------------------------------------------------------ K or V gather
+    const bool is_v = warp == 7;
     const int32_t* lst = a.kidx + row * a.nkb;
     const float* shl = a.kshift + row * a.nkb;
     const int64_t tok_stride = static_cast<int64_t>(a.Hh) * D;  // elements between consecutive tokens
-    const __nv_bfloat16* kbase = a.k + (static_cast<int64_t>(b) * a.S * a.Hh + hd) * D;
-    const __nv_bfloat16* vbase = a.v + (static_cast<int64_t>(b) * a.S * a.Hh + hd) * D;
+    const __nv_bfloat16* base = (is_v ? a.v : a.k) + (static_cast<int64_t>(b) * a.S * a.Hh + hd) * D;
+    uint64_t* full = is_v ? v_full : k_full;
+    uint64_t* empty = is_v ? v_empty : k_empty;
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % kStages;
-      if (n >= kStages && !__all_sync(0xffffffffu, mbar_wait(kv_empty + s, ((n / kStages) - 1) & 1, abort_flag)))
+      if (n >= kStages && !__all_sync(0xffffffffu, mbar_wait(empty + s, ((n / kStages) - 1) & 1, abort_flag)))
         break;
       int j = -1;
-      float sh = -INFINITY;
       if (lane < 16) {
         const int e = 16 * n + lane;
+        float sh = -INFINITY;
         if (e < cnt) {
           const int jj = __ldg(lst + e);
           if (jj < 0 || jj >= a.nkb) {
-            report(NABLA_ERR_DEVICE_BOUNDS);
+            if (!is_v) report(NABLA_ERR_DEVICE_BOUNDS);
           } else {
             j = jj;
             sh = __ldg(shl + e) * 1.4426950408889634f;
           }
         }
-        float* sd = shift_s + s * 64 + 4 * lane;
-        const float w = j >= 0 ? sh : -INFINITY;
-        sd[0] = w;
-        sd[1] = w;
-        sd[2] = w;
-        sd[3] = w;
+        if (is_v) {
+          float* sd = shift_s + s * 64 + 4 * lane;
+          const float w = j >= 0 ? sh : -INFINITY;
+          sd[0] = w;
+          sd[1] = w;
+          sd[2] = w;
+          sd[3] = w;
+        }
       }
-      unsigned char* kd = sm + L::kK + s * L::kKVBytes;
-      unsigned char* vd = sm + L::kV + s * L::kKVBytes;
+      unsigned char* dstage = sm + (is_v ? L::kV : L::kK) + s * L::kKVBytes;
       for (int x = lane; x < 64 * kRowChunks; x += 32) {
         const int kr = x / kRowChunks, cc = x - kr * kRowChunks;
         const int jj = __shfl_sync(0xffffffffu, j, kr >> 2);
         const bool valid = jj >= 0;
         const int64_t off = valid ? (static_cast<int64_t>(jj) * 4 + (kr & 3)) * tok_stride + cc * 8 : 0;
         const int dst = (cc >> 3) * (64 * 128) + kr * 128 + (((cc & 7) ^ (kr & 7)) << 4);
-        cp_async16_zfill(kd + dst, kbase + off, valid);
-        cp_async16_zfill(vd + dst, vbase + off, valid);
+        cp_async16_zfill(dstage + dst, base + off, valid);
       }
       cp_async_commit();
       cp_async_wait<0>();
       fence_proxy_async_smem();
-      mbar_arrive(kv_full + s);
+      mbar_arrive(full + s);
     }
     cp_async_wait<0>();
   } else if (warp == 5) {
@@ -179,7 +191,7 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
       tc_fence_after();
       for (int n = 0; ok && n < n_tiles; ++n) {
         const int s = n % kStages;
-        if (!mbar_wait(kv_full + s, (n / kStages) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(k_full + s, (n / kStages) & 1, abort_flag)) { ok = false; break; }
         if (n >= 2 && !mbar_wait(pv_done + (n & 1), ((n - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kb = sK + s * L::kKVBytes;
@@ -192,6 +204,7 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
           umma_bf16_ss(tS, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full + (n & 1));
+        umma_commit(k_empty + s);
       }
       umma_commit(mma_drain);
       mbar_wait_drain(mma_drain, 0);
@@ -204,7 +217,7 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
       for (int m = 0; ok && m < n_tiles; ++m) {
         const int s = m % kStages;
         if (!mbar_wait(p_full + (m & 1), (m >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(kv_full + s, (m / kStages) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(v_full + s, (m / kStages) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t pa = (m & 1) ? tS1 : tS0;
         const uint32_t vb = sV + s * L::kKVBytes;
@@ -214,7 +227,7 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
           umma_bf16_ts(tO, pa + kk * 8, bd, kIdescPV, (m > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(pv_done + (m & 1));
-        umma_commit(kv_empty + s);
+        umma_commit(v_empty + s);
       }
       umma_commit(mma_drain);
       mbar_wait_drain(mma_drain, 0);
@@ -227,8 +240,10 @@ __global__ void __launch_bounds__(kABAttnThreads, 2)
     bool ok = true;
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % kStages;
-      // the shifts of this tile are published with the stage's full barrier
-      if (!__all_sync(0xffffffffu, mbar_wait(kv_full + s, (n / kStages) & 1, abort_flag) &&
+      // the shifts of this tile are published with its V stage's full
+      // barrier (that stage is refilled only after this tile's PV, so the
+      // barrier cannot run a phase ahead of this wait)
+      if (!__all_sync(0xffffffffu, mbar_wait(v_full + s, (n / kStages) & 1, abort_flag) &&
                                        mbar_wait(s_full + (n & 1), (n >> 1) & 1, abort_flag))) {
         ok = false;
         break;
