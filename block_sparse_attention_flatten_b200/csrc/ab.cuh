@@ -77,8 +77,10 @@ __global__ void __launch_bounds__(256) ab_key_means_kernel(const __nv_bfloat16* 
 //     distances of query t to centroids 4*half .. 4*half+3 (diff rounded to
 //     fp32, then an fmaf chain over d ascending), keeps the nearest (ties to
 //     the lower index) and settles with its partner lane;
+//   members: one warp lists each cluster's queries in ascending token order
+//     (ballots over 32 queries at a time);
 //   update: thread owns (c, d) pairs; the fp32 sum over the cluster's
-//     queries in ascending token order, one division by the count; an empty
+//     listed queries in that order, one division by the count; an empty
 //     cluster keeps its centroid.
 __global__ void __launch_bounds__(256) ab_kmeans_kernel(const __nv_bfloat16* __restrict__ q,
                                                         float* __restrict__ centT, int32_t* __restrict__ counts,
@@ -91,6 +93,8 @@ __global__ void __launch_bounds__(256) ab_kmeans_kernel(const __nv_bfloat16* __r
   float* mu = x + kABQBlock * ld;         // [8][D]
   int* asg = reinterpret_cast<int*>(mu + kABClusters * D);  // [128]
   int* cnt = asg + kABQBlock;             // [8]
+  int* mem = cnt + kABClusters;           // [8][128]: each cluster's queries, ascending
+  int* mcount = mem + kABClusters * kABQBlock;  // [8]
   const int tid = threadIdx.x;
   const int chunks = D >> 3;  // 16-byte chunks of one head's slice of a token row
   for (int u = tid; u < kABQBlock * chunks; u += blockDim.x) {
@@ -142,16 +146,33 @@ __global__ void __launch_bounds__(256) ab_kmeans_kernel(const __nv_bfloat16* __r
     // the lower half's candidate has the lower index: it wins ties
     if (half == 0) asg[t] = (obd < bd) ? obest : best;
     __syncthreads();
-    // update: pairs (c, d), c = u / D
+    // members of each cluster, ascending
+    if (tid < 32) {
+      const int lane = tid;
+      int nb[kABClusters];
+#pragma unroll
+      for (int c = 0; c < kABClusters; ++c) nb[c] = 0;
+      for (int s0 = 0; s0 < kABQBlock; s0 += 32) {
+        const int a_s = asg[s0 + lane];
+#pragma unroll
+        for (int c = 0; c < kABClusters; ++c) {
+          const unsigned bal = __ballot_sync(0xffffffffu, a_s == c);
+          if (a_s == c) mem[c * kABQBlock + nb[c] + __popc(bal & ((1u << lane) - 1u))] = s0 + lane;
+          nb[c] += __popc(bal);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kABClusters; ++c)
+        if (lane == c) mcount[c] = nb[c];
+    }
+    __syncthreads();
+    // update: pairs (c, d), c = u / D (one c per warp: D >= 32)
     for (int u = tid; u < kABClusters * D; u += blockDim.x) {
       const int c = u / D, d = u - c * D;
+      const int n = mcount[c];
+      const int* mc = mem + c * kABQBlock;
       float acc = 0.f;
-      int n = 0;
-      for (int s = 0; s < kABQBlock; ++s)
-        if (asg[s] == c) {
-          acc = __fadd_rn(acc, x[s * ld + d]);
-          ++n;
-        }
+      for (int e = 0; e < n; ++e) acc = __fadd_rn(acc, x[mc[e] * ld + d]);
       if (n > 0) mu[u] = __fdiv_rn(acc, static_cast<float>(n));
       if (d == 0) cnt[c] = n;
     }
@@ -167,7 +188,8 @@ __global__ void __launch_bounds__(256) ab_kmeans_kernel(const __nv_bfloat16* __r
 }
 
 inline size_t ab_kmeans_smem(int D) {
-  return (static_cast<size_t>(kABQBlock) * (D + 1) + kABClusters * D) * 4 + kABQBlock * 4 + kABClusters * 4;
+  return (static_cast<size_t>(kABQBlock) * (D + 1) + kABClusters * D) * 4 + kABQBlock * 4 + kABClusters * 4 +
+         kABClusters * kABQBlock * 4 + kABClusters * 4;
 }
 
 struct ABSelectArgs {
