@@ -159,3 +159,54 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 64, 8, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         nabla.flatten(x, 1, 8, 8)
+
+
+def _c_caller_source():
+    """A plain C program that includes the header, takes the address of
+    every declared function (so the link must resolve them all) and calls
+    the host-only paths: the error strings, the workspace size arithmetic
+    and an argument rejection, none of which touches a GPU."""
+    fns = header_functions()
+    table = ",\n    ".join(f"(void (*)(void))&{f}" for f in fns)
+    return f"""#include <stdio.h>
+#include <string.h>
+#include "nabla.h"
+
+static void (*const every_entry_point[])(void) = {{
+    {table}
+}};
+
+int main(void) {{
+  nabla_params prm;
+  size_t ws;
+  int rc;
+  memset(&prm, 0, sizeof prm);
+  prm.P = 8;
+  prm.thr = 0.9f;
+  ws = nabla_mask_workspace_bytes(1, 2, 64, 4, 16, 16, &prm);
+  /* grid 4 x 16 x 16 = 16 blocks: pooled Q and K, fp32 [1][2][64][16]
+     each, then the block scores, fp32 [1][2][16][16] */
+  rc = nabla_flatten(NULL, NULL, 1, 4, 16, 16, 8, 128, NULL);
+  printf("%u %zu %d %s\\n", (unsigned)(sizeof every_entry_point / sizeof every_entry_point[0]), ws, rc,
+         nabla_strerror(NABLA_ERR_INVALID));
+  return 0;
+}}
+"""
+
+
+@pytest.mark.parametrize("compiler", [["gcc", "-std=c99", "-pedantic"], ["g++", "-std=c++17", "-x", "c++"]],
+                         ids=["c99", "c++17"])
+def test_header_compiles_links_and_rejects_from_c(lib, tmp_path, compiler):
+    import subprocess
+    src = tmp_path / "caller.c"
+    src.write_text(_c_caller_source())
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(nbuild.LIB)
+    cmd = compiler + ["-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                      "-L", libdir, "-lnabla", f"-Wl,-rpath,{libdir}"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split(maxsplit=3)
+    assert int(out[0]) == len(header_functions())
+    assert int(out[1]) == 2 * 4 * 2 * 64 * 16 + 4 * 2 * 16 * 16
+    assert int(out[2]) == nabla.NABLA_ERR_INVALID  # null pointers: rejected before any CUDA call
+    assert out[3].strip() == nabla.strerror(nabla.NABLA_ERR_INVALID)
