@@ -1,6 +1,7 @@
-"""The N > 1 path of bench.py on the CPU: two gloo ranks run the same
+"""bench.py on the CPU: the N > 1 path, where two gloo ranks run the same
 aggregation the GPU ranks run over NCCL (one independent replica per rank,
-no data exchange; the job's time is the slowest rank's)."""
+no data exchange; the job's time is the slowest rank's), the peak
+choice, and the reference arm's contract line."""
 import os
 import socket
 import sys
@@ -73,3 +74,42 @@ def test_peak_choice_follows_the_timed_region(tmp_path, monkeypatch):
     assert (peak, burst) == (1615.5, 1615.5) and "burst" in kind
     monkeypatch.setattr(bench, "ROOT", str(tmp_path / "absent"))
     assert bench.tensor_peak(22.0)[0] == 1590.0 and bench.tensor_peak(2000.0)[0] == 1400.0
+
+
+def _bench(args, env_extra=None):
+    import subprocess
+    env = dict(os.environ, **(env_extra or {}))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, capture_output=True, text=True,
+                          env=env, timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the CPU oracle, the one other place the
+    benchmark runs it) prints one JSON line with the contract's keys, the
+    GPU arm's metric and unit, and an e2e object with no host copies."""
+    import json
+
+    sys.path.insert(0, ROOT)
+    import bench
+    r = _bench(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "3"])
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
+    assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["config"]["workload"] == bench.CONFIGS["tiny"].name
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    r = _bench(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "3"],
+               {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_bench_rejects_fewer_than_three_warmup_steps():
+    r = _bench(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0 and "warmup" in r.stderr
