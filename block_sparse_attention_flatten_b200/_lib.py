@@ -5,6 +5,11 @@ dtype and layout, allocates missing outputs with torch (the library itself
 allocates no device memory), and passes raw device pointers, sizes and the
 current CUDA stream to the C entry point of the same name (include/nabla.h).
 There is no CPU fallback: a missing library or a non-CUDA tensor raises.
+
+To capture calls in a CUDA graph, pass every output and workspace
+preallocated (then nothing here allocates, and the calls launch only on the
+capturing stream); get_status and validate_mask synchronise and stay
+outside a capture.
 """
 from __future__ import annotations
 
